@@ -1,0 +1,309 @@
+"""CPU float64 oracle of the FNO spectral-convolution block and of the small FNO
+network built from it.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports, calls or links
+this module: only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` do.  It shares no code, tables or helpers with the CUDA
+library, and it never reads a value the CUDA library produced.
+
+Sources (web pages; cited by title and section):
+
+* [MPFNO] "Model-Parallel Fourier Neural Operators as Learned Surrogates for
+  Large-Scale Parametric PDEs" (review page), section "Proposed method": the
+  network is the original FNO -- a lifting, four spectral blocks of embedding
+  width 20, a projection -- and its spectral convolution is the operation
+  written in FNO's linear-algebra form; gradients come from automatic
+  differentiation (same section, last item).
+* [MPTRAIN] "Guaranteed approximation bounds and efficient mixed-precision
+  training for neural operators" (summary page), "key insights": the Fourier
+  transform may run below full precision, the spectral contraction is a
+  memory-bound half-precision tensor contraction, and a tanh pre-activation is
+  applied before the Fourier transform.
+
+The pages do not print the block's equations.  The oracle computes the
+standard FNO block, with the readings listed below; each is repeated in the
+repository's design notes.
+
+Notation: ``x`` has shape ``[B, C, N_0, ..., N_{d-1}]``; the last axis is the
+real-FFT axis.  The kept mode set ``K`` holds, on each non-last axis ``j``, the
+wavenumbers ``0..m_j-1`` followed by ``N_j-m_j..N_j-1`` (positive block first,
+negative block second), and on the last axis ``0..m_{d-1}-1``; ``K`` is
+flattened row-major in that order.  ``theta(k, n) = 2*pi*sum_j k_j n_j / N_j``.
+
+Readings (where the pages are silent):
+
+1. Forward transform unnormalised, inverse scaled by ``1/N`` (``N = prod N_j``).
+2. Inverse of the half spectrum: ``y[n] = (1/N) sum_{k in K} c_k Re(Y_k e^{+i theta})``
+   with ``c_k = 1`` when ``k_{d-1} = 0`` or ``k_{d-1} = N_{d-1}/2`` and 2 otherwise
+   (the imaginary part of a DC/Nyquist column is dropped, as a C2R inverse does).
+3. GELU is the exact erf form ``p * Phi(p)``.
+4. tanh pre-activation feeds the spectral branch only; the 1x1 path sees raw x.
+5. Complex gradient convention: ``dZ = dL/dRe Z + i dL/dIm Z``.
+
+Parity pins: ``tests/test_oracle.py`` (closed forms, invariants, brute force,
+library DFT, finite differences, hand-derived fixtures under ``tests/golden``).
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+TANH_PREACT = 1
+NO_ACT = 2
+
+_SQRT1_2 = 1.0 / math.sqrt(2.0)
+_INV_SQRT_2PI = 1.0 / math.sqrt(2.0 * math.pi)
+
+
+# --------------------------------------------------------------------------
+# mode bookkeeping
+# --------------------------------------------------------------------------
+
+def axis_wavenumbers(n_points: int, m: int, last: bool) -> np.ndarray:
+    """Kept wavenumbers of one axis, in storage order (reading 1 of the header)."""
+    if last:
+        if not 1 <= m <= n_points // 2 + 1:
+            raise ValueError("last-axis modes out of range")
+        return np.arange(m)
+    if not 1 <= 2 * m <= n_points:
+        raise ValueError("non-last-axis modes out of range")
+    return np.concatenate([np.arange(m), np.arange(n_points - m, n_points)])
+
+
+def kept_shape(grid, modes):
+    d = len(grid)
+    return tuple(len(axis_wavenumbers(grid[j], modes[j], j == d - 1)) for j in range(d))
+
+
+def num_modes(grid, modes) -> int:
+    return int(np.prod(kept_shape(grid, modes)))
+
+
+def mode_weights(grid, modes) -> np.ndarray:
+    """``c_k`` over the flattened K (reading 2): 1 on the DC/Nyquist column, else 2."""
+    d = len(grid)
+    kl = axis_wavenumbers(grid[-1], modes[-1], True)
+    nl = grid[-1]
+    c_last = np.where((kl == 0) | ((nl % 2 == 0) & (kl == nl // 2)), 1.0, 2.0)
+    lead = int(np.prod(kept_shape(grid, modes)[:-1])) if d > 1 else 1
+    return np.tile(c_last, lead)
+
+
+def _exp_matrix(n_points: int, ks: np.ndarray, sign: int) -> np.ndarray:
+    """``E[k, n] = exp(sign * 2 pi i ((k n) mod N) / N)`` for the kept ``k``."""
+    n = np.arange(n_points)
+    phase = 2.0 * np.pi * (np.outer(ks, n) % n_points) / n_points
+    return np.cos(phase) + sign * 1j * np.sin(phase)
+
+
+# --------------------------------------------------------------------------
+# the two truncated transforms
+# --------------------------------------------------------------------------
+
+def truncated_dft(s: np.ndarray, modes) -> np.ndarray:
+    """``S[b, c, k] = sum_n s[b, c, n] exp(-i theta(k, n))`` for ``k`` in K.
+
+    The d-dimensional sum is applied one axis at a time with explicit
+    exponential matrices (the sum is separable; this only reorders it).
+    Returns ``[B, C, |K|]`` complex128.
+    """
+    s = np.asarray(s)
+    b, c = s.shape[:2]
+    grid = s.shape[2:]
+    d = len(grid)
+    out = s.astype(np.complex128)
+    for j in range(d - 1, -1, -1):
+        ks = axis_wavenumbers(grid[j], modes[j], j == d - 1)
+        e = _exp_matrix(grid[j], ks, -1)                       # [kept_j, N_j]
+        out = np.moveaxis(np.tensordot(out, e, axes=([2 + j], [1])), -1, 2 + j)
+    return out.reshape(b, c, -1)
+
+
+def inverse_sum(v: np.ndarray, grid, modes) -> np.ndarray:
+    """``u[b, c, n] = sum_{k in K} Re(v[b, c, k] exp(+i theta(k, n)))`` (no scale).
+
+    ``v`` is ``[B, C, |K|]`` complex; returns ``[B, C, *grid]`` float64.
+    """
+    v = np.asarray(v, dtype=np.complex128)
+    b, c = v.shape[:2]
+    d = len(grid)
+    out = v.reshape((b, c) + kept_shape(grid, modes))
+    for j in range(d):
+        ks = axis_wavenumbers(grid[j], modes[j], j == d - 1)
+        e = _exp_matrix(grid[j], ks, +1)                       # [kept_j, N_j]
+        out = np.moveaxis(np.tensordot(out, e, axes=([2 + j], [0])), -1, 2 + j)
+    return out.real.copy()
+
+
+# --------------------------------------------------------------------------
+# activations
+# --------------------------------------------------------------------------
+
+try:  # vectorised library erf; math.erf element by element otherwise
+    from scipy.special import erf as _erf
+except ImportError:  # pragma: no cover
+    def _erf(z):
+        return np.vectorize(math.erf, otypes=[np.float64])(z)
+
+
+def gelu(p: np.ndarray) -> np.ndarray:
+    """Exact GELU ``p * Phi(p)``, ``Phi`` the standard normal CDF (reading 3)."""
+    p = np.asarray(p, dtype=np.float64)
+    return 0.5 * p * (1.0 + _erf(p * _SQRT1_2))
+
+
+def gelu_grad(p: np.ndarray) -> np.ndarray:
+    """``d/dp [p Phi(p)] = Phi(p) + p phi(p)``."""
+    p = np.asarray(p, dtype=np.float64)
+    return 0.5 * (1.0 + _erf(p * _SQRT1_2)) + p * _INV_SQRT_2PI * np.exp(-0.5 * p * p)
+
+
+# --------------------------------------------------------------------------
+# spectral convolution and block
+# --------------------------------------------------------------------------
+
+def _pointwise(mat: np.ndarray, v: np.ndarray) -> np.ndarray:
+    """``out[b, o, n] = sum_i mat[o, i] v[b, i, n]`` (a 1x1 convolution)."""
+    return np.einsum("oi,bi...->bo...", np.asarray(mat, np.float64), v)
+
+
+def _outer_sum(u: np.ndarray, v: np.ndarray) -> np.ndarray:
+    """``out[o, i] = sum_{b, n} u[b, o, n] v[b, i, n]`` over batch and grid points."""
+    u2 = np.asarray(u, np.float64).reshape(u.shape[0], u.shape[1], -1)
+    v2 = np.asarray(v, np.float64).reshape(v.shape[0], v.shape[1], -1)
+    return np.einsum("bon,bin->oi", u2, v2)
+
+
+def _bcast(vec: np.ndarray, d: int) -> np.ndarray:
+    return np.asarray(vec, np.float64).reshape((1, -1) + (1,) * d)
+
+
+def spectral_conv_fwd(x, r, modes, flags: int = 0):
+    """Spectral branch of the block.
+
+    ``s = tanh(x)`` if TANH_PREACT ([MPTRAIN] key insights) else ``x``;
+    ``xhat = DFT_K(s)``; ``yhat[b,o,k] = sum_i xhat[b,i,k] r[i,o,k]``;
+    ``y = (1/N) sum_k c_k Re(yhat e^{+i theta})``.
+    Returns ``(y, xhat)``.
+    """
+    x = np.asarray(x, np.float64)
+    grid = x.shape[2:]
+    s = np.tanh(x) if flags & TANH_PREACT else x
+    xhat = truncated_dft(s, modes)
+    yhat = np.einsum("bik,iok->bok", xhat, np.asarray(r, np.complex128))
+    w = mode_weights(grid, modes) / float(np.prod(grid))
+    return inverse_sum(yhat * w, grid, modes), xhat
+
+
+def spectral_conv_bwd(x, r, xhat, dy, modes, flags: int = 0):
+    """Adjoint of :func:`spectral_conv_fwd` (gradients by differentiation, [MPFNO]).
+
+    ``dyhat = (c_k/N) DFT_K(dy)``; ``dR = sum_b conj(xhat) dyhat``;
+    ``dxhat = sum_o dyhat conj(R)``; ``ds = sum_k Re(dxhat e^{+i theta})``;
+    ``dx = ds (1 - tanh^2 x)`` under TANH_PREACT, else ``ds``.
+    Returns ``(dx, dR)``.
+    """
+    x = np.asarray(x, np.float64)
+    grid = x.shape[2:]
+    r = np.asarray(r, np.complex128)
+    w = mode_weights(grid, modes) / float(np.prod(grid))
+    dyhat = truncated_dft(np.asarray(dy, np.float64), modes) * w
+    d_r = np.einsum("bik,bok->iok", np.conj(xhat), dyhat)
+    dxhat = np.einsum("bok,iok->bik", dyhat, np.conj(r))
+    ds = inverse_sum(dxhat, grid, modes)
+    if flags & TANH_PREACT:
+        ds = ds * (1.0 - np.tanh(x) ** 2)
+    return ds, d_r
+
+
+def block_fwd(x, r, w, bias, modes, flags: int = 0):
+    """``pre = spectral(x) + W x + b``; ``y = GELU(pre)`` unless NO_ACT.
+
+    Returns ``(y, pre, xhat)``.
+    """
+    x = np.asarray(x, np.float64)
+    d = x.ndim - 2
+    y_spec, xhat = spectral_conv_fwd(x, r, modes, flags)
+    pre = y_spec + _pointwise(w, x) + _bcast(bias, d)
+    y = pre if flags & NO_ACT else gelu(pre)
+    return y, pre, xhat
+
+
+def block_bwd(x, r, w, pre, xhat, dy, modes, flags: int = 0):
+    """Adjoint of :func:`block_fwd`: returns ``(dx, dR, dW, db)``.
+
+    ``dz = dy * GELU'(pre)``; ``db = sum dz``; ``dW = sum dz x^T``;
+    ``dx = W^T dz + spectral_bwd(dz)``.
+    """
+    x = np.asarray(x, np.float64)
+    dy = np.asarray(dy, np.float64)
+    dz = dy if flags & NO_ACT else dy * gelu_grad(pre)
+    spatial = tuple(range(2, x.ndim))
+    db = dz.sum(axis=(0,) + spatial)
+    d_w = _outer_sum(dz, x)
+    dx_spec, d_r = spectral_conv_bwd(x, r, xhat, dz, modes, flags)
+    dx = _pointwise(np.asarray(w, np.float64).T, dz) + dx_spec
+    return dx, d_r, d_w, db
+
+
+# --------------------------------------------------------------------------
+# network: lift -> L blocks -> projection ([MPFNO] "original FNO architecture")
+# --------------------------------------------------------------------------
+
+def forward(a, params, modes, flags: int = 0, save: bool = False):
+    """``v_0 = P a + p``; ``v_{l+1} = block_l(v_l)``; ``u = Q2 GELU(Q1 v_L + q1) + q2``.
+
+    ``params`` is a dict with ``P, p, R (list), W (list), b (list), Q1, q1, Q2, q2``.
+    Returns ``u`` or ``(u, saves)`` with the per-layer block inputs, pre-activations,
+    spectra and the projection's hidden pre-activation.
+    """
+    a = np.asarray(a, np.float64)
+    d = a.ndim - 2
+    v = _pointwise(params["P"], a) + _bcast(params["p"], d)
+    xs, pres, xhats = [], [], []
+    for r, w, bias in zip(params["R"], params["W"], params["b"]):
+        xs.append(v)
+        v, pre, xhat = block_fwd(v, r, w, bias, modes, flags)
+        pres.append(pre)
+        xhats.append(xhat)
+    h = _pointwise(params["Q1"], v) + _bcast(params["q1"], d)
+    u = _pointwise(params["Q2"], gelu(h)) + _bcast(params["q2"], d)
+    if not save:
+        return u
+    return u, {"x": xs, "pre": pres, "xhat": xhats, "v_last": v, "h": h}
+
+
+def backward(a, params, saves, du, modes, flags: int = 0):
+    """Adjoint of :func:`forward`: gradients of every parameter (and of ``a``)."""
+    a = np.asarray(a, np.float64)
+    du = np.asarray(du, np.float64)
+    spatial = tuple(range(2, a.ndim))
+    h, v = saves["h"], saves["v_last"]
+    g = gelu(h)
+    grads = {
+        "Q2": _outer_sum(du, g),
+        "q2": du.sum(axis=(0,) + spatial),
+    }
+    dh = _pointwise(np.asarray(params["Q2"], np.float64).T, du) * gelu_grad(h)
+    grads["Q1"] = _outer_sum(dh, v)
+    grads["q1"] = dh.sum(axis=(0,) + spatial)
+    dv = _pointwise(np.asarray(params["Q1"], np.float64).T, dh)
+    n_layers = len(params["R"])
+    d_r, d_w, d_b = [None] * n_layers, [None] * n_layers, [None] * n_layers
+    for l in range(n_layers - 1, -1, -1):
+        dv, d_r[l], d_w[l], d_b[l] = block_bwd(
+            saves["x"][l], params["R"][l], params["W"][l], saves["pre"][l],
+            saves["xhat"][l], dv, modes, flags)
+    grads["R"], grads["W"], grads["b"] = d_r, d_w, d_b
+    grads["P"] = _outer_sum(dv, a)
+    grads["p"] = dv.sum(axis=(0,) + spatial)
+    grads["a"] = _pointwise(np.asarray(params["P"], np.float64).T, dv)
+    return grads
+
+
+def mse(u, target):
+    """``L = mean((u - t)^2)`` over every element and ``dL/du = 2 (u - t) / numel``."""
+    diff = np.asarray(u, np.float64) - np.asarray(target, np.float64)
+    return float(np.mean(diff * diff)), 2.0 * diff / diff.size
