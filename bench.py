@@ -1,0 +1,409 @@
+#!/usr/bin/env python
+"""Benchmark of the FNO hot path on B200: one step = one forward pass of the 2D
+FNO network (lift 3->32, four spectral blocks of width 32 with 16x16 modes on a
+256x256 grid, projection 32->128->1, float32) over a batch of 16 synthetic
+log-resistivity fields, through the library's C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fno|reference]
+
+Prints one JSON line (rank 0).  With N > 1 (launched by torch.distributed.run)
+every rank runs its own batch of 16 (weak scaling, batch-sharded data
+parallelism: the forward has no exchange step, so there is no collective on
+the data path); the step time is the maximum over ranks.
+
+``--impl reference`` times the CPU float64 oracle instead (rank 0 only; one
+sample of the batch per step).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "FNO block samples/sec at 1 B200; achieved HBM GB/s & tensor-pipe util vs peak"
+DEFAULT_WORKLOAD = "fno2d_f32_b16_w32_256sq_m16"
+FLUSH_BYTES = 512 << 20          # > 126 MB L2: written between timed steps
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("fno", "reference"), default="fno")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="bound on the CPU-oracle sample of the fno arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing
+# --------------------------------------------------------------------------
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend: str):
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=180))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            import torch
+            if torch.cuda.is_available():
+                self.pg.barrier(device_ids=[self.local])
+            else:
+                self.pg.barrier()
+
+    def max(self, v: float) -> float:
+        if not self.pg:
+            return v
+        import torch
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# --------------------------------------------------------------------------
+# clocks (NVML, read only)
+# --------------------------------------------------------------------------
+
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+            0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+            0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons every few ms while running."""
+
+    def __init__(self, index: int):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # pragma: no cover - no NVML
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._nv:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thr:
+            self._thr.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples),
+                "reasons": [n for bit, n in _REASONS.items() if self.reasons & bit]}
+
+
+# --------------------------------------------------------------------------
+# the workload
+# --------------------------------------------------------------------------
+
+def workload_config(wl, n_gpus):
+    return {"workload": wl.name, "description": wl.description, "batch_per_gpu": wl.batch,
+            "global_batch": wl.batch * n_gpus, "grid": list(wl.grid), "modes": list(wl.modes),
+            "width": wl.width, "in_channels": wl.in_ch, "hidden": wl.hidden,
+            "blocks": wl.n_layers, "storage": wl.dtype,
+            "l2": "flushed between timed steps (512 MiB write outside the step events)",
+            "parallelism": f"dp{n_gpus} (batch-sharded, no data-path collective)"}
+
+
+def algorithmic_bytes(tag: str, wl) -> float:
+    """Bytes a kernel must move per launch (each operand once) for the workload."""
+    s = 4 if wl.dtype == "f32" else 2
+    act = wl.batch * wl.width * wl.points * s
+    k = wl.modes[-1]
+    for m in wl.modes[:-1]:
+        k *= 2 * m
+    spec = wl.batch * wl.width * k * 8
+    r = wl.width * wl.width * k * 2 * s
+    table = {
+        "fwd_transform": act + spec,                 # read x, write spectrum
+        "epi_block_fwd": 2 * act + spec,             # read x, write y, read spectrum
+        "mix_fwd": 2 * spec + r,
+        "lift": wl.batch * wl.in_ch * wl.points * s + act,
+        "proj_fwd": act + wl.batch * wl.out_ch * wl.points * s,
+    }
+    return float(table.get(tag, 0.0))
+
+
+def kernel_source_sha(tag: str) -> str:
+    files = {"fwd_transform": "transform.cu", "fwd_finish": "transform.cu",
+             "epi_block_fwd": "epilogue.cu", "mix_fwd": "mix.cu", "lift": "net.cu",
+             "proj_fwd": "net.cu"}
+    path = os.path.join(ROOT, "fourier_neural_spectral_fno_b200", "csrc", files.get(tag, ""))
+    if not os.path.isfile(path):
+        return ""
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def measured_traffic(tag: str, wl):
+    """ncu DRAM bytes per launch from profiles/traffic.json, or None when absent
+    or when the kernel's source changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(path))[wl.name][tag]
+    except Exception:
+        return None
+    if rec.get("source_sha") != kernel_source_sha(tag):
+        return None
+    return rec.get("bytes_per_launch")
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        return float(json.load(open(path))["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def cpu_threads() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max(i.get("num_threads", 1) for i in info) if info else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_samples(wl, inp, n_samples):
+    import oracle as O
+    return O.forward(inp["a"][:n_samples], inp["params"], wl.modes)
+
+
+def cpu_baseline(wl, inp, seconds):
+    """The oracle on a bounded sample of the workload (whole samples, one at a
+    time, until `seconds` of CPU work or the batch is done)."""
+    done, t0 = 0, time.perf_counter()
+    while done < wl.batch and (time.perf_counter() - t0) < seconds:
+        oracle_samples(wl, {"a": inp["a"][done:done + 1], "params": inp["params"]}, 1)
+        done += 1
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": "samples/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{done} of {wl.batch} samples of the workload, full grid, all blocks, "
+                      f"float64 NumPy, {dt:.1f} s"}
+
+
+# --------------------------------------------------------------------------
+# arms
+# --------------------------------------------------------------------------
+
+def run_reference(args, dist):
+    from fourier_neural_spectral_fno_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    if dist.rank != 0:
+        return
+    inp = synth.make_network_inputs(wl)
+    for i in range(args.warmup):
+        oracle_samples(wl, {"a": inp["a"][i % wl.batch:i % wl.batch + 1], "params": inp["params"]}, 1)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle_samples(wl, {"a": inp["a"][i % wl.batch:i % wl.batch + 1], "params": inp["params"]}, 1)
+    dt = time.perf_counter() - t0
+    value = args.steps / dt
+    cores = cpu_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "samples/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(wl, args.gpus),
+            "cpu_baseline": {"value": value, "unit": "samples/s", "cores": cores, "kind": "oracle",
+                             "sample": "one sample of the batch per step (full grid, all blocks)"},
+            "e2e": {"value": value, "unit": "samples/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_fno(args, dist):
+    import numpy as np
+    import torch
+
+    from fourier_neural_spectral_fno_b200 import capi, synth
+
+    wl = synth.WORKLOADS[args.workload]
+    torch.cuda.set_device(dist.local)
+    dev = torch.device("cuda", dist.local)
+    capi.load()
+
+    inp = synth.make_network_inputs(wl)
+    tdt = torch.float32 if wl.dtype == "f32" else (torch.float16 if wl.dtype == "f16" else torch.bfloat16)
+
+    def up(v):
+        v = np.asarray(v)
+        if np.iscomplexobj(v):
+            v = np.stack([v.real, v.imag], -1)
+        return torch.from_numpy(np.ascontiguousarray(v)).to(dev).to(tdt)
+
+    params = {k: ([up(x) for x in v] if isinstance(v, list) else up(v))
+              for k, v in inp["params"].items()}
+    cp = capi.make_params(params)
+    desc = capi.net_desc(wl.batch, wl.grid, wl.modes, wl.in_ch, wl.width, wl.hidden, wl.out_ch,
+                         wl.n_layers, wl.dtype, capi.FNO_TANH_PREACT if wl.tanh else 0)
+    a = up(inp["a"])
+    u = torch.empty((wl.batch, wl.out_ch) + wl.grid, dtype=tdt, device=dev)
+    ws = torch.empty(capi.fno_net_workspace_size(desc, capi.FNO_OP_NET_FWD), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        capi.fno_forward(desc, a, cp, u, None, ws, stream)
+
+    for _ in range(args.warmup):
+        step()
+    launches = capi.last_launch_count()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, events around each step, L2 flushed between
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    reg0, reg1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        reg0.record()
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            starts[i].record()
+            step()
+            ends[i].record()
+        reg1.record()
+        torch.cuda.synchronize()
+    dist.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = dist.max(sum(step_ms) / len(step_ms))
+    region_ms = dist.max(reg0.elapsed_time(reg1))
+    value = dist.world * wl.batch / (ms / 1e3)
+
+    # ---- per-kernel device time (second pass, profiling events on)
+    capi.fno_profile_enable(True)
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        step()
+    torch.cuda.synchronize()
+    capi.fno_profile_enable(False)
+    stats = capi.fno_profile_read()
+    dom = max(stats, key=lambda t: stats[t]["total_ms"])
+    avg_ms = stats[dom]["total_ms"] / stats[dom]["launches"]
+    peak, peak_src = hbm_peak()
+    alg = algorithmic_bytes(dom, wl)
+    achieved = alg / (avg_ms / 1e3) / 1e9 if alg else None
+    roofline = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak,
+                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, copy)",
+                "unit": "GB/s", "frac": (achieved / peak) if achieved else None,
+                "traffic": measured_traffic(dom, wl), "avg_launch_ms": avg_ms,
+                "algorithmic_bytes_per_launch": alg}
+    per_step = {t: round(v["total_ms"] / args.steps, 4) for t, v in sorted(
+        stats.items(), key=lambda kv: -kv[1]["total_ms"])}
+
+    # ---- end to end through the public API with host buffers
+    a_host = torch.empty(a.shape, dtype=tdt, pin_memory=True)
+    a_host.copy_(a.cpu())
+    u_host = torch.empty(u.shape, dtype=tdt, pin_memory=True)
+    e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        a.copy_(a_host, non_blocking=True)
+        step()
+        u_host.copy_(u, non_blocking=True)
+    torch.cuda.synchronize()
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e_steps):
+        a.copy_(a_host, non_blocking=True)
+        step()
+        u_host.copy_(u, non_blocking=True)
+        stream.synchronize()
+        float(u_host.view(-1)[0])           # the host reads the step's result
+    e1.record()
+    torch.cuda.synchronize()
+    e_ms = dist.max(e0.elapsed_time(e1) / e_steps)
+    e2e = {"value": dist.world * wl.batch / (e_ms / 1e3), "unit": "samples/s",
+           "h2d_bytes_per_step": a.numel() * a.element_size(),
+           "d2h_bytes_per_step": u.numel() * u.element_size(), "ms_per_step": e_ms}
+
+    clocks = clk.summary()
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, inp, args.cpu_seconds)
+
+    if dist.rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "samples/s", "n_gpus": dist.world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "region_ms_per_step_incl_flush": region_ms / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": wl.dtype, "data": "synthetic", "config": workload_config(wl, dist.world),
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches * args.steps, "launches_per_step": launches,
+                "clocks": clocks, "kernels_ms_per_step": per_step}
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    dist = Dist()
+    if args.impl == "reference":
+        run_reference(args, dist)      # rank 0 only; no process group needed
+        return
+    dist.init("nccl")
+    try:
+        run_fno(args, dist)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,121 @@
+// Internal kernel interface of the FNO library: geometry, argument blocks and
+// launchers.  Nothing here is part of the public C ABI (include/fno.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace fno {
+
+constexpr int kMaxWidth = 64;   // channels held in registers per grid point
+constexpr int kMaxAxis = 4096;  // longest axis whose twiddle table fits shared memory
+
+// Grid geometry of one block, flattened to at most three axes:
+//   outer axis (d == 3: axis 0), slab axis (d >= 2: axis d-2), last axis.
+// Missing axes have length 1 and a single kept mode.
+struct Geom {
+  int d;
+  long long B;
+  int O, mO, QO;    // outer axis length, modes, kept count (2 mO or 1)
+  int S, mS, QS;    // slab axis
+  int NL, mL;       // last (real-FFT) axis
+  long long N;      // points per channel = O * S * NL
+  long long K;      // kept modes = QO * QS * mL
+  float inv_n;      // 1 / N
+};
+
+enum LoadMode { LOAD_PLAIN = 0, LOAD_TANH = 1, LOAD_DZ = 2 };
+enum EpiMode { EPI_SPEC = 0, EPI_BLOCK_FWD = 1, EPI_SPEC_BWD = 2, EPI_BLOCK_BWD = 3 };
+
+// dtype codes match include/fno.h
+enum { DT_F32 = 0, DT_F16 = 1, DT_BF16 = 2 };
+
+struct Launch {
+  cudaStream_t stream;
+  int *count;       // incremented per kernel launch
+  int num_sms;
+};
+
+// Bracket every kernel launch: launch_begin records a CUDA event on the launch
+// stream when per-kernel timing is on (fno_profile_enable); launch_end records
+// the closing event under `tag` and counts the launch.
+void launch_begin(const Launch &L);
+void launch_end(const Launch &L, const char *tag);
+
+// ---- forward truncated transform (S0-S2) ----------------------------------
+// in0 (and in1 for LOAD_DZ) are [B][C][N]; out xhat [B][C][K] float2.
+// zpart scratch: fwd_zpart_floats() floats.
+int fwd_bands(const Geom &g, long long planes, int num_sms);
+size_t fwd_zpart_bytes(const Geom &g, long long C);
+cudaError_t launch_fwd_transform(const Launch &L, const Geom &g, int dtype, int load_mode,
+                                 long long C, const void *in0, const void *in1, float2 *zpart,
+                                 float2 *xhat);
+
+// ---- mixing (S3) -----------------------------------------------------------
+// yhat[b,o,k] = (c_k / N) sum_i xhat[b,i,k] R[i,o,k]
+cudaError_t launch_mix_fwd(const Launch &L, const Geom &g, int dtype, int Ci, int Co,
+                           const float2 *xhat, const void *R, float2 *yhat);
+// dR[i,o,k] = sum_b conj(xhat[b,i,k]) (c_k/N) D[b,o,k]
+cudaError_t launch_mix_bwd_dr(const Launch &L, const Geom &g, int Ci, int Co,
+                              const float2 *xhat, const float2 *D, float *dR);
+// dxhat[b,i,k] = sum_o (c_k/N) D[b,o,k] conj(R[i,o,k])
+cudaError_t launch_mix_bwd_dx(const Launch &L, const Geom &g, int dtype, int Ci, int Co,
+                              const float2 *D, const void *R, float2 *dxhat);
+
+// ---- inverse of the outer axis (d == 3) -----------------------------------
+size_t inv_expand_bytes(const Geom &g, long long C);
+cudaError_t launch_inv_expand(const Launch &L, const Geom &g, long long C, const float2 *V,
+                              float2 *Z);
+
+// ---- inverse of slab + last axis with fused epilogue (S4, S6 epilogue) ----
+struct EpiArgs {
+  const float2 *Z;  // [B][Cs][O][QS][mL]
+  const void *x;    // [B][Ci][N]
+  const void *W;    // [Co][Ci]
+  const void *bias; // [Co]
+  const void *dy;   // [B][Co][N]
+  const void *pre;  // [B][Co][N]
+  void *out;        // y (fwd modes, [B][Co][N]) or dx (bwd modes, [B][Ci][N])
+  void *pre_out;    // optional [B][Co][N]
+  float *partial;   // bwd: per-CTA partial sums of dW/db, [grid][Co][Ci+1]
+  int Ci, Co;
+  int act, tanh_pre;
+};
+int epi_grid(const Geom &g, int mode, int num_sms);
+size_t epi_partial_bytes(const Geom &g, int Ci, int Co, int num_sms);
+cudaError_t launch_epilogue(const Launch &L, const Geom &g, int dtype, int mode,
+                            const EpiArgs &a);
+
+size_t epi_smem_bytes(const Geom &g, int mode, int Ci, int Co);
+
+// Sum per-CTA partials: partial[p * stride + offset + r * (cols + 1) + c] over p
+// into out_main[r * cols + c] (c < cols) and out_last[r] (c == cols); float32,
+// overwritten.  Either output may be NULL.
+cudaError_t launch_reduce_rows(const Launch &L, const float *partial, int nparts,
+                               long long stride, long long offset, int rows, int cols,
+                               float *out_main, float *out_last);
+
+// CTAs of every kernel that writes per-CTA partial sums (fixed, so workspace
+// sizes do not depend on the device).
+constexpr int kPartialCTAs = 296;
+
+// ---- lift / projection / loss (S5) ----------------------------------------
+cudaError_t launch_lift(const Launch &L, const Geom &g, int dtype, int in_ch, int width,
+                        const void *a, const void *P, const void *p, void *v);
+cudaError_t launch_proj_fwd(const Launch &L, const Geom &g, int dtype, int width, int hidden,
+                            int out_ch, const void *v, const void *Q1, const void *q1,
+                            const void *Q2, const void *q2, void *u);
+int proj_bwd_grid(const Geom &g, int num_sms);
+size_t proj_bwd_partial_floats(int width, int hidden, int out_ch);
+size_t proj_bwd_smem_bytes(int width, int hidden, int out_ch);
+cudaError_t launch_proj_bwd(const Launch &L, const Geom &g, int dtype, int width, int hidden,
+                            int out_ch, const void *v, const void *du, const void *Q1,
+                            const void *q1, const void *Q2, void *dv, float *partial);
+int lift_bwd_grid(const Geom &g, int num_sms);
+cudaError_t launch_lift_bwd(const Launch &L, const Geom &g, int dtype, int in_ch, int width,
+                            const void *a, const void *dv, float *partial);
+cudaError_t launch_mse(const Launch &L, long long n, int dtype, const void *u, const void *t,
+                       float *loss, void *du);
+
+}  // namespace fno

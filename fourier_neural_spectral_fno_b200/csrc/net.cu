@@ -1,0 +1,442 @@
+// Pointwise network stages around the spectral blocks (step S5): the lifting
+// v = P a + p, the projection u = Q2 GELU(Q1 v + q1) + q2, their adjoints,
+// and the mean-squared-error loss of the training step.
+//
+// One thread owns one grid point.  Parameter gradients are reduced per CTA in
+// shared memory over a persistent loop of point tiles and written as per-CTA
+// partials, which a second kernel sums in a fixed order (deterministic).
+#include "fno_common.cuh"
+#include "fno_kernels.cuh"
+
+namespace fno {
+
+namespace {
+
+constexpr int NT = 256;      // threads of the forward pointwise kernels
+constexpr int PB = 128;      // points per tile of the backward kernels
+constexpr int HC = 32;       // projection hidden units per chunk
+constexpr int kMaxIn = 8;    // lift input channels
+constexpr int kMaxOut = 4;   // projection output channels
+
+template <typename T>
+__global__ void __launch_bounds__(NT)
+    k_lift(const T *__restrict__ a, const T *__restrict__ P, const T *__restrict__ p,
+           T *__restrict__ v, long long B, long long N, int in_ch, int width) {
+  __shared__ float Ps[kMaxWidth * kMaxIn], ps[kMaxWidth];
+  for (int e = threadIdx.x; e < width * in_ch; e += NT) Ps[e] = to_f<T>(P[e]);
+  for (int e = threadIdx.x; e < width; e += NT) ps[e] = to_f<T>(p[e]);
+  __syncthreads();
+  for (long long t = (long long)blockIdx.x * NT + threadIdx.x; t < B * N;
+       t += (long long)gridDim.x * NT) {
+    const long long b = t / N, n = t - b * N;
+    float aj[kMaxIn];
+#pragma unroll
+    for (int j = 0; j < kMaxIn; ++j) aj[j] = j < in_ch ? ldf<T>(a + (b * in_ch + j) * N + n) : 0.f;
+    for (int c = 0; c < width; ++c) {
+      float s = ps[c];
+#pragma unroll
+      for (int j = 0; j < kMaxIn; ++j)
+        if (j < in_ch) s = fmaf(Ps[c * in_ch + j], aj[j], s);
+      v[(b * width + c) * N + n] = from_f<T>(s);
+    }
+  }
+}
+
+template <typename T, int CMAX>
+__global__ void __launch_bounds__(NT)
+    k_proj_fwd(const T *__restrict__ v, const T *__restrict__ Q1, const T *__restrict__ q1,
+               const T *__restrict__ Q2, const T *__restrict__ q2, T *__restrict__ u, long long B,
+               long long N, int width, int hidden, int out_ch) {
+  extern __shared__ __align__(16) float psm[];
+  const int ld = (width + 3) & ~3;
+  float *Q1s = psm;                    // [hidden][ld]
+  float *q1s = Q1s + hidden * ld;      // [hidden]
+  float *Q2s = q1s + hidden;           // [out][hidden]
+  for (int e = threadIdx.x; e < hidden * ld; e += NT) {
+    const int h = e / ld, c = e - h * ld;
+    Q1s[e] = c < width ? to_f<T>(Q1[h * width + c]) : 0.f;
+  }
+  for (int e = threadIdx.x; e < hidden; e += NT) q1s[e] = to_f<T>(q1[e]);
+  for (int e = threadIdx.x; e < out_ch * hidden; e += NT) Q2s[e] = to_f<T>(Q2[e]);
+  __syncthreads();
+  for (long long t = (long long)blockIdx.x * NT + threadIdx.x; t < B * N;
+       t += (long long)gridDim.x * NT) {
+    const long long b = t / N, n = t - b * N;
+    float vr[CMAX];
+#pragma unroll
+    for (int c = 0; c < CMAX; ++c) vr[c] = c < width ? ldf<T>(v + (b * width + c) * N + n) : 0.f;
+    float uo[kMaxOut];
+#pragma unroll
+    for (int o = 0; o < kMaxOut; ++o) uo[o] = o < out_ch ? to_f<T>(q2[o]) : 0.f;
+    for (int h = 0; h < hidden; ++h) {
+      const float4 *qp = reinterpret_cast<const float4 *>(Q1s + h * ld);
+      float z = q1s[h];
+#pragma unroll
+      for (int c4 = 0; c4 < CMAX / 4; ++c4) {
+        if (4 * c4 < width) {
+          const float4 q = qp[c4];
+          z = fmaf(q.x, vr[4 * c4], z);
+          z = fmaf(q.y, vr[4 * c4 + 1], z);
+          z = fmaf(q.z, vr[4 * c4 + 2], z);
+          z = fmaf(q.w, vr[4 * c4 + 3], z);
+        }
+      }
+      const float gz = gelu_f(z);
+#pragma unroll
+      for (int o = 0; o < kMaxOut; ++o)
+        if (o < out_ch) uo[o] = fmaf(Q2s[o * hidden + h], gz, uo[o]);
+    }
+#pragma unroll
+    for (int o = 0; o < kMaxOut; ++o)
+      if (o < out_ch) u[(b * out_ch + o) * N + n] = from_f<T>(uo[o]);
+  }
+}
+
+struct ProjBwdLayout {
+  size_t Q1s, q1s, Q2s, vs, dus, dhs, gs, acc1, acc2, total;
+  int ld;
+};
+
+__host__ __device__ inline ProjBwdLayout proj_bwd_layout(int width, int hidden, int out_ch) {
+  ProjBwdLayout l;
+  l.ld = (width + 3) & ~3;
+  size_t off = 0;
+  l.Q1s = off; off += sizeof(float) * (size_t)hidden * l.ld;
+  l.q1s = off; off += sizeof(float) * hidden;
+  l.Q2s = off; off += sizeof(float) * (size_t)out_ch * hidden;
+  l.vs = off; off += sizeof(float) * (size_t)(width + 1) * (PB + 1);
+  l.dus = off; off += sizeof(float) * (size_t)out_ch * PB;
+  l.dhs = off; off += sizeof(float) * (size_t)HC * PB;
+  l.gs = off; off += sizeof(float) * (size_t)HC * (PB + 1);
+  l.acc1 = off; off += sizeof(float) * (size_t)hidden * (width + 1);
+  l.acc2 = off; off += sizeof(float) * (size_t)out_ch * (hidden + 1);
+  l.total = (off + 15) & ~(size_t)15;
+  return l;
+}
+
+// Projection adjoint: dv, and per-CTA partials of dQ1|dq1 ([hidden][width+1])
+// followed by dQ2|dq2 ([out][hidden+1]).
+template <typename T, int CMAX>
+__global__ void __launch_bounds__(PB)
+    k_proj_bwd(const T *__restrict__ v, const T *__restrict__ du, const T *__restrict__ Q1,
+               const T *__restrict__ q1, const T *__restrict__ Q2, T *__restrict__ dv,
+               float *__restrict__ partial, long long B, long long N, int width, int hidden,
+               int out_ch) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const ProjBwdLayout lay = proj_bwd_layout(width, hidden, out_ch);
+  const int ld = lay.ld;
+  float *Q1s = reinterpret_cast<float *>(smem + lay.Q1s);
+  float *q1s = reinterpret_cast<float *>(smem + lay.q1s);
+  float *Q2s = reinterpret_cast<float *>(smem + lay.Q2s);
+  float *v_s = reinterpret_cast<float *>(smem + lay.vs);
+  float *du_s = reinterpret_cast<float *>(smem + lay.dus);
+  float *dh_s = reinterpret_cast<float *>(smem + lay.dhs);
+  float *g_s = reinterpret_cast<float *>(smem + lay.gs);
+  float *acc1 = reinterpret_cast<float *>(smem + lay.acc1);
+  float *acc2 = reinterpret_cast<float *>(smem + lay.acc2);
+  const int tid = threadIdx.x;
+  for (int e = tid; e < hidden * ld; e += PB) {
+    const int h = e / ld, c = e - h * ld;
+    Q1s[e] = c < width ? to_f<T>(Q1[h * width + c]) : 0.f;
+  }
+  for (int e = tid; e < hidden; e += PB) q1s[e] = to_f<T>(q1[e]);
+  for (int e = tid; e < out_ch * hidden; e += PB) Q2s[e] = to_f<T>(Q2[e]);
+  for (int e = tid; e < hidden * (width + 1); e += PB) acc1[e] = 0.f;
+  for (int e = tid; e < out_ch * (hidden + 1); e += PB) acc2[e] = 0.f;
+
+  const long long total = B * N;
+  const long long ntiles = (total + PB - 1) / PB;
+  for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const long long t = tile * PB + tid;
+    const bool valid = t < total;
+    const long long b = valid ? t / N : 0, n = valid ? t - b * N : 0;
+    __syncthreads();
+    float vr[CMAX], dvr[CMAX];
+#pragma unroll
+    for (int c = 0; c < CMAX; ++c) {
+      vr[c] = (valid && c < width) ? ldf<T>(v + (b * width + c) * N + n) : 0.f;
+      dvr[c] = 0.f;
+      if (c < width) v_s[c * (PB + 1) + tid] = vr[c];
+    }
+    v_s[width * (PB + 1) + tid] = valid ? 1.f : 0.f;
+    float dur[kMaxOut];
+#pragma unroll
+    for (int o = 0; o < kMaxOut; ++o) {
+      dur[o] = (valid && o < out_ch) ? ldf<T>(du + (b * out_ch + o) * N + n) : 0.f;
+      if (o < out_ch) du_s[o * PB + tid] = dur[o];
+    }
+    for (int hc = 0; hc < hidden; hc += HC) {
+      __syncthreads();  // previous chunk's reductions are done with dh_s / g_s
+      for (int hh = 0; hh < HC; ++hh) {
+        const int h = hc + hh;
+        float dh = 0.f, gz = 0.f;
+        if (h < hidden && valid) {
+          const float4 *qp = reinterpret_cast<const float4 *>(Q1s + h * ld);
+          float z = q1s[h];
+#pragma unroll
+          for (int c4 = 0; c4 < CMAX / 4; ++c4) {
+            if (4 * c4 < width) {
+              const float4 q = qp[c4];
+              z = fmaf(q.x, vr[4 * c4], z);
+              z = fmaf(q.y, vr[4 * c4 + 1], z);
+              z = fmaf(q.z, vr[4 * c4 + 2], z);
+              z = fmaf(q.w, vr[4 * c4 + 3], z);
+            }
+          }
+          gz = gelu_f(z);
+          float dg = 0.f;
+#pragma unroll
+          for (int o = 0; o < kMaxOut; ++o)
+            if (o < out_ch) dg = fmaf(Q2s[o * hidden + h], dur[o], dg);
+          dh = dg * gelu_grad_f(z);
+#pragma unroll
+          for (int c4 = 0; c4 < CMAX / 4; ++c4) {
+            if (4 * c4 < width) {
+              const float4 q = qp[c4];
+              dvr[4 * c4] = fmaf(q.x, dh, dvr[4 * c4]);
+              dvr[4 * c4 + 1] = fmaf(q.y, dh, dvr[4 * c4 + 1]);
+              dvr[4 * c4 + 2] = fmaf(q.z, dh, dvr[4 * c4 + 2]);
+              dvr[4 * c4 + 3] = fmaf(q.w, dh, dvr[4 * c4 + 3]);
+            }
+          }
+        }
+        dh_s[hh * PB + tid] = dh;
+        g_s[hh * (PB + 1) + tid] = gz;
+      }
+      __syncthreads();
+      const int hn = min(HC, hidden - hc);
+      for (int e = tid; e < hn * (width + 1); e += PB) {
+        const int hh = e / (width + 1), c = e - hh * (width + 1);
+        const float *dr = dh_s + hh * PB;
+        const float *vrow = v_s + c * (PB + 1);
+        float s = 0.f;
+#pragma unroll 8
+        for (int k = 0; k < PB; ++k) s = fmaf(dr[k], vrow[k], s);
+        acc1[(hc + hh) * (width + 1) + c] += s;
+      }
+      for (int e = tid; e < out_ch * hn; e += PB) {
+        const int o = e / hn, hh = e - o * hn;
+        const float *dr = du_s + o * PB;
+        const float *gr = g_s + hh * (PB + 1);
+        float s = 0.f;
+#pragma unroll 8
+        for (int k = 0; k < PB; ++k) s = fmaf(dr[k], gr[k], s);
+        acc2[o * (hidden + 1) + hc + hh] += s;
+      }
+    }
+    for (int o = tid; o < out_ch; o += PB) {
+      float s = 0.f;
+      for (int k = 0; k < PB; ++k) s += du_s[o * PB + k];
+      acc2[o * (hidden + 1) + hidden] += s;
+    }
+    if (valid) {
+#pragma unroll
+      for (int c = 0; c < CMAX; ++c)
+        if (c < width) dv[(b * width + c) * N + n] = from_f<T>(dvr[c]);
+    }
+  }
+  __syncthreads();
+  const long long stride = (long long)hidden * (width + 1) + (long long)out_ch * (hidden + 1);
+  float *dst = partial + blockIdx.x * stride;
+  for (int e = tid; e < hidden * (width + 1); e += PB) dst[e] = acc1[e];
+  for (int e = tid; e < out_ch * (hidden + 1); e += PB) dst[hidden * (width + 1) + e] = acc2[e];
+}
+
+// Lift adjoint: per-CTA partials of dP|dp ([width][in+1]).
+template <typename T>
+__global__ void __launch_bounds__(PB)
+    k_lift_bwd(const T *__restrict__ a, const T *__restrict__ dv, float *__restrict__ partial,
+               long long B, long long N, int in_ch, int width) {
+  __shared__ float dv_s[kMaxWidth * PB];
+  __shared__ float a_s[(kMaxIn + 1) * (PB + 1)];
+  __shared__ float acc[kMaxWidth * (kMaxIn + 1)];
+  const int tid = threadIdx.x;
+  for (int e = tid; e < width * (in_ch + 1); e += PB) acc[e] = 0.f;
+  const long long total = B * N;
+  const long long ntiles = (total + PB - 1) / PB;
+  for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const long long t = tile * PB + tid;
+    const bool valid = t < total;
+    const long long b = valid ? t / N : 0, n = valid ? t - b * N : 0;
+    __syncthreads();
+    for (int c = 0; c < width; ++c)
+      dv_s[c * PB + tid] = valid ? ldf<T>(dv + (b * width + c) * N + n) : 0.f;
+    for (int j = 0; j < in_ch; ++j)
+      a_s[j * (PB + 1) + tid] = valid ? ldf<T>(a + (b * in_ch + j) * N + n) : 0.f;
+    a_s[in_ch * (PB + 1) + tid] = valid ? 1.f : 0.f;
+    __syncthreads();
+    for (int e = tid; e < width * (in_ch + 1); e += PB) {
+      const int c = e / (in_ch + 1), j = e - c * (in_ch + 1);
+      float s = 0.f;
+      for (int k = 0; k < PB; ++k) s = fmaf(dv_s[c * PB + k], a_s[j * (PB + 1) + k], s);
+      acc[e] += s;
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < width * (in_ch + 1); e += PB)
+    partial[(long long)blockIdx.x * width * (in_ch + 1) + e] = acc[e];
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+    k_mse(const T *__restrict__ u, const T *__restrict__ tg, float *__restrict__ loss,
+          T *__restrict__ du, long long n) {
+  __shared__ float red[8];
+  const float inv_n = 1.0f / (float)n;
+  float s = 0.f;
+  for (long long i = (long long)blockIdx.x * 256 + threadIdx.x; i < n;
+       i += (long long)gridDim.x * 256) {
+    const float d = ldf<T>(u + i) - ldf<T>(tg + i);
+    s = fmaf(d, d, s);
+    if (du) du[i] = from_f<T>(2.0f * d * inv_n);
+  }
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int w = 0; w < 8; ++w) t += red[w];
+    atomicAdd(loss, t * inv_n);
+  }
+}
+
+int pointwise_grid(long long total, int num_sms) {
+  const long long want = (total + NT - 1) / NT;
+  const long long cap = (long long)num_sms * 16;
+  return (int)(want < cap ? want : cap);
+}
+
+}  // namespace
+
+#define FNO_DISPATCH_T(dtype, ...)                                \
+  do {                                                            \
+    if ((dtype) == DT_F32) {                                      \
+      using T = float;                                            \
+      __VA_ARGS__;                                                \
+    } else if ((dtype) == DT_F16) {                               \
+      using T = __half;                                           \
+      __VA_ARGS__;                                                \
+    } else {                                                      \
+      using T = __nv_bfloat16;                                    \
+      __VA_ARGS__;                                                \
+    }                                                             \
+  } while (0)
+
+cudaError_t launch_lift(const Launch &L, const Geom &g, int dtype, int in_ch, int width,
+                        const void *a, const void *P, const void *p, void *v) {
+  const int grid = pointwise_grid(g.B * g.N, L.num_sms);
+  launch_begin(L);
+  FNO_DISPATCH_T(dtype, k_lift<T><<<grid, NT, 0, L.stream>>>(
+                            (const T *)a, (const T *)P, (const T *)p, (T *)v, g.B, g.N, in_ch,
+                            width));
+  launch_end(L, "lift");
+  return cudaGetLastError();
+}
+
+template <typename T, int CMAX>
+static cudaError_t proj_fwd_t(const Launch &L, const Geom &g, int width, int hidden, int out_ch,
+                              const void *v, const void *Q1, const void *q1, const void *Q2,
+                              const void *q2, void *u) {
+  const int ld = (width + 3) & ~3;
+  const size_t smem = sizeof(float) * ((size_t)hidden * ld + hidden + (size_t)out_ch * hidden);
+  auto kern = k_proj_fwd<T, CMAX>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  kern<<<pointwise_grid(g.B * g.N, L.num_sms), NT, smem, L.stream>>>(
+      (const T *)v, (const T *)Q1, (const T *)q1, (const T *)Q2, (const T *)q2, (T *)u, g.B, g.N,
+      width, hidden, out_ch);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_proj_fwd(const Launch &L, const Geom &g, int dtype, int width, int hidden,
+                            int out_ch, const void *v, const void *Q1, const void *q1,
+                            const void *Q2, const void *q2, void *u) {
+  cudaError_t err;
+  launch_begin(L);
+  FNO_DISPATCH_T(dtype, {
+    if (width <= 16)
+      err = proj_fwd_t<T, 16>(L, g, width, hidden, out_ch, v, Q1, q1, Q2, q2, u);
+    else if (width <= 32)
+      err = proj_fwd_t<T, 32>(L, g, width, hidden, out_ch, v, Q1, q1, Q2, q2, u);
+    else
+      err = proj_fwd_t<T, 64>(L, g, width, hidden, out_ch, v, Q1, q1, Q2, q2, u);
+  });
+  launch_end(L, "proj_fwd");
+  return err;
+}
+
+int proj_bwd_grid(const Geom &g, int num_sms) {
+  const long long ntiles = (g.B * g.N + PB - 1) / PB;
+  const long long cap = kPartialCTAs;
+  return (int)(ntiles < cap ? ntiles : cap);
+}
+
+size_t proj_bwd_partial_floats(int width, int hidden, int out_ch) {
+  return (size_t)hidden * (width + 1) + (size_t)out_ch * (hidden + 1);
+}
+
+size_t proj_bwd_smem_bytes(int width, int hidden, int out_ch) {
+  return proj_bwd_layout(width, hidden, out_ch).total;
+}
+
+template <typename T, int CMAX>
+static cudaError_t proj_bwd_t(const Launch &L, const Geom &g, int width, int hidden, int out_ch,
+                              const void *v, const void *du, const void *Q1, const void *q1,
+                              const void *Q2, void *dv, float *partial, int grid) {
+  const size_t smem = proj_bwd_layout(width, hidden, out_ch).total;
+  auto kern = k_proj_bwd<T, CMAX>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  kern<<<grid, PB, smem, L.stream>>>((const T *)v, (const T *)du, (const T *)Q1, (const T *)q1,
+                                     (const T *)Q2, (T *)dv, partial, g.B, g.N, width, hidden,
+                                     out_ch);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_proj_bwd(const Launch &L, const Geom &g, int dtype, int width, int hidden,
+                            int out_ch, const void *v, const void *du, const void *Q1,
+                            const void *q1, const void *Q2, void *dv, float *partial) {
+  const int grid = proj_bwd_grid(g, L.num_sms);
+  cudaError_t err;
+  launch_begin(L);
+  FNO_DISPATCH_T(dtype, {
+    if (width <= 16)
+      err = proj_bwd_t<T, 16>(L, g, width, hidden, out_ch, v, du, Q1, q1, Q2, dv, partial, grid);
+    else if (width <= 32)
+      err = proj_bwd_t<T, 32>(L, g, width, hidden, out_ch, v, du, Q1, q1, Q2, dv, partial, grid);
+    else
+      err = proj_bwd_t<T, 64>(L, g, width, hidden, out_ch, v, du, Q1, q1, Q2, dv, partial, grid);
+  });
+  launch_end(L, "proj_bwd");
+  return err;
+}
+
+int lift_bwd_grid(const Geom &g, int num_sms) {
+  const long long ntiles = (g.B * g.N + PB - 1) / PB;
+  const long long cap = kPartialCTAs;
+  return (int)(ntiles < cap ? ntiles : cap);
+}
+
+cudaError_t launch_lift_bwd(const Launch &L, const Geom &g, int dtype, int in_ch, int width,
+                            const void *a, const void *dv, float *partial) {
+  const int grid = lift_bwd_grid(g, L.num_sms);
+  launch_begin(L);
+  FNO_DISPATCH_T(dtype, k_lift_bwd<T><<<grid, PB, 0, L.stream>>>((const T *)a, (const T *)dv,
+                                                                 partial, g.B, g.N, in_ch,
+                                                                 width));
+  launch_end(L, "lift_bwd");
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mse(const Launch &L, long long n, int dtype, const void *u, const void *t,
+                       float *loss, void *du) {
+  cudaError_t err = cudaMemsetAsync(loss, 0, sizeof(float), L.stream);
+  if (err != cudaSuccess) return err;
+  long long want = (n + 255) / 256;
+  const int grid = (int)(want < 4LL * L.num_sms ? (want > 0 ? want : 1) : 4LL * L.num_sms);
+  launch_begin(L);
+  FNO_DISPATCH_T(dtype, k_mse<T><<<grid, 256, 0, L.stream>>>((const T *)u, (const T *)t, loss,
+                                                             (T *)du, n));
+  launch_end(L, "mse");
+  return cudaGetLastError();
+}
+
+}  // namespace fno

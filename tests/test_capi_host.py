@@ -1,0 +1,165 @@
+"""Host-side tests of the C ABI (no GPU needed): the library loads, exports every
+function include/fno.h declares, its structs have the C layout, and argument
+validation rejects bad calls before anything is enqueued."""
+
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+from fourier_neural_spectral_fno_b200 import build, capi, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fno.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return capi.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fno_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 12
+    for name in names:
+        assert hasattr(lib, name), name
+    assert sorted(capi.EXPORTED) == names
+
+
+def test_version_string(lib):
+    assert b"sm_100a" in lib.fno_version()
+
+
+LAYOUT_PROG = r"""
+#include <stdio.h>
+#include <stddef.h>
+#include "fno.h"
+#define F(T, f) printf(#T "." #f " %zu\n", offsetof(T, f));
+int main(void) {
+  printf("fno_block_desc %zu\n", sizeof(fno_block_desc));
+  F(fno_block_desc, ndim) F(fno_block_desc, dtype) F(fno_block_desc, flags) F(fno_block_desc, cin)
+  F(fno_block_desc, cout) F(fno_block_desc, batch) F(fno_block_desc, grid) F(fno_block_desc, modes)
+  printf("fno_net_desc %zu\n", sizeof(fno_net_desc));
+  F(fno_net_desc, in_channels) F(fno_net_desc, width) F(fno_net_desc, hidden)
+  F(fno_net_desc, out_channels) F(fno_net_desc, n_layers) F(fno_net_desc, batch)
+  F(fno_net_desc, grid) F(fno_net_desc, modes)
+  printf("fno_params %zu\n", sizeof(fno_params));
+  F(fno_params, P) F(fno_params, p) F(fno_params, R) F(fno_params, W) F(fno_params, b)
+  F(fno_params, Q1) F(fno_params, q1) F(fno_params, Q2) F(fno_params, q2)
+  printf("fno_grads %zu\n", sizeof(fno_grads));
+  F(fno_grads, R) F(fno_grads, q2)
+  return 0;
+}
+"""
+
+
+def test_struct_layout_matches_c():
+    with tempfile.TemporaryDirectory() as d:
+        src = os.path.join(d, "layout.c")
+        exe = os.path.join(d, "layout")
+        open(src, "w").write(LAYOUT_PROG)
+        subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), src, "-o", exe], check=True)
+        out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout
+    got = dict(line.rsplit(" ", 1) for line in out.strip().splitlines())
+    cls = {"fno_block_desc": capi.BlockDesc, "fno_net_desc": capi.NetDesc,
+           "fno_params": capi.Params, "fno_grads": capi.Grads}
+    for key, val in got.items():
+        if "." in key:
+            s, f = key.split(".")
+            assert getattr(cls[s], f).offset == int(val), key
+        else:
+            assert ctypes.sizeof(cls[key]) == int(val), key
+
+
+@pytest.mark.parametrize("name", synth.WORKLOAD_ORDER)
+def test_workspace_sizes_for_every_workload(lib, name):
+    wl = synth.WORKLOADS[name]
+    flags = capi.FNO_TANH_PREACT if wl.tanh else 0
+    if wl.kind == "block":
+        d = capi.block_desc(wl.batch, wl.width, wl.width, wl.grid, wl.modes, wl.dtype, flags)
+        for op in (0, 1, 2, 3):
+            assert capi.fno_workspace_size(d, op) > 0
+    else:
+        d = capi.net_desc(wl.batch, wl.grid, wl.modes, wl.in_ch, wl.width, wl.hidden, wl.out_ch,
+                          wl.n_layers, wl.dtype, flags)
+        assert capi.fno_net_workspace_size(d, capi.FNO_OP_NET_FWD) > 0
+        assert capi.fno_net_workspace_size(d, capi.FNO_OP_NET_BWD) > 0
+        assert capi.fno_net_saves_size(d) > 0
+
+
+@pytest.mark.parametrize("grid,modes,code", [
+    ((64, 64), (33, 12), capi.FNO_ERR_INVALID_ARG),   # 2m > N on a non-last axis
+    ((64, 64), (12, 34), capi.FNO_ERR_INVALID_ARG),   # m > N/2+1 on the last axis
+    ((64, 64), (0, 12), capi.FNO_ERR_INVALID_ARG),
+    ((8192, 64), (12, 12), capi.FNO_ERR_UNSUPPORTED),  # axis longer than the twiddle tables
+    ((64, 256), (12, 100), capi.FNO_ERR_UNSUPPORTED),  # more than 64 last-axis modes
+])
+def test_invalid_descriptors(lib, grid, modes, code):
+    d = capi.block_desc(2, 4, 4, grid, modes)
+    assert lib.fno_workspace_size(ctypes.byref(d), capi.FNO_OP_BLOCK_FWD) == 0
+    rc = lib.fno_block_fwd(ctypes.byref(d), 256, 256, 256, 256, 256, None, None, 256, 1 << 30, None)
+    assert rc == code, capi.last_error()
+    assert capi.last_error()
+
+
+def test_invalid_channels_and_dtype(lib):
+    d = capi.block_desc(2, 0, 4, (16, 16), (4, 4))
+    assert lib.fno_block_fwd(ctypes.byref(d), 256, 256, 256, 256, 256, None, None, 256, 1 << 30,
+                             None) == capi.FNO_ERR_INVALID_ARG
+    d = capi.block_desc(2, 65, 4, (16, 16), (4, 4))
+    assert lib.fno_block_fwd(ctypes.byref(d), 256, 256, 256, 256, 256, None, None, 256, 1 << 30,
+                             None) == capi.FNO_ERR_UNSUPPORTED
+    d = capi.block_desc(2, 4, 4, (16, 16), (4, 4))
+    d.dtype = 7
+    assert lib.fno_spectral_conv_fwd(ctypes.byref(d), 256, 256, 256, None, 256, 1 << 30,
+                                     None) == capi.FNO_ERR_INVALID_ARG
+    d.dtype = 0
+    d.flags = 8
+    assert lib.fno_spectral_conv_fwd(ctypes.byref(d), 256, 256, 256, None, 256, 1 << 30,
+                                     None) == capi.FNO_ERR_INVALID_ARG
+    assert lib.fno_spectral_conv_fwd(None, 256, 256, 256, None, 256, 1 << 30,
+                                     None) == capi.FNO_ERR_INVALID_ARG
+
+
+def test_null_misaligned_and_workspace(lib):
+    d = capi.block_desc(2, 4, 4, (16, 16), (4, 4))
+    need = capi.fno_workspace_size(d, capi.FNO_OP_SPECTRAL_FWD)
+    f = lib.fno_spectral_conv_fwd
+    assert f(ctypes.byref(d), None, 256, 256, None, 256, need, None) == capi.FNO_ERR_INVALID_ARG
+    assert "x" in capi.last_error()
+    assert f(ctypes.byref(d), 0x1008, 256, 256, None, 256, need, None) == capi.FNO_ERR_INVALID_ARG
+    assert "aligned" in capi.last_error()
+    assert f(ctypes.byref(d), 256, 256, 256, 0x104, 256, need, None) == capi.FNO_ERR_INVALID_ARG
+    assert f(ctypes.byref(d), 256, 256, 256, None, 256, need - 1, None) == capi.FNO_ERR_WORKSPACE
+    assert f(ctypes.byref(d), 256, 256, 256, None, None, need, None) == capi.FNO_ERR_INVALID_ARG
+    bw = lib.fno_block_bwd
+    assert bw(ctypes.byref(d), 256, 256, 256, None, None, 256, 256, 256, 256, 256, 256, 1 << 30,
+              None) == capi.FNO_ERR_INVALID_ARG          # pre_save required with GELU
+    assert "pre_save" in capi.last_error()
+
+
+def test_network_validation(lib):
+    d = capi.net_desc(2, (16, 16), (4, 4), 3, 8, n_layers=0)
+    assert lib.fno_net_workspace_size(ctypes.byref(d), capi.FNO_OP_NET_FWD) == 0
+    d = capi.net_desc(2, (16, 16), (4, 4), 3, 8, out_channels=5)
+    assert lib.fno_net_saves_size(ctypes.byref(d)) == 0
+    d = capi.net_desc(2, (16, 16), (4, 4), 3, 8)
+    p = capi.Params()
+    assert lib.fno_forward(ctypes.byref(d), 256, ctypes.byref(p), 256, None, 256, 1 << 30,
+                           None) == capi.FNO_ERR_INVALID_ARG
+    assert lib.fno_mse(0, 0, 256, 256, 256, None, None) == capi.FNO_ERR_INVALID_ARG
+
+
+def test_missing_library_raises(tmp_path):
+    with pytest.raises(capi.FnoError):
+        capi.load(str(tmp_path / "libfno.so"))

@@ -1,0 +1,196 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle, element by
+element, on seeded inputs at sizes that span several tiles and ragged tails.
+
+Tolerances: relative L2 error 1e-5 for float32 storage, 1e-2 for float16 /
+bfloat16 storage with float32 accumulation."""
+
+import numpy as np
+import pytest
+
+import oracle as O
+from fourier_neural_spectral_fno_b200 import capi, synth
+
+from fno_testlib import (TOL, assert_close, dev, dev_complex, empty, flags_of, grads_like, host,
+                         host_complex, oracle_flags, params_to_device)
+
+pytestmark = pytest.mark.gpu
+
+# (grid, modes): 1D, 2D with ragged row tiles / column chunks, odd lengths, all
+# modes kept, 3D with ragged slabs
+SHAPES = [
+    ((100,), (20,)),
+    ((16, 12), (4, 5)),
+    ((15, 9), (5, 5)),
+    ((8, 8), (4, 5)),
+    ((70, 130), (6, 9)),
+    ((6, 10, 12), (2, 3, 4)),
+    ((20, 9, 70), (5, 4, 11)),
+]
+
+
+def _block_inputs(grid, modes, batch, ci, co, dtype, seed=0, bias=True):
+    rng = np.random.default_rng(seed)
+    x = synth.quantize(rng.standard_normal((batch, ci) + tuple(grid)), dtype)
+    k = capi.num_modes(grid, modes)
+    r = synth.quantize_complex(synth.spectral_weights(rng, ci, co, k) * (ci * co) / np.sqrt(ci), dtype)
+    w = synth.quantize(rng.uniform(-1, 1, (co, ci)) / np.sqrt(ci), dtype)
+    b = synth.quantize(rng.uniform(-0.5, 0.5, co) if bias else np.zeros(co), dtype)
+    dy = synth.quantize(rng.standard_normal((batch, co) + tuple(grid)), dtype)
+    return x, r, w, b, dy
+
+
+@pytest.mark.parametrize("grid,modes", SHAPES)
+@pytest.mark.parametrize("dtype,tanh", [("f32", False), ("f32", True), ("f16", True),
+                                        ("bf16", False)])
+def test_spectral_conv_fwd(grid, modes, dtype, tanh):
+    b_, ci, co = 3, 5, 4
+    x, r, _, _, _ = _block_inputs(grid, modes, b_, ci, co, dtype)
+    flags = flags_of(tanh=tanh)
+    d = capi.block_desc(b_, ci, co, grid, modes, dtype, flags)
+    k = capi.num_modes(grid, modes)
+    y = empty((b_, co) + grid, dtype)
+    xh = empty((b_, ci, k, 2))
+    capi.fno_spectral_conv_fwd(d, dev(x, dtype), dev_complex(r, dtype), y, xh)
+    y_ref, xh_ref = O.spectral_conv_fwd(x, r, modes, oracle_flags(flags))
+    assert_close(host_complex(xh), xh_ref, TOL["f32"] if dtype == "f32" else 2e-5, "xhat")
+    assert_close(host(y), y_ref, TOL[dtype], "y")
+
+
+@pytest.mark.parametrize("grid,modes", SHAPES)
+@pytest.mark.parametrize("dtype,flags", [("f32", 0), ("f32", 2), ("f16", 1), ("bf16", 0)])
+def test_block_fwd(grid, modes, dtype, flags):
+    b_, ci, co = 2, 6, 7
+    x, r, w, b, _ = _block_inputs(grid, modes, b_, ci, co, dtype, seed=1)
+    d = capi.block_desc(b_, ci, co, grid, modes, dtype, flags)
+    k = capi.num_modes(grid, modes)
+    y = empty((b_, co) + grid, dtype)
+    pre = empty((b_, co) + grid, dtype)
+    xh = empty((b_, ci, k, 2))
+    capi.fno_block_fwd(d, dev(x, dtype), dev_complex(r, dtype), dev(w, dtype), dev(b, dtype), y,
+                       pre, xh)
+    y_ref, pre_ref, xh_ref = O.block_fwd(x, r, w, b, modes, oracle_flags(flags))
+    assert_close(host(pre), pre_ref, TOL[dtype], "pre")
+    assert_close(host(y), y_ref, TOL[dtype], "y")
+    assert_close(host_complex(xh), xh_ref, 2e-5, "xhat")
+
+
+@pytest.mark.parametrize("grid,modes", SHAPES)
+@pytest.mark.parametrize("dtype,tanh,give_xhat", [("f32", False, True), ("f32", True, False),
+                                                  ("f16", True, True), ("bf16", False, False)])
+def test_spectral_conv_bwd(grid, modes, dtype, tanh, give_xhat):
+    b_, ci, co = 3, 4, 5
+    x, r, _, _, dy = _block_inputs(grid, modes, b_, ci, co, dtype, seed=2)
+    flags = flags_of(tanh=tanh)
+    d = capi.block_desc(b_, ci, co, grid, modes, dtype, flags)
+    k = capi.num_modes(grid, modes)
+    _, xh_ref = O.spectral_conv_fwd(x, r, modes, oracle_flags(flags))
+    xh = dev_complex(xh_ref) if give_xhat else None
+    dx = empty((b_, ci) + grid, dtype)
+    dr = empty((ci, co, k, 2))
+    capi.fno_spectral_conv_bwd(d, dev(x, dtype), xh, dev_complex(r, dtype), dev(dy, dtype), dx, dr)
+    dx_ref, dr_ref = O.spectral_conv_bwd(x, r, xh_ref, dy, modes, oracle_flags(flags))
+    assert_close(host(dx), dx_ref, TOL[dtype], "dx")
+    assert_close(host_complex(dr), dr_ref, TOL[dtype] if dtype != "f32" else 1e-5, "dR")
+
+
+@pytest.mark.parametrize("grid,modes", SHAPES)
+@pytest.mark.parametrize("dtype,flags,give_xhat", [("f32", 0, True), ("f32", 1, False),
+                                                   ("f32", 2, True), ("f16", 1, True),
+                                                   ("bf16", 0, False)])
+def test_block_bwd(grid, modes, dtype, flags, give_xhat):
+    b_, ci, co = 2, 5, 6
+    x, r, w, b, dy = _block_inputs(grid, modes, b_, ci, co, dtype, seed=3)
+    d = capi.block_desc(b_, ci, co, grid, modes, dtype, flags)
+    k = capi.num_modes(grid, modes)
+    y_ref, pre_ref, xh_ref = O.block_fwd(x, r, w, b, modes, oracle_flags(flags))
+    pre_q = synth.quantize(pre_ref, dtype)          # what the forward saved
+    dx = empty((b_, ci) + grid, dtype)
+    dr = empty((ci, co, k, 2))
+    dw = empty((co, ci))
+    db = empty((co,))
+    capi.fno_block_bwd(d, dev(x, dtype), dev_complex(r, dtype), dev(w, dtype), dev(pre_q, dtype),
+                       dev_complex(xh_ref) if give_xhat else None, dev(dy, dtype), dx, dr, dw, db)
+    dx_ref, dr_ref, dw_ref, db_ref = O.block_bwd(x, r, w, pre_q, xh_ref, dy, modes,
+                                                 oracle_flags(flags))
+    tol = TOL[dtype]
+    assert_close(host(dx), dx_ref, tol, "dx")
+    assert_close(host_complex(dr), dr_ref, tol, "dR")
+    assert_close(host(dw), dw_ref, tol, "dW")
+    assert_close(host(db), db_ref, tol, "db")
+
+
+def test_block_bwd_wide_channels_f32():
+    grid, modes = (32, 40), (5, 7)
+    x, r, w, b, dy = _block_inputs(grid, modes, 3, 64, 48, "f32", seed=4)
+    d = capi.block_desc(3, 64, 48, grid, modes)
+    y_ref, pre_ref, xh_ref = O.block_fwd(x, r, w, b, modes)
+    y = empty((3, 48) + grid)
+    pre = empty((3, 48) + grid)
+    capi.fno_block_fwd(d, dev(x), dev_complex(r), dev(w), dev(b), y, pre)
+    assert_close(host(y), y_ref, 1e-5, "y")
+    k = capi.num_modes(grid, modes)
+    dx, dr, dw, db = empty((3, 64) + grid), empty((64, 48, k, 2)), empty((48, 64)), empty((48,))
+    capi.fno_block_bwd(d, dev(x), dev_complex(r), dev(w), pre, None, dev(dy), dx, dr, dw, db)
+    dx_ref, dr_ref, dw_ref, db_ref = O.block_bwd(x, r, w, host(pre), xh_ref, dy, modes)
+    assert_close(host(dx), dx_ref, 1e-5, "dx")
+    assert_close(host_complex(dr), dr_ref, 1e-5, "dR")
+    assert_close(host(dw), dw_ref, 1e-5, "dW")
+    assert_close(host(db), db_ref, 1e-5, "db")
+
+
+def _tiny_network(grid, modes, dtype, batch=2, width=6, hidden=9, layers=2, in_ch=None):
+    in_ch = in_ch or 1 + len(grid)
+    wl = synth.Workload("tiny", "network", dtype, batch, tuple(grid), tuple(modes), width,
+                        in_ch=in_ch, hidden=hidden, n_layers=layers, backward=True)
+    inp = synth.make_network_inputs(wl)
+    p = inp["params"]
+    p["R"] = [synth.quantize_complex(r * width * width / np.sqrt(width), dtype) for r in p["R"]]
+    p["b"] = [synth.quantize(np.linspace(-0.3, 0.3, width), dtype) for _ in p["b"]]
+    return wl, inp
+
+
+@pytest.mark.parametrize("grid,modes", [((16, 12), (4, 5)), ((40, 70), (6, 9)),
+                                        ((6, 10, 12), (2, 3, 4)), ((100,), (20,))])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_network_forward_backward_mse(grid, modes, dtype):
+    import torch
+    wl, inp = _tiny_network(grid, modes, dtype)
+    a, params, tgt = inp["a"], inp["params"], inp["target"]
+    d = capi.net_desc(wl.batch, grid, modes, wl.in_ch, wl.width, wl.hidden, 1, wl.n_layers, dtype)
+    pd = params_to_device(params, dtype)
+    cp = capi.make_params(pd)
+    saves = torch.empty(capi.fno_net_saves_size(d), dtype=torch.uint8, device="cuda")
+    u = empty((wl.batch, 1) + grid, dtype)
+    a_d = dev(a, dtype)
+    capi.fno_forward(d, a_d, cp, u, saves)
+    u_ref, sv = O.forward(a, params, modes, save=True)
+    assert_close(host(u), u_ref, TOL[dtype], "u")
+    # forward without saves gives the same result
+    u2 = empty((wl.batch, 1) + grid, dtype)
+    capi.fno_forward(d, a_d, cp, u2)
+    assert torch.equal(u, u2)
+    loss = torch.empty(1, dtype=torch.float32, device="cuda")
+    du = empty(u.shape, dtype)
+    capi.fno_mse(u, dev(tgt, dtype), loss, du, dtype)
+    loss_ref, du_ref = O.mse(host(u), tgt)
+    assert abs(float(loss.item()) - loss_ref) <= 1e-5 * abs(loss_ref) + 1e-7
+    assert_close(host(du), du_ref, TOL[dtype], "du")
+    gd = grads_like(params)
+    capi.fno_backward(d, a_d, cp, saves, du, capi.make_grads(gd))
+    g_ref = O.backward(a, params, sv, host(du), modes)
+    tol = TOL[dtype] if dtype != "f32" else 2e-5
+    for key in ("P", "p", "Q1", "q1", "Q2", "q2"):
+        assert_close(host(gd[key]), g_ref[key], tol, key)
+    for key in ("R", "W", "b"):
+        for l in range(wl.n_layers):
+            got = host_complex(gd[key][l]) if key == "R" else host(gd[key][l])
+            assert_close(got, g_ref[key][l], tol, f"{key}[{l}]")
+
+
+def test_launch_count_is_reported():
+    grid, modes = (16, 12), (4, 5)
+    x, r, w, b, _ = _block_inputs(grid, modes, 2, 3, 3, "f32")
+    d = capi.block_desc(2, 3, 3, grid, modes)
+    y = empty((2, 3) + grid)
+    capi.fno_block_fwd(d, dev(x), dev_complex(r), dev(w), dev(b), y)
+    assert capi.last_launch_count() == 4   # transform, finish, mix, epilogue
