@@ -43,7 +43,8 @@ EXPORTED = (
     "fno_last_error", "fno_version", "fno_last_launch_count", "fno_workspace_size",
     "fno_net_workspace_size", "fno_net_saves_size", "fno_spectral_conv_fwd",
     "fno_spectral_conv_bwd", "fno_block_fwd", "fno_block_bwd", "fno_forward", "fno_backward",
-    "fno_mse", "fno_profile_enable", "fno_profile_read",
+    "fno_mse", "fno_profile_enable", "fno_profile_read", "fno_set_tensor_cores",
+    "fno_device_error",
 )
 
 
@@ -119,6 +120,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
                              sz, vp]),
         "fno_mse": (i, [ctypes.c_int64, i, vp, vp, vp, vp, vp]),
         "fno_profile_enable": (i, [i]),
+        "fno_set_tensor_cores": (i, [i]),
+        "fno_device_error": (i, [i]),
         "fno_profile_read": (i, [ctypes.POINTER(KernelStat), i]),
     }
     for name, (res, args) in sig.items():
@@ -314,3 +317,13 @@ def fno_profile_read(max_kernels: int = 64) -> Dict[str, Dict[str, float]]:
         raise FnoError(n, last_error())
     return {arr[i].name.decode(): {"launches": arr[i].launches, "total_ms": arr[i].total_ms}
             for i in range(n)}
+
+
+def fno_set_tensor_cores(enable: bool) -> bool:
+    """Use the tcgen05 kernels where shapes allow (True) or the CUDA-core ones."""
+    return bool(load().fno_set_tensor_cores(1 if enable else 0))
+
+
+def fno_device_error(clear: bool = True) -> None:
+    """Raise if a bounded device-side wait expired since the last clear."""
+    _check(load().fno_device_error(1 if clear else 0))

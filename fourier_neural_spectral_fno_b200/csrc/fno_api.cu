@@ -17,6 +17,7 @@ namespace {
 
 thread_local char g_err[512] = "";
 thread_local int g_launches = 0;
+int g_use_tc = 1;   // tensor-core kernels where the shape allows (fno_set_tensor_cores)
 
 int fail(int code, const char *fmt, ...) {
   va_list ap;
@@ -114,7 +115,7 @@ int check_block(const fno_block_desc *d, Geom *g) {
 
 // Workspace map of a block operation.
 struct BlockWs {
-  size_t zpart, xhat, yhat, zexp, dxhat, partial, total;
+  size_t zpart, xhat, yhat, zexp, u, dxhat, partial, total;
 };
 
 BlockWs block_ws(const Geom &g, int Ci, int Co, int op) {
@@ -133,6 +134,8 @@ BlockWs block_ws(const Geom &g, int Ci, int Co, int op) {
   off += al(cplx * (size_t)(g.B * Cmax * g.K));
   w.zexp = off;
   off += al(inv_expand_bytes(g, Cmax));
+  w.u = off;                          // spectrum inverted along the slab axis
+  off += al(inv_slab_bytes(g, Cmax));
   w.dxhat = off;
   w.partial = off;
   if (op == FNO_OP_SPECTRAL_BWD || op == FNO_OP_BLOCK_BWD) {
@@ -171,10 +174,43 @@ std::vector<ProfRec> g_prof;   // event pool; the first g_prof_used entries are 
 size_t g_prof_used = 0;
 bool g_prof_on = false;
 
+__device__ int g_fno_device_error;   // set by kernels whose bounded waits expire
+
+int *device_error_word() {
+  static int *addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (!addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fno_device_error) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    addr[dev] = static_cast<int *>(p);
+  }
+  return addr[dev];
+}
+
 Launch make_launch(fno_stream_t s) {
   g_launches = 0;
-  Launch L{reinterpret_cast<cudaStream_t>(s), &g_launches, device_sms()};
+  Launch L{reinterpret_cast<cudaStream_t>(s), &g_launches, device_sms(), g_use_tc,
+           device_error_word()};
   return L;
+}
+
+cudaError_t run_epilogue(const Launch &L, const Geom &g, int dtype, int mode, const EpiArgs &a,
+                         unsigned char *ws, const BlockWs &w) {
+  if (L.tc && epi_tc_supported(g, dtype, mode, a.Ci, a.Co)) {
+    float2 *U = reinterpret_cast<float2 *>(ws + w.u);
+    const int cs = mode == EPI_SPEC_BWD ? a.Ci : a.Co;
+    cudaError_t e = launch_inv_slab(L, g, cs, a.Z, U);
+    if (e != cudaSuccess) return e;
+    return launch_epilogue_tc(L, g, dtype, mode, a, U);
+  }
+  return launch_epilogue(L, g, dtype, mode, a);
 }
 
 // ---------------------------------------------------------------------------
@@ -210,7 +246,7 @@ int run_forward(const Launch &L, const Geom &g, int dtype, unsigned flags, int C
   a.Co = Co;
   a.act = !(flags & FNO_NO_ACT);
   a.tanh_pre = (flags & FNO_TANH_PREACT) ? 1 : 0;
-  FNO_TRY(launch_epilogue(L, g, dtype, epi_mode, a), "epilogue");
+  FNO_TRY(run_epilogue(L, g, dtype, epi_mode, a, ws, w), "epilogue");
   return FNO_OK;
 }
 
@@ -254,7 +290,7 @@ int run_backward(const Launch &L, const Geom &g, int dtype, unsigned flags, int 
   a.tanh_pre = (flags & FNO_TANH_PREACT) ? 1 : 0;
   float *partial = reinterpret_cast<float *>(ws + w.partial);
   a.partial = partial;
-  FNO_TRY(launch_epilogue(L, g, dtype, block ? EPI_BLOCK_BWD : EPI_SPEC_BWD, a), "epilogue");
+  FNO_TRY(run_epilogue(L, g, dtype, block ? EPI_BLOCK_BWD : EPI_SPEC_BWD, a, ws, w), "epilogue");
   if (block) {
     const int nparts = epi_grid(g, EPI_BLOCK_BWD, L.num_sms);
     FNO_TRY(launch_reduce_rows(L, partial, nparts, (long long)Co * (Ci + 1), 0, Co, Ci, dW, db),
@@ -387,6 +423,28 @@ const char *fno_last_error(void) { return g_err; }
 const char *fno_version(void) { return "fno-b200 0.1 (sm_100a)"; }
 
 int fno_last_launch_count(void) { return g_launches; }
+
+int fno_set_tensor_cores(int enable) {
+  const int prev = g_use_tc;
+  g_use_tc = enable ? 1 : 0;
+  return prev;
+}
+
+int fno_device_error(int clear) {
+  int *p = device_error_word();
+  if (!p) return fail(FNO_ERR_CUDA, "no CUDA device");
+  int v = 0;
+  cudaError_t e = cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (clear && v) {
+    const int zero = 0;
+    e = cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+  }
+  if (v) return fail(FNO_ERR_TIMEOUT, "a bounded device-side wait expired (results invalid)");
+  g_err[0] = 0;
+  return FNO_OK;
+}
 
 int fno_profile_enable(int on) {
   std::lock_guard<std::mutex> lk(g_prof_mu);

@@ -35,6 +35,8 @@ struct Launch {
   cudaStream_t stream;
   int *count;       // incremented per kernel launch
   int num_sms;
+  int tc;           // use the tensor-core kernels where the shape allows
+  int *err;         // device error word (bounded waits that expired)
 };
 
 // Bracket every kernel launch: launch_begin records a CUDA event on the launch
@@ -51,6 +53,12 @@ size_t fwd_zpart_bytes(const Geom &g, long long C);
 cudaError_t launch_fwd_transform(const Launch &L, const Geom &g, int dtype, int load_mode,
                                  long long C, const void *in0, const void *in1, float2 *zpart,
                                  float2 *xhat);
+
+// ---- tensor-core variants (transform_tc.cu, epilogue_tc.cu) ----------------
+bool s1_tc_supported(const Geom &g, int dtype);
+int s1_tc_bands(const Geom &g);
+cudaError_t launch_s1_tc(const Launch &L, const Geom &g, int dtype, int load_mode, long long C,
+                         const void *in0, const void *in1, float2 *zpart, int *err);
 
 // ---- mixing (S3) -----------------------------------------------------------
 // yhat[b,o,k] = (c_k / N) sum_i xhat[b,i,k] R[i,o,k]
@@ -83,6 +91,15 @@ struct EpiArgs {
   int act, tanh_pre;
 };
 int epi_grid(const Geom &g, int mode, int num_sms);
+// tensor-core epilogue: U = spectrum inverted along the slab axis,
+// [B][Cs][O][S][mL] float2 (launch_inv_slab), then one GEMM per 128-point tile
+bool epi_tc_supported(const Geom &g, int dtype, int mode, int Ci, int Co);
+size_t inv_slab_bytes(const Geom &g, long long C);
+cudaError_t launch_inv_slab(const Launch &L, const Geom &g, long long C, const float2 *Z,
+                            float2 *U);
+struct EpiArgs;
+cudaError_t launch_epilogue_tc(const Launch &L, const Geom &g, int dtype, int mode,
+                               const EpiArgs &a, const float2 *U);
 size_t epi_partial_bytes(const Geom &g, int Ci, int Co, int num_sms);
 cudaError_t launch_epilogue(const Launch &L, const Geom &g, int dtype, int mode,
                             const EpiArgs &a);

@@ -232,6 +232,9 @@ cudaError_t launch_fwd_slab_t(const Launch &L, int load_mode, dim3 grid, size_t 
 
 }  // namespace
 
+cudaError_t launch_fwd_slab(const Launch &L, const Geom &g, int dtype, int load_mode, long long C,
+                            const void *in0, const void *in1, float2 *zpart, int nb);
+
 int fwd_bands(const Geom &g, long long planes, int num_sms) {
   // Enough CTAs for several waves, with bands of whole row tiles.
   const int tiles = (g.S + FS_RT - 1) / FS_RT;
@@ -244,29 +247,27 @@ int fwd_bands(const Geom &g, long long planes, int num_sms) {
 
 size_t fwd_zpart_bytes(const Geom &g, long long C) {
   const long long planes = g.B * C * g.O;
-  return sizeof(float2) * (size_t)fwd_bands(g, planes, 148) * planes * g.QS * g.mL;
+  long long nb = fwd_bands(g, planes, 148);
+  const long long ntc = s1_tc_bands(g);
+  if (ntc > nb) nb = ntc;
+  return sizeof(float2) * (size_t)nb * planes * g.QS * g.mL;
 }
 
 cudaError_t launch_fwd_transform(const Launch &L, const Geom &g, int dtype, int load_mode,
                                  long long C, const void *in0, const void *in1, float2 *zpart,
                                  float2 *xhat) {
   const long long planes = g.B * C * g.O;
-  const int nb = fwd_bands(g, planes, 148);
-  const int tiles = (g.S + FS_RT - 1) / FS_RT;
-  const int tiles_per_band = (tiles + nb - 1) / nb;
-  FwdSlabArgs args{in0, in1, zpart, planes, g.S, g.NL, g.mL, g.mS, g.QS, tiles_per_band * FS_RT};
-  const size_t smem = fwd_slab_smem(g.S, g.NL, g.mL, g.QS);
-  dim3 grid((unsigned)planes, (unsigned)nb);
+  int nb;
   cudaError_t err;
-  launch_begin(L);
-  if (dtype == DT_F32)
-    err = launch_fwd_slab_t<float>(L, load_mode, grid, smem, args);
-  else if (dtype == DT_F16)
-    err = launch_fwd_slab_t<__half>(L, load_mode, grid, smem, args);
-  else
-    err = launch_fwd_slab_t<__nv_bfloat16>(L, load_mode, grid, smem, args);
-  launch_end(L, load_mode == LOAD_DZ ? "fwd_transform_dz" : "fwd_transform");
-  if (err != cudaSuccess) return err;
+  if (L.tc && s1_tc_supported(g, dtype)) {
+    nb = s1_tc_bands(g);
+    err = launch_s1_tc(L, g, dtype, load_mode, C, in0, in1, zpart, L.err);
+    if (err != cudaSuccess) return err;
+  } else {
+    nb = fwd_bands(g, planes, 148);
+    err = launch_fwd_slab(L, g, dtype, load_mode, C, in0, in1, zpart, nb);
+    if (err != cudaSuccess) return err;
+  }
   const long long BC = g.B * C;
   const int QSmL = g.QS * g.mL;
   const long long n = BC * QSmL;
@@ -276,6 +277,27 @@ cudaError_t launch_fwd_transform(const Launch &L, const Geom &g, int dtype, int 
                                                                        g.O, g.mO, g.QO, QSmL);
   launch_end(L, "fwd_finish");
   return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_slab(const Launch &L, const Geom &g, int dtype, int load_mode, long long C,
+                            const void *in0, const void *in1, float2 *zpart, int nb) {
+  const long long planes = g.B * C * g.O;
+  const int tiles = (g.S + FS_RT - 1) / FS_RT;
+  const int tiles_per_band = (tiles + nb - 1) / nb;
+  FwdSlabArgs args{in0, in1, zpart, planes, g.S, g.NL, g.mL, g.mS, g.QS, tiles_per_band * FS_RT};
+  const size_t smem = fwd_slab_smem(g.S, g.NL, g.mL, g.QS);
+  dim3 grid((unsigned)planes, (unsigned)nb);
+  cudaError_t err;
+  (void)tiles;
+  launch_begin(L);
+  if (dtype == DT_F32)
+    err = launch_fwd_slab_t<float>(L, load_mode, grid, smem, args);
+  else if (dtype == DT_F16)
+    err = launch_fwd_slab_t<__half>(L, load_mode, grid, smem, args);
+  else
+    err = launch_fwd_slab_t<__nv_bfloat16>(L, load_mode, grid, smem, args);
+  launch_end(L, load_mode == LOAD_DZ ? "fwd_transform_dz" : "fwd_transform");
+  return err;
 }
 
 size_t inv_expand_bytes(const Geom &g, long long C) {

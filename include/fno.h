@@ -151,6 +151,18 @@ const char *fno_version(void);
 /* Number of kernel launches the last successful call on this thread enqueued. */
 int fno_last_launch_count(void);
 
+/* Kernel selection: 1 (default) uses the tcgen05 tensor-core kernels wherever
+ * the shape allows them, 0 forces the CUDA-core kernels everywhere (both are
+ * complete implementations; the switch exists to compare them).  Process-wide;
+ * returns the previous setting. */
+int fno_set_tensor_cores(int enable);
+
+/* Synchronises the current device and reads the library's device error word,
+ * which a kernel sets when one of its bounded waits on the tensor-core
+ * pipeline expires (its results are then invalid).  Returns FNO_OK or
+ * FNO_ERR_TIMEOUT; clear != 0 resets the word. */
+int fno_device_error(int clear);
+
 /* Per-kernel timing.  fno_profile_enable(1) starts a recording: from then on
  * every kernel the library launches (on any thread) is bracketed by a pair of
  * CUDA events recorded on its launch stream; fno_profile_enable(0) stops
