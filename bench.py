@@ -176,13 +176,17 @@ def algorithmic_bytes(tag: str, wl) -> float:
         "lift": wl.batch * wl.in_ch * wl.points * s + act,
         "proj_fwd": act + wl.batch * wl.out_ch * wl.points * s,
     }
+    for base in ("fwd_transform", "epi_block_fwd", "proj_fwd"):
+        table[base + "_tc"] = table[base]
     return float(table.get(tag, 0.0))
 
 
 def kernel_source_sha(tag: str) -> str:
     files = {"fwd_transform": "transform.cu", "fwd_finish": "transform.cu",
              "epi_block_fwd": "epilogue.cu", "mix_fwd": "mix.cu", "lift": "net.cu",
-             "proj_fwd": "net.cu"}
+             "proj_fwd": "net.cu", "fwd_transform_tc": "transform_tc.cu",
+             "epi_block_fwd_tc": "epilogue_tc.cu", "inv_slab": "epilogue_tc.cu",
+             "proj_fwd_tc": "net_tc.cu"}
     path = os.path.join(ROOT, "fourier_neural_spectral_fno_b200", "csrc", files.get(tag, ""))
     if not os.path.isfile(path):
         return ""

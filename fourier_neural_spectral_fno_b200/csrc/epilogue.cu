@@ -119,10 +119,8 @@ __global__ void __launch_bounds__(PTS) k_epilogue(EpiArgs a, Geom g) {
       const int row = r_first + rl;
       const float2 *z = a.Z + (((b * Cs + c) * O + outer) * QS) * (long long)mL + k;
       float2 s = make_float2(0.f, 0.f);
-      for (int q = 0; q < QS; ++q) {
-        const int ks = QS == 1 ? 0 : kept_k(q, g.mS, S);
-        cfma(s, __ldg(z + (long long)q * mL), twS[(int)(((long long)ks * row) % S)]);
-      }
+      KeptIndex ki(QS == 1 ? 0 : g.mS, S, row);
+      for (int q = 0; q < QS; ++q) cfma(s, __ldg(z + (long long)q * mL), twS[ki.next()]);
       U[(rl * mL + k) * Csp + c] = s;
     }
     if (Cs & 1)

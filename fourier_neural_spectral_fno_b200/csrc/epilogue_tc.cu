@@ -20,7 +20,8 @@ namespace fno {
 
 namespace {
 
-constexpr int TC_THREADS = 128;
+constexpr int TC_THREADS = 128;   // tile rows = TMEM lanes
+constexpr int EPI_THREADS = 256;  // two warps per TMEM lane quarter, splitting channel groups
 constexpr int TMEM_COLS = 256;
 
 template <typename T> struct EKind {
@@ -45,11 +46,20 @@ template <> struct EKind<__nv_bfloat16> {
 __host__ __device__ inline int rup(int v, int m) { return (v + m - 1) / m * m; }
 __host__ __device__ inline size_t al16(size_t v) { return (v + 15) & ~(size_t)15; }
 
+constexpr int UMAX = 16;   // spectrum values per thread per tile (B operand)
+
+// Tile plan.  TMEM columns: D [0, NP); then the spectral A block of each
+// last-axis tile offset ("variant"), resident for the whole kernel; then the
+// x block, restaged per tile.  tf32 keeps hi and lo copies of both blocks.
 struct EpiTcGeom {
-  int Rt;       // slab rows per tile
-  int KS;       // spectral K (Rt * 2 mL), padded to KSp
-  int KSp, KXp, KA, NP;
-  int dcol;     // TMEM column of D
+  int Rt;        // slab rows per tile (NL < 128) or 1
+  int nvar;      // distinct tile offsets along the last axis
+  int KS, KSp;   // spectral K and its 16-padded width
+  int KXp, KA, NP;
+  int cs_cols;   // TMEM columns of one spectral variant (hi + lo)
+  int x_col;     // first TMEM column of the x block
+  int total_cols;
+  int upt;       // spectrum values each thread loads per tile
   size_t bhi, blo, twL, bias, mbar, tbase, total;
   uint32_t sbo;
 };
@@ -57,17 +67,20 @@ struct EpiTcGeom {
 __host__ __device__ inline EpiTcGeom epi_tc_geom(const Geom &g, int mode, int Ci, int Co, int eb,
                                                  bool tf32) {
   EpiTcGeom e;
-  const int kstep = tf32 ? 8 : 16;
   e.Rt = g.NL >= 128 ? 1 : 128 / g.NL;
+  e.nvar = g.NL >= 128 ? g.NL / 128 : 1;
   e.KS = e.Rt * 2 * g.mL;
-  (void)kstep;
-  e.KSp = rup(e.KS, 16);                          // 16-element staging granule
+  e.KSp = rup(e.KS, 16);
   e.KXp = mode == EPI_BLOCK_FWD ? rup(Ci, 16) : 0;
   e.KA = e.KSp + e.KXp;
-  const int cout = (mode == EPI_SPEC_BWD) ? Ci : Co;
-  e.NP = rup(cout, 16);
-  const int acols = tf32 ? 2 * e.KA : e.KA / 2;
-  e.dcol = rup(acols, 32);
+  const int cs = (mode == EPI_SPEC_BWD) ? Ci : Co;
+  e.NP = rup(cs, 16);
+  const int per = tf32 ? 2 : 1;                 // columns per 2 elements: tf32 2 (x hi+lo), 16-bit 1/2
+  e.cs_cols = tf32 ? 2 * e.KSp : e.KSp / 2;
+  e.x_col = e.NP + e.nvar * e.cs_cols;
+  e.total_cols = e.x_col + (tf32 ? 2 * e.KXp : e.KXp / 2);
+  (void)per;
+  e.upt = (e.Rt * cs * g.mL + 127) / 128;
   e.sbo = (uint32_t)(e.KA * eb / 16) * 128u;
   size_t off = 0;
   const size_t bbytes = (size_t)e.NP * e.KA * eb;
@@ -82,15 +95,14 @@ __host__ __device__ inline EpiTcGeom epi_tc_geom(const Geom &g, int mode, int Ci
 }
 
 // byte offset of element (n, k) in a K-major no-swizzle B operand
-__device__ __forceinline__ size_t boff(int n, int k, int eb, uint32_t sbo) {
+__host__ __device__ __forceinline__ uint32_t boff(int n, int k, int eb, uint32_t sbo) {
   const int kb = k * eb;
-  return (size_t)(n >> 3) * sbo + (kb >> 4) * 128 + (n & 7) * 16 + (kb & 15);
+  return (uint32_t)(n >> 3) * sbo + (kb >> 4) * 128 + (n & 7) * 16 + (kb & 15);
 }
 
 template <typename T>
-__device__ __forceinline__ void bstore(unsigned char *bhi, unsigned char *blo, int n, int k,
-                                       uint32_t sbo, float v) {
-  const size_t o = boff(n, k, EKind<T>::EB, sbo);
+__device__ __forceinline__ void bstore_at(unsigned char *bhi, unsigned char *blo, uint32_t o,
+                                          float v) {
   if (EKind<T>::tf32) {
     uint32_t hi, lo;
     tc::split_tf32(v, hi, lo);
@@ -109,27 +121,28 @@ struct EpiTcArgs {
   int Ci, Co, act, tanh_pre;
 };
 
-// stage 16 A columns [c0, c0 + 16) of this thread's row into TMEM
+// stage 16 A elements into TMEM: tf32 -> hi at col, lo at col + lo_off;
+// 16-bit -> 8 packed columns at col
 template <typename T>
-__device__ __forceinline__ void stage16(uint32_t taddr_hi, uint32_t taddr_lo, const float (&v)[16]) {
+__device__ __forceinline__ void stage16(uint32_t col, uint32_t lo_off, const float (&v)[16]) {
   if (EKind<T>::tf32) {
     uint32_t hi[16], lo[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) tc::split_tf32(v[i], hi[i], lo[i]);
-    tc::tmem_st16(taddr_hi, hi);
-    tc::tmem_st16(taddr_lo, lo);
+    tc::tmem_st16(col, hi);
+    tc::tmem_st16(col + lo_off, lo);
   } else {
     uint32_t pk[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
       pk[i] = EKind<T>::fmt == tc::FMT_BF16 ? tc::pack_bf16(v[2 * i], v[2 * i + 1])
                                              : tc::pack_f16(v[2 * i], v[2 * i + 1]);
-    tc::tmem_st8(taddr_hi, pk);
+    tc::tmem_st8(col, pk);
   }
 }
 
 template <typename T, int MODE, int CX>
-__global__ void __launch_bounds__(TC_THREADS) k_epi_tc(EpiTcArgs a, Geom g) {
+__global__ void __launch_bounds__(EPI_THREADS) k_epi_tc(EpiTcArgs a, Geom g) {
   using K = EKind<T>;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int Ci = a.Ci, Co = a.Co;
@@ -140,7 +153,9 @@ __global__ void __launch_bounds__(TC_THREADS) k_epi_tc(EpiTcArgs a, Geom g) {
   float *bias_s = reinterpret_cast<float *>(smem + e.bias);
   uint64_t *mbar = reinterpret_cast<uint64_t *>(smem + e.mbar);
   uint32_t *tbase_s = reinterpret_cast<uint32_t *>(smem + e.tbase);
-  const int t = threadIdx.x, warp = t >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int t = tid & (TC_THREADS - 1);   // tile row (point) = TMEM lane
+  const int half = tid >> 7;              // channel groups g with g % 2 == half
   const int NL = g.NL, S = g.S, mL = g.mL, O = g.O;
   const int Cs = MODE == EPI_SPEC_BWD ? Ci : Co;     // spectral output channels
   const long long SN = (long long)S * NL;
@@ -149,12 +164,11 @@ __global__ void __launch_bounds__(TC_THREADS) k_epi_tc(EpiTcArgs a, Geom g) {
     tc::tmem_alloc(tbase_s, TMEM_COLS);
     tc::tmem_relinquish();
   }
-  if (t == 0) tc::mbar_init(mbar, 1);
+  if (tid == 0) tc::mbar_init(mbar, 1);
   build_twiddles(twL, NL);
-  // constant part of B: zero everything, then W in columns [KSp, KSp + Ci)
-  {
+  {  // B: zero, then W in columns [KSp, KSp + Ci)
     const size_t bbytes = (size_t)e.NP * e.KA * K::EB;
-    for (size_t i = t * 16; i < bbytes; i += TC_THREADS * 16) {
+    for (size_t i = tid * 16; i < bbytes; i += EPI_THREADS * 16) {
       *reinterpret_cast<uint4 *>(bhi + i) = make_uint4(0, 0, 0, 0);
       if (K::tf32) *reinterpret_cast<uint4 *>(blo + i) = make_uint4(0, 0, 0, 0);
     }
@@ -162,79 +176,143 @@ __global__ void __launch_bounds__(TC_THREADS) k_epi_tc(EpiTcArgs a, Geom g) {
   __syncthreads();
   if (MODE == EPI_BLOCK_FWD) {
     const T *W = reinterpret_cast<const T *>(a.W);
-    for (int i = t; i < Co * Ci; i += TC_THREADS)
-      bstore<T>(bhi, blo, i / Ci, e.KSp + i % Ci, e.sbo, to_f<T>(W[i]));
+    for (int i = tid; i < Co * Ci; i += EPI_THREADS)
+      bstore_at<T>(bhi, blo, boff(i / Ci, e.KSp + i % Ci, K::EB, e.sbo), to_f<T>(W[i]));
     const T *bias = reinterpret_cast<const T *>(a.bias);
-    for (int o = t; o < Co; o += TC_THREADS) bias_s[o] = bias ? to_f<T>(bias[o]) : 0.f;
+    for (int o = tid; o < Co; o += EPI_THREADS) bias_s[o] = bias ? to_f<T>(bias[o]) : 0.f;
   }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tbase = *tbase_s;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  const uint32_t idesc = tc::instr_desc(K::fmt, 128, e.NP);
-  const uint32_t bhi_a = tc::smem_u32(bhi), blo_a = tc::smem_u32(blo);
-  const uint32_t acol_lo = K::tf32 ? (uint32_t)e.KA : 0u;   // A_lo column offset
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+  const uint32_t arow = tbase + lane_off;
+  const uint32_t lo_spec = K::tf32 ? (uint32_t)e.KSp : 0u;   // lo copy offset (columns)
+  const uint32_t lo_x = K::tf32 ? (uint32_t)e.KXp : 0u;
+
+  // resident spectral A block per variant: row t = point n0 + t (NL >= 128) or
+  // point t of the Rt rows (NL < 128): (cos, -sin)(2 pi k n / NL) in the slot
+  // of the point's row, zeros elsewhere
+  for (int v = 0; v < e.nvar; ++v) {
+    const int n = e.Rt > 1 ? t % NL : v * 128 + t;
+    const int rl = e.Rt > 1 ? t / NL : 0;
+    const uint32_t c0v = arow + e.NP + v * e.cs_cols;
+    int r = 0, k = 0, par = 0, idx = 0;
+    for (int c0 = 0; c0 < e.KSp; c0 += 16) {
+      float vals[16];
+      const bool mine = ((c0 >> 4) & 1) == half;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float val = 0.f;
+        if (c0 + i < e.KS) {
+          if (r == rl) {
+            const float2 w = twL[idx];
+            val = par ? -w.y : w.x;
+          }
+          if (par) {
+            ++k;
+            idx += n;
+            if (idx >= NL) idx -= NL;
+            if (k == mL) {
+              k = 0;
+              ++r;
+              idx = 0;
+            }
+          }
+          par ^= 1;
+        }
+        vals[i] = val;
+      }
+      if (mine) stage16<T>(c0v + (K::tf32 ? c0 : c0 / 2), lo_spec, vals);
+    }
+  }
+  tc::tmem_wait_st();
+
+  // this thread's share of the B spectral block: element i = t + 128 j of the
+  // tile's [Rt][Cs][mL] spectrum, its offset inside the tile's U rows and its
+  // smem position (row o, column r 2 mL + 2 k)
+  int u_off[UMAX / 2];
+  uint32_t b_off[UMAX / 2];
+#pragma unroll
+  for (int j = 0; j < UMAX / 2; ++j) {
+    const int i = tid + EPI_THREADS * j;
+    u_off[j] = -1;
+    b_off[j] = 0;
+    if (i < e.Rt * Cs * mL) {
+      const int k = i % mL, rest = i / mL;
+      const int o = rest % Cs, r = rest / Cs;
+      u_off[j] = (o * O * S + r) * mL + k;
+      b_off[j] = boff(o, r * 2 * mL + 2 * k, K::EB, e.sbo);
+    }
+  }
+
   const T *x = reinterpret_cast<const T *>(a.x);
   T *out = reinterpret_cast<T *>(a.out);
   T *pre_out = reinterpret_cast<T *>(a.pre_out);
-
+  const uint32_t idesc = tc::instr_desc(K::fmt, 128, e.NP);
+  const uint32_t bhi_a = tc::smem_u32(bhi), blo_a = tc::smem_u32(blo);
+  const long long cstride = (long long)O * SN;     // channel stride of activations
   const int tps = (int)(SN / TC_THREADS);          // tiles per slab
   const long long ntiles = g.B * O * tps;
-  uint32_t phase = 0;
-  bool ok = true;
+  const long long per_cta = (ntiles + gridDim.x - 1) / gridDim.x;
+  const long long t_begin = blockIdx.x * per_cta;
+  const long long t_end = t_begin + per_cta < ntiles ? t_begin + per_cta : ntiles;
 
-  for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+  constexpr int GPH = CX / 32 > 0 ? CX / 32 : 1;   // channel groups (of 16) per half
+  float xr[GPH * 16];
+  float2 ur[UMAX / 2];
+  auto fetch = [&](long long tile) {
     const long long slab = tile / tps;
     const long long pbase = (tile - slab * tps) * (long long)TC_THREADS;
     const long long b = slab / O;
     const int outer = (int)(slab - b * O);
-    const int row0 = (int)(pbase / NL);
-    const long long p = pbase + t;
-    const int n = (int)(p % NL);
-    const int rl = (int)(p / NL) - row0;
-
-    // (1) spectral part of B for this tile's rows: B[o][rl*2mL + 2k (+1)] = U
-    for (int i = t; i < e.Rt * Cs * mL; i += TC_THREADS) {
-      const int k = i % mL;
-      const int rest = i / mL;
-      const int o = rest % Cs, r = rest / Cs;
-      const float2 u = __ldg(a.U + ((((b * Cs + o) * O + outer) * S) + row0 + r) * (long long)mL + k);
-      const int col = r * 2 * mL + 2 * k;
-      bstore<T>(bhi, blo, o, col, e.sbo, u.x);
-      bstore<T>(bhi, blo, o, col + 1, e.sbo, u.y);
-    }
-    // (2) A = [basis | x] for this thread's point
-    {
-      const uint32_t arow = tbase + lane_off;
-      for (int c0 = 0; c0 < e.KSp; c0 += 16) {
-        float v[16];
+    if (MODE == EPI_BLOCK_FWD) {
+      const T *xp = x + (b * Ci * O + outer) * SN + pbase + t;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int j = c0 + i;
-          float val = 0.f;
-          if (j < e.KS) {
-            const int r = j / (2 * mL), jj = j - r * 2 * mL;
-            if (r == rl) {
-              const float2 w = twL[((jj >> 1) * n) % NL];
-              val = (jj & 1) ? -w.y : w.x;
-            }
-          }
-          v[i] = val;
-        }
-        stage16<T>(arow + (K::tf32 ? c0 : c0 / 2), arow + acol_lo + c0, v);
+      for (int gi = 0; gi < GPH; ++gi) {
+        const int c0 = (2 * gi + half) * 16;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          xr[gi * 16 + i] = c0 + i < Ci ? ldf<T>(xp + (long long)(c0 + i) * cstride) : 0.f;
       }
-      if (MODE == EPI_BLOCK_FWD) {
-        const long long xb = (b * Ci * O + outer) * SN + p;
-        for (int c0 = 0; c0 < e.KXp; c0 += 16) {
-          float v[16];
+    }
+    const long long ub = ((b * Cs * O + outer) * S + pbase / NL) * (long long)mL;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int ci = c0 + i;
-            v[i] = (ci < Ci) ? ldf<T>(x + xb + (long long)ci * O * SN) : 0.f;
-          }
-          const int col = e.KSp + c0;
-          stage16<T>(arow + (K::tf32 ? col : col / 2), arow + acol_lo + col, v);
+    for (int j = 0; j < UMAX / 2; ++j)
+      if (u_off[j] >= 0) ur[j] = __ldg(a.U + ub + u_off[j]);
+  };
+
+  uint32_t phase = 0;
+  bool ok = true;
+  long long prev_key = -1;
+  if (t_begin < t_end) fetch(t_begin);
+  for (long long tile = t_begin; tile < t_end; ++tile) {
+    const long long slab = tile / tps;
+    const long long pbase = (tile - slab * tps) * (long long)TC_THREADS;
+    const long long key = slab * S + pbase / NL;    // (slab, first row)
+    const int variant = e.Rt > 1 ? 0 : (int)(pbase % NL) / 128;
+    // (1) B spectral block (only when the tile's rows change)
+    if (key != prev_key) {
+#pragma unroll
+      for (int j = 0; j < UMAX / 2; ++j) {
+        if (u_off[j] >= 0) {
+          bstore_at<T>(bhi, blo, b_off[j], ur[j].x);
+          bstore_at<T>(bhi, blo, b_off[j] + K::EB, ur[j].y);
+        }
+      }
+      prev_key = key;
+    }
+    // (2) x block of A
+    if (MODE == EPI_BLOCK_FWD) {
+      const uint32_t xc = arow + e.x_col;
+#pragma unroll
+      for (int gi = 0; gi < GPH; ++gi) {
+        const int c0 = (2 * gi + half) * 16;
+        if (c0 < e.KXp) {
+          float vals[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) vals[i] = xr[gi * 16 + i];
+          stage16<T>(xc + (K::tf32 ? c0 : c0 / 2), lo_x, vals);
         }
       }
     }
@@ -242,51 +320,64 @@ __global__ void __launch_bounds__(TC_THREADS) k_epi_tc(EpiTcArgs a, Geom g) {
     tc::fence_proxy_async_smem();
     tc::fence_before_sync();
     __syncthreads();
-    // (3) one thread issues the MMAs
-    if (t == 0) {
+    // (3) one thread issues the MMAs: spectral K steps then x K steps
+    if (tid == 0) {
       tc::fence_after_sync();
-      const int nsteps = e.KA / K::KSTEP;
-      for (int s = 0; s < nsteps; ++s) {
+      const uint32_t aspec = tbase + e.NP + variant * e.cs_cols;
+      const uint32_t ax = tbase + e.x_col;
+      const int ns = e.KSp / K::KSTEP, nx = e.KXp / K::KSTEP;
+      for (int s = 0; s < ns + nx; ++s) {
         const uint64_t bh = tc::smem_desc_kmajor(bhi_a + s * 256, 128, e.sbo);
-        const uint32_t acolh = tbase + s * 8;   // 8 columns per K step (tf32 or packed 16-bit)
+        const uint32_t acol = s < ns ? aspec + s * 8 : ax + (s - ns) * 8;
+        const uint32_t alo = s < ns ? lo_spec : lo_x;
         if (K::tf32) {
           const uint64_t bl = tc::smem_desc_kmajor(blo_a + s * 256, 128, e.sbo);
-          tc::mma_tf32_ts(tbase + e.dcol, acolh, bh, idesc, s > 0 ? 1u : 0u);
-          tc::mma_tf32_ts(tbase + e.dcol, acolh, bl, idesc, 1u);
-          tc::mma_tf32_ts(tbase + e.dcol, acolh + acol_lo, bh, idesc, 1u);
+          tc::mma_tf32_ts(tbase, acol, bh, idesc, s > 0 ? 1u : 0u);
+          tc::mma_tf32_ts(tbase, acol, bl, idesc, 1u);
+          tc::mma_tf32_ts(tbase, acol + alo, bh, idesc, 1u);
         } else {
-          tc::mma_f16_ts(tbase + e.dcol, acolh, bh, idesc, s > 0 ? 1u : 0u);
+          tc::mma_f16_ts(tbase, acol, bh, idesc, s > 0 ? 1u : 0u);
         }
       }
       tc::mma_commit(mbar);
     }
-    // (4) epilogue
+    // (4) prefetch the next tile while the MMAs run
+    if (tile + 1 < t_end) fetch(tile + 1);
+    // (5) epilogue
     ok = tc::mbar_wait(mbar, phase & 1, a.err);
     phase++;
     tc::fence_after_sync();
-    const long long ob = (b * Cs * O + outer) * SN + p;
+    const long long b = slab / O;
+    const int outer = (int)(slab - b * O);
+    const long long ob = (b * Cs * O + outer) * SN + pbase + t;
 #pragma unroll
-    for (int c0 = 0; c0 < CX; c0 += 16) {
+    for (int gi = 0; gi < GPH; ++gi) {
+      const int c0 = (2 * gi + half) * 16;
+      T *op = out + ob + (long long)c0 * cstride;
+      T *pp = pre_out ? pre_out + ob + (long long)c0 * cstride : nullptr;
+      const T *xq = x + ob + (long long)c0 * cstride;
       if (c0 < Cs) {
         uint32_t dv[16];
-        tc::tmem_ld16(tbase + lane_off + e.dcol + c0, dv);
+        tc::tmem_ld16(arow + c0, dv);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int o = c0 + i;
           if (o < Cs) {
             float val = __uint_as_float(dv[i]);
-            const long long oi = ob + (long long)o * O * SN;
             if (MODE == EPI_BLOCK_FWD) {
               val += bias_s[o];
-              if (pre_out) pre_out[oi] = from_f<T>(val);
+              if (pp) *pp = from_f<T>(val);
               if (a.act) val = gelu_f(val);
             } else if (MODE == EPI_SPEC_BWD && a.tanh_pre) {
-              const float th = tanhf(ldf<T>(x + oi));
+              const float th = tanhf(ldf<T>(xq));
               val *= 1.f - th * th;
             }
-            out[oi] = from_f<T>(val);
+            *op = from_f<T>(val);
           }
+          op += cstride;
+          if (pp) pp += cstride;
+          xq += cstride;
         }
       }
     }
@@ -300,26 +391,42 @@ __global__ void __launch_bounds__(TC_THREADS) k_epi_tc(EpiTcArgs a, Geom g) {
 }
 
 // U[b, c, outer, r, k] = sum_q Z[b, c, outer, q, k] exp(+2 pi i kS(q) r / S)
+// One CTA per (b, c, outer) slab; a thread owns one row r and four modes.
 __global__ void __launch_bounds__(256) k_inv_slab(const float2 *__restrict__ Z,
                                                   float2 *__restrict__ U, int S, int mS, int QS,
                                                   int mL) {
   extern __shared__ __align__(1024) unsigned char smem[];
+  const int mLp = (mL + 3) & ~3;
   float2 *twS = reinterpret_cast<float2 *>(smem);
-  float2 *zs = twS + S;                      // [QS][mL]
+  float2 *zs = twS + ((S + 1) & ~1);          // [QS][mLp], 16-byte aligned rows
   const long long slab = blockIdx.x;
   build_twiddles(twS, S);
   const float2 *z = Z + slab * QS * mL;
-  for (int i = threadIdx.x; i < QS * mL; i += blockDim.x) zs[i] = z[i];
+  for (int i = threadIdx.x; i < QS * mLp; i += blockDim.x) {
+    const int q = i / mLp, k = i - q * mLp;
+    zs[i] = k < mL ? z[q * mL + k] : make_float2(0.f, 0.f);
+  }
   __syncthreads();
   float2 *u = U + slab * (long long)S * mL;
-  for (int i = threadIdx.x; i < S * mL; i += blockDim.x) {
-    const int r = i / mL, k = i - r * mL;
-    float2 s = make_float2(0.f, 0.f);
+  const int mLg = mLp / 4;
+  for (int i = threadIdx.x; i < S * mLg; i += blockDim.x) {
+    const int r = i / mLg, kg = i - r * mLg;
+    float2 acc[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[j] = make_float2(0.f, 0.f);
+    KeptIndex ki(QS == 1 ? 0 : mS, S, r);
     for (int q = 0; q < QS; ++q) {
-      const int ks = QS == 1 ? 0 : kept_k(q, mS, S);
-      cfma(s, zs[q * mL + k], twS[(int)(((long long)ks * r) % S)]);
+      const float2 w = twS[ki.next()];
+      const float4 z01 = *reinterpret_cast<const float4 *>(zs + q * mLp + 4 * kg);
+      const float4 z23 = *reinterpret_cast<const float4 *>(zs + q * mLp + 4 * kg + 2);
+      cfma(acc[0], make_float2(z01.x, z01.y), w);
+      cfma(acc[1], make_float2(z01.z, z01.w), w);
+      cfma(acc[2], make_float2(z23.x, z23.y), w);
+      cfma(acc[3], make_float2(z23.z, z23.w), w);
     }
-    u[i] = s;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (4 * kg + j < mL) u[r * mL + 4 * kg + j] = acc[j];
   }
 }
 
@@ -329,7 +436,7 @@ cudaError_t launch_epi_tc_m(const Launch &L, const Geom &g, const EpiTcArgs &a, 
   const EpiTcGeom e = epi_tc_geom(g, MODE, a.Ci, a.Co, EKind<T>::EB, EKind<T>::tf32);
   auto go = [&](auto kern) {
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)e.total);
-    kern<<<grid, TC_THREADS, e.total, L.stream>>>(a, g);
+    kern<<<grid, EPI_THREADS, e.total, L.stream>>>(a, g);
   };
   if (cmax <= 16) go(k_epi_tc<T, MODE, 16>);
   else if (cmax <= 32) go(k_epi_tc<T, MODE, 32>);
@@ -354,7 +461,8 @@ bool epi_tc_supported(const Geom &g, int dtype, int mode, int Ci, int Co) {
   if (SN % 128 != 0) return false;
   const bool tf32 = dtype == DT_F32;
   const EpiTcGeom e = epi_tc_geom(g, mode, Ci, Co, tf32 ? 4 : 2, tf32);
-  if (e.dcol + e.NP > TMEM_COLS) return false;
+  if (e.total_cols > TMEM_COLS) return false;
+  if (e.Rt * ((mode == EPI_SPEC_BWD) ? Ci : Co) * g.mL > (UMAX / 2) * EPI_THREADS) return false;
   return e.total <= 227 * 1024;
 }
 
@@ -365,7 +473,7 @@ size_t inv_slab_bytes(const Geom &g, long long C) {
 cudaError_t launch_inv_slab(const Launch &L, const Geom &g, long long C, const float2 *Z,
                             float2 *U) {
   const long long slabs = g.B * C * g.O;
-  const size_t smem = sizeof(float2) * ((size_t)g.S + (size_t)g.QS * g.mL);
+  const size_t smem = sizeof(float2) * ((size_t)((g.S + 1) & ~1) + (size_t)g.QS * ((g.mL + 3) & ~3));
   launch_begin(L);
   k_inv_slab<<<(unsigned)slabs, 256, smem, L.stream>>>(Z, U, g.S, g.mS, g.QS, g.mL);
   launch_end(L, "inv_slab");

@@ -78,6 +78,28 @@ __device__ __forceinline__ void build_twiddles(float2 *tw, int n) {
 // kept wavenumber of storage slot q on a non-last axis (positive block first)
 __device__ __forceinline__ int kept_k(int q, int m, int n) { return q < m ? q : n - 2 * m + q; }
 
+// (k * r) mod n for 0 <= k, r < n <= 4096 (fits in 32 bits)
+__device__ __forceinline__ int mulmod(int k, int r, int n) { return (k * r) % n; }
+
+// Walks the twiddle index (kept_k(q, m, n) * r) mod n over q = 0, 1, ...:
+// the positive block starts at 0 and the negative block at ((n - m) r) mod n,
+// each advancing by r.  With m == 0 (a single kept mode, k = 0) it stays 0.
+struct KeptIndex {
+  int idx, step, n, m, q;
+  __device__ __forceinline__ KeptIndex(int m_, int n_, int r) : idx(0), step(r % n_), n(n_), m(m_), q(0) {}
+  __device__ __forceinline__ int next() {
+    const int cur = idx;
+    ++q;
+    if (q == m) {
+      idx = mulmod(n - m, step, n);
+    } else {
+      idx += step;
+      if (idx >= n) idx -= n;
+    }
+    return cur;
+  }
+};
+
 // ---------------------------------------------------------------------------
 // activations
 // ---------------------------------------------------------------------------

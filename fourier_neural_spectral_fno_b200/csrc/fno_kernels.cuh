@@ -123,6 +123,10 @@ cudaError_t launch_lift(const Launch &L, const Geom &g, int dtype, int in_ch, in
 cudaError_t launch_proj_fwd(const Launch &L, const Geom &g, int dtype, int width, int hidden,
                             int out_ch, const void *v, const void *Q1, const void *q1,
                             const void *Q2, const void *q2, void *u);
+bool proj_tc_supported(const Geom &g, int dtype, int width, int hidden, int out_ch);
+cudaError_t launch_proj_fwd_tc(const Launch &L, const Geom &g, int dtype, int width, int hidden,
+                               int out_ch, const void *v, const void *Q1, const void *q1,
+                               const void *Q2, const void *q2, void *u);
 int proj_bwd_grid(const Geom &g, int num_sms);
 size_t proj_bwd_partial_floats(int width, int hidden, int out_ch);
 size_t proj_bwd_smem_bytes(int width, int hidden, int out_ch);

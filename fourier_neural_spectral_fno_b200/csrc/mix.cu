@@ -13,7 +13,7 @@ namespace fno {
 namespace {
 
 constexpr int MX_THREADS = 128;
-constexpr int MX_BT = 8;  // batch entries per thread
+constexpr int MX_BT = 4;  // batch entries per thread
 
 __device__ __forceinline__ float weight_of(long long k, int mL, int NL, float inv_n) {
   return mode_weight((int)(k % mL), NL, inv_n);
@@ -30,11 +30,15 @@ __global__ void __launch_bounds__(MX_THREADS)
   float2 acc[MX_BT];
 #pragma unroll
   for (int j = 0; j < MX_BT; ++j) acc[j] = make_float2(0.f, 0.f);
+  const T *rp = R + 2 * ((long long)o * K + k);
+  const long long rstride = 2LL * Co * K;
+  const float2 *xp = xhat + b0 * Ci * K + k;
+#pragma unroll 8
   for (int i = 0; i < Ci; ++i) {
-    const float2 r = ldc<T>(R + 2 * (((long long)i * Co + o) * K + k));
+    const float2 r = ldc<T>(rp + i * rstride);
 #pragma unroll
     for (int j = 0; j < MX_BT; ++j)
-      if (b0 + j < B) cfma(acc[j], __ldg(xhat + ((b0 + j) * Ci + i) * K + k), r);
+      if (b0 + j < B) cfma(acc[j], __ldg(xp + (j * Ci + i) * K), r);
   }
   const float w = weight_of(k, mL, NL, inv_n);
 #pragma unroll

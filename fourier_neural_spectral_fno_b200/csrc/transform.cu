@@ -125,9 +125,11 @@ __global__ void __launch_bounds__(FS_THREADS) k_fwd_slab(FwdSlabArgs a) {
       const int q = p / mL, k = p - q * mL;
       const int ks = QS == 1 ? 0 : kept_k(q, a.mS, S);
       float2 s = acc2[p];
+      int idx = mulmod(ks, rt0, S);
       for (int r = 0; r < nrows; ++r) {
-        const int row = rt0 + r;
-        cfma_conj_b(s, X1[r * mL + k], twS[(int)(((long long)ks * row) % S)]);
+        cfma_conj_b(s, X1[r * mL + k], twS[idx]);
+        idx += ks;
+        if (idx >= S) idx -= S;
       }
       acc2[p] = s;
     }
@@ -162,8 +164,13 @@ __global__ void __launch_bounds__(256) k_fwd_finish(const float2 *__restrict__ z
   }
   for (int q0 = 0; q0 < QO; q0 += 16) {
     float2 acc[16];
+    int idx[16], stp[16];
 #pragma unroll
-    for (int q = 0; q < 16; ++q) acc[q] = make_float2(0.f, 0.f);
+    for (int q = 0; q < 16; ++q) {
+      acc[q] = make_float2(0.f, 0.f);
+      idx[q] = 0;
+      stp[q] = q0 + q < QO ? kept_k(q0 + q, mO, O) : 0;
+    }
     for (int n0 = 0; n0 < O; ++n0) {
       float2 z = make_float2(0.f, 0.f);
       for (int band = 0; band < nbands; ++band) {
@@ -173,10 +180,9 @@ __global__ void __launch_bounds__(256) k_fwd_finish(const float2 *__restrict__ z
       }
 #pragma unroll
       for (int q = 0; q < 16; ++q) {
-        if (q0 + q < QO) {
-          const int k0 = kept_k(q0 + q, mO, O);
-          cfma_conj_b(acc[q], z, twO[(int)(((long long)k0 * n0) % O)]);
-        }
+        if (q0 + q < QO) cfma_conj_b(acc[q], z, twO[idx[q]]);
+        idx[q] += stp[q];
+        if (idx[q] >= O) idx[q] -= O;
       }
     }
 #pragma unroll
@@ -200,10 +206,8 @@ __global__ void __launch_bounds__(256) k_inv_expand(const float2 *__restrict__ V
   const int n0 = (int)(rest % O);
   const long long bc = rest / O;
   float2 s = make_float2(0.f, 0.f);
-  for (int q0 = 0; q0 < QO; ++q0) {
-    const int k0 = kept_k(q0, mO, O);
-    cfma(s, V[(bc * QO + q0) * QSmL + p], twO[(int)(((long long)k0 * n0) % O)]);
-  }
+  KeptIndex ki(mO, O, n0);
+  for (int q0 = 0; q0 < QO; ++q0) cfma(s, V[(bc * QO + q0) * QSmL + p], twO[ki.next()]);
   Z[t] = s;
 }
 

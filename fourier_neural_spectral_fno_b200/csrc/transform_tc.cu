@@ -53,9 +53,11 @@ template <> struct Kind<__nv_bfloat16> {
 };
 
 struct S1Layout {
-  size_t fhi, flo, twL, twS, x1, mbar, tbase, total;
+  size_t fhi, flo, twL, twS, x1, xs, mbar, tbase, total;
   int x1_ld, mLp;
 };
+
+constexpr int XS_LD = 144;   // bytes per staged row chunk (128 + 16 pad: conflict-free rows)
 
 __host__ __device__ inline size_t al16(size_t v) { return (v + 15) & ~(size_t)15; }
 
@@ -69,7 +71,12 @@ __host__ __device__ inline S1Layout s1_layout(int S, int NL, int mL, int NP, int
   l.flo = off; if (tf32) off = al16(off + fbytes);
   l.twL = off; off = al16(off + sizeof(float2) * NL);
   l.twS = off; off = al16(off + sizeof(float2) * S);
-  l.x1 = off; off = al16(off + sizeof(float) * (size_t)TC_THREADS * l.x1_ld);
+  // the staged row chunks (chunk loop) and the X1 copy (after it) share space
+  const size_t x1b = sizeof(float) * (size_t)TC_THREADS * l.x1_ld;
+  const size_t xsb = 2 * (size_t)TC_THREADS * XS_LD;
+  l.x1 = off;
+  l.xs = off;
+  off = al16(off + (x1b > xsb ? x1b : xsb));
   l.mbar = off; off = al16(off + 2 * sizeof(uint64_t));
   l.tbase = off; off = al16(off + sizeof(uint32_t));
   // keep at most two CTAs per SM so their TMEM allocations always fit
@@ -88,6 +95,24 @@ __device__ __forceinline__ float elem(const uint4 (&raw)[8], int i) {
   }
 }
 
+// apply the load transform (tanh, or dz = dy * GELU'(pre)) to one 16-byte
+// piece, keeping the storage format
+template <typename T, int LOAD>
+__device__ __forceinline__ uint4 transform16(uint4 v0, uint4 v1) {
+  if (LOAD == LOAD_PLAIN) return v0;
+  constexpr int NE = 16 / sizeof(T);
+  T *a = reinterpret_cast<T *>(&v0);
+  const T *b = reinterpret_cast<const T *>(&v1);
+#pragma unroll
+  for (int i = 0; i < NE; ++i) {
+    float x = to_f<T>(a[i]);
+    if (LOAD == LOAD_TANH) x = tanhf(x);
+    if (LOAD == LOAD_DZ) x *= gelu_grad_f(to_f<T>(b[i]));
+    a[i] = from_f<T>(x);
+  }
+  return v0;
+}
+
 template <typename T, int LOAD>
 __global__ void __launch_bounds__(TC_THREADS) k_s1_tc(S1Args a) {
   using K = Kind<T>;
@@ -104,6 +129,7 @@ __global__ void __launch_bounds__(TC_THREADS) k_s1_tc(S1Args a) {
   float *x1s = reinterpret_cast<float *>(smem + lay.x1);
   uint64_t *mbar = reinterpret_cast<uint64_t *>(smem + lay.mbar);
   uint32_t *tbase_s = reinterpret_cast<uint32_t *>(smem + lay.tbase);
+  unsigned char *xs = smem + lay.xs;       // [2][128][XS_LD] staged row chunks
   const int t = threadIdx.x, warp = t >> 5;
 
   if (warp == 0) {
@@ -155,41 +181,56 @@ __global__ void __launch_bounds__(TC_THREADS) k_s1_tc(S1Args a) {
 
   for (long long tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
     const long long row0 = tile * TC_THREADS;
-    const long long my_row = row0 + t;
-    const bool valid = my_row < a.total_rows;
-    const uint4 *src0 = reinterpret_cast<const uint4 *>(in0 + (valid ? my_row : 0) * NL);
-    const uint4 *src1 = LOAD == LOAD_DZ ? reinterpret_cast<const uint4 *>(in1 + (valid ? my_row : 0) * NL)
-                                        : nullptr;
-    uint4 r0[8], r1[8], n0[8], n1[8];
+    // coalesced loading: thread t fetches 16-byte piece (t & 7) of rows
+    // (t >> 3) + 16 j, j < 8, for every 128-byte chunk of the row
+    const int seg = t & 7;
+    const uint4 *src0[8];
+    const uint4 *src1[8];
+    bool rv[8];
 #pragma unroll
-    for (int v = 0; v < 8; ++v) {
-      r0[v] = valid ? __ldg(src0 + v) : make_uint4(0, 0, 0, 0);
-      if (LOAD == LOAD_DZ) r1[v] = valid ? __ldg(src1 + v) : make_uint4(0, 0, 0, 0);
+    for (int j = 0; j < 8; ++j) {
+      const long long row = row0 + (t >> 3) + 16 * j;
+      rv[j] = row < a.total_rows;
+      const long long rr = rv[j] ? row : 0;
+      src0[j] = reinterpret_cast<const uint4 *>(in0 + rr * NL) + seg;
+      src1[j] = LOAD == LOAD_DZ ? reinterpret_cast<const uint4 *>(in1 + rr * NL) + seg : nullptr;
+    }
+    uint4 p0[8], p1[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      p0[j] = rv[j] ? __ldg(src0[j]) : make_uint4(0, 0, 0, 0);
+      if (LOAD == LOAD_DZ) p1[j] = rv[j] ? __ldg(src1[j]) : make_uint4(0, 0, 0, 0);
     }
     for (int c = 0; c < nchunks; ++c, ++g) {
+      const uint32_t buf = g & 1;
+      unsigned char *xb = xs + buf * (TC_THREADS * XS_LD);
+      // (1) transformed pieces of chunk c -> shared memory
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<uint4 *>(xb + ((t >> 3) + 16 * j) * XS_LD + seg * 16) =
+            transform16<T, LOAD>(p0[j], LOAD == LOAD_DZ ? p1[j] : p0[j]);
+      // (2) prefetch chunk c + 1
       if (c + 1 < nchunks) {
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          n0[v] = valid ? __ldg(src0 + (c + 1) * 8 + v) : make_uint4(0, 0, 0, 0);
-          if (LOAD == LOAD_DZ) n1[v] = valid ? __ldg(src1 + (c + 1) * 8 + v) : make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < 8; ++j) {
+          p0[j] = rv[j] ? __ldg(src0[j] + (c + 1) * 8) : make_uint4(0, 0, 0, 0);
+          if (LOAD == LOAD_DZ) p1[j] = rv[j] ? __ldg(src1[j] + (c + 1) * 8) : make_uint4(0, 0, 0, 0);
         }
       }
-      const uint32_t buf = g & 1;
+      // (3) the A buffer of chunk c - 2 must be free
       if (g >= 2) ok = tc::mbar_wait(&mbar[buf], ((g - 2) >> 1) & 1, a.err);
       if (__syncthreads_or(!ok)) { ok = false; break; }
       tc::fence_after_sync();
+      // (4) this thread's row of the chunk -> A operand in TMEM
+      uint4 r0[8];
+#pragma unroll
+      for (int v = 0; v < 8; ++v) r0[v] = *reinterpret_cast<const uint4 *>(xb + t * XS_LD + v * 16);
       const uint32_t acol = tbase + lane_off + A_COL0 + buf * ACOLS;
-      // stage the chunk as the A operand (transform applied on the way)
 #pragma unroll
       for (int h = 0; h < CW / 16; ++h) {      // 16 elements per step
         float xv[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float v = elem<T>(r0, h * 16 + i);
-          if (LOAD == LOAD_TANH) v = tanhf(v);
-          if (LOAD == LOAD_DZ) v *= gelu_grad_f(elem<T>(r1, h * 16 + i));
-          xv[i] = v;
-        }
+        for (int i = 0; i < 16; ++i) xv[i] = elem<T>(r0, h * 16 + i);
         if (K::tf32) {
           uint32_t hi[16], lo[16];
 #pragma unroll
@@ -226,11 +267,6 @@ __global__ void __launch_bounds__(TC_THREADS) k_s1_tc(S1Args a) {
           }
         }
         tc::mma_commit(&mbar[buf]);
-      }
-#pragma unroll
-      for (int v = 0; v < 8; ++v) {
-        r0[v] = n0[v];
-        if (LOAD == LOAD_DZ) r1[v] = n1[v];
       }
     }
     if (!ok) break;

@@ -168,7 +168,9 @@ def _tiny_network(grid, modes, dtype, batch=2, width=6, hidden=9, layers=2, in_c
 
 
 @pytest.mark.parametrize("grid,modes", [((16, 12), (4, 5)), ((40, 70), (6, 9)),
-                                        ((6, 10, 12), (2, 3, 4)), ((100,), (20,))])
+                                        ((6, 10, 12), (2, 3, 4)), ((100,), (20,)),
+                                        ((64, 64), (10, 12)), ((8, 16, 64), (2, 4, 8)),
+                                        ((256,), (40,))])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_network_forward_backward_mse(grid, modes, dtype):
     import torch
