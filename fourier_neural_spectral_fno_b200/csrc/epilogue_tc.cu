@@ -56,6 +56,7 @@ struct EpiTcGeom {
   int nvar;      // distinct tile offsets along the last axis
   int KS, KSp;   // spectral K and its 16-padded width
   int KXp, KA, NP;
+  int DC;        // TMEM columns of D: tf32 keeps A B_hi and A B_lo side by side (2 NP)
   int cs_cols;   // TMEM columns of one spectral variant (hi + lo)
   int x_col;     // first TMEM column of the x block
   int total_cols;
@@ -75,17 +76,19 @@ __host__ __device__ inline EpiTcGeom epi_tc_geom(const Geom &g, int mode, int Ci
   e.KA = e.KSp + e.KXp;
   const int cs = (mode == EPI_SPEC_BWD) ? Ci : Co;
   e.NP = rup(cs, 16);
-  const int per = tf32 ? 2 : 1;                 // columns per 2 elements: tf32 2 (x hi+lo), 16-bit 1/2
+  e.DC = tf32 ? 2 * e.NP : e.NP;
   e.cs_cols = tf32 ? 2 * e.KSp : e.KSp / 2;
-  e.x_col = e.NP + e.nvar * e.cs_cols;
+  e.x_col = e.DC + e.nvar * e.cs_cols;
   e.total_cols = e.x_col + (tf32 ? 2 * e.KXp : e.KXp / 2);
-  (void)per;
   e.upt = (e.Rt * cs * g.mL + 127) / 128;
   e.sbo = (uint32_t)(e.KA * eb / 16) * 128u;
+  // B rows [0, NP) hold the hi split and rows [NP, 2 NP) the lo split (tf32), so
+  // one MMA of width 2 NP applies both
   size_t off = 0;
   const size_t bbytes = (size_t)e.NP * e.KA * eb;
-  e.bhi = off; off = al16(off + bbytes);
-  e.blo = off; if (tf32) off = al16(off + bbytes);
+  e.bhi = off;
+  e.blo = off + bbytes;
+  off = al16(off + (tf32 ? 2 : 1) * bbytes);
   e.twL = off; off = al16(off + sizeof(float2) * g.NL);
   e.bias = off; off = al16(off + sizeof(float) * 64);
   e.mbar = off; off = al16(off + sizeof(uint64_t));
@@ -167,11 +170,9 @@ __global__ void __launch_bounds__(EPI_THREADS) k_epi_tc(EpiTcArgs a, Geom g) {
   if (tid == 0) tc::mbar_init(mbar, 1);
   build_twiddles(twL, NL);
   {  // B: zero, then W in columns [KSp, KSp + Ci)
-    const size_t bbytes = (size_t)e.NP * e.KA * K::EB;
-    for (size_t i = tid * 16; i < bbytes; i += EPI_THREADS * 16) {
+    const size_t bbytes = (size_t)e.NP * e.KA * K::EB * (K::tf32 ? 2 : 1);
+    for (size_t i = tid * 16; i < bbytes; i += EPI_THREADS * 16)
       *reinterpret_cast<uint4 *>(bhi + i) = make_uint4(0, 0, 0, 0);
-      if (K::tf32) *reinterpret_cast<uint4 *>(blo + i) = make_uint4(0, 0, 0, 0);
-    }
   }
   __syncthreads();
   if (MODE == EPI_BLOCK_FWD) {
@@ -196,7 +197,7 @@ __global__ void __launch_bounds__(EPI_THREADS) k_epi_tc(EpiTcArgs a, Geom g) {
   for (int v = 0; v < e.nvar; ++v) {
     const int n = e.Rt > 1 ? t % NL : v * 128 + t;
     const int rl = e.Rt > 1 ? t / NL : 0;
-    const uint32_t c0v = arow + e.NP + v * e.cs_cols;
+    const uint32_t c0v = arow + e.DC + v * e.cs_cols;
     int r = 0, k = 0, par = 0, idx = 0;
     for (int c0 = 0; c0 < e.KSp; c0 += 16) {
       float vals[16];
@@ -233,24 +234,27 @@ __global__ void __launch_bounds__(EPI_THREADS) k_epi_tc(EpiTcArgs a, Geom g) {
   // smem position (row o, column r 2 mL + 2 k)
   int u_off[UMAX / 2];
   uint32_t b_off[UMAX / 2];
+  float u_bias[UMAX / 2];   // bias added to the k = 0 real column (basis cos 0 = 1)
 #pragma unroll
   for (int j = 0; j < UMAX / 2; ++j) {
     const int i = tid + EPI_THREADS * j;
     u_off[j] = -1;
     b_off[j] = 0;
+    u_bias[j] = 0.f;
     if (i < e.Rt * Cs * mL) {
       const int k = i % mL, rest = i / mL;
       const int o = rest % Cs, r = rest / Cs;
       u_off[j] = (o * O * S + r) * mL + k;
       b_off[j] = boff(o, r * 2 * mL + 2 * k, K::EB, e.sbo);
+      if (MODE == EPI_BLOCK_FWD && k == 0) u_bias[j] = bias_s[o];
     }
   }
 
   const T *x = reinterpret_cast<const T *>(a.x);
   T *out = reinterpret_cast<T *>(a.out);
   T *pre_out = reinterpret_cast<T *>(a.pre_out);
-  const uint32_t idesc = tc::instr_desc(K::fmt, 128, e.NP);
-  const uint32_t bhi_a = tc::smem_u32(bhi), blo_a = tc::smem_u32(blo);
+  const uint32_t idesc = tc::instr_desc(K::fmt, 128, e.DC);
+  const uint32_t bhi_a = tc::smem_u32(bhi);
   const long long cstride = (long long)O * SN;     // channel stride of activations
   const int tps = (int)(SN / TC_THREADS);          // tiles per slab
   const long long ntiles = g.B * O * tps;
@@ -258,49 +262,75 @@ __global__ void __launch_bounds__(EPI_THREADS) k_epi_tc(EpiTcArgs a, Geom g) {
   const long long t_begin = blockIdx.x * per_cta;
   const long long t_end = t_begin + per_cta < ntiles ? t_begin + per_cta : ntiles;
 
+  // Tile cursor: tiles of a CTA are consecutive, so (b, outer, row0, n0) is
+  // advanced incrementally (no 64-bit division per tile).
+  struct Cursor {
+    long long b;
+    int outer, row0, n0;   // first row of the tile and its last-axis offset
+  };
+  Cursor cur{0, 0, 0, 0};
+  if (t_begin < t_end) {
+    const long long slab = t_begin / tps;
+    const int pb = (int)(t_begin - slab * tps) * TC_THREADS;
+    cur.b = slab / O;
+    cur.outer = (int)(slab - cur.b * O);
+    cur.row0 = pb / NL;
+    cur.n0 = pb - cur.row0 * NL;
+  }
+  auto advance = [&](Cursor c) {
+    if (NL >= TC_THREADS) {
+      c.n0 += TC_THREADS;
+      if (c.n0 == NL) { c.n0 = 0; ++c.row0; }
+    } else {
+      c.row0 += e.Rt;
+    }
+    if (c.row0 == S) {
+      c.row0 = 0;
+      if (++c.outer == O) { c.outer = 0; ++c.b; }
+    }
+    return c;
+  };
+
   constexpr int GPH = CX / 32 > 0 ? CX / 32 : 1;   // channel groups (of 16) per half
   float xr[GPH * 16];
   float2 ur[UMAX / 2];
-  auto fetch = [&](long long tile) {
-    const long long slab = tile / tps;
-    const long long pbase = (tile - slab * tps) * (long long)TC_THREADS;
-    const long long b = slab / O;
-    const int outer = (int)(slab - b * O);
+  auto fetch = [&](const Cursor &c) {
+    const long long pt = (long long)c.row0 * NL + c.n0 + t;
     if (MODE == EPI_BLOCK_FWD) {
-      const T *xp = x + (b * Ci * O + outer) * SN + pbase + t;
+      const T *xp = x + (c.b * Ci * O + c.outer) * SN + pt;
 #pragma unroll
       for (int gi = 0; gi < GPH; ++gi) {
         const int c0 = (2 * gi + half) * 16;
+        const T *xq = xp + (long long)c0 * cstride;
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          xr[gi * 16 + i] = c0 + i < Ci ? ldf<T>(xp + (long long)(c0 + i) * cstride) : 0.f;
+        for (int i = 0; i < 16; ++i) {
+          xr[gi * 16 + i] = c0 + i < Ci ? ldf<T>(xq) : 0.f;
+          xq += cstride;
+        }
       }
     }
-    const long long ub = ((b * Cs * O + outer) * S + pbase / NL) * (long long)mL;
+    const float2 *up = a.U + ((c.b * Cs * O + c.outer) * S + c.row0) * (long long)mL;
 #pragma unroll
     for (int j = 0; j < UMAX / 2; ++j)
-      if (u_off[j] >= 0) ur[j] = __ldg(a.U + ub + u_off[j]);
+      if (u_off[j] >= 0) ur[j] = __ldg(up + u_off[j]);
   };
 
   uint32_t phase = 0;
   bool ok = true;
-  long long prev_key = -1;
-  if (t_begin < t_end) fetch(t_begin);
+  if (t_begin < t_end) fetch(cur);
   for (long long tile = t_begin; tile < t_end; ++tile) {
-    const long long slab = tile / tps;
-    const long long pbase = (tile - slab * tps) * (long long)TC_THREADS;
-    const long long key = slab * S + pbase / NL;    // (slab, first row)
-    const int variant = e.Rt > 1 ? 0 : (int)(pbase % NL) / 128;
+    const Cursor c = cur;
+    const bool new_rows = tile == t_begin || NL < TC_THREADS || c.n0 == 0;
+    const int variant = e.Rt > 1 ? 0 : c.n0 / TC_THREADS;
     // (1) B spectral block (only when the tile's rows change)
-    if (key != prev_key) {
+    if (new_rows) {
 #pragma unroll
       for (int j = 0; j < UMAX / 2; ++j) {
         if (u_off[j] >= 0) {
-          bstore_at<T>(bhi, blo, b_off[j], ur[j].x);
+          bstore_at<T>(bhi, blo, b_off[j], ur[j].x + u_bias[j]);
           bstore_at<T>(bhi, blo, b_off[j] + K::EB, ur[j].y);
         }
       }
-      prev_key = key;
     }
     // (2) x block of A
     if (MODE == EPI_BLOCK_FWD) {
@@ -320,64 +350,87 @@ __global__ void __launch_bounds__(EPI_THREADS) k_epi_tc(EpiTcArgs a, Geom g) {
     tc::fence_proxy_async_smem();
     tc::fence_before_sync();
     __syncthreads();
-    // (3) one thread issues the MMAs: spectral K steps then x K steps
+    // (3) one thread issues the MMAs: spectral K steps then x K steps; for
+    // tf32 each K step is A_hi [B_hi; B_lo] + A_lo [B_hi; B_lo]
     if (tid == 0) {
       tc::fence_after_sync();
-      const uint32_t aspec = tbase + e.NP + variant * e.cs_cols;
+      const uint32_t aspec = tbase + e.DC + variant * e.cs_cols;
       const uint32_t ax = tbase + e.x_col;
       const int ns = e.KSp / K::KSTEP, nx = e.KXp / K::KSTEP;
       for (int s = 0; s < ns + nx; ++s) {
-        const uint64_t bh = tc::smem_desc_kmajor(bhi_a + s * 256, 128, e.sbo);
+        const uint64_t bd = tc::smem_desc_kmajor(bhi_a + s * 256, 128, e.sbo);
         const uint32_t acol = s < ns ? aspec + s * 8 : ax + (s - ns) * 8;
-        const uint32_t alo = s < ns ? lo_spec : lo_x;
         if (K::tf32) {
-          const uint64_t bl = tc::smem_desc_kmajor(blo_a + s * 256, 128, e.sbo);
-          tc::mma_tf32_ts(tbase, acol, bh, idesc, s > 0 ? 1u : 0u);
-          tc::mma_tf32_ts(tbase, acol, bl, idesc, 1u);
-          tc::mma_tf32_ts(tbase, acol + alo, bh, idesc, 1u);
+          const uint32_t alo = s < ns ? lo_spec : lo_x;
+          tc::mma_tf32_ts(tbase, acol, bd, idesc, s > 0 ? 1u : 0u);
+          tc::mma_tf32_ts(tbase, acol + alo, bd, idesc, 1u);
         } else {
-          tc::mma_f16_ts(tbase, acol, bh, idesc, s > 0 ? 1u : 0u);
+          tc::mma_f16_ts(tbase, acol, bd, idesc, s > 0 ? 1u : 0u);
         }
       }
       tc::mma_commit(mbar);
     }
     // (4) prefetch the next tile while the MMAs run
-    if (tile + 1 < t_end) fetch(tile + 1);
+    if (tile + 1 < t_end) {
+      cur = advance(c);
+      fetch(cur);
+    }
     // (5) epilogue
     ok = tc::mbar_wait(mbar, phase & 1, a.err);
     phase++;
     tc::fence_after_sync();
-    const long long b = slab / O;
-    const int outer = (int)(slab - b * O);
-    const long long ob = (b * Cs * O + outer) * SN + pbase + t;
+    const long long ob = (c.b * Cs * O + c.outer) * SN + (long long)c.row0 * NL + c.n0 + t;
 #pragma unroll
     for (int gi = 0; gi < GPH; ++gi) {
       const int c0 = (2 * gi + half) * 16;
-      T *op = out + ob + (long long)c0 * cstride;
-      T *pp = pre_out ? pre_out + ob + (long long)c0 * cstride : nullptr;
-      const T *xq = x + ob + (long long)c0 * cstride;
       if (c0 < Cs) {
         uint32_t dv[16];
         tc::tmem_ld16(arow + c0, dv);
-        tc::tmem_wait_ld();
+        float v[16];
+        if (K::tf32) {
+          uint32_t dl[16];
+          tc::tmem_ld16(arow + e.NP + c0, dl);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; i += 2)
+            f2unpack(f2add(f2pack(__uint_as_float(dv[i]), __uint_as_float(dv[i + 1])),
+                           f2pack(__uint_as_float(dl[i]), __uint_as_float(dl[i + 1]))),
+                     v[i], v[i + 1]);
+        } else {
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(dv[i]);
+        }
+        const int nv = Cs - c0 < 16 ? Cs - c0 : 16;
+        T *op = out + ob + (long long)c0 * cstride;
+        if (MODE == EPI_BLOCK_FWD) {
+          if (pre_out) {
+            T *pp = pre_out + ob + (long long)c0 * cstride;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              if (i < nv) *pp = from_f<T>(v[i]);
+              pp += cstride;
+            }
+          }
+          if (a.act) {
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) gelu2(v[i], v[i + 1]);
+          }
+        } else if (MODE == EPI_SPEC_BWD && a.tanh_pre) {
+          const T *xq = x + ob + (long long)c0 * cstride;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            if (i < nv) {
+              const float th = tanhf(ldf<T>(xq));
+              v[i] *= 1.f - th * th;
+            }
+            xq += cstride;
+          }
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const int o = c0 + i;
-          if (o < Cs) {
-            float val = __uint_as_float(dv[i]);
-            if (MODE == EPI_BLOCK_FWD) {
-              val += bias_s[o];
-              if (pp) *pp = from_f<T>(val);
-              if (a.act) val = gelu_f(val);
-            } else if (MODE == EPI_SPEC_BWD && a.tanh_pre) {
-              const float th = tanhf(ldf<T>(xq));
-              val *= 1.f - th * th;
-            }
-            *op = from_f<T>(val);
-          }
+          if (i < nv) *op = from_f<T>(v[i]);
           op += cstride;
-          if (pp) pp += cstride;
-          xq += cstride;
         }
       }
     }
@@ -461,7 +514,7 @@ bool epi_tc_supported(const Geom &g, int dtype, int mode, int Ci, int Co) {
   if (SN % 128 != 0) return false;
   const bool tf32 = dtype == DT_F32;
   const EpiTcGeom e = epi_tc_geom(g, mode, Ci, Co, tf32 ? 4 : 2, tf32);
-  if (e.total_cols > TMEM_COLS) return false;
+  if (e.total_cols > TMEM_COLS || e.DC > 256) return false;
   if (e.Rt * ((mode == EPI_SPEC_BWD) ? Ci : Co) * g.mL > (UMAX / 2) * EPI_THREADS) return false;
   return e.total <= 227 * 1024;
 }

@@ -194,12 +194,14 @@ __global__ void __launch_bounds__(TC_THREADS)
       tc::tmem_ld16(arow + h0, dv);
       tc::tmem_wait_ld();
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float z = __uint_as_float(dv[i]) + q1s[h0 + i];
-        const float gz = gelu_f(z);
+      for (int i = 0; i < 16; i += 2) {
+        float z0 = __uint_as_float(dv[i]) + q1s[h0 + i];
+        float z1 = __uint_as_float(dv[i + 1]) + q1s[h0 + i + 1];
+        gelu2(z0, z1);
 #pragma unroll
         for (int o = 0; o < kMaxOut; ++o)
-          if (o < out_ch) acc[o] = fmaf(q2s[o * e.HP + h0 + i], gz, acc[o]);
+          if (o < out_ch)
+            acc[o] = fmaf(q2s[o * e.HP + h0 + i + 1], z1, fmaf(q2s[o * e.HP + h0 + i], z0, acc[o]));
       }
     }
     const long long b = cur / tpb;

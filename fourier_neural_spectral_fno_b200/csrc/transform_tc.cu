@@ -169,8 +169,12 @@ __global__ void __launch_bounds__(TC_THREADS) k_s1_tc(S1Args a) {
   tc::fence_after_sync();
   const uint32_t tbase = *tbase_s;
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  const uint32_t idesc = tc::instr_desc(K::fmt, 128, NP);
-  const uint32_t fhi_a = tc::smem_u32(fhi), flo_a = tc::smem_u32(flo);
+  // tf32: F rows [0, NP) hold the hi split and [NP, 2 NP) the lo split (contiguous),
+  // so A [F_hi; F_lo] is one MMA of width 2 NP; D keeps both halves
+  const int DC = K::tf32 ? 2 * NP : NP;
+  const uint32_t idesc = tc::instr_desc(K::fmt, 128, DC);
+  const uint32_t fhi_a = tc::smem_u32(fhi);
+  (void)flo;
 
   const T *in0 = reinterpret_cast<const T *>(a.in0);
   const T *in1 = reinterpret_cast<const T *>(a.in1);
@@ -258,9 +262,7 @@ __global__ void __launch_bounds__(TC_THREADS) k_s1_tc(S1Args a) {
           const uint64_t bh = tc::smem_desc_kmajor(fhi_a + gs * 256, 128, sbo);
           const uint32_t acc = (c | s) ? 1u : 0u;
           if (K::tf32) {
-            const uint64_t bl = tc::smem_desc_kmajor(flo_a + gs * 256, 128, sbo);
             tc::mma_tf32_ts(tbase, a0 + s * 8, bh, idesc, acc);
-            tc::mma_tf32_ts(tbase, a0 + s * 8, bl, idesc, 1u);
             tc::mma_tf32_ts(tbase, a0 + 32 + s * 8, bh, idesc, 1u);
           } else {
             tc::mma_f16_ts(tbase, a0 + s * 8, bh, idesc, acc);
@@ -280,7 +282,15 @@ __global__ void __launch_bounds__(TC_THREADS) k_s1_tc(S1Args a) {
     for (int c0 = 0; c0 < NP; c0 += 16) {
       uint32_t v[16];
       tc::tmem_ld16(tbase + lane_off + c0, v);
-      tc::tmem_wait_ld();
+      if (K::tf32) {
+        uint32_t vl[16];
+        tc::tmem_ld16(tbase + lane_off + NP + c0, vl);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(vl[i]));
+      } else {
+        tc::tmem_wait_ld();
+      }
 #pragma unroll
       for (int i = 0; i < 16; i += 4) {
         if (c0 + i < 2 * lay.mLp)
@@ -310,8 +320,28 @@ __global__ void __launch_bounds__(TC_THREADS) k_s1_tc(S1Args a) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
       const float *xr = x1s + (si * rows_per_slab) * lay.x1_ld + kg * 8;
-      int idx = (int)(((long long)ks * r_off) % S);
-      for (int r = 0; r < rows_per_slab; ++r) {
+      int idx = mulmod(ks, r_off % S, S);
+      int r = 0;
+      for (; r + 4 <= rows_per_slab; r += 4) {     // four rows per step: loads ahead of FMAs
+        float2 w[4];
+        float4 p0[4], p1[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          w[u] = twS[idx];
+          idx += ks;
+          if (idx >= S) idx -= S;
+          p0[u] = *reinterpret_cast<const float4 *>(xr + (r + u) * lay.x1_ld);
+          p1[u] = *reinterpret_cast<const float4 *>(xr + (r + u) * lay.x1_ld + 4);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          cfma_conj_b(acc[0], make_float2(p0[u].x, p0[u].y), w[u]);
+          cfma_conj_b(acc[1], make_float2(p0[u].z, p0[u].w), w[u]);
+          cfma_conj_b(acc[2], make_float2(p1[u].x, p1[u].y), w[u]);
+          cfma_conj_b(acc[3], make_float2(p1[u].z, p1[u].w), w[u]);
+        }
+      }
+      for (; r < rows_per_slab; ++r) {
         const float2 w = twS[idx];
         idx += ks;
         if (idx >= S) idx -= S;
@@ -361,7 +391,7 @@ bool s1_tc_supported(const Geom &g, int dtype) {
   if ((g.NL * eb) % 128 != 0) return false;
   if (!(g.S % 128 == 0 || 128 % g.S == 0)) return false;
   const int np = ((2 * g.mL + 15) / 16) * 16;
-  if (np > 128) return false;
+  if ((dtype == DT_F32 ? 2 * np : np) > 128) return false;   // D must fit below the A buffers
   const S1Layout l = s1_layout(g.S, g.NL, g.mL, np, eb, dtype == DT_F32);
   return l.total <= 227 * 1024;
 }
