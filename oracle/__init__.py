@@ -3,4 +3,5 @@ from .fno_oracle import *  # noqa: F401,F403
 from .fno_oracle import (axis_wavenumbers, kept_shape, num_modes, mode_weights,
                          truncated_dft, inverse_sum, gelu, gelu_grad,
                          spectral_conv_fwd, spectral_conv_bwd, block_fwd,
-                         block_bwd, forward, backward, mse, TANH_PREACT, NO_ACT)
+                         block_bwd, forward, backward, mse, lift, projection,
+                         TANH_PREACT, NO_ACT)

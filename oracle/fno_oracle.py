@@ -252,6 +252,20 @@ def block_bwd(x, r, w, pre, xhat, dy, modes, flags: int = 0):
 # network: lift -> L blocks -> projection ([MPFNO] "original FNO architecture")
 # --------------------------------------------------------------------------
 
+def lift(a, p_mat, p_vec):
+    """Lifting ``v_0 = P a + p`` (pointwise over the grid)."""
+    a = np.asarray(a, np.float64)
+    return _pointwise(p_mat, a) + _bcast(p_vec, a.ndim - 2)
+
+
+def projection(v, q1_mat, q1_vec, q2_mat, q2_vec):
+    """Projection ``u = Q2 GELU(Q1 v + q1) + q2`` (pointwise over the grid)."""
+    v = np.asarray(v, np.float64)
+    d = v.ndim - 2
+    h = _pointwise(q1_mat, v) + _bcast(q1_vec, d)
+    return _pointwise(q2_mat, gelu(h)) + _bcast(q2_vec, d)
+
+
 def forward(a, params, modes, flags: int = 0, save: bool = False):
     """``v_0 = P a + p``; ``v_{l+1} = block_l(v_l)``; ``u = Q2 GELU(Q1 v_L + q1) + q2``.
 
@@ -261,7 +275,7 @@ def forward(a, params, modes, flags: int = 0, save: bool = False):
     """
     a = np.asarray(a, np.float64)
     d = a.ndim - 2
-    v = _pointwise(params["P"], a) + _bcast(params["p"], d)
+    v = lift(a, params["P"], params["p"])
     xs, pres, xhats = [], [], []
     for r, w, bias in zip(params["R"], params["W"], params["b"]):
         xs.append(v)
@@ -269,7 +283,7 @@ def forward(a, params, modes, flags: int = 0, save: bool = False):
         pres.append(pre)
         xhats.append(xhat)
     h = _pointwise(params["Q1"], v) + _bcast(params["q1"], d)
-    u = _pointwise(params["Q2"], gelu(h)) + _bcast(params["q2"], d)
+    u = projection(v, params["Q1"], params["q1"], params["Q2"], params["q2"])
     if not save:
         return u
     return u, {"x": xs, "pre": pres, "xhat": xhats, "v_last": v, "h": h}
