@@ -44,8 +44,10 @@ EXPORTED = (
     "fno_net_workspace_size", "fno_net_saves_size", "fno_spectral_conv_fwd",
     "fno_spectral_conv_bwd", "fno_block_fwd", "fno_block_bwd", "fno_forward", "fno_backward",
     "fno_mse", "fno_profile_enable", "fno_profile_read", "fno_set_tensor_cores",
-    "fno_device_error",
+    "fno_device_error", "fno_spectral_conv_fwd_noalloc",
 )
+
+FNO_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class FnoError(RuntimeError):
@@ -121,6 +123,7 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "fno_mse": (i, [ctypes.c_int64, i, vp, vp, vp, vp, vp]),
         "fno_profile_enable": (i, [i]),
         "fno_set_tensor_cores": (i, [i]),
+        "fno_spectral_conv_fwd_noalloc": (i, [bd, vp, vp, vp, vp, vp]),
         "fno_device_error": (i, [i]),
         "fno_profile_read": (i, [ctypes.POINTER(KernelStat), i]),
     }
@@ -327,3 +330,10 @@ def fno_set_tensor_cores(enable: bool) -> bool:
 def fno_device_error(clear: bool = True) -> None:
     """Raise if a bounded device-side wait expired since the last clear."""
     _check(load().fno_device_error(1 if clear else 0))
+
+
+def fno_spectral_conv_fwd_noalloc(desc, x, R, y, xhat_save=None, stream=None):
+    """fno_spectral_conv_fwd with the library's built-in scratch (no workspace)."""
+    _check(load().fno_spectral_conv_fwd_noalloc(ctypes.byref(desc), _ptr(x), _ptr(R), _ptr(y),
+                                                _ptr(xhat_save), _stream(stream)))
+    return y

@@ -386,6 +386,13 @@ SavesMap saves_map(const fno_net_desc *d, const Geom &g) {
 
 namespace fno {
 
+void set_last_error(const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+}
+
 void launch_begin(const Launch &L) {
   if (!g_prof_on) return;
   std::lock_guard<std::mutex> lk(g_prof_mu);

@@ -39,6 +39,9 @@ struct Launch {
   int *err;         // device error word (bounded waits that expired)
 };
 
+// Set the thread-local message fno_last_error() returns.
+void set_last_error(const char *fmt, ...);
+
 // Bracket every kernel launch: launch_begin records a CUDA event on the launch
 // stream when per-kernel timing is on (fno_profile_enable); launch_end records
 // the closing event under `tag` and counts the launch.

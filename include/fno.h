@@ -195,6 +195,33 @@ int fno_spectral_conv_fwd(const fno_block_desc *desc, const void *x, const void 
                           void *y, float *xhat_save, void *ws, size_t ws_bytes,
                           fno_stream_t stream);
 
+/* Bytes of the scratch array built into the library for
+ * fno_spectral_conv_fwd_noalloc (per GPU that loads the library). */
+#define FNO_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* fno_spectral_conv_fwd for callers that cannot allocate device memory.
+ * The pages have no counterpart; this is a deployment convenience.  Some
+ * callers own no allocator at all: a plugin inside a host application that
+ * keeps every device byte in its own pool, or code that runs where a
+ * cudaMalloc would stall the stream or is simply not permitted.  Such a caller
+ * passes only inputs and outputs; the scratch lives in a fixed device array of
+ * FNO_NOALLOC_SCRATCH_BYTES compiled into the library, which every GPU that
+ * loads the library holds until the process exits.  This call allocates and
+ * frees nothing, on the host or the device.
+ *   - Problems whose fno_workspace_size(desc, FNO_OP_SPECTRAL_FWD) exceeds the
+ *     array are rejected with FNO_ERR_WORKSPACE and a message naming both sizes.
+ *   - The first call on each device looks up the array's device address (a
+ *     host-side lookup that requires that device to be current).  Make that first
+ *     call before any stream capture.
+ *   - All calls share the one array, which keeps whatever the last call left in
+ *     it; every scratch byte this operation reads it has first written, so
+ *     nothing needs clearing.  Calls whose work overlaps on the GPU (concurrent
+ *     streams, or several host threads on one device) race on the array:
+ *     serialise them.
+ * Arguments, layouts and results are those of fno_spectral_conv_fwd. */
+int fno_spectral_conv_fwd_noalloc(const fno_block_desc *desc, const void *x, const void *R,
+                                  void *y, float *xhat_save, fno_stream_t stream);
+
 /* Adjoint of fno_spectral_conv_fwd.  Inputs: x (needed for tanh'), xhat_save
  * from the forward (may be NULL: then it is recomputed from x), R, dy
  * [B][Co][grid].  Outputs: dx [B][Ci][grid] (storage dtype),
