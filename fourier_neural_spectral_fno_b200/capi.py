@@ -322,9 +322,14 @@ def fno_profile_read(max_kernels: int = 64) -> Dict[str, Dict[str, float]]:
             for i in range(n)}
 
 
-def fno_set_tensor_cores(enable: bool) -> bool:
-    """Use the tcgen05 kernels where shapes allow (True) or the CUDA-core ones."""
-    return bool(load().fno_set_tensor_cores(1 if enable else 0))
+def fno_set_tensor_cores(mode) -> int:
+    """Kernel selection: 1 / True = tcgen05 kernels with the TMA pipelines where
+    shapes allow, 2 = tcgen05 kernels without the pipelines, 0 / False = the
+    CUDA-core kernels.  Returns the previous setting."""
+    m = int(mode)
+    if m not in (0, 1, 2):
+        raise ValueError("tensor-core mode must be 0, 1 or 2")
+    return int(load().fno_set_tensor_cores(m))
 
 
 def fno_device_error(clear: bool = True) -> None:

@@ -1,0 +1,607 @@
+// Fused block epilogue (step S4, forward) as a warp-specialised, TMA-fed
+// tcgen05 pipeline.
+//
+// The arithmetic is the per-tile GEMM of the tensor-core epilogue: for a tile
+// of 128 consecutive grid points of one (sample, outer index) slab
+//     pre[p, o] = sum_j basis[p, j] U[o, j] + sum_i x[p, i] W[o, i] + b[o]
+// with basis = (cos, -sin)(2 pi k n / N_L) of the point's last-axis index n
+// and U the spectrum already inverted along the slab axis (k_inv_slab).  The
+// difference is the schedule: every role runs in its own warps and the tiles
+// stream through the SM, so HBM traffic, staging, MMAs and the GELU epilogue
+// of consecutive tiles overlap.
+//
+//   warp 13       TMA producer: x tile [Ci][128] and U rows [Co][Rt 2 mL] of
+//                 tile j into ring stage j % NS (mbarrier transaction count)
+//   warps 0-3     staging: U -> B operand (smem, K-major core matrices,
+//                 tf32 hi/lo split, bias folded into the k = 0 column), x ->
+//                 A operand (TMEM, one lane per point); double-buffered
+//   warp 12       one thread issues the MMAs of tile j into D buffer j % 2
+//   warps 4-11    epilogue: D -> registers, bias already in, optional pre
+//                 store, GELU, coalesced y stores; two warps per TMEM lane
+//                 quarter, each owning half of the channel groups
+//
+// Hand-offs (all mbarriers, every wait bounded):
+//   full[s]   TMA -> staging (transaction bytes)   empty[s]  staging -> TMA
+//   aready[i] staging -> MMA                       mdone[i]  MMA -> epilogue
+//   dempty[i] epilogue -> MMA                      (mdone also frees A/B)
+// A waiter never falls two phases behind its barrier: each barrier's next
+// phase needs an action that follows the wait in program order.
+#include <string.h>
+
+#include "fno_common.cuh"
+#include "fno_kernels.cuh"
+#include "tc_util.cuh"
+#include "tma_util.cuh"
+
+namespace fno {
+
+namespace {
+
+constexpr int ROWS = 128;                  // points per tile = TMEM lanes
+constexpr int NCONV = 4;                   // staging warps
+constexpr int NEPI = 8;                    // epilogue warps
+constexpr int WARP_MMA = NCONV + NEPI;     // 12
+constexpr int WARP_TMA = WARP_MMA + 1;     // 13
+constexpr int THREADS = (WARP_TMA + 1) * 32;
+constexpr int MAX_STAGES = 6;
+constexpr size_t kSmemMax = 227 * 1024;
+
+template <typename T> struct PKind {
+  static constexpr bool tf32 = false;
+  static constexpr int EB = 2;
+  static constexpr int KSTEP = 16;
+  static constexpr int fmt = tc::FMT_F16;
+  static constexpr CUtensorMapDataType tmap = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+};
+template <> struct PKind<float> {
+  static constexpr bool tf32 = true;
+  static constexpr int EB = 4;
+  static constexpr int KSTEP = 8;
+  static constexpr int fmt = tc::FMT_TF32;
+  static constexpr CUtensorMapDataType tmap = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+};
+template <> struct PKind<__nv_bfloat16> {
+  static constexpr bool tf32 = false;
+  static constexpr int EB = 2;
+  static constexpr int KSTEP = 16;
+  static constexpr int fmt = tc::FMT_BF16;
+  static constexpr CUtensorMapDataType tmap = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+};
+
+__host__ __device__ inline int rup(int v, int m) { return (v + m - 1) / m * m; }
+__host__ __device__ inline size_t alg(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Tile plan.  TMEM columns: two D buffers [0, 2 DC), the resident spectral A
+// block of every last-axis tile offset ("variant"), then NA x-blocks of A.
+// Shared memory: NS ring stages (x tile, U rows), NA B buffers (hi rows then
+// lo rows), the last-axis twiddles, the bias, mbarriers.
+struct PipeGeom {
+  int Rt, nvar, KS, KSp, KXp, KA, NP, DC, cs_cols, ax_cols;
+  int NA, NS;
+  int col_spec, col_x, used_cols, cols;
+  uint32_t sbo, x_bytes, u_bytes;
+  size_t uoff, stage, bhalf, bbuf, b, tw, bias, bar, tbase, total;
+};
+
+__host__ __device__ inline PipeGeom pipe_geom(const Geom &g, bool has_x, int Ci, int Co, int eb,
+                                              bool tf32) {
+  PipeGeom e;
+  e.Rt = g.NL >= ROWS ? 1 : ROWS / g.NL;
+  e.nvar = g.NL >= ROWS ? g.NL / ROWS : 1;
+  e.KS = e.Rt * 2 * g.mL;
+  e.KSp = rup(e.KS, 16);
+  e.KXp = has_x ? rup(Ci, 16) : 0;
+  e.KA = e.KSp + e.KXp;
+  e.NP = rup(Co, 16);
+  e.DC = tf32 ? 2 * e.NP : e.NP;
+  e.cs_cols = tf32 ? 2 * e.KSp : e.KSp / 2;
+  e.ax_cols = tf32 ? 2 * e.KXp : e.KXp / 2;
+  e.col_spec = 2 * e.DC;
+  e.col_x = e.col_spec + e.nvar * e.cs_cols;
+  e.NA = e.col_x + 2 * e.ax_cols <= 512 ? 2 : 1;
+  e.used_cols = e.col_x + e.NA * e.ax_cols;
+  e.cols = 32;
+  while (e.cols < e.used_cols && e.cols < 1024) e.cols *= 2;
+  e.sbo = (uint32_t)(e.KA * eb / 16) * 128u;
+  e.x_bytes = has_x ? (uint32_t)(Ci * ROWS * eb) : 0u;
+  e.u_bytes = (uint32_t)(Co * e.KS * 4);
+  e.uoff = alg(e.x_bytes, 128);
+  e.stage = alg(e.uoff + e.u_bytes, 1024);
+  e.bhalf = (size_t)e.NP * e.KA * eb;
+  e.bbuf = alg((tf32 ? 2 : 1) * e.bhalf, 1024);
+  const size_t fixed = e.NA * e.bbuf + alg(sizeof(float2) * g.NL, 128) + sizeof(float) * 64 +
+                       sizeof(uint64_t) * (2 * MAX_STAGES + 6) + 16;
+  const size_t room = kSmemMax > fixed ? kSmemMax - fixed : 0;
+  const size_t ns = room / e.stage;
+  e.NS = (int)(ns < (size_t)MAX_STAGES ? ns : (size_t)MAX_STAGES);
+  size_t off = 0;
+  off += (size_t)(e.NS > 0 ? e.NS : 0) * e.stage;
+  e.b = off; off += e.NA * e.bbuf;
+  e.tw = off; off = alg(off + sizeof(float2) * g.NL, 128);
+  e.bias = off; off += sizeof(float) * 64;
+  e.bar = off; off += sizeof(uint64_t) * (2 * MAX_STAGES + 6);
+  e.tbase = off; off += 16;
+  // one CTA per SM: the TMEM allocation may take all 512 columns
+  e.total = off < 116 * 1024 ? 116 * 1024 : off;
+  return e;
+}
+
+// byte offset of element (n, k) in a K-major no-swizzle B operand
+__host__ __device__ __forceinline__ uint32_t boff(int n, int k, int eb, uint32_t sbo) {
+  const int kb = k * eb;
+  return (uint32_t)(n >> 3) * sbo + (kb >> 4) * 128 + (n & 7) * 16 + (kb & 15);
+}
+
+template <typename T>
+__device__ __forceinline__ void bstore1(unsigned char *bh, size_t bhalf, uint32_t o, float v) {
+  if (PKind<T>::tf32) {
+    uint32_t hi, lo;
+    tc::split_tf32(v, hi, lo);
+    *reinterpret_cast<uint32_t *>(bh + o) = hi;
+    *reinterpret_cast<uint32_t *>(bh + bhalf + o) = lo;
+  } else {
+    *reinterpret_cast<T *>(bh + o) = from_f<T>(v);
+  }
+}
+
+// four K-consecutive elements (k multiple of 4) in one store per half
+template <typename T>
+__device__ __forceinline__ void bstore4(unsigned char *bh, size_t bhalf, uint32_t o, float4 v) {
+  if (PKind<T>::tf32) {
+    uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+    tc::split_tf32(v.x, h0, l0);
+    tc::split_tf32(v.y, h1, l1);
+    tc::split_tf32(v.z, h2, l2);
+    tc::split_tf32(v.w, h3, l3);
+    *reinterpret_cast<uint4 *>(bh + o) = make_uint4(h0, h1, h2, h3);
+    *reinterpret_cast<uint4 *>(bh + bhalf + o) = make_uint4(l0, l1, l2, l3);
+  } else if (PKind<T>::fmt == tc::FMT_BF16) {
+    *reinterpret_cast<uint2 *>(bh + o) = make_uint2(tc::pack_bf16(v.x, v.y), tc::pack_bf16(v.z, v.w));
+  } else {
+    *reinterpret_cast<uint2 *>(bh + o) = make_uint2(tc::pack_f16(v.x, v.y), tc::pack_f16(v.z, v.w));
+  }
+}
+
+// 16 A elements of this thread's lane into TMEM (tf32: hi at col, lo at col + lo_off)
+template <typename T>
+__device__ __forceinline__ void stage16(uint32_t col, uint32_t lo_off, const float (&v)[16]) {
+  if (PKind<T>::tf32) {
+    uint32_t hi[16], lo[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) tc::split_tf32(v[i], hi[i], lo[i]);
+    tc::tmem_st16(col, hi);
+    tc::tmem_st16(col + lo_off, lo);
+  } else {
+    uint32_t pk[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      pk[i] = PKind<T>::fmt == tc::FMT_BF16 ? tc::pack_bf16(v[2 * i], v[2 * i + 1])
+                                             : tc::pack_f16(v[2 * i], v[2 * i + 1]);
+    tc::tmem_st8(col, pk);
+  }
+}
+
+struct PipeArgs {
+  const void *W, *bias;
+  void *out, *pre_out;
+  int *err;
+  int Ci, Co, act;
+};
+
+// tile cursor (tiles of a CTA are consecutive)
+struct Cursor {
+  long long b;
+  int outer, row0, n0;
+};
+
+__device__ __forceinline__ Cursor cursor_at(long long tile, int tps, const Geom &g) {
+  Cursor c{0, 0, 0, 0};
+  const long long slab = tile / tps;
+  const int pb = (int)(tile - slab * tps) * ROWS;
+  c.b = slab / g.O;
+  c.outer = (int)(slab - c.b * g.O);
+  c.row0 = pb / g.NL;
+  c.n0 = pb - c.row0 * g.NL;
+  return c;
+}
+
+__device__ __forceinline__ void cursor_next(Cursor &c, int Rt, const Geom &g) {
+  if (g.NL >= ROWS) {
+    c.n0 += ROWS;
+    if (c.n0 == g.NL) {
+      c.n0 = 0;
+      ++c.row0;
+    }
+  } else {
+    c.row0 += Rt;
+  }
+  if (c.row0 == g.S) {
+    c.row0 = 0;
+    if (++c.outer == g.O) {
+      c.outer = 0;
+      ++c.b;
+    }
+  }
+}
+
+template <typename T, bool HAS_X, int CX>
+__global__ void __launch_bounds__(THREADS, 1)
+    k_epi_pipe(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmu,
+               PipeArgs a, Geom g) {
+  using K = PKind<T>;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const int Ci = a.Ci, Co = a.Co;
+  const PipeGeom e = pipe_geom(g, HAS_X, Ci, Co, K::EB, K::tf32);
+  unsigned char *bbase = smem + e.b;
+  float2 *twL = reinterpret_cast<float2 *>(smem + e.tw);
+  float *bias_s = reinterpret_cast<float *>(smem + e.bias);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + e.bar);
+  uint64_t *empty = full + MAX_STAGES;
+  uint64_t *aready = empty + MAX_STAGES;
+  uint64_t *mdone = aready + 2;
+  uint64_t *dempty = mdone + 2;
+  uint32_t *tbase_s = reinterpret_cast<uint32_t *>(smem + e.tbase);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int NL = g.NL, mL = g.mL;
+  const long long SN = (long long)g.S * NL;
+
+  if (warp == 0) {
+    tc::tmem_alloc(tbase_s, e.cols);
+    tc::tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int s = 0; s < MAX_STAGES; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], NCONV);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&aready[i], NCONV);
+      tc::mbar_init(&mdone[i], 1);
+      tc::mbar_init(&dempty[i], NEPI);
+    }
+    tma::fence_barrier_init();
+  }
+  if (warp == WARP_TMA && lane == 0) {
+    if (HAS_X) tma::prefetch_map(&tmx);
+    tma::prefetch_map(&tmu);
+  }
+  build_twiddles(twL, NL);
+  for (size_t i = (size_t)tid * 16; i < e.NA * e.bbuf; i += THREADS * 16)
+    *reinterpret_cast<uint4 *>(bbase + i) = make_uint4(0, 0, 0, 0);
+  __syncthreads();
+  if (HAS_X) {  // W in columns [KSp, KSp + Ci) of every B buffer; bias
+    const T *W = reinterpret_cast<const T *>(a.W);
+    for (int i = tid; i < Co * Ci; i += THREADS) {
+      const int o = i / Ci, c = i - o * Ci;
+      const float w = to_f<T>(W[i]);
+      const uint32_t off = boff(o, e.KSp + c, K::EB, e.sbo);
+      for (int nb = 0; nb < e.NA; ++nb) bstore1<T>(bbase + nb * e.bbuf, e.bhalf, off, w);
+    }
+  }
+  {
+    const T *bias = reinterpret_cast<const T *>(a.bias);
+    for (int o = tid; o < 64; o += THREADS)
+      bias_s[o] = (HAS_X && bias && o < Co) ? to_f<T>(bias[o]) : 0.f;
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = *tbase_s;
+
+  const int tps = (int)(SN / ROWS);              // tiles per slab
+  const long long ntiles = g.B * g.O * tps;
+  const long long per_cta = (ntiles + gridDim.x - 1) / gridDim.x;
+  const long long t_begin = blockIdx.x * per_cta;
+  const long long t_end = t_begin + per_cta < ntiles ? t_begin + per_cta : ntiles;
+  const int ntl = t_begin < t_end ? (int)(t_end - t_begin) : 0;
+
+  if (warp == WARP_TMA) {
+    // ---------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      Cursor c = cursor_at(t_begin, tps, g);
+      int j = 0;
+      for (; j < ntl; ++j) {
+        const int s = j % e.NS;
+        if (j >= e.NS && !tc::mbar_wait(&empty[s], ((j / e.NS) - 1) & 1, a.err)) break;
+        tma::arrive_expect_tx(&full[s], e.x_bytes + e.u_bytes);
+        unsigned char *st = smem + (size_t)s * e.stage;
+        if (HAS_X)
+          tma::load_4d(st, &tmx, &full[s], c.row0 * NL + c.n0, c.outer, 0, (int)c.b);
+        tma::load_4d(st + e.uoff, &tmu, &full[s], c.row0 * 2 * mL, c.outer, 0, (int)c.b);
+        cursor_next(c, e.Rt, g);
+      }
+      // every issued load lands before the CTA may exit
+      for (int jj = j - 1; jj >= 0 && jj >= j - e.NS; --jj)
+        tc::mbar_wait(&full[jj % e.NS], (jj / e.NS) & 1, nullptr);
+    }
+  } else if (warp == WARP_MMA) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      Cursor c = cursor_at(t_begin, tps, g);
+      const uint32_t idesc = tc::instr_desc(K::fmt, ROWS, e.DC);
+      const uint32_t lo_spec = K::tf32 ? (uint32_t)e.KSp : 0u;
+      const uint32_t lo_x = K::tf32 ? (uint32_t)e.KXp : 0u;
+      const int ns = e.KSp / K::KSTEP, nx = e.KXp / K::KSTEP;
+      int j = 0;
+      for (; j < ntl; ++j) {
+        bool ok = tc::mbar_wait(&aready[j & 1], (j >> 1) & 1, a.err);
+        if (ok && j >= 2) ok = tc::mbar_wait(&dempty[j & 1], ((j - 2) >> 1) & 1, a.err);
+        if (!ok) break;
+        tc::fence_after_sync();
+        const int variant = e.Rt > 1 ? 0 : c.n0 / ROWS;
+        const int ab = e.NA == 2 ? (j & 1) : 0;
+        const uint32_t d = tbase + (uint32_t)((j & 1) * e.DC);
+        const uint32_t aspec = tbase + e.col_spec + variant * e.cs_cols;
+        const uint32_t ax = tbase + e.col_x + ab * e.ax_cols;
+        const uint32_t b_a = tc::smem_u32(bbase + ab * e.bbuf);
+        for (int s = 0; s < ns + nx; ++s) {
+          const uint64_t bd = tc::smem_desc_kmajor(b_a + s * 256, 128, e.sbo);
+          const uint32_t acol = s < ns ? aspec + s * 8 : ax + (s - ns) * 8;
+          if (K::tf32) {
+            tc::mma_tf32_ts(d, acol, bd, idesc, s > 0 ? 1u : 0u);
+            tc::mma_tf32_ts(d, acol + (s < ns ? lo_spec : lo_x), bd, idesc, 1u);
+          } else {
+            tc::mma_f16_ts(d, acol, bd, idesc, s > 0 ? 1u : 0u);
+          }
+        }
+        tc::mma_commit(&mdone[j & 1]);
+        cursor_next(c, e.Rt, g);
+      }
+      // no MMA may still run when TMEM is freed
+      if (j > 0) tc::mbar_wait(&mdone[(j - 1) & 1], ((j - 1) >> 1) & 1, nullptr);
+    }
+  } else if (warp < NCONV) {
+    // ---------------------------------------------------------- staging
+    const int t = tid;                                  // point / TMEM lane
+    const uint32_t arow = tbase + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lo_spec = K::tf32 ? (uint32_t)e.KSp : 0u;
+    const uint32_t lo_x = K::tf32 ? (uint32_t)e.KXp : 0u;
+    // resident spectral A block per variant: row t = point n0 + t (NL >= 128)
+    // or point t of the Rt rows (NL < 128): (cos, -sin)(2 pi k n / NL) in the
+    // slot of the point's row, zeros elsewhere
+    for (int v = 0; v < e.nvar; ++v) {
+      const int n = e.Rt > 1 ? t % NL : v * ROWS + t;
+      const int rl = e.Rt > 1 ? t / NL : 0;
+      const uint32_t c0v = arow + e.col_spec + v * e.cs_cols;
+      int r = 0, k = 0, par = 0, idx = 0;
+      for (int c0 = 0; c0 < e.KSp; c0 += 16) {
+        float vals[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float val = 0.f;
+          if (c0 + i < e.KS) {
+            if (r == rl) {
+              const float2 w = twL[idx];
+              val = par ? -w.y : w.x;
+            }
+            if (par) {
+              ++k;
+              idx += n;
+              if (idx >= NL) idx -= NL;
+              if (k == mL) {
+                k = 0;
+                ++r;
+                idx = 0;
+              }
+            }
+            par ^= 1;
+          }
+          vals[i] = val;
+        }
+        stage16<T>(c0v + (K::tf32 ? c0 : c0 / 2), lo_spec, vals);
+      }
+    }
+    const int njb = e.KS / 4;                           // 16-byte chunks per U row
+    const int nchunk = rup(Co, 8) * njb;
+    const int two_ml = 2 * mL;
+    for (int j = 0; j < ntl; ++j) {
+      const int s = j % e.NS;
+      const int ab = e.NA == 2 ? (j & 1) : 0;
+      bool ok = tc::mbar_wait(&full[s], (j / e.NS) & 1, a.err);
+      if (ok && j >= e.NA)
+        ok = tc::mbar_wait(&mdone[(j - e.NA) & 1], ((j - e.NA) >> 1) & 1, a.err);
+      if (!ok) break;
+      tc::fence_after_sync();
+      const unsigned char *st = smem + (size_t)s * e.stage;
+      // B spectral block: U rows -> K-major core matrices.  Chunk order walks
+      // 8-row groups diagonally so a quarter warp touches 8 distinct 16-byte
+      // bank groups on both the read and the write side.
+      {
+        const float *us = reinterpret_cast<const float *>(st + e.uoff);
+        unsigned char *bh = bbase + ab * e.bbuf;
+        for (int i = t; i < nchunk; i += ROWS) {
+          const int o8 = i / (8 * njb), rem = i - o8 * 8 * njb;
+          const int ol = rem & 7, jrot = rem >> 3;
+          const int jb = (jrot + ol) % njb;
+          const int o = o8 * 8 + ol;
+          if (o < Co) {
+            float4 v = *reinterpret_cast<const float4 *>(us + o * e.KS + 4 * jb);
+            if (HAS_X && (4 * jb) % two_ml == 0) v.x += bias_s[o];
+            bstore4<T>(bh, e.bhalf, boff(o, 4 * jb, K::EB, e.sbo), v);
+          }
+        }
+      }
+      if (HAS_X) {
+        const T *xs = reinterpret_cast<const T *>(st);
+        const uint32_t xc = arow + e.col_x + ab * e.ax_cols;
+#pragma unroll
+        for (int c0 = 0; c0 < CX; c0 += 16) {
+          if (c0 < e.KXp) {
+            float vals[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              vals[i] = c0 + i < Ci ? to_f<T>(xs[(c0 + i) * ROWS + t]) : 0.f;
+            stage16<T>(xc + (K::tf32 ? c0 : c0 / 2), lo_x, vals);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) tma::arrive(&empty[s]);            // the stage may be refilled
+      tc::tmem_wait_st();
+      tc::fence_proxy_async_smem();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tma::arrive(&aready[j & 1]);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue
+    const int q = warp & 3, half = (warp - NCONV) >> 2;
+    const int t = q * 32 + lane;
+    const uint32_t arow = tbase + ((uint32_t)(q * 32) << 16);
+    const long long cstride = (long long)g.O * SN;
+    T *out = reinterpret_cast<T *>(a.out);
+    T *pre_out = reinterpret_cast<T *>(a.pre_out);
+    constexpr int GPH = CX / 32 > 0 ? CX / 32 : 1;     // channel groups (of 16) per half
+    Cursor c = cursor_at(t_begin, tps, g);
+    for (int j = 0; j < ntl; ++j) {
+      if (!tc::mbar_wait(&mdone[j & 1], (j >> 1) & 1, a.err)) break;
+      tc::fence_after_sync();
+      const uint32_t dcol = arow + (uint32_t)((j & 1) * e.DC);
+      float v[GPH][16];
+#pragma unroll
+      for (int gi = 0; gi < GPH; ++gi) {
+        const int c0 = (2 * gi + half) * 16;
+        if (c0 < Co) {
+          uint32_t dv[16];
+          tc::tmem_ld16(dcol + c0, dv);
+          if (K::tf32) {
+            uint32_t dl[16];
+            tc::tmem_ld16(dcol + e.NP + c0, dl);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; i += 2)
+              f2unpack(f2add(f2pack(__uint_as_float(dv[i]), __uint_as_float(dv[i + 1])),
+                             f2pack(__uint_as_float(dl[i]), __uint_as_float(dl[i + 1]))),
+                       v[gi][i], v[gi][i + 1]);
+          } else {
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[gi][i] = __uint_as_float(dv[i]);
+          }
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tma::arrive(&dempty[j & 1]);       // D buffer may be overwritten
+      const long long ob =
+          (c.b * Co * g.O + c.outer) * SN + (long long)c.row0 * NL + c.n0 + t;
+#pragma unroll
+      for (int gi = 0; gi < GPH; ++gi) {
+        const int c0 = (2 * gi + half) * 16;
+        if (c0 < Co) {
+          const int nv = Co - c0 < 16 ? Co - c0 : 16;
+          if (HAS_X && pre_out) {
+            T *pp = pre_out + ob + (long long)c0 * cstride;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              if (i < nv) *pp = from_f<T>(v[gi][i]);
+              pp += cstride;
+            }
+          }
+          if (HAS_X && a.act) {
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) gelu2(v[gi][i], v[gi][i + 1]);
+          }
+          T *op = out + ob + (long long)c0 * cstride;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            if (i < nv) *op = from_f<T>(v[gi][i]);
+            op += cstride;
+          }
+        }
+      }
+      cursor_next(c, e.Rt, g);
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tbase, e.cols);
+  }
+}
+
+template <typename T, bool HAS_X>
+cudaError_t launch_pipe_t(const Launch &L, const Geom &g, const PipeArgs &a, const void *x,
+                          const float2 *U) {
+  using K = PKind<T>;
+  const PipeGeom e = pipe_geom(g, HAS_X, a.Ci, a.Co, K::EB, K::tf32);
+  const long long SN = (long long)g.S * g.NL;
+  CUtensorMap tmx, tmu;
+  memset(&tmx, 0, sizeof(tmx));
+  if (HAS_X) {
+    const uint64_t dims[4] = {(uint64_t)SN, (uint64_t)g.O, (uint64_t)a.Ci, (uint64_t)g.B};
+    const uint64_t str[3] = {(uint64_t)SN * K::EB, (uint64_t)g.O * SN * K::EB,
+                             (uint64_t)a.Ci * g.O * SN * K::EB};
+    const uint32_t box[4] = {(uint32_t)ROWS, 1u, (uint32_t)a.Ci, 1u};
+    if (!encode_tmap_4d(&tmx, K::tmap, x, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t row = (uint64_t)g.S * 2 * g.mL;   // floats of one (b, o, outer) slab
+    const uint64_t dims[4] = {row, (uint64_t)g.O, (uint64_t)a.Co, (uint64_t)g.B};
+    const uint64_t str[3] = {row * 4, (uint64_t)g.O * row * 4, (uint64_t)a.Co * g.O * row * 4};
+    const uint32_t box[4] = {(uint32_t)e.KS, 1u, (uint32_t)a.Co, 1u};
+    if (!encode_tmap_4d(&tmu, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, U, dims, str, box))
+      return cudaErrorInvalidValue;
+  }
+  const long long ntiles = g.B * g.O * (SN / ROWS);
+  const int grid = (int)(ntiles < L.num_sms ? ntiles : L.num_sms);
+  auto go = [&](auto kern) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)e.total);
+    kern<<<grid, THREADS, e.total, L.stream>>>(tmx, tmu, a, g);
+  };
+  const int cmax = a.Co > a.Ci ? a.Co : a.Ci;
+  if (cmax <= 16) go(k_epi_pipe<T, HAS_X, 16>);
+  else if (cmax <= 32) go(k_epi_pipe<T, HAS_X, 32>);
+  else go(k_epi_pipe<T, HAS_X, 64>);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool epi_pipe_supported(const Geom &g, int dtype, int mode, int Ci, int Co, const void *x,
+                        const void *U) {
+  if (mode != EPI_SPEC && mode != EPI_BLOCK_FWD) return false;
+  const bool has_x = mode == EPI_BLOCK_FWD;
+  if (!(g.NL % ROWS == 0 || ROWS % g.NL == 0)) return false;
+  const long long SN = (long long)g.S * g.NL;
+  if (SN % ROWS != 0 || SN > (1LL << 30) || g.B > (1LL << 30)) return false;
+  // U rows through TMA: 16-byte aligned row starts and box widths
+  if (g.mL % 2 != 0) return false;
+  if ((reinterpret_cast<uintptr_t>(U) & 15) != 0) return false;
+  if (has_x && (reinterpret_cast<uintptr_t>(x) & 15) != 0) return false;
+  const bool tf32 = dtype == DT_F32;
+  const PipeGeom e = pipe_geom(g, has_x, Ci, Co, tf32 ? 4 : 2, tf32);
+  if (e.KS > 256 || e.DC > 256 || e.used_cols > 512) return false;
+  if (e.NS < 2 || e.total > kSmemMax) return false;
+  return true;
+}
+
+cudaError_t launch_epi_pipe(const Launch &L, const Geom &g, int dtype, int mode,
+                            const EpiArgs &ea, const float2 *U) {
+  PipeArgs a{};
+  a.W = ea.W;
+  a.bias = ea.bias;
+  a.out = ea.out;
+  a.pre_out = ea.pre_out;
+  a.err = L.err;
+  a.Ci = ea.Ci;
+  a.Co = ea.Co;
+  a.act = ea.act;
+  const bool has_x = mode == EPI_BLOCK_FWD;
+  launch_begin(L);
+  cudaError_t err;
+  if (dtype == DT_F32)
+    err = has_x ? launch_pipe_t<float, true>(L, g, a, ea.x, U)
+                : launch_pipe_t<float, false>(L, g, a, ea.x, U);
+  else if (dtype == DT_F16)
+    err = has_x ? launch_pipe_t<__half, true>(L, g, a, ea.x, U)
+                : launch_pipe_t<__half, false>(L, g, a, ea.x, U);
+  else
+    err = has_x ? launch_pipe_t<__nv_bfloat16, true>(L, g, a, ea.x, U)
+                : launch_pipe_t<__nv_bfloat16, false>(L, g, a, ea.x, U);
+  launch_end(L, has_x ? "epi_block_fwd_pipe" : "epi_spec_pipe");
+  return err;
+}
+
+}  // namespace fno

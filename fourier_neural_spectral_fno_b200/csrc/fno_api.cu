@@ -203,9 +203,14 @@ Launch make_launch(fno_stream_t s) {
 
 cudaError_t run_epilogue(const Launch &L, const Geom &g, int dtype, int mode, const EpiArgs &a,
                          unsigned char *ws, const BlockWs &w) {
+  float2 *U = reinterpret_cast<float2 *>(ws + w.u);
+  const int cs = mode == EPI_SPEC_BWD ? a.Ci : a.Co;
+  if (L.tc == 1 && epi_pipe_supported(g, dtype, mode, a.Ci, a.Co, a.x, U)) {
+    cudaError_t e = launch_inv_slab(L, g, cs, a.Z, U);
+    if (e != cudaSuccess) return e;
+    return launch_epi_pipe(L, g, dtype, mode, a, U);
+  }
   if (L.tc && epi_tc_supported(g, dtype, mode, a.Ci, a.Co)) {
-    float2 *U = reinterpret_cast<float2 *>(ws + w.u);
-    const int cs = mode == EPI_SPEC_BWD ? a.Ci : a.Co;
     cudaError_t e = launch_inv_slab(L, g, cs, a.Z, U);
     if (e != cudaSuccess) return e;
     return launch_epilogue_tc(L, g, dtype, mode, a, U);
@@ -433,7 +438,7 @@ int fno_last_launch_count(void) { return g_launches; }
 
 int fno_set_tensor_cores(int enable) {
   const int prev = g_use_tc;
-  g_use_tc = enable ? 1 : 0;
+  g_use_tc = enable == 2 ? 2 : enable ? 1 : 0;
   return prev;
 }
 

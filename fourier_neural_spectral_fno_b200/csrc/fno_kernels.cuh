@@ -35,7 +35,7 @@ struct Launch {
   cudaStream_t stream;
   int *count;       // incremented per kernel launch
   int num_sms;
-  int tc;           // use the tensor-core kernels where the shape allows
+  int tc;           // 1: tensor-core kernels + TMA pipelines, 2: without pipelines, 0: none
   int *err;         // device error word (bounded waits that expired)
 };
 
@@ -103,6 +103,12 @@ cudaError_t launch_inv_slab(const Launch &L, const Geom &g, long long C, const f
 struct EpiArgs;
 cudaError_t launch_epilogue_tc(const Launch &L, const Geom &g, int dtype, int mode,
                                const EpiArgs &a, const float2 *U);
+// warp-specialised TMA pipeline for the forward epilogue modes (EPI_SPEC,
+// EPI_BLOCK_FWD); same inputs as launch_epilogue_tc
+bool epi_pipe_supported(const Geom &g, int dtype, int mode, int Ci, int Co, const void *x,
+                        const void *U);
+cudaError_t launch_epi_pipe(const Launch &L, const Geom &g, int dtype, int mode,
+                            const EpiArgs &a, const float2 *U);
 size_t epi_partial_bytes(const Geom &g, int Ci, int Co, int num_sms);
 cudaError_t launch_epilogue(const Launch &L, const Geom &g, int dtype, int mode,
                             const EpiArgs &a);

@@ -152,9 +152,10 @@ const char *fno_version(void);
 int fno_last_launch_count(void);
 
 /* Kernel selection: 1 (default) uses the tcgen05 tensor-core kernels wherever
- * the shape allows them, 0 forces the CUDA-core kernels everywhere (both are
- * complete implementations; the switch exists to compare them).  Process-wide;
- * returns the previous setting. */
+ * the shape allows them, including the warp-specialised TMA pipelines; 2 uses
+ * the tensor-core kernels without the TMA pipelines; 0 forces the CUDA-core
+ * kernels everywhere.  All are complete implementations; the switch exists to
+ * compare them.  Process-wide; returns the previous setting. */
 int fno_set_tensor_cores(int enable);
 
 /* Synchronises the current device and reads the library's device error word,

@@ -35,10 +35,11 @@ SHAPES = [
 ]
 
 
-@pytest.fixture(autouse=True, params=[True, False], ids=["tc", "cudacore"])
+@pytest.fixture(autouse=True, params=[1, 2, 0], ids=["tc", "tc_nopipe", "cudacore"])
 def kernel_path(request):
-    """Every parity test runs on the tcgen05 kernels (where the shape allows)
-    and on the CUDA-core kernels; no bounded device wait may expire."""
+    """Every parity test runs on the tcgen05 kernels with the TMA pipelines,
+    on the tcgen05 kernels without them (where the shape allows either) and on
+    the CUDA-core kernels; no bounded device wait may expire."""
     capi.fno_set_tensor_cores(request.param)
     yield request.param
     capi.fno_device_error(clear=True)
