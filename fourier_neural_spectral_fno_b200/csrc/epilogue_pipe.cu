@@ -297,17 +297,22 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp == WARP_TMA) {
     // ---------------------------------------------------------- TMA producer
-    if (lane == 0) {
+    // (the whole warp walks the loop and waits; lane 0 issues)
+    {
       Cursor c = cursor_at(t_begin, tps, g);
       int j = 0;
       for (; j < ntl; ++j) {
         const int s = j % e.NS;
-        if (j >= e.NS && !tc::mbar_wait(&empty[s], ((j / e.NS) - 1) & 1, a.err)) break;
-        tma::arrive_expect_tx(&full[s], e.x_bytes + e.u_bytes);
-        unsigned char *st = smem + (size_t)s * e.stage;
-        if (HAS_X)
-          tma::load_4d(st, &tmx, &full[s], c.row0 * NL + c.n0, c.outer, 0, (int)c.b);
-        tma::load_4d(st + e.uoff, &tmu, &full[s], c.row0 * 2 * mL, c.outer, 0, (int)c.b);
+        const bool ok = j < e.NS || tc::mbar_wait(&empty[s], ((j / e.NS) - 1) & 1, a.err);
+        if (!__all_sync(0xffffffffu, ok)) break;     // warp-uniform exit
+        if (lane == 0) {
+          tma::arrive_expect_tx(&full[s], e.x_bytes + e.u_bytes);
+          unsigned char *st = smem + (size_t)s * e.stage;
+          if (HAS_X)
+            tma::load_4d(st, &tmx, &full[s], c.row0 * NL + c.n0, c.outer, 0, (int)c.b);
+          tma::load_4d(st + e.uoff, &tmu, &full[s], c.row0 * 2 * mL, c.outer, 0, (int)c.b);
+        }
+        __syncwarp();
         cursor_next(c, e.Rt, g);
       }
       // every issued load lands before the CTA may exit
@@ -316,35 +321,50 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp == WARP_MMA) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // (the whole warp walks the loop and waits; lane 0 issues)
+    {
       Cursor c = cursor_at(t_begin, tps, g);
       const uint32_t idesc = tc::instr_desc(K::fmt, ROWS, e.DC);
       const uint32_t lo_spec = K::tf32 ? (uint32_t)e.KSp : 0u;
       const uint32_t lo_x = K::tf32 ? (uint32_t)e.KXp : 0u;
       const int ns = e.KSp / K::KSTEP, nx = e.KXp / K::KSTEP;
+      // B descriptors of both buffers; one K step advances the start address by
+      // 256 bytes (16 in descriptor units, no carry out of the 14-bit field)
+      const uint64_t bdesc0 = tc::smem_desc_kmajor(tc::smem_u32(bbase), 128, e.sbo);
+      const uint64_t bdesc1 =
+          tc::smem_desc_kmajor(tc::smem_u32(bbase + (e.NA - 1) * e.bbuf), 128, e.sbo);
       int j = 0;
       for (; j < ntl; ++j) {
         bool ok = tc::mbar_wait(&aready[j & 1], (j >> 1) & 1, a.err);
         if (ok && j >= 2) ok = tc::mbar_wait(&dempty[j & 1], ((j - 2) >> 1) & 1, a.err);
-        if (!ok) break;
+        if (!__all_sync(0xffffffffu, ok)) break;
         tc::fence_after_sync();
         const int variant = e.Rt > 1 ? 0 : c.n0 / ROWS;
         const int ab = e.NA == 2 ? (j & 1) : 0;
         const uint32_t d = tbase + (uint32_t)((j & 1) * e.DC);
-        const uint32_t aspec = tbase + e.col_spec + variant * e.cs_cols;
-        const uint32_t ax = tbase + e.col_x + ab * e.ax_cols;
-        const uint32_t b_a = tc::smem_u32(bbase + ab * e.bbuf);
-        for (int s = 0; s < ns + nx; ++s) {
-          const uint64_t bd = tc::smem_desc_kmajor(b_a + s * 256, 128, e.sbo);
-          const uint32_t acol = s < ns ? aspec + s * 8 : ax + (s - ns) * 8;
-          if (K::tf32) {
-            tc::mma_tf32_ts(d, acol, bd, idesc, s > 0 ? 1u : 0u);
-            tc::mma_tf32_ts(d, acol + (s < ns ? lo_spec : lo_x), bd, idesc, 1u);
-          } else {
-            tc::mma_f16_ts(d, acol, bd, idesc, s > 0 ? 1u : 0u);
+        // one thread issues; operands advance by constants (tf32: the A_hi and
+        // A_lo products of each K step, both against [B_hi; B_lo])
+        if (lane == 0) {
+          uint64_t bd = ab ? bdesc1 : bdesc0;
+          uint32_t acol = tbase + e.col_spec + variant * e.cs_cols;
+          uint32_t lo = lo_spec;
+          for (int s = 0; s < ns + nx; ++s) {
+            if (s == ns) {
+              acol = tbase + e.col_x + ab * e.ax_cols;
+              lo = lo_x;
+            }
+            if (K::tf32) {
+              tc::mma_tf32_ts(d, acol, bd, idesc, s > 0 ? 1u : 0u);
+              tc::mma_tf32_ts(d, acol + lo, bd, idesc, 1u);
+            } else {
+              tc::mma_f16_ts(d, acol, bd, idesc, s > 0 ? 1u : 0u);
+            }
+            acol += 8;
+            bd += 16;
           }
+          tc::mma_commit(&mdone[j & 1]);
         }
-        tc::mma_commit(&mdone[j & 1]);
+        __syncwarp();
         cursor_next(c, e.Rt, g);
       }
       // no MMA may still run when TMEM is freed
@@ -394,19 +414,57 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int njb = e.KS / 4;                           // 16-byte chunks per U row
     const int nchunk = rup(Co, 8) * njb;
     const int two_ml = 2 * mL;
+    // This thread's chunks of the B spectral block are the same for every
+    // tile: chunk i = t + 128 m.  Chunk order walks 8-row groups diagonally so a
+    // quarter warp touches 8 distinct 16-byte bank groups on both the read and
+    // the write side.  Packed per slot: source float index (low 16 bits), B byte
+    // offset (high 16 bits); bias_mask bit m: add the bias (k = 0 real column).
+    constexpr int MAXSLOT = 8;
+    uint32_t slot[MAXSLOT];
+    float slot_bias[MAXSLOT];
+    const bool slots_fit = nchunk <= MAXSLOT * ROWS && e.bhalf <= 65536;
+#pragma unroll
+    for (int m = 0; m < MAXSLOT; ++m) {
+      slot[m] = 0xffffffffu;
+      slot_bias[m] = 0.f;
+      const int i = t + ROWS * m;
+      if (slots_fit && i < nchunk) {
+        const int o8 = i / (8 * njb), rem = i - o8 * 8 * njb;
+        const int ol = rem & 7, jrot = rem >> 3;
+        const int jb = (jrot + ol) % njb;
+        const int o = o8 * 8 + ol;
+        if (o < Co) {
+          slot[m] = (uint32_t)(o * e.KS + 4 * jb) | (boff(o, 4 * jb, K::EB, e.sbo) << 16);
+          if (HAS_X && (4 * jb) % two_ml == 0) slot_bias[m] = bias_s[o];
+        }
+      }
+    }
     for (int j = 0; j < ntl; ++j) {
       const int s = j % e.NS;
       const int ab = e.NA == 2 ? (j & 1) : 0;
       bool ok = tc::mbar_wait(&full[s], (j / e.NS) & 1, a.err);
       if (ok && j >= e.NA)
         ok = tc::mbar_wait(&mdone[(j - e.NA) & 1], ((j - e.NA) >> 1) & 1, a.err);
-      if (!ok) break;
+      if (!__all_sync(0xffffffffu, ok)) break;      // warp-uniform exit
       tc::fence_after_sync();
       const unsigned char *st = smem + (size_t)s * e.stage;
-      // B spectral block: U rows -> K-major core matrices.  Chunk order walks
-      // 8-row groups diagonally so a quarter warp touches 8 distinct 16-byte
-      // bank groups on both the read and the write side.
-      {
+      // B spectral block: U rows -> K-major core matrices
+      if (slots_fit) {
+        const float *us = reinterpret_cast<const float *>(st + e.uoff);
+        unsigned char *bh = bbase + ab * e.bbuf;
+        float4 v[MAXSLOT];
+#pragma unroll
+        for (int m = 0; m < MAXSLOT; ++m)
+          if (slot[m] != 0xffffffffu)
+            v[m] = *reinterpret_cast<const float4 *>(us + (slot[m] & 0xffffu));
+#pragma unroll
+        for (int m = 0; m < MAXSLOT; ++m) {
+          if (slot[m] != 0xffffffffu) {
+            v[m].x += slot_bias[m];
+            bstore4<T>(bh, e.bhalf, slot[m] >> 16, v[m]);
+          }
+        }
+      } else {
         const float *us = reinterpret_cast<const float *>(st + e.uoff);
         unsigned char *bh = bbase + ab * e.bbuf;
         for (int i = t; i < nchunk; i += ROWS) {
@@ -454,7 +512,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     constexpr int GPH = CX / 32 > 0 ? CX / 32 : 1;     // channel groups (of 16) per half
     Cursor c = cursor_at(t_begin, tps, g);
     for (int j = 0; j < ntl; ++j) {
-      if (!tc::mbar_wait(&mdone[j & 1], (j >> 1) & 1, a.err)) break;
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&mdone[j & 1], (j >> 1) & 1, a.err))) break;
       tc::fence_after_sync();
       const uint32_t dcol = arow + (uint32_t)((j & 1) * e.DC);
       float v[GPH][16];
@@ -464,7 +522,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (c0 < Co) {
           uint32_t dv[16];
           tc::tmem_ld16(dcol + c0, dv);
-          if (K::tf32) {
+          if (K::tf32) {   // A [B_hi; B_lo]: add the two column halves
             uint32_t dl[16];
             tc::tmem_ld16(dcol + e.NP + c0, dl);
             tc::tmem_wait_ld();

@@ -254,7 +254,7 @@ __global__ void __launch_bounds__(EPI_THREADS) k_epi_tc(EpiTcArgs a, Geom g) {
   T *out = reinterpret_cast<T *>(a.out);
   T *pre_out = reinterpret_cast<T *>(a.pre_out);
   const uint32_t idesc = tc::instr_desc(K::fmt, 128, e.DC);
-  const uint32_t bhi_a = tc::smem_u32(bhi);
+  const uint64_t bdesc0 = tc::smem_desc_kmajor(tc::smem_u32(bhi), 128, e.sbo);
   const long long cstride = (long long)O * SN;     // channel stride of activations
   const int tps = (int)(SN / TC_THREADS);          // tiles per slab
   const long long ntiles = g.B * O * tps;
@@ -357,16 +357,30 @@ __global__ void __launch_bounds__(EPI_THREADS) k_epi_tc(EpiTcArgs a, Geom g) {
       const uint32_t aspec = tbase + e.DC + variant * e.cs_cols;
       const uint32_t ax = tbase + e.x_col;
       const int ns = e.KSp / K::KSTEP, nx = e.KXp / K::KSTEP;
-      for (int s = 0; s < ns + nx; ++s) {
-        const uint64_t bd = tc::smem_desc_kmajor(bhi_a + s * 256, 128, e.sbo);
-        const uint32_t acol = s < ns ? aspec + s * 8 : ax + (s - ns) * 8;
+      uint64_t bd = bdesc0;            // +256 bytes (16 units) per K step
+      uint32_t acol = aspec;
+#pragma unroll 4
+      for (int s = 0; s < ns; ++s) {
         if (K::tf32) {
-          const uint32_t alo = s < ns ? lo_spec : lo_x;
           tc::mma_tf32_ts(tbase, acol, bd, idesc, s > 0 ? 1u : 0u);
-          tc::mma_tf32_ts(tbase, acol + alo, bd, idesc, 1u);
+          tc::mma_tf32_ts(tbase, acol + lo_spec, bd, idesc, 1u);
         } else {
           tc::mma_f16_ts(tbase, acol, bd, idesc, s > 0 ? 1u : 0u);
         }
+        bd += 16;
+        acol += 8;
+      }
+      acol = ax;
+#pragma unroll 4
+      for (int s = 0; s < nx; ++s) {
+        if (K::tf32) {
+          tc::mma_tf32_ts(tbase, acol, bd, idesc, (ns + s) > 0 ? 1u : 0u);
+          tc::mma_tf32_ts(tbase, acol + lo_x, bd, idesc, 1u);
+        } else {
+          tc::mma_f16_ts(tbase, acol, bd, idesc, (ns + s) > 0 ? 1u : 0u);
+        }
+        bd += 16;
+        acol += 8;
       }
       tc::mma_commit(mbar);
     }

@@ -174,7 +174,7 @@ __device__ __forceinline__ f32x2 f2splat(float c) { return f2pack(c, c); }
 // x = |p| / (1.95 sqrt 2) - 1 is one fused multiply-add.
 __device__ __forceinline__ void gelu2(float &a, float &b) {
   const float ta = fminf(fabsf(a), 5.5154328f), tb = fminf(fabsf(b), 5.5154328f);
-  const f32x2 x = f2fma(f2pack(ta, tb), f2splat(0.36262512f), f2splat(-1.0f));
+  const f32x2 x = f2fma(f2pack(ta, tb), f2splat(0.36261886f), f2splat(-1.0f));
   f32x2 e = f2splat(0.0026791077f);
   e = f2fma(e, x, f2splat(-0.0049660155f));
   e = f2fma(e, x, f2splat(-0.013497429f));

@@ -119,7 +119,8 @@ __global__ void __launch_bounds__(TC_THREADS)
   const uint32_t tbase = *tbase_s;
   const uint32_t arow = tbase + ((uint32_t)(warp * 32) << 16);
   const uint32_t idesc = tc::instr_desc(K::fmt, 128, e.HP);
-  const uint32_t bhi_a = tc::smem_u32(bhi), blo_a = tc::smem_u32(blo);
+  const uint64_t bh0 = tc::smem_desc_kmajor(tc::smem_u32(bhi), 128, e.sbo);
+  const uint64_t bl0 = tc::smem_desc_kmajor(tc::smem_u32(blo), 128, e.sbo);
   float q2b[kMaxOut];
 #pragma unroll
   for (int o = 0; o < kMaxOut; ++o) q2b[o] = o < out_ch ? to_f<T>(q2[o]) : 0.f;
@@ -167,17 +168,20 @@ __global__ void __launch_bounds__(TC_THREADS)
     if (t == 0) {
       tc::fence_after_sync();
       const int ns = e.Cp / K::KSTEP;
+      uint64_t bh = bh0, bl = bl0;      // +256 bytes (16 units) per K step
+      uint32_t a0 = tbase + e.acol;
+#pragma unroll 4
       for (int s = 0; s < ns; ++s) {
-        const uint64_t bh = tc::smem_desc_kmajor(bhi_a + s * 256, 128, e.sbo);
-        const uint32_t a0 = tbase + e.acol + s * 8;
         if (K::tf32) {
-          const uint64_t bl = tc::smem_desc_kmajor(blo_a + s * 256, 128, e.sbo);
           tc::mma_tf32_ts(tbase, a0, bh, idesc, s > 0 ? 1u : 0u);
           tc::mma_tf32_ts(tbase, a0, bl, idesc, 1u);
           tc::mma_tf32_ts(tbase, a0 + e.Cp, bh, idesc, 1u);
         } else {
           tc::mma_f16_ts(tbase, a0, bh, idesc, s > 0 ? 1u : 0u);
         }
+        bh += 16;
+        bl += 16;
+        a0 += 8;
       }
       tc::mma_commit(mbar);
     }

@@ -162,10 +162,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *mbar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait: returns false (and sets *err) if the phase did not complete.
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or about `ns` nanoseconds pass, instead of re-polling the barrier
+// word (busy polling by many warps measurably slows the tensor pipe).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *mbar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(mbar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: returns false (and sets *err) if the phase did not complete
+// within about two seconds (2^17 suspensions of at most 16 us each, plus a
+// first unhinted probe so that completed phases return at once).
 __device__ __forceinline__ bool mbar_wait(uint64_t *mbar, uint32_t parity, int *err) {
-  for (int i = 0; i < (1 << 22); ++i)
-    if (mbar_try_wait(mbar, parity)) return true;
+  if (mbar_try_wait(mbar, parity)) return true;
+  for (int i = 0; i < (1 << 17); ++i)
+    if (mbar_try_wait_sleep(mbar, parity, 16384u)) return true;
   if (err) atomicExch(err, 1);
   return false;
 }

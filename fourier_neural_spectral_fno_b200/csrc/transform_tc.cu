@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(TC_THREADS) k_s1_tc(S1Args a) {
   // so A [F_hi; F_lo] is one MMA of width 2 NP; D keeps both halves
   const int DC = K::tf32 ? 2 * NP : NP;
   const uint32_t idesc = tc::instr_desc(K::fmt, 128, DC);
-  const uint32_t fhi_a = tc::smem_u32(fhi);
+  const uint64_t fdesc0 = tc::smem_desc_kmajor(tc::smem_u32(fhi), 128, sbo);
   (void)flo;
 
   const T *in0 = reinterpret_cast<const T *>(a.in0);
@@ -256,11 +256,13 @@ __global__ void __launch_bounds__(TC_THREADS) k_s1_tc(S1Args a) {
       if (t == 0) {
         tc::fence_after_sync();
         const uint32_t a0 = tbase + A_COL0 + buf * ACOLS;
+        // descriptors advance by constants (256 bytes = 16 units per K step)
+        const uint64_t bh0 = fdesc0 + (uint64_t)(c * 4 * 16);
+        const uint32_t acc0 = c ? 1u : 0u;
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
-          const uint32_t gs = (uint32_t)c * 4 + s;
-          const uint64_t bh = tc::smem_desc_kmajor(fhi_a + gs * 256, 128, sbo);
-          const uint32_t acc = (c | s) ? 1u : 0u;
+          const uint64_t bh = bh0 + (uint64_t)(s * 16);
+          const uint32_t acc = s ? 1u : acc0;
           if (K::tf32) {
             tc::mma_tf32_ts(tbase, a0 + s * 8, bh, idesc, acc);
             tc::mma_tf32_ts(tbase, a0 + 32 + s * 8, bh, idesc, 1u);

@@ -43,3 +43,15 @@ def test_gelu_from_polynomial_matches_exact_gelu():
     assert np.max(np.abs(gelu - exact)) < 3e-7
     big = np.abs(exact) > 0.1          # away from the cancelling negative tail
     assert np.max(np.abs(gelu - exact)[big] / np.abs(exact)[big]) < 2e-6
+
+
+def test_paired_gelu_matches_scalar_coefficients():
+    """The paired GELU (gelu2) evaluates the same polynomial as erf_pos: its
+    f2splat literals are the scalar coefficients, preceded by the variable
+    change x = |p| / (1.95 sqrt 2) - 1 (the scale to float32 rounding)."""
+    body = open(HDR).read().split("void gelu2(float &a, float &b)")[1].split("f2unpack(e")[0]
+    vals = [float(v) for v in re.findall(r"f2splat\((-?\d+\.\d+(?:e-?\d+)?)f\)", body)]
+    assert len(vals) == 2 + gen_erf_poly.DEGREE + 1
+    assert np.float32(vals[0]) == np.float32(1.0 / (1.95 * np.sqrt(2.0)))
+    assert vals[1] == -1.0
+    np.testing.assert_array_equal(np.float32(vals[2:]), np.float32(_compiled_coefficients()))
