@@ -63,6 +63,12 @@ int s1_tc_bands(const Geom &g);
 cudaError_t launch_s1_tc(const Launch &L, const Geom &g, int dtype, int load_mode, long long C,
                          const void *in0, const void *in1, float2 *zpart, int *err);
 
+// warp-specialised TMA pipeline for the forward transform (LOAD_PLAIN /
+// LOAD_TANH): writes the same per-band partial sums as launch_s1_tc
+bool fwd_pipe_supported(const Geom &g, int dtype, int load_mode, const void *in0);
+cudaError_t launch_fwd_pipe(const Launch &L, const Geom &g, int dtype, int load_mode,
+                            long long C, const void *in0, float2 *zpart);
+
 // ---- mixing (S3) -----------------------------------------------------------
 // yhat[b,o,k] = (c_k / N) sum_i xhat[b,i,k] R[i,o,k]
 cudaError_t launch_mix_fwd(const Launch &L, const Geom &g, int dtype, int Ci, int Co,

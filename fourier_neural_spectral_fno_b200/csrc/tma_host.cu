@@ -34,7 +34,7 @@ EncodeTiledFn encode_fn() {
 
 bool encode_tmap_4d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
                     const uint64_t dims[4], const uint64_t strides_bytes[3],
-                    const uint32_t box[4]) {
+                    const uint32_t box[4], bool swizzle128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) {
     set_last_error("cuTensorMapEncodeTiled is not available from the driver");
@@ -49,7 +49,8 @@ bool encode_tmap_4d(CUtensorMap *map, CUtensorMapDataType dtype, const void *bas
   }
   for (int i = 0; i < 3; ++i) gs[i] = strides_bytes[i];
   const CUresult r = fn(map, dtype, 4, const_cast<void *>(base), gd, gs, bx, es,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     set_last_error("cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);

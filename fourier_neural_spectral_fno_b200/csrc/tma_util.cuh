@@ -55,11 +55,12 @@ __device__ __forceinline__ void fence_barrier_init() {
 
 }  // namespace tma
 
-// Host: encode a 4-D tiled tensor map (no interleave, no swizzle, no OOB fill).
-// dims[0] is the contiguous axis; strides_bytes[i] is the byte stride of axis
-// i + 1.  Returns false (message set) if the driver refuses the map.
+// Host: encode a 4-D tiled tensor map (no interleave, no OOB fill; optional
+// 128-byte swizzle, whose box rows must then be exactly 128 bytes).  dims[0] is
+// the contiguous axis; strides_bytes[i] is the byte stride of axis i + 1.
+// Returns false (message set) if the driver refuses the map.
 bool encode_tmap_4d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
                     const uint64_t dims[4], const uint64_t strides_bytes[3],
-                    const uint32_t box[4]);
+                    const uint32_t box[4], bool swizzle128 = false);
 
 }  // namespace fno

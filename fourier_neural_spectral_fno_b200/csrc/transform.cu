@@ -263,7 +263,11 @@ cudaError_t launch_fwd_transform(const Launch &L, const Geom &g, int dtype, int 
   const long long planes = g.B * C * g.O;
   int nb;
   cudaError_t err;
-  if (L.tc && s1_tc_supported(g, dtype)) {
+  if (L.tc == 1 && fwd_pipe_supported(g, dtype, load_mode, in0)) {
+    nb = s1_tc_bands(g);
+    err = launch_fwd_pipe(L, g, dtype, load_mode, C, in0, zpart);
+    if (err != cudaSuccess) return err;
+  } else if (L.tc && s1_tc_supported(g, dtype)) {
     nb = s1_tc_bands(g);
     err = launch_s1_tc(L, g, dtype, load_mode, C, in0, in1, zpart, L.err);
     if (err != cudaSuccess) return err;

@@ -32,6 +32,13 @@ SHAPES = [
     ((8, 16, 64), (2, 4, 8)),
     ((128,), (30,)),
     ((384, 64), (40, 33)),
+    # shapes the pipelined forward transform takes (128-row bands, 128-byte
+    # column chunks, <= 16 last-axis and <= 32 slab-axis modes); 96-wide rows
+    # are whole chunks in float32 only
+    ((128, 64), (8, 8)),
+    ((256, 96), (16, 12)),
+    ((384, 128), (10, 16)),
+    ((4, 128, 64), (2, 8, 8)),
 ]
 
 
