@@ -139,6 +139,12 @@ cudaError_t launch_proj_fwd(const Launch &L, const Geom &g, int dtype, int width
                             int out_ch, const void *v, const void *Q1, const void *q1,
                             const void *Q2, const void *q2, void *u);
 bool proj_tc_supported(const Geom &g, int dtype, int width, int hidden, int out_ch);
+// warp-specialised TMA pipeline for the projection
+bool proj_pipe_supported(const Geom &g, int dtype, int width, int hidden, int out_ch,
+                         const void *v);
+cudaError_t launch_proj_pipe(const Launch &L, const Geom &g, int dtype, int width, int hidden,
+                             int out_ch, const void *v, const void *Q1, const void *q1,
+                             const void *Q2, const void *q2, void *u);
 cudaError_t launch_proj_fwd_tc(const Launch &L, const Geom &g, int dtype, int width, int hidden,
                                int out_ch, const void *v, const void *Q1, const void *q1,
                                const void *Q2, const void *q2, void *u);

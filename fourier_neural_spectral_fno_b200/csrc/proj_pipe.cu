@@ -1,0 +1,430 @@
+// Projection u = Q2 GELU(Q1 v + q1) + q2 (step S5) as a warp-specialised,
+// TMA-fed tcgen05 pipeline.
+//
+// A tile is 128 consecutive grid points of one sample.  The hidden layer
+// h[p, :] = v[p, :] Q1^T is an MMA chain with A = v (point p <-> TMEM lane p)
+// and B = Q1 (K-major, resident in shared memory); it never leaves the SM:
+// epilogue warps read it from tensor memory, add q1, apply GELU and contract
+// with Q2 on the CUDA cores.  Float32 storage: three tf32 passes (v_hi Q1_hi +
+// v_hi Q1_lo + v_lo Q1_hi); 16-bit storage: one kind::f16 pass.
+//
+//   warp 13      TMA producer: v tile [width][128] into ring stage j % NS
+//   warps 0-3    staging: v -> A operand in TMEM (tf32 head / remainder)
+//   warp 12      MMA issuer: tile j into D buffer j % 2
+//   warps 4-11   epilogue: two warps per TMEM lane quarter, each taking half of
+//                the hidden units; the halves' Q2 partial sums meet in shared
+//                memory and one half stores u
+// Every wait is a bounded mbarrier wait; exits are warp-uniform, and the
+// epilogue warps share one named barrier per tile.
+#include <string.h>
+
+#include "fno_common.cuh"
+#include "fno_kernels.cuh"
+#include "tc_util.cuh"
+#include "tma_util.cuh"
+
+namespace fno {
+
+namespace {
+
+constexpr int ROWS = 128;
+constexpr int NCONV = 4;
+constexpr int NEPI = 8;
+constexpr int WARP_MMA = NCONV + NEPI;     // 12
+constexpr int WARP_TMA = WARP_MMA + 1;     // 13
+constexpr int THREADS = (WARP_TMA + 1) * 32;
+constexpr int MAX_STAGES = 6;
+constexpr int kMaxOut = 4;
+constexpr size_t kSmemMax = 227 * 1024;
+
+template <typename T> struct QKind {
+  static constexpr bool tf32 = false;
+  static constexpr int EB = 2;
+  static constexpr int KSTEP = 16;
+  static constexpr int fmt = tc::FMT_F16;
+  static constexpr CUtensorMapDataType tmap = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+};
+template <> struct QKind<float> {
+  static constexpr bool tf32 = true;
+  static constexpr int EB = 4;
+  static constexpr int KSTEP = 8;
+  static constexpr int fmt = tc::FMT_TF32;
+  static constexpr CUtensorMapDataType tmap = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+};
+template <> struct QKind<__nv_bfloat16> {
+  static constexpr bool tf32 = false;
+  static constexpr int EB = 2;
+  static constexpr int KSTEP = 16;
+  static constexpr int fmt = tc::FMT_BF16;
+  static constexpr CUtensorMapDataType tmap = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+};
+
+__host__ __device__ inline int rup(int v, int m) { return (v + m - 1) / m * m; }
+__host__ __device__ inline size_t alg(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Plan.  TMEM: two D buffers [0, 2 HP), then two A buffers (tf32: head and
+// remainder, 2 Cp columns each).  Shared memory: the ring (v tiles), B = Q1
+// (head block, then remainder block), q1, Q2, the half-sum exchange, barriers.
+struct ProjGeom {
+  int Cp, HP, ax_cols, col_a, used, NS;
+  uint32_t sbo, x_bytes;
+  size_t stage, bhalf, b, q1, q2, red, bar, tbase, total;
+};
+
+__host__ __device__ inline ProjGeom proj_geom(int width, int hidden, int eb, bool tf32) {
+  ProjGeom e;
+  e.Cp = rup(width, 16);
+  e.HP = rup(hidden, 32);                 // two halves of whole 16-column groups
+  e.ax_cols = tf32 ? 2 * e.Cp : e.Cp / 2;
+  e.col_a = 2 * e.HP;
+  e.used = e.col_a + 2 * e.ax_cols;
+  e.sbo = (uint32_t)(e.Cp * eb / 16) * 128u;
+  e.x_bytes = (uint32_t)(width * ROWS * eb);
+  e.stage = alg(e.x_bytes, 1024);
+  e.bhalf = (size_t)e.HP * e.Cp * eb;
+  const size_t fixed = alg((tf32 ? 2 : 1) * e.bhalf, 1024) + sizeof(float) * e.HP +
+                       sizeof(float) * kMaxOut * e.HP + sizeof(float) * 2 * kMaxOut * ROWS +
+                       sizeof(uint64_t) * (2 * MAX_STAGES + 8) + 16;
+  const size_t room = kSmemMax > fixed ? kSmemMax - fixed : 0;
+  const size_t ns = room / e.stage;
+  e.NS = (int)(ns < (size_t)MAX_STAGES ? ns : (size_t)MAX_STAGES);
+  size_t off = (size_t)e.NS * e.stage;
+  e.b = off; off = alg(off + (tf32 ? 2 : 1) * e.bhalf, 1024);
+  e.q1 = off; off += sizeof(float) * e.HP;
+  e.q2 = off; off += sizeof(float) * kMaxOut * e.HP;
+  e.red = off; off += sizeof(float) * 2 * kMaxOut * ROWS;
+  off = alg(off, 8);
+  e.bar = off; off += sizeof(uint64_t) * (2 * MAX_STAGES + 8);
+  e.tbase = off; off += 16;
+  e.total = off < 116 * 1024 ? 116 * 1024 : off;
+  return e;
+}
+
+__host__ __device__ __forceinline__ uint32_t boff(int n, int k, int eb, uint32_t sbo) {
+  const int kb = k * eb;
+  return (uint32_t)(n >> 3) * sbo + (kb >> 4) * 128 + (n & 7) * 16 + (kb & 15);
+}
+
+// named barrier over the eight epilogue warps
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ bool epi_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 1, 256, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
+struct ProjArgs {
+  const void *Q1, *q1, *Q2, *q2;
+  void *u;
+  int *err;
+  long long B, N;
+  int width, hidden, out_ch;
+};
+
+// 16 A elements of this thread's lane into TMEM (tf32: head at col, remainder
+// at col + lo_off)
+template <typename T>
+__device__ __forceinline__ void stage16(uint32_t col, uint32_t lo_off, const float (&v)[16]) {
+  if (QKind<T>::tf32) {
+    uint32_t hi[16], lo[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) tc::split_tf32(v[i], hi[i], lo[i]);
+    tc::tmem_st16(col, hi);
+    tc::tmem_st16(col + lo_off, lo);
+  } else {
+    uint32_t pk[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      pk[i] = QKind<T>::fmt == tc::FMT_BF16 ? tc::pack_bf16(v[2 * i], v[2 * i + 1])
+                                             : tc::pack_f16(v[2 * i], v[2 * i + 1]);
+    tc::tmem_st8(col, pk);
+  }
+}
+
+template <typename T, int CX>
+__global__ void __launch_bounds__(THREADS, 1)
+    k_proj_pipe(const __grid_constant__ CUtensorMap tmv, ProjArgs a) {
+  using K = QKind<T>;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const int width = a.width, hidden = a.hidden, out_ch = a.out_ch;
+  const ProjGeom e = proj_geom(width, hidden, K::EB, K::tf32);
+  unsigned char *bsm = smem + e.b;
+  float *q1s = reinterpret_cast<float *>(smem + e.q1);
+  float *q2s = reinterpret_cast<float *>(smem + e.q2);
+  float *red = reinterpret_cast<float *>(smem + e.red);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + e.bar);
+  uint64_t *empty = full + MAX_STAGES;
+  uint64_t *aready = empty + MAX_STAGES;   // [2]
+  uint64_t *mdone = aready + 2;            // [2]
+  uint64_t *dempty = mdone + 2;            // [2]
+  uint64_t *fin = dempty + 2;              // [1]
+  uint32_t *tbase_s = reinterpret_cast<uint32_t *>(smem + e.tbase);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long N = a.N;
+
+  if (warp == 0) {
+    tc::tmem_alloc(tbase_s, 512);
+    tc::tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int s = 0; s < MAX_STAGES; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], NCONV);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&aready[i], NCONV);
+      tc::mbar_init(&mdone[i], 1);
+      tc::mbar_init(&dempty[i], NEPI);
+    }
+    tc::mbar_init(fin, 1);
+    tma::fence_barrier_init();
+  }
+  if (warp == WARP_TMA && lane == 0) tma::prefetch_map(&tmv);
+  for (size_t i = (size_t)tid * 16; i < (K::tf32 ? 2 : 1) * e.bhalf; i += THREADS * 16)
+    *reinterpret_cast<uint4 *>(bsm + i) = make_uint4(0, 0, 0, 0);
+  __syncthreads();
+  {  // B = Q1 [hidden][width] (head rows block, remainder block), q1, Q2
+    const T *Q1 = reinterpret_cast<const T *>(a.Q1);
+    for (int i = tid; i < hidden * width; i += THREADS) {
+      const int h = i / width, c = i - h * width;
+      const float v = to_f<T>(Q1[i]);
+      const uint32_t o = boff(h, c, K::EB, e.sbo);
+      if (K::tf32) {
+        uint32_t hi, lo;
+        tc::split_tf32(v, hi, lo);
+        *reinterpret_cast<uint32_t *>(bsm + o) = hi;
+        *reinterpret_cast<uint32_t *>(bsm + e.bhalf + o) = lo;
+      } else {
+        *reinterpret_cast<T *>(bsm + o) = from_f<T>(v);
+      }
+    }
+    const T *q1 = reinterpret_cast<const T *>(a.q1);
+    const T *Q2 = reinterpret_cast<const T *>(a.Q2);
+    for (int h = tid; h < e.HP; h += THREADS) q1s[h] = h < hidden ? to_f<T>(q1[h]) : 0.f;
+    for (int i = tid; i < kMaxOut * e.HP; i += THREADS) {
+      const int o = i / e.HP, h = i - o * e.HP;
+      q2s[i] = (o < out_ch && h < hidden) ? to_f<T>(Q2[o * hidden + h]) : 0.f;
+    }
+  }
+  tc::fence_proxy_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = *tbase_s;
+
+  const long long tpb = N / ROWS;
+  const long long ntiles = a.B * tpb;
+  const long long per_cta = (ntiles + gridDim.x - 1) / gridDim.x;
+  const long long t_begin = blockIdx.x * per_cta;
+  const long long t_end = t_begin + per_cta < ntiles ? t_begin + per_cta : ntiles;
+  const int ntl = t_begin < t_end ? (int)(t_end - t_begin) : 0;
+
+  if (warp == WARP_TMA) {
+    // ------------------------------------------------------------ TMA producer
+    int j = 0;
+    for (; j < ntl; ++j) {
+      const int s = j % e.NS;
+      const bool w = j < e.NS || tc::mbar_wait(&empty[s], ((j / e.NS) - 1) & 1, a.err);
+      if (!__all_sync(0xffffffffu, w)) break;
+      if (lane == 0) {
+        const long long tile = t_begin + j;
+        const long long b = tile / tpb;
+        const int n0 = (int)((tile - b * tpb) * ROWS);
+        tma::arrive_expect_tx(&full[s], e.x_bytes);
+        tma::load_4d(smem + (size_t)s * e.stage, &tmv, &full[s], n0, 0, 0, (int)b);
+      }
+      __syncwarp();
+    }
+    for (int jj = j - 1; jj >= 0 && jj >= j - e.NS; --jj)
+      tc::mbar_wait(&full[jj % e.NS], (jj / e.NS) & 1, nullptr);
+  } else if (warp < NCONV) {
+    // ------------------------------------------------------------ staging
+    const int t = tid;
+    const uint32_t arow = tbase + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lo_off = K::tf32 ? (uint32_t)e.Cp : 0u;
+    for (int j = 0; j < ntl; ++j) {
+      const int s = j % e.NS;
+      bool w = tc::mbar_wait(&full[s], (j / e.NS) & 1, a.err);
+      if (w && j >= 2) w = tc::mbar_wait(&mdone[j & 1], ((j - 2) >> 1) & 1, a.err);
+      if (!__all_sync(0xffffffffu, w)) break;
+      tc::fence_after_sync();
+      const T *xs = reinterpret_cast<const T *>(smem + (size_t)s * e.stage);
+      const uint32_t ac = arow + e.col_a + (j & 1) * e.ax_cols;
+#pragma unroll
+      for (int c0 = 0; c0 < CX; c0 += 16) {
+        if (c0 < e.Cp) {
+          float vals[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) vals[i] = c0 + i < width ? to_f<T>(xs[(c0 + i) * ROWS + t]) : 0.f;
+          stage16<T>(ac + (K::tf32 ? c0 : c0 / 2), lo_off, vals);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) tma::arrive(&empty[s]);
+      tc::tmem_wait_st();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tma::arrive(&aready[j & 1]);
+    }
+  } else if (warp == WARP_MMA) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t idesc = tc::instr_desc(K::fmt, ROWS, e.HP);
+    const uint64_t bh0 = tc::smem_desc_kmajor(tc::smem_u32(bsm), 128, e.sbo);
+    const uint64_t bl0 = tc::smem_desc_kmajor(tc::smem_u32(bsm + e.bhalf), 128, e.sbo);
+    const int ns = e.Cp / K::KSTEP;
+    for (int j = 0; j < ntl; ++j) {
+      bool w = tc::mbar_wait(&aready[j & 1], (j >> 1) & 1, a.err);
+      if (w && j >= 2) w = tc::mbar_wait(&dempty[j & 1], ((j - 2) >> 1) & 1, a.err);
+      if (!__all_sync(0xffffffffu, w)) break;
+      tc::fence_after_sync();
+      if (lane == 0) {
+        const uint32_t d = tbase + (uint32_t)((j & 1) * e.HP);
+        uint32_t a0 = tbase + e.col_a + (j & 1) * e.ax_cols;
+        uint64_t bh = bh0, bl = bl0;
+        for (int ks = 0; ks < ns; ++ks) {
+          if (K::tf32) {
+            tc::mma_tf32_ts(d, a0, bh, idesc, ks > 0 ? 1u : 0u);
+            tc::mma_tf32_ts(d, a0, bl, idesc, 1u);
+            tc::mma_tf32_ts(d, a0 + e.Cp, bh, idesc, 1u);
+          } else {
+            tc::mma_f16_ts(d, a0, bh, idesc, ks > 0 ? 1u : 0u);
+          }
+          a0 += 8;
+          bh += 16;
+          bl += 16;
+        }
+        tc::mma_commit(&mdone[j & 1]);
+      }
+      __syncwarp();
+    }
+    if (lane == 0) tc::mma_commit(fin);   // covers every MMA this CTA issued
+    __syncwarp();
+    tc::mbar_wait(fin, 0, nullptr);
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3, half = (warp - NCONV) >> 2;
+    const int t = q * 32 + lane;
+    const uint32_t arow = tbase + ((uint32_t)(q * 32) << 16);
+    const int hbeg = half * (e.HP / 2), hend = hbeg + e.HP / 2;
+    T *u = reinterpret_cast<T *>(a.u);
+    const T *q2 = reinterpret_cast<const T *>(a.q2);
+    float q2b[kMaxOut];
+#pragma unroll
+    for (int o = 0; o < kMaxOut; ++o) q2b[o] = o < out_ch ? to_f<T>(q2[o]) : 0.f;
+    for (int j = 0; j < ntl; ++j) {
+      if (!epi_all(tc::mbar_wait(&mdone[j & 1], (j >> 1) & 1, a.err))) break;
+      tc::fence_after_sync();
+      const uint32_t dcol = arow + (uint32_t)((j & 1) * e.HP);
+      float acc[kMaxOut];
+#pragma unroll
+      for (int o = 0; o < kMaxOut; ++o) acc[o] = 0.f;
+      for (int h0 = hbeg; h0 < hend; h0 += 16) {
+        uint32_t dv[16];
+        tc::tmem_ld16(dcol + h0, dv);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+          float z0 = __uint_as_float(dv[i]) + q1s[h0 + i];
+          float z1 = __uint_as_float(dv[i + 1]) + q1s[h0 + i + 1];
+          gelu2(z0, z1);
+#pragma unroll
+          for (int o = 0; o < kMaxOut; ++o)
+            if (o < out_ch)
+              acc[o] = fmaf(q2s[o * e.HP + h0 + i + 1], z1, fmaf(q2s[o * e.HP + h0 + i], z0, acc[o]));
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tma::arrive(&dempty[j & 1]);
+      float *rb = red + (j & 1) * kMaxOut * ROWS;
+      if (half == 1) {
+#pragma unroll
+        for (int o = 0; o < kMaxOut; ++o)
+          if (o < out_ch) rb[o * ROWS + t] = acc[o];
+      }
+      epi_sync();
+      if (half == 0) {
+        const long long tile = t_begin + j;
+        const long long b = tile / tpb;
+        const long long n = (tile - b * tpb) * ROWS + t;
+#pragma unroll
+        for (int o = 0; o < kMaxOut; ++o)
+          if (o < out_ch) u[(b * out_ch + o) * N + n] = from_f<T>(acc[o] + rb[o * ROWS + t] + q2b[o]);
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tbase, 512);
+  }
+}
+
+template <typename T>
+cudaError_t launch_t(const Launch &L, const Geom &g, const ProjArgs &a, const void *v) {
+  using K = QKind<T>;
+  const ProjGeom e = proj_geom(a.width, a.hidden, K::EB, K::tf32);
+  CUtensorMap tmv;
+  memset(&tmv, 0, sizeof(tmv));
+  const uint64_t dims[4] = {(uint64_t)g.N, 1u, (uint64_t)a.width, (uint64_t)g.B};
+  const uint64_t rowb = (uint64_t)g.N * K::EB;
+  const uint64_t str[3] = {rowb, rowb, rowb * (uint64_t)a.width};
+  const uint32_t box[4] = {(uint32_t)ROWS, 1u, (uint32_t)a.width, 1u};
+  if (!encode_tmap_4d(&tmv, K::tmap, v, dims, str, box)) return cudaErrorInvalidValue;
+  const long long ntiles = g.B * (g.N / ROWS);
+  const int grid = (int)(ntiles < L.num_sms ? ntiles : L.num_sms);
+  auto go = [&](auto kern) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)e.total);
+    kern<<<grid, THREADS, e.total, L.stream>>>(tmv, a);
+  };
+  if (a.width <= 16) go(k_proj_pipe<T, 16>);
+  else if (a.width <= 32) go(k_proj_pipe<T, 32>);
+  else go(k_proj_pipe<T, 64>);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool proj_pipe_supported(const Geom &g, int dtype, int width, int hidden, int out_ch,
+                         const void *v) {
+  if (g.N % ROWS != 0 || g.N > (1LL << 30) || g.B > (1LL << 30)) return false;
+  if (out_ch > kMaxOut || width > 64 || hidden < 1) return false;
+  if ((reinterpret_cast<uintptr_t>(v) & 15) != 0) return false;
+  const bool tf32 = dtype == DT_F32;
+  const ProjGeom e = proj_geom(width, hidden, tf32 ? 4 : 2, tf32);
+  if (e.HP > 256 || e.used > 512) return false;
+  return e.NS >= 2 && e.total <= kSmemMax;
+}
+
+cudaError_t launch_proj_pipe(const Launch &L, const Geom &g, int dtype, int width, int hidden,
+                             int out_ch, const void *v, const void *Q1, const void *q1,
+                             const void *Q2, const void *q2, void *u) {
+  ProjArgs a{};
+  a.Q1 = Q1;
+  a.q1 = q1;
+  a.Q2 = Q2;
+  a.q2 = q2;
+  a.u = u;
+  a.err = L.err;
+  a.B = g.B;
+  a.N = g.N;
+  a.width = width;
+  a.hidden = hidden;
+  a.out_ch = out_ch;
+  launch_begin(L);
+  cudaError_t err = dtype == DT_F32   ? launch_t<float>(L, g, a, v)
+                    : dtype == DT_F16 ? launch_t<__half>(L, g, a, v)
+                                      : launch_t<__nv_bfloat16>(L, g, a, v);
+  launch_end(L, "proj_fwd_pipe");
+  return err;
+}
+
+}  // namespace fno

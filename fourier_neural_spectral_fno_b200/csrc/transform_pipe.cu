@@ -6,10 +6,11 @@
 // cores:
 //   S1  X1[r, j] = sum_n x[r, n] F[j, n]       F[2k] = cos(2 pi k n / N_L),
 //                                              F[2k+1] = -sin(2 pi k n / N_L)
-//       A = x straight from the TMA ring (K-major, 128-byte swizzle); for
-//       float32 storage the staging warps overwrite each element with its tf32
-//       head and put the remainder in tensor memory, so the two MMAs per K step
-//       are A_head [F_hi; F_lo] and A_rest [F_hi; F_lo] (three significant
+//       16-bit storage: A = x straight from the TMA ring (K-major, 128-byte
+//       swizzle).  Float32: the staging warps read each chunk row once and put
+//       its tf32 head and remainder in tensor memory (A from TMEM keeps the
+//       shared-memory port for TMA and F), so the two MMAs per K step are
+//       A_head [F_hi; F_lo] and A_rest [F_hi; F_lo] (three significant
 //       products, ~21 bits).
 //   S2  Z[q, k] = sum_r X1[r, k] exp(-i theta(q, r_off + r)),
 //       theta(q, r) = 2 pi kS(q) r / S, as one MMA chain with A = the resident
@@ -19,6 +20,7 @@
 //
 //   warp 8       TMA producer: 128-byte column chunks of the tile's 128 rows
 //   warps 0-3    staging (thread = row): tanh if asked, tf32 head / remainder
+//                into TMEM (float32; the stage is then released at once)
 //   warp 9       MMA issuer (S1 of tile j, then S2 of tile j - 1)
 //   warps 4-7    X1 readout -> B operand of S2; Z readout, band phase, store
 //
@@ -44,6 +46,7 @@ constexpr int THREADS = 10 * 32;
 constexpr int MAX_STAGES = 8;
 constexpr size_t kSmemMax = 227 * 1024;
 constexpr int CHUNK_BYTES = 128;         // one swizzle atom row
+constexpr int NABUF = 3;                 // A buffers in TMEM (float32 staging ring)
 
 template <typename T> struct FKind {
   static constexpr bool tf32 = false;
@@ -67,7 +70,10 @@ template <> struct FKind<__nv_bfloat16> {
 __host__ __device__ inline int rup(int v, int m) { return (v + m - 1) / m * m; }
 __host__ __device__ inline size_t alg(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Plan.  TMEM: D1 x2 [0, 2 DC1), A_rest x2 (tf32), A2 (128 columns), D2 x2.
+// Plan.  TMEM: D1 x2 [0, 2 DC1), a ring of NA = 3 A buffers (tf32: head +
+// remainder, 64 columns each; staging runs up to two chunks ahead of the
+// MMAs), A2 (128 columns), one D2 (its readout always precedes the next tile's
+// S2, which waits for the B2 that follows that readout).
 // Shared memory: the TMA ring (the twiddle tables alias it during set-up), F,
 // the padded X1 transpose, B2, the readout exchange, the band phases, barriers.
 struct PipeGeom {
@@ -90,7 +96,7 @@ __host__ __device__ inline PipeGeom fpipe_geom(int S, int NL, int mL, int eb, bo
   e.nch = NL / e.CW;
   e.x1ld = 2 * mL + 1;
   e.col_alo = 2 * e.DC1;
-  e.col_a2 = e.col_alo + (tf32 ? 2 * 32 : 0);
+  e.col_a2 = e.col_alo + (tf32 ? NABUF * 64 : 0);
   e.col_d2 = e.col_a2 + ROWS;
   e.cols = 512;
   e.fsbo = (uint32_t)(NL * eb / 16) * 128u;
@@ -187,12 +193,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + e.bar);
   uint64_t *empty = full + MAX_STAGES;
   uint64_t *cready = empty + MAX_STAGES;
-  uint64_t *lofree = cready + MAX_STAGES;   // [2]
-  uint64_t *d1full = lofree + 2;            // [2]
+  uint64_t *lofree = cready + MAX_STAGES;   // [NABUF] A buffer free
+  uint64_t *d1full = lofree + NABUF;        // [2]
   uint64_t *d1free = d1full + 2;            // [2]
   uint64_t *b2ready = d1free + 2;           // [1]
   uint64_t *s2done = b2ready + 1;           // [2]
   uint64_t *d2free = s2done + 2;            // [2]
+  uint64_t *fin = d2free + 2;               // [1] all MMAs of the CTA done
   uint32_t *tbase_s = reinterpret_cast<uint32_t *>(smem + e.tbase);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -203,17 +210,18 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (tid == 0) {
     for (int s = 0; s < MAX_STAGES; ++s) {
       tc::mbar_init(&full[s], 1);
-      tc::mbar_init(&empty[s], 1);
+      tc::mbar_init(&empty[s], K::tf32 ? NSTAGE_WARPS : 1);   // tf32: staging frees it
       tc::mbar_init(&cready[s], NSTAGE_WARPS);
     }
+    for (int i = 0; i < NABUF; ++i) tc::mbar_init(&lofree[i], 1);
     for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&lofree[i], 1);
       tc::mbar_init(&d1full[i], 1);
       tc::mbar_init(&d1free[i], 4);
       tc::mbar_init(&s2done[i], 1);
       tc::mbar_init(&d2free[i], 4);
     }
     tc::mbar_init(b2ready, 4);
+    tc::mbar_init(fin, 1);
     tma::fence_barrier_init();
   }
   if (warp == WARP_TMA && lane == 0) tma::prefetch_map(&tmx);
@@ -319,7 +327,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int c = 0; c < nch; ++c, ++g) {
         const int s = g % e.NS;
         bool w = tc::mbar_wait(&full[s], (g / e.NS) & 1, a.err);
-        if (K::tf32 && w && g >= 2) w = tc::mbar_wait(&lofree[g & 1], ((g - 2) >> 1) & 1, a.err);
+        if (K::tf32 && w && g >= NABUF)
+          w = tc::mbar_wait(&lofree[g % NABUF], ((g / NABUF) - 1) & 1, a.err);
         if (!__all_sync(0xffffffffu, w)) {
           ok = false;
           break;
@@ -332,27 +341,25 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int p = 0; p < 8; ++p) pc[p] = *reinterpret_cast<const uint4 *>(rowp + ((p ^ (r & 7)) << 4));
           if (K::tf32) {
-            uint32_t lo[32];
+            // head / remainder of the 32 values into A buffer g & 1: head
+            // columns [0, 32), remainder [32, 64)
+            const uint32_t acol = lrow + e.col_alo + (g % NABUF) * 64;
 #pragma unroll
-            for (int p = 0; p < 8; ++p) {
-              uint32_t *u = reinterpret_cast<uint32_t *>(&pc[p]);
+            for (int hlf = 0; hlf < 2; ++hlf) {
+              uint32_t hi[16], lo[16];
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                float v = __uint_as_float(u[i]);
-                if (LOAD == LOAD_TANH) v = tanhf(v);
-                const uint32_t hb = __float_as_uint(v) & 0xFFFFE000u;
-                lo[p * 4 + i] = __float_as_uint(v - __uint_as_float(hb));
-                u[i] = hb;
+              for (int p = 0; p < 4; ++p) {
+                const uint32_t *u = reinterpret_cast<const uint32_t *>(&pc[hlf * 4 + p]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  float v = __uint_as_float(u[i]);
+                  if (LOAD == LOAD_TANH) v = tanhf(v);
+                  tc::split_tf32(v, hi[p * 4 + i], lo[p * 4 + i]);
+                }
               }
-              *reinterpret_cast<uint4 *>(rowp + ((p ^ (r & 7)) << 4)) = pc[p];
+              tc::tmem_st16(acol + hlf * 16, hi);
+              tc::tmem_st16(acol + 32 + hlf * 16, lo);
             }
-            uint32_t l16[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) l16[i] = lo[i];
-            tc::tmem_st16(lrow + e.col_alo + (g & 1) * 32, l16);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) l16[i] = lo[16 + i];
-            tc::tmem_st16(lrow + e.col_alo + (g & 1) * 32 + 16, l16);
           } else {
 #pragma unroll
             for (int p = 0; p < 8; ++p) {
@@ -367,7 +374,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         tc::fence_before_sync();
         __syncwarp();
-        if (lane == 0) tma::arrive(&cready[s]);
+        if (lane == 0) {
+          if (K::tf32) tma::arrive(&empty[s]);   // the row data now lives in TMEM
+          tma::arrive(&cready[s]);
+        }
       }
     }
   } else if (warp == WARP_MMA) {
@@ -378,11 +388,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint64_t b2desc = tc::smem_desc_kmajor(tc::smem_u32(b2), 128, e.b2sbo);
     auto issue_s2 = [&](int jj) -> bool {   // S2 of local tile jj
       bool w = tc::mbar_wait(b2ready, jj & 1, a.err);
-      if (w && jj >= 2) w = tc::mbar_wait(&d2free[jj & 1], ((jj - 2) >> 1) & 1, a.err);
+      if (w && jj >= 1) w = tc::mbar_wait(&d2free[0], (jj - 1) & 1, a.err);
       if (!__all_sync(0xffffffffu, w)) return false;
       tc::fence_after_sync();
       if (lane == 0) {
-        const uint32_t d2 = tbase + e.col_d2 + (uint32_t)((jj & 1) * 2 * e.NP);
+        const uint32_t d2 = tbase + e.col_d2;
         uint64_t bd = b2desc;
         uint32_t acol = tbase + e.col_a2;
         for (int ks = 0; ks < ROWS / 8; ++ks) {
@@ -413,17 +423,21 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (lane == 0) {
           uint64_t ad = desc_sw128(tc::smem_u32(smem + (size_t)s * e.stage));
           uint64_t bd = fdesc + (uint64_t)(c * 4 * 16);
-          const uint32_t alo = tbase + e.col_alo + (g & 1) * 32;
+          const uint32_t ahi = tbase + e.col_alo + (g % NABUF) * 64;
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
             const uint32_t acc = (c | ks) ? 1u : 0u;
-            mma_ss(d1, ad, bd, id1, acc, K::tf32);
-            if (K::tf32) tc::mma_tf32_ts(d1, alo + ks * 8, bd, id1, 1u);
+            if (K::tf32) {
+              tc::mma_tf32_ts(d1, ahi + ks * 8, bd, id1, acc);
+              tc::mma_tf32_ts(d1, ahi + 32 + ks * 8, bd, id1, 1u);
+            } else {
+              mma_ss(d1, ad, bd, id1, acc, false);
+            }
             ad += 2;     // 32 bytes along K inside the swizzle atom
             bd += 16;    // 256 bytes: next K step of F
           }
-          tc::mma_commit(&empty[s]);
-          if (K::tf32) tc::mma_commit(&lofree[g & 1]);
+          if (K::tf32) tc::mma_commit(&lofree[g % NABUF]);   // A buffer free
+          else tc::mma_commit(&empty[s]);                 // stage free
           if (c == nch - 1) tc::mma_commit(&d1full[j & 1]);
         }
         __syncwarp();
@@ -432,9 +446,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (j >= 1 && !issue_s2(j - 1)) ok = false;
     }
     if (ok && ntl > 0) ok = issue_s2(ntl - 1);
-    // no MMA may still run when TMEM is freed
-    if (ntl > 0) tc::mbar_wait(&s2done[(ntl - 1) & 1], ((ntl - 1) >> 1) & 1, nullptr);
-    if (g > 0) tc::mbar_wait(&empty[(g - 1) % e.NS], ((g - 1) / e.NS) & 1, nullptr);
+    // no MMA may still run when TMEM is freed: one last commit covers them all
+    if (lane == 0) tc::mma_commit(fin);
+    __syncwarp();
+    tc::mbar_wait(fin, 0, nullptr);
   } else {
     // ------------------------------------------------------------ X1 / Z warps
     const int blk = warp - WARP_X1;                 // lane quarter
@@ -444,7 +459,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto readout_s2 = [&](int jj) -> bool {         // Z of local tile jj
       if (!x1_all(tc::mbar_wait(&s2done[jj & 1], (jj >> 1) & 1, a.err))) return false;
       tc::fence_after_sync();
-      const uint32_t d2 = lrow + e.col_d2 + (uint32_t)((jj & 1) * 2 * e.NP);
+      const uint32_t d2 = lrow + e.col_d2;
       float val[32];
 #pragma unroll
       for (int c0 = 0; c0 < 32; c0 += 16) {
@@ -459,7 +474,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) tma::arrive(&d2free[jj & 1]);
+      if (lane == 0) tma::arrive(&d2free[0]);
       // cos rows = blk 0 (+ blk 2), sin rows = blk 1 (+ blk 3)
       if (blk >= 2) {
 #pragma unroll
@@ -614,7 +629,7 @@ bool fwd_pipe_supported(const Geom &g, int dtype, int load_mode, const void *in0
   const bool tf32 = dtype == DT_F32;
   const PipeGeom e = fpipe_geom(g.S, g.NL, g.mL, eb, tf32);
   if (e.NS < 2 || e.total > kSmemMax) return false;
-  if (e.col_d2 + 4 * e.NP > 512) return false;
+  if (e.col_d2 + 2 * e.NP > 512) return false;
   return true;
 }
 
