@@ -179,6 +179,8 @@ def algorithmic_bytes(tag: str, wl) -> float:
     for base in ("fwd_transform", "epi_block_fwd", "proj_fwd"):
         table[base + "_tc"] = table[base]
     table["epi_block_fwd_pipe"] = table["epi_block_fwd"]
+    table["fwd_transform_pipe"] = table["fwd_transform"]
+    table["proj_fwd_pipe"] = table["proj_fwd"]
     return float(table.get(tag, 0.0))
 
 
@@ -187,7 +189,8 @@ def kernel_source_sha(tag: str) -> str:
              "epi_block_fwd": "epilogue.cu", "mix_fwd": "mix.cu", "lift": "net.cu",
              "proj_fwd": "net.cu", "fwd_transform_tc": "transform_tc.cu",
              "epi_block_fwd_tc": "epilogue_tc.cu", "inv_slab": "epilogue_tc.cu",
-             "proj_fwd_tc": "net_tc.cu", "epi_block_fwd_pipe": "epilogue_pipe.cu"}
+             "proj_fwd_tc": "net_tc.cu", "epi_block_fwd_pipe": "epilogue_pipe.cu",
+             "fwd_transform_pipe": "transform_pipe.cu", "proj_fwd_pipe": "proj_pipe.cu"}
     path = os.path.join(ROOT, "fourier_neural_spectral_fno_b200", "csrc", files.get(tag, ""))
     if not os.path.isfile(path):
         return ""

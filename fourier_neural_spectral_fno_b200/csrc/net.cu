@@ -42,6 +42,76 @@ __global__ void __launch_bounds__(NT)
   }
 }
 
+// Lift for rows whose length is a multiple of 4: a thread takes 4 consecutive
+// points, loads each input channel as one vector, and writes each of the width
+// output channels as one vector (weights broadcast from shared memory).
+template <typename T> struct Vec4;
+template <> struct Vec4<float> {
+  using raw = float4;
+  __device__ static void load(const float *p, float (&v)[4]) {
+    const float4 r = *reinterpret_cast<const float4 *>(p);
+    v[0] = r.x; v[1] = r.y; v[2] = r.z; v[3] = r.w;
+  }
+  __device__ static void store(float *p, const float (&v)[4]) {
+    *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+};
+template <typename T> struct Vec4 {   // 16-bit storage: 8-byte vectors
+  __device__ static void load(const T *p, float (&v)[4]) {
+    const uint2 r = *reinterpret_cast<const uint2 *>(p);
+    const T *h = reinterpret_cast<const T *>(&r);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = to_f<T>(h[i]);
+  }
+  __device__ static void store(T *p, const float (&v)[4]) {
+    uint2 r;
+    T *h = reinterpret_cast<T *>(&r);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = from_f<T>(v[i]);
+    *reinterpret_cast<uint2 *>(p) = r;
+  }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(NT)
+    k_lift4(const T *__restrict__ a, const T *__restrict__ P, const T *__restrict__ p,
+            T *__restrict__ v, long long B, long long N, int in_ch, int width) {
+  __shared__ float Ps[kMaxWidth * kMaxIn], ps[kMaxWidth];
+  for (int e = threadIdx.x; e < width * in_ch; e += NT) Ps[e] = to_f<T>(P[e]);
+  for (int e = threadIdx.x; e < width; e += NT) ps[e] = to_f<T>(p[e]);
+  __syncthreads();
+  const long long N4 = N / 4;
+  for (long long t = (long long)blockIdx.x * NT + threadIdx.x; t < B * N4;
+       t += (long long)gridDim.x * NT) {
+    const long long b = t / N4, n = (t - b * N4) * 4;
+    float x[kMaxIn][4];
+    const T *ap = a + b * in_ch * N + n;
+#pragma unroll
+    for (int j = 0; j < kMaxIn; ++j) {
+      if (j < in_ch) Vec4<T>::load(ap + j * N, x[j]);
+    }
+    T *vp = v + b * width * N + n;
+    const float *pw = Ps;
+    for (int c = 0; c < width; ++c) {
+      float o[4];
+      const float bc = ps[c];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[i] = bc;
+#pragma unroll
+      for (int j = 0; j < kMaxIn; ++j) {
+        if (j < in_ch) {
+          const float w = pw[j];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) o[i] = fmaf(w, x[j][i], o[i]);
+        }
+      }
+      pw += in_ch;
+      Vec4<T>::store(vp, o);
+      vp += N;
+    }
+  }
+}
+
 template <typename T, int CMAX>
 __global__ void __launch_bounds__(NT)
     k_proj_fwd(const T *__restrict__ v, const T *__restrict__ Q1, const T *__restrict__ q1,
@@ -324,11 +394,21 @@ int pointwise_grid(long long total, int num_sms) {
 
 cudaError_t launch_lift(const Launch &L, const Geom &g, int dtype, int in_ch, int width,
                         const void *a, const void *P, const void *p, void *v) {
-  const int grid = pointwise_grid(g.B * g.N, L.num_sms);
+  const size_t vb = dtype == DT_F32 ? 16 : 8;   // vector bytes of 4 elements
+  const bool vec = g.N % 4 == 0 && (reinterpret_cast<uintptr_t>(a) % vb) == 0 &&
+                   (reinterpret_cast<uintptr_t>(v) % vb) == 0;
   launch_begin(L);
-  FNO_DISPATCH_T(dtype, k_lift<T><<<grid, NT, 0, L.stream>>>(
-                            (const T *)a, (const T *)P, (const T *)p, (T *)v, g.B, g.N, in_ch,
-                            width));
+  if (vec) {
+    const int grid = pointwise_grid(g.B * g.N / 4, L.num_sms);
+    FNO_DISPATCH_T(dtype, k_lift4<T><<<grid, NT, 0, L.stream>>>(
+                              (const T *)a, (const T *)P, (const T *)p, (T *)v, g.B, g.N, in_ch,
+                              width));
+  } else {
+    const int grid = pointwise_grid(g.B * g.N, L.num_sms);
+    FNO_DISPATCH_T(dtype, k_lift<T><<<grid, NT, 0, L.stream>>>(
+                              (const T *)a, (const T *)P, (const T *)p, (T *)v, g.B, g.N, in_ch,
+                              width));
+  }
   launch_end(L, "lift");
   return cudaGetLastError();
 }

@@ -330,14 +330,21 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc::tmem_ld16(dcol + h0, dv);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; i += 2) {
-          float z0 = __uint_as_float(dv[i]) + q1s[h0 + i];
-          float z1 = __uint_as_float(dv[i + 1]) + q1s[h0 + i + 1];
+        for (int i = 0; i < 16; i += 4) {   // q1 / Q2 as 16-byte vectors
+          const float4 qa = *reinterpret_cast<const float4 *>(q1s + h0 + i);
+          float z0 = __uint_as_float(dv[i]) + qa.x;
+          float z1 = __uint_as_float(dv[i + 1]) + qa.y;
+          float z2 = __uint_as_float(dv[i + 2]) + qa.z;
+          float z3 = __uint_as_float(dv[i + 3]) + qa.w;
           gelu2(z0, z1);
+          gelu2(z2, z3);
 #pragma unroll
-          for (int o = 0; o < kMaxOut; ++o)
-            if (o < out_ch)
-              acc[o] = fmaf(q2s[o * e.HP + h0 + i + 1], z1, fmaf(q2s[o * e.HP + h0 + i], z0, acc[o]));
+          for (int o = 0; o < kMaxOut; ++o) {
+            if (o < out_ch) {
+              const float4 qb = *reinterpret_cast<const float4 *>(q2s + o * e.HP + h0 + i);
+              acc[o] = fmaf(qb.w, z3, fmaf(qb.z, z2, fmaf(qb.y, z1, fmaf(qb.x, z0, acc[o]))));
+            }
+          }
         }
       }
       tc::fence_before_sync();

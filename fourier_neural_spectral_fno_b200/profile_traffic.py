@@ -1,0 +1,96 @@
+"""Record per-launch DRAM traffic of the library's kernels from an ncu capture.
+
+Reads the CSV that ``ncu -i <report> --page raw --csv`` prints (a capture that
+collected ``dram__bytes_read.sum`` and ``dram__bytes_write.sum``), averages the
+launches of each kernel, and stores them in ``profiles/traffic.json`` under the
+workload name, keyed by the kernel's timing tag together with the hash of the
+source file it was built from (bench.py ignores a record whose source changed).
+
+    ncu -i report.ncu-rep --page raw --csv > raw.csv
+    python -m fourier_neural_spectral_fno_b200.profile_traffic raw.csv \
+        fno2d_f32_b16_w32_256sq_m16
+"""
+
+from __future__ import annotations
+
+import csv
+import hashlib
+import json
+import os
+import sys
+from collections import defaultdict
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CSRC = os.path.join(ROOT, "fourier_neural_spectral_fno_b200", "csrc")
+
+# kernel symbol prefix -> (timing tag, source file)
+KERNELS = {
+    "k_epi_pipe": ("epi_block_fwd_pipe", "epilogue_pipe.cu"),
+    "k_fwd_pipe": ("fwd_transform_pipe", "transform_pipe.cu"),
+    "k_proj_pipe": ("proj_fwd_pipe", "proj_pipe.cu"),
+    "k_epi_tc": ("epi_block_fwd_tc", "epilogue_tc.cu"),
+    "k_s1_tc": ("fwd_transform_tc", "transform_tc.cu"),
+    "k_proj_tc": ("proj_fwd_tc", "net_tc.cu"),
+    "k_inv_slab": ("inv_slab", "epilogue_tc.cu"),
+    "k_mix_fwd": ("mix_fwd", "mix.cu"),
+    "k_fwd_finish": ("fwd_finish", "transform.cu"),
+    "k_lift4": ("lift", "net.cu"),
+    "k_lift": ("lift", "net.cu"),
+}
+
+
+def source_sha(fname: str) -> str:
+    with open(os.path.join(CSRC, fname), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def _kernel_key(name: str):
+    base = name.split("(")[0].split("<")[0].split("::")[-1].strip()
+    return KERNELS.get(base)
+
+
+def parse(csv_path: str):
+    rows = list(csv.reader(open(csv_path)))
+    hdr = rows[0]
+    col = {h: i for i, h in enumerate(hdr)}
+    acc = defaultdict(lambda: [0.0, 0.0, 0])
+    for r in rows[2:]:                       # row 1 holds the units
+        key = _kernel_key(r[col["Kernel Name"]])
+        if key is None:
+            continue
+        try:
+            rd = float(r[col["dram__bytes_read.sum"]])
+            wr = float(r[col["dram__bytes_write.sum"]])
+        except (KeyError, ValueError):
+            continue
+        unit = rows[1][col["dram__bytes_read.sum"]]
+        scale = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}.get(unit, 1.0)
+        a = acc[key]
+        a[0] += rd * scale
+        a[1] += wr * scale
+        a[2] += 1
+    return acc
+
+
+def main(argv) -> int:
+    if len(argv) != 3:
+        print(__doc__)
+        return 2
+    acc = parse(argv[1])
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        data = json.load(open(path))
+    except Exception:
+        data = {}
+    wl = data.setdefault(argv[2], {})
+    for (tag, src), (rd, wr, n) in sorted(acc.items()):
+        wl[tag] = {"bytes_per_launch": (rd + wr) / n, "read_bytes": rd / n,
+                   "write_bytes": wr / n, "launches": n, "source_sha": source_sha(src)}
+        print(f"{tag:22s} {src:18s} read {rd / n / 1e6:8.1f} MB  write {wr / n / 1e6:8.1f} MB")
+    with open(path, "w") as f:
+        json.dump(data, f, indent=1)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main(sys.argv))
