@@ -10,7 +10,9 @@
 //
 //   warp 13      TMA producer: v tile [width][128] into ring stage j % NS
 //   warps 0-3    staging: v -> A operand in TMEM (tf32 head / remainder)
-//   warp 12      MMA issuer: tile j into D buffer j % 2
+//   warp 12      MMA issuer: tile j into D buffer j % 2; its one mbarrier wait
+//                per tile (aready) also means the D buffer is free, since the
+//                staging warps wait for the epilogue before arriving
 //   warps 4-11   epilogue: two warps per TMEM lane quarter, each taking half of
 //                the hidden units; the halves' Q2 partial sums meet in shared
 //                memory and one half stores u
@@ -253,6 +255,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int s = j % e.NS;
       bool w = tc::mbar_wait(&full[s], (j / e.NS) & 1, a.err);
       if (w && j >= 2) w = tc::mbar_wait(&mdone[j & 1], ((j - 2) >> 1) & 1, a.err);
+      // aready(j) also carries "D buffer j % 2 is free" to the MMA thread
+      if (w && j >= 2) w = tc::mbar_wait(&dempty[j & 1], ((j - 2) >> 1) & 1, a.err);
       if (!__all_sync(0xffffffffu, w)) break;
       tc::fence_after_sync();
       const T *xs = reinterpret_cast<const T *>(smem + (size_t)s * e.stage);
@@ -280,8 +284,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint64_t bl0 = tc::smem_desc_kmajor(tc::smem_u32(bsm + e.bhalf), 128, e.sbo);
     const int ns = e.Cp / K::KSTEP;
     for (int j = 0; j < ntl; ++j) {
-      bool w = tc::mbar_wait(&aready[j & 1], (j >> 1) & 1, a.err);
-      if (w && j >= 2) w = tc::mbar_wait(&dempty[j & 1], ((j - 2) >> 1) & 1, a.err);
+      const bool w = tc::mbar_wait(&aready[j & 1], (j >> 1) & 1, a.err);
       if (!__all_sync(0xffffffffu, w)) break;
       tc::fence_after_sync();
       if (lane == 0) {

@@ -21,7 +21,10 @@
 //   warp 8       TMA producer: 128-byte column chunks of the tile's 128 rows
 //   warps 0-3    staging (thread = row): tanh if asked, tf32 head / remainder
 //                into TMEM (float32; the stage is then released at once)
-//   warp 9       MMA issuer (S1 of tile j, then S2 of tile j - 1)
+//   warp 9       MMA issuer (S1 of tile j, then S2 of tile j - 1); it waits only
+//                on chunk-ready and B2-ready barriers (each mbarrier operation in
+//                the issuing thread costs tensor-pipe time), the staging and
+//                readout warps fold the buffer-free conditions into those
 //   warps 4-7    X1 readout -> B operand of S2; Z readout, band phase, store
 //
 // Every wait is a bounded mbarrier wait; every role leaves its loop on a
@@ -198,8 +201,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t *d1free = d1full + 2;            // [2]
   uint64_t *b2ready = d1free + 2;           // [1]
   uint64_t *s2done = b2ready + 1;           // [2]
-  uint64_t *d2free = s2done + 2;            // [2]
-  uint64_t *fin = d2free + 2;               // [1] all MMAs of the CTA done
+  uint64_t *fin = s2done + 2;               // [1] all MMAs of the CTA done
   uint32_t *tbase_s = reinterpret_cast<uint32_t *>(smem + e.tbase);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -218,7 +220,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc::mbar_init(&d1full[i], 1);
       tc::mbar_init(&d1free[i], 4);
       tc::mbar_init(&s2done[i], 1);
-      tc::mbar_init(&d2free[i], 4);
     }
     tc::mbar_init(b2ready, 4);
     tc::mbar_init(fin, 1);
@@ -329,6 +330,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         bool w = tc::mbar_wait(&full[s], (g / e.NS) & 1, a.err);
         if (K::tf32 && w && g >= NABUF)
           w = tc::mbar_wait(&lofree[g % NABUF], ((g / NABUF) - 1) & 1, a.err);
+        // chunk 0 of tile j also carries "D1 buffer j % 2 is free" to the MMA
+        if (w && c == 0 && j >= 2) w = tc::mbar_wait(&d1free[j & 1], ((j - 2) >> 1) & 1, a.err);
         if (!__all_sync(0xffffffffu, w)) {
           ok = false;
           break;
@@ -387,8 +390,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint64_t fdesc = tc::smem_desc_kmajor(tc::smem_u32(fsm), 128, e.fsbo);
     const uint64_t b2desc = tc::smem_desc_kmajor(tc::smem_u32(b2), 128, e.b2sbo);
     auto issue_s2 = [&](int jj) -> bool {   // S2 of local tile jj
-      bool w = tc::mbar_wait(b2ready, jj & 1, a.err);
-      if (w && jj >= 1) w = tc::mbar_wait(&d2free[0], (jj - 1) & 1, a.err);
+      // b2ready(jj) follows the readout of D2 for tile jj - 1 in the readout
+      // warps' own order, so D2 is free as well
+      const bool w = tc::mbar_wait(b2ready, jj & 1, a.err);
       if (!__all_sync(0xffffffffu, w)) return false;
       tc::fence_after_sync();
       if (lane == 0) {
@@ -408,10 +412,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     int g = 0;
     bool ok = true;
     for (int j = 0; j < ntl && ok; ++j) {
-      if (j >= 2 && !__all_sync(0xffffffffu, tc::mbar_wait(&d1free[j & 1], ((j - 2) >> 1) & 1, a.err))) {
-        ok = false;
-        break;
-      }
       const uint32_t d1 = tbase + (uint32_t)((j & 1) * e.DC1);
       for (int c = 0; c < nch; ++c, ++g) {
         const int s = g % e.NS;
@@ -474,7 +474,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) tma::arrive(&d2free[0]);
       // cos rows = blk 0 (+ blk 2), sin rows = blk 1 (+ blk 3)
       if (blk >= 2) {
 #pragma unroll
