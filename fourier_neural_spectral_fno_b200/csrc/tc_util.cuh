@@ -12,9 +12,9 @@
 //        (n / 8) * SBO + (k_bytes / 16) * 128 + (n % 8) * 16 + k_bytes % 16
 //    i.e. LBO = 128 B between K-adjacent core matrices and SBO = (K bytes / 16)
 //    * 128 B between 8-row groups.
-//  * Every spin on an mbarrier is bounded; on expiry the kernel records an
-//    error word and carries on (results are then invalid, the host reports
-//    FNO_ERR_TIMEOUT).
+//  * Every spin on an mbarrier is bounded (about two seconds of suspended
+//    waits); on expiry the kernel records an error word and carries on
+//    (results are then invalid, the host reports FNO_ERR_TIMEOUT).
 #pragma once
 
 #include <cuda_runtime.h>
