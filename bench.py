@@ -157,7 +157,12 @@ def workload_config(wl, n_gpus):
             "width": wl.width, "in_channels": wl.in_ch, "hidden": wl.hidden,
             "blocks": wl.n_layers, "storage": wl.dtype,
             "l2": "flushed between timed steps (512 MiB write outside the step events)",
-            "parallelism": f"dp{n_gpus} (batch-sharded, no data-path collective)"}
+            "step": ("training: forward + MSE + backward" +
+                     (" + NCCL gradient all-reduce" if n_gpus > 1 else "")
+                     if wl.backward and wl.kind == "network" else "forward"),
+            "parallelism": (f"dp{n_gpus} (batch-sharded" +
+                            (", gradient all-reduce)" if wl.backward and wl.kind == "network"
+                             and n_gpus > 1 else ", no data-path collective)"))}
 
 
 def algorithmic_bytes(tag: str, wl) -> float:
@@ -179,6 +184,10 @@ def algorithmic_bytes(tag: str, wl) -> float:
     for base in ("fwd_transform", "epi_block_fwd", "proj_fwd"):
         table[base + "_tc"] = table[base]
     table["epi_block_fwd_pipe"] = table["epi_block_fwd"]
+    table["epi_block_bwd"] = 4 * act + spec         # read dy, pre, x; write dx; read spectrum
+    table["fwd_transform_dz"] = 2 * act + spec      # read dy, pre; write spectrum
+    table["fwd_transform_tc_dz"] = table["fwd_transform_dz"]
+    table["proj_bwd"] = 2 * act + 2 * wl.batch * wl.out_ch * wl.points * s
     table["fwd_transform_pipe"] = table["fwd_transform"]
     table["proj_fwd_pipe"] = table["proj_fwd"]
     return float(table.get(tag, 0.0))
@@ -228,8 +237,22 @@ def cpu_threads() -> int:
 
 
 def oracle_samples(wl, inp, n_samples):
+    """The oracle's step on the first n_samples of the batch: the forward, and
+    for training workloads the MSE and the backward as well."""
     import oracle as O
-    return O.forward(inp["a"][:n_samples], inp["params"], wl.modes)
+    a = inp["a"][:n_samples]
+    if not (wl.backward and wl.kind == "network"):
+        return O.forward(a, inp["params"], wl.modes)
+    u, sv = O.forward(a, inp["params"], wl.modes, save=True)
+    _, du = O.mse(u, inp["target"][:n_samples])
+    return O.backward(a, inp["params"], sv, du, wl.modes)
+
+
+def _one_sample(inp, i):
+    one = {"a": inp["a"][i:i + 1], "params": inp["params"]}
+    if inp.get("target") is not None:
+        one["target"] = inp["target"][i:i + 1]
+    return one
 
 
 def cpu_baseline(wl, inp, seconds):
@@ -237,7 +260,7 @@ def cpu_baseline(wl, inp, seconds):
     time, until `seconds` of CPU work or the batch is done)."""
     done, t0 = 0, time.perf_counter()
     while done < wl.batch and (time.perf_counter() - t0) < seconds:
-        oracle_samples(wl, {"a": inp["a"][done:done + 1], "params": inp["params"]}, 1)
+        oracle_samples(wl, _one_sample(inp, done), 1)
         done += 1
     dt = time.perf_counter() - t0
     return {"value": done / dt, "unit": "samples/s", "cores": cpu_threads(), "kind": "oracle",
@@ -256,10 +279,10 @@ def run_reference(args, dist):
         return
     inp = synth.make_network_inputs(wl)
     for i in range(args.warmup):
-        oracle_samples(wl, {"a": inp["a"][i % wl.batch:i % wl.batch + 1], "params": inp["params"]}, 1)
+        oracle_samples(wl, _one_sample(inp, i % wl.batch), 1)
     t0 = time.perf_counter()
     for i in range(args.steps):
-        oracle_samples(wl, {"a": inp["a"][i % wl.batch:i % wl.batch + 1], "params": inp["params"]}, 1)
+        oracle_samples(wl, _one_sample(inp, i % wl.batch), 1)
     dt = time.perf_counter() - t0
     value = args.steps / dt
     cores = cpu_threads()
@@ -302,13 +325,42 @@ def run_fno(args, dist):
                          wl.n_layers, wl.dtype, capi.FNO_TANH_PREACT if wl.tanh else 0)
     a = up(inp["a"])
     u = torch.empty((wl.batch, wl.out_ch) + wl.grid, dtype=tdt, device=dev)
-    ws = torch.empty(capi.fno_net_workspace_size(desc, capi.FNO_OP_NET_FWD), dtype=torch.uint8,
-                     device=dev)
+    train = wl.backward and wl.kind == "network"
+    ws_bytes = capi.fno_net_workspace_size(desc, capi.FNO_OP_NET_FWD)
+    if train:
+        ws_bytes = max(ws_bytes, capi.fno_net_workspace_size(desc, capi.FNO_OP_NET_BWD))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step():
-        capi.fno_forward(desc, a, cp, u, None, ws, stream)
+    if train:
+        # forward (keeping the saves), MSE against the target, backward into
+        # float32 gradients; with several ranks the gradients are summed by one
+        # NCCL all-reduce (the cotangent carries the global-mean scaling)
+        from fourier_neural_spectral_fno_b200 import dp
+        saves = torch.empty(capi.fno_net_saves_size(desc), dtype=torch.uint8, device=dev)
+        target = up(inp["target"])
+        loss = torch.empty(1, dtype=torch.float32, device=dev)
+        du = torch.empty_like(u)
+        grads = {k: ([torch.empty(np.shape(x) + ((2,) if np.iscomplexobj(x) else ()),
+                                  dtype=torch.float32, device=dev) for x in v]
+                     if isinstance(v, list) else
+                     torch.empty(np.shape(v), dtype=torch.float32, device=dev))
+                 for k, v in inp["params"].items()}
+        cg = capi.make_grads(grads)
+        scale = dp.mse_scale(u.numel(), u.numel() * dist.world)
+
+        def step():
+            capi.fno_forward(desc, a, cp, u, saves, ws, stream)
+            capi.fno_mse(u, target, loss, du, wl.dtype, stream)
+            if scale != 1.0:
+                du.mul_(scale)
+            capi.fno_backward(desc, a, cp, saves, du, cg, ws, stream)
+            if dist.world > 1:
+                dp.allreduce_grads(grads)
+    else:
+        def step():
+            capi.fno_forward(desc, a, cp, u, None, ws, stream)
 
     for _ in range(args.warmup):
         step()
@@ -358,30 +410,37 @@ def run_fno(args, dist):
         stats.items(), key=lambda kv: -kv[1]["total_ms"])}
 
     # ---- end to end through the public API with host buffers
-    a_host = torch.empty(a.shape, dtype=tdt, pin_memory=True)
-    a_host.copy_(a.cpu())
-    u_host = torch.empty(u.shape, dtype=tdt, pin_memory=True)
+    ins = [a, target] if train else [a]            # the step's inputs
+    out = loss if train else u                     # the step's result the host reads
+    ins_host = []
+    for t in ins:
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t.cpu())
+        ins_host.append(h)
+    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     e_steps = max(3, min(args.steps, 20))
     for _ in range(2):
-        a.copy_(a_host, non_blocking=True)
+        for t, h in zip(ins, ins_host):
+            t.copy_(h, non_blocking=True)
         step()
-        u_host.copy_(u, non_blocking=True)
+        out_host.copy_(out, non_blocking=True)
     torch.cuda.synchronize()
     dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(e_steps):
-        a.copy_(a_host, non_blocking=True)
+        for t, h in zip(ins, ins_host):
+            t.copy_(h, non_blocking=True)
         step()
-        u_host.copy_(u, non_blocking=True)
+        out_host.copy_(out, non_blocking=True)
         stream.synchronize()
-        float(u_host.view(-1)[0])           # the host reads the step's result
+        float(out_host.view(-1)[0])           # the host reads the step's result
     e1.record()
     torch.cuda.synchronize()
     e_ms = dist.max(e0.elapsed_time(e1) / e_steps)
     e2e = {"value": dist.world * wl.batch / (e_ms / 1e3), "unit": "samples/s",
-           "h2d_bytes_per_step": a.numel() * a.element_size(),
-           "d2h_bytes_per_step": u.numel() * u.element_size(), "ms_per_step": e_ms}
+           "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in ins),
+           "d2h_bytes_per_step": out.numel() * out.element_size(), "ms_per_step": e_ms}
 
     clocks = clk.summary()
     cpu = None
