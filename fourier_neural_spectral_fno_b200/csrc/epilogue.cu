@@ -47,12 +47,11 @@ __host__ __device__ inline EpiLayout epi_layout(const Geom &g, int mode, int Ci,
   l.dz = off;
   l.xs = off;
   l.acc = off;
-  if (mode == EPI_BLOCK_BWD) {
-    off = align16(off + sizeof(float) * (size_t)Co * pts);
+  if (mode == EPI_BLOCK_BWD) {   // dz and x of the tile, rows padded to pts + 1
+    off = align16(off + sizeof(float) * (size_t)Co * (pts + 1));
     l.xs = off;
     off = align16(off + sizeof(float) * (size_t)(Ci + 1) * (pts + 1));
     l.acc = off;
-    off = align16(off + sizeof(float) * (size_t)Co * (Ci + 1));
   }
   l.total = off;
   return l;
@@ -70,7 +69,6 @@ __global__ void __launch_bounds__(PTS) k_epilogue(EpiArgs a, Geom g) {
   float *bias_s = reinterpret_cast<float *>(smem + lay.bias);
   float *dz_s = reinterpret_cast<float *>(smem + lay.dz);
   float *x_s = reinterpret_cast<float *>(smem + lay.xs);
-  float *acc_s = reinterpret_cast<float *>(smem + lay.acc);
 
   const int tid = threadIdx.x;
   const int Cs = (MODE <= EPI_BLOCK_FWD) ? Co : Ci;
@@ -99,8 +97,19 @@ __global__ void __launch_bounds__(PTS) k_epilogue(EpiArgs a, Geom g) {
       const int o = e / lay.Wld, i = e - o * lay.Wld;
       Wsm[e] = i < Ci ? to_f<T>(W[o * Ci + i]) : 0.f;
     }
-    for (int e = tid; e < Co * (Ci + 1); e += PTS) acc_s[e] = 0.f;
   }
+  // block backward: this thread's share of dW (a 4 x 8 block of [Co][Ci]) and
+  // of db (row tid), accumulated in registers over all of the CTA's tiles
+  constexpr int OB = 4, IB = 8;
+  const int nib = (Ci + IB - 1) / IB;
+  const int nblk = ((Co + OB - 1) / OB) * nib;
+  const int ob = tid / (nib > 0 ? nib : 1), ib = tid - ob * (nib > 0 ? nib : 1);
+  float accw[OB][IB];
+  float accb = 0.f;
+#pragma unroll
+  for (int k = 0; k < OB; ++k)
+#pragma unroll
+    for (int m = 0; m < IB; ++m) accw[k][m] = 0.f;
 
   for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
     const long long slab = tile / tiles_per_slab;
@@ -119,8 +128,12 @@ __global__ void __launch_bounds__(PTS) k_epilogue(EpiArgs a, Geom g) {
       const int row = r_first + rl;
       const float2 *z = a.Z + (((b * Cs + c) * O + outer) * QS) * (long long)mL + k;
       float2 s = make_float2(0.f, 0.f);
-      KeptIndex ki(QS == 1 ? 0 : g.mS, S, row);
-      for (int q = 0; q < QS; ++q) cfma(s, __ldg(z + (long long)q * mL), twS[ki.next()]);
+      if (a.U) {   // precomputed slab inverse
+        s = a.U[(((b * Cs + c) * O + outer) * (long long)S + row) * mL + k];
+      } else {
+        KeptIndex ki(QS == 1 ? 0 : g.mS, S, row);
+        for (int q = 0; q < QS; ++q) cfma(s, __ldg(z + (long long)q * mL), twS[ki.next()]);
+      }
       U[(rl * mL + k) * Csp + c] = s;
     }
     if (Cs & 1)
@@ -140,7 +153,7 @@ __global__ void __launch_bounds__(PTS) k_epilogue(EpiArgs a, Geom g) {
           const float d = ldf<T>(dy + base_o + o * cstride);
           dz = a.act ? d * gelu_grad_f(ldf<T>(pre + base_o + o * cstride)) : d;
         }
-        dz_s[o * PTS + tid] = dz;
+        dz_s[o * (PTS + 1) + tid] = dz;
       }
       for (int i = 0; i < Ci; ++i)
         x_s[i * (PTS + 1) + tid] = valid ? ldf<T>(x + base_i + i * cstride) : 0.f;
@@ -224,7 +237,7 @@ __global__ void __launch_bounds__(PTS) k_epilogue(EpiArgs a, Geom g) {
           }
         }
         for (int o = 0; o < Co; ++o) {
-          const float dzo = dz_s[o * PTS + tid];
+          const float dzo = dz_s[o * (PTS + 1) + tid];
           const float4 *wp = reinterpret_cast<const float4 *>(Wsm + o * lay.Wld);
 #pragma unroll
           for (int i4 = 0; i4 < CMAX / 4; ++i4) {
@@ -243,22 +256,41 @@ __global__ void __launch_bounds__(PTS) k_epilogue(EpiArgs a, Geom g) {
       }
     }
     if (MODE == EPI_BLOCK_BWD) {
-      // dW[o][i] (i < Ci) and db[o] (i == Ci) partial sums over this tile
-      for (int e = tid; e < Co * (Ci + 1); e += PTS) {
-        const int o = e / (Ci + 1), i = e - o * (Ci + 1);
-        const float *dzr = dz_s + o * PTS;
-        const float *xr = x_s + i * (PTS + 1);
-        float s = 0.f;
-#pragma unroll 8
-        for (int t = 0; t < PTS; ++t) s = fmaf(dzr[t], xr[t], s);
-        acc_s[e] += s;
+      // dW[o][i] += sum_p dz[o][p] x[i][p] over this tile's points (4 x 8
+      // outer products per point from shared memory), db[o] += sum_p dz[o][p]
+      if (tid < nblk) {
+        for (int pp = 0; pp < PTS; ++pp) {
+          float dzv[OB], xv[IB];
+#pragma unroll
+          for (int k = 0; k < OB; ++k)
+            dzv[k] = ob * OB + k < Co ? dz_s[(ob * OB + k) * (PTS + 1) + pp] : 0.f;
+#pragma unroll
+          for (int m = 0; m < IB; ++m)
+            xv[m] = ib * IB + m < Ci ? x_s[(ib * IB + m) * (PTS + 1) + pp] : 0.f;
+#pragma unroll
+          for (int k = 0; k < OB; ++k)
+#pragma unroll
+            for (int m = 0; m < IB; ++m) accw[k][m] = fmaf(dzv[k], xv[m], accw[k][m]);
+        }
+      }
+      if (tid < Co) {
+        const float *dzr = dz_s + tid * (PTS + 1);
+        for (int pp = 0; pp < PTS; ++pp) accb += dzr[pp];
       }
     }
   }
   if (MODE == EPI_BLOCK_BWD) {
-    __syncthreads();
     float *dst = a.partial + (long long)blockIdx.x * Co * (Ci + 1);
-    for (int e = tid; e < Co * (Ci + 1); e += PTS) dst[e] = acc_s[e];
+    if (tid < nblk) {
+#pragma unroll
+      for (int k = 0; k < OB; ++k)
+#pragma unroll
+        for (int m = 0; m < IB; ++m) {
+          const int o = ob * OB + k, i = ib * IB + m;
+          if (o < Co && i < Ci) dst[o * (Ci + 1) + i] = accw[k][m];
+        }
+    }
+    if (tid < Co) dst[tid * (Ci + 1) + Ci] = accb;
   }
 }
 

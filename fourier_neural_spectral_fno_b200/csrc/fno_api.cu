@@ -204,7 +204,8 @@ Launch make_launch(fno_stream_t s) {
 cudaError_t run_epilogue(const Launch &L, const Geom &g, int dtype, int mode, const EpiArgs &a,
                          unsigned char *ws, const BlockWs &w) {
   float2 *U = reinterpret_cast<float2 *>(ws + w.u);
-  const int cs = mode == EPI_SPEC_BWD ? a.Ci : a.Co;
+  // channels of the spectrum being inverted: Ci for the backward modes (dxhat)
+  const int cs = (mode == EPI_SPEC_BWD || mode == EPI_BLOCK_BWD) ? a.Ci : a.Co;
   if (L.tc == 1 && epi_pipe_supported(g, dtype, mode, a.Ci, a.Co, a.x, U)) {
     cudaError_t e = launch_inv_slab(L, g, cs, a.Z, U);
     if (e != cudaSuccess) return e;
@@ -214,6 +215,15 @@ cudaError_t run_epilogue(const Launch &L, const Geom &g, int dtype, int mode, co
     cudaError_t e = launch_inv_slab(L, g, cs, a.Z, U);
     if (e != cudaSuccess) return e;
     return launch_epilogue_tc(L, g, dtype, mode, a, U);
+  }
+  if (mode == EPI_BLOCK_BWD && g.S > 1) {
+    // the block backward reads the slab-axis inverse once per row instead of
+    // recomputing it in every tile
+    cudaError_t e = launch_inv_slab(L, g, cs, a.Z, U);
+    if (e != cudaSuccess) return e;
+    EpiArgs b = a;
+    b.U = U;
+    return launch_epilogue(L, g, dtype, mode, b);
   }
   return launch_epilogue(L, g, dtype, mode, a);
 }

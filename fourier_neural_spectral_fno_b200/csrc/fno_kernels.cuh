@@ -96,6 +96,8 @@ struct EpiArgs {
   void *out;        // y (fwd modes, [B][Co][N]) or dx (bwd modes, [B][Ci][N])
   void *pre_out;    // optional [B][Co][N]
   float *partial;   // bwd: per-CTA partial sums of dW/db, [grid][Co][Ci+1]
+  const float2 *U;  // optional: the spectrum already inverted along the slab axis,
+                    // [B][Cs][O][S][mL] (launch_inv_slab); NULL: computed per tile
   int Ci, Co;
   int act, tanh_pre;
 };
