@@ -275,14 +275,44 @@ __global__ void __launch_bounds__(PB)
       }
       __syncthreads();
       const int hn = min(HC, hidden - hc);
-      for (int e = tid; e < hn * (width + 1); e += PB) {
-        const int hh = e / (width + 1), c = e - hh * (width + 1);
-        const float *dr = dh_s + hh * PB;
-        const float *vrow = v_s + c * (PB + 1);
-        float s = 0.f;
-#pragma unroll 8
-        for (int k = 0; k < PB; ++k) s = fmaf(dr[k], vrow[k], s);
-        acc1[(hc + hh) * (width + 1) + c] += s;
+      {
+        // dQ1[h][c] over this tile's points as 4 x 4 blocks (h, c) per thread:
+        // 8 shared-memory loads feed 16 multiply-adds per point
+        constexpr int HB = 4, CB = 4;
+        const int ncb = (width + CB - 1) / CB;
+        const int nblk = ((hn + HB - 1) / HB) * ncb;
+        for (int blk = tid; blk < nblk; blk += PB) {
+          const int hb = blk / ncb, cb = blk - hb * ncb;
+          float acc[HB][CB];
+#pragma unroll
+          for (int i = 0; i < HB; ++i)
+#pragma unroll
+            for (int j = 0; j < CB; ++j) acc[i][j] = 0.f;
+          for (int k = 0; k < PB; ++k) {
+            float dv4[HB], v4[CB];
+#pragma unroll
+            for (int i = 0; i < HB; ++i) dv4[i] = hb * HB + i < hn ? dh_s[(hb * HB + i) * PB + k] : 0.f;
+#pragma unroll
+            for (int j = 0; j < CB; ++j) v4[j] = cb * CB + j < width ? v_s[(cb * CB + j) * (PB + 1) + k] : 0.f;
+#pragma unroll
+            for (int i = 0; i < HB; ++i)
+#pragma unroll
+              for (int j = 0; j < CB; ++j) acc[i][j] = fmaf(dv4[i], v4[j], acc[i][j]);
+          }
+#pragma unroll
+          for (int i = 0; i < HB; ++i)
+#pragma unroll
+            for (int j = 0; j < CB; ++j)
+              if (hb * HB + i < hn && cb * CB + j < width)
+                acc1[(hc + hb * HB + i) * (width + 1) + cb * CB + j] += acc[i][j];
+        }
+        // bias column: dq1[h] = sum_p dh[h][p]
+        for (int hh = tid; hh < hn; hh += PB) {
+          const float *dr = dh_s + hh * PB;
+          float sacc = 0.f;
+          for (int k = 0; k < PB; ++k) sacc += dr[k];
+          acc1[(hc + hh) * (width + 1) + width] += sacc;
+        }
       }
       for (int e = tid; e < out_ch * hn; e += PB) {
         const int o = e / hn, hh = e - o * hn;
