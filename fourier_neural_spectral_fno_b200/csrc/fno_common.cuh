@@ -138,6 +138,12 @@ __device__ __forceinline__ float norm_cdf(float p) {
   return 0.5f + 0.5f * copysignf(e, p);
 }
 __device__ __forceinline__ float gelu_f(float p) { return p * norm_cdf(p); }
+// GELU and its derivative from one evaluation of the normal CDF
+__device__ __forceinline__ void gelu_and_grad_f(float p, float &g, float &dg) {
+  const float cdf = norm_cdf(p);
+  g = p * cdf;
+  dg = cdf + p * 0.39894228040143267794f * expf(-0.5f * p * p);
+}
 __device__ __forceinline__ float gelu_grad_f(float p) {
   return norm_cdf(p) + p * 0.39894228040143267794f * expf(-0.5f * p * p);
 }

@@ -253,12 +253,13 @@ __global__ void __launch_bounds__(PB)
               z = fmaf(q.w, vr[4 * c4 + 3], z);
             }
           }
-          gz = gelu_f(z);
+          float gp;
+          gelu_and_grad_f(z, gz, gp);
           float dg = 0.f;
 #pragma unroll
           for (int o = 0; o < kMaxOut; ++o)
             if (o < out_ch) dg = fmaf(Q2s[o * hidden + h], dur[o], dg);
-          dh = dg * gelu_grad_f(z);
+          dh = dg * gp;
 #pragma unroll
           for (int c4 = 0; c4 < CMAX / 4; ++c4) {
             if (4 * c4 < width) {
