@@ -185,9 +185,12 @@ __host__ __device__ inline ProjBwdLayout proj_bwd_layout(int width, int hidden, 
 }
 
 // Projection adjoint: dv, and per-CTA partials of dQ1|dq1 ([hidden][width+1])
-// followed by dQ2|dq2 ([out][hidden+1]).
+// followed by dQ2|dq2 ([out][hidden+1]).  Two threads per point of a tile,
+// each taking half of every hidden chunk; their dv contributions meet in
+// shared memory at the end of the tile.
+constexpr int PBT = 2 * PB;   // threads of k_proj_bwd
 template <typename T, int CMAX>
-__global__ void __launch_bounds__(PB)
+__global__ void __launch_bounds__(PBT)
     k_proj_bwd(const T *__restrict__ v, const T *__restrict__ du, const T *__restrict__ Q1,
                const T *__restrict__ q1, const T *__restrict__ Q2, T *__restrict__ dv,
                float *__restrict__ partial, long long B, long long N, int width, int hidden,
@@ -205,19 +208,20 @@ __global__ void __launch_bounds__(PB)
   float *acc1 = reinterpret_cast<float *>(smem + lay.acc1);
   float *acc2 = reinterpret_cast<float *>(smem + lay.acc2);
   const int tid = threadIdx.x;
-  for (int e = tid; e < hidden * ld; e += PB) {
+  const int pt = tid & (PB - 1), half = tid / PB;   // point of the tile, hidden half
+  for (int e = tid; e < hidden * ld; e += PBT) {
     const int h = e / ld, c = e - h * ld;
     Q1s[e] = c < width ? to_f<T>(Q1[h * width + c]) : 0.f;
   }
-  for (int e = tid; e < hidden; e += PB) q1s[e] = to_f<T>(q1[e]);
-  for (int e = tid; e < out_ch * hidden; e += PB) Q2s[e] = to_f<T>(Q2[e]);
-  for (int e = tid; e < hidden * (width + 1); e += PB) acc1[e] = 0.f;
-  for (int e = tid; e < out_ch * (hidden + 1); e += PB) acc2[e] = 0.f;
+  for (int e = tid; e < hidden; e += PBT) q1s[e] = to_f<T>(q1[e]);
+  for (int e = tid; e < out_ch * hidden; e += PBT) Q2s[e] = to_f<T>(Q2[e]);
+  for (int e = tid; e < hidden * (width + 1); e += PBT) acc1[e] = 0.f;
+  for (int e = tid; e < out_ch * (hidden + 1); e += PBT) acc2[e] = 0.f;
 
   const long long total = B * N;
   const long long ntiles = (total + PB - 1) / PB;
   for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    const long long t = tile * PB + tid;
+    const long long t = tile * PB + pt;
     const bool valid = t < total;
     const long long b = valid ? t / N : 0, n = valid ? t - b * N : 0;
     __syncthreads();
@@ -226,18 +230,18 @@ __global__ void __launch_bounds__(PB)
     for (int c = 0; c < CMAX; ++c) {
       vr[c] = (valid && c < width) ? ldf<T>(v + (b * width + c) * N + n) : 0.f;
       dvr[c] = 0.f;
-      if (c < width) v_s[c * (PB + 1) + tid] = vr[c];
+      if (c < width && half == 0) v_s[c * (PB + 1) + pt] = vr[c];
     }
-    v_s[width * (PB + 1) + tid] = valid ? 1.f : 0.f;
+    if (half == 0) v_s[width * (PB + 1) + pt] = valid ? 1.f : 0.f;
     float dur[kMaxOut];
 #pragma unroll
     for (int o = 0; o < kMaxOut; ++o) {
       dur[o] = (valid && o < out_ch) ? ldf<T>(du + (b * out_ch + o) * N + n) : 0.f;
-      if (o < out_ch) du_s[o * PB + tid] = dur[o];
+      if (o < out_ch && half == 0) du_s[o * PB + pt] = dur[o];
     }
     for (int hc = 0; hc < hidden; hc += HC) {
       __syncthreads();  // previous chunk's reductions are done with dh_s / g_s
-      for (int hh = 0; hh < HC; ++hh) {
+      for (int hh = half * (HC / 2); hh < (half + 1) * (HC / 2); ++hh) {
         const int h = hc + hh;
         float dh = 0.f, gz = 0.f;
         if (h < hidden && valid) {
@@ -271,8 +275,8 @@ __global__ void __launch_bounds__(PB)
             }
           }
         }
-        dh_s[hh * PB + tid] = dh;
-        g_s[hh * (PB + 1) + tid] = gz;
+        dh_s[hh * PB + pt] = dh;
+        g_s[hh * (PB + 1) + pt] = gz;
       }
       __syncthreads();
       const int hn = min(HC, hidden - hc);
@@ -282,7 +286,7 @@ __global__ void __launch_bounds__(PB)
         constexpr int HB = 4, CB = 4;
         const int ncb = (width + CB - 1) / CB;
         const int nblk = ((hn + HB - 1) / HB) * ncb;
-        for (int blk = tid; blk < nblk; blk += PB) {
+        for (int blk = tid; blk < nblk; blk += PBT) {
           const int hb = blk / ncb, cb = blk - hb * ncb;
           float acc[HB][CB];
 #pragma unroll
@@ -308,14 +312,14 @@ __global__ void __launch_bounds__(PB)
                 acc1[(hc + hb * HB + i) * (width + 1) + cb * CB + j] += acc[i][j];
         }
         // bias column: dq1[h] = sum_p dh[h][p]
-        for (int hh = tid; hh < hn; hh += PB) {
+        for (int hh = tid; hh < hn; hh += PBT) {
           const float *dr = dh_s + hh * PB;
           float sacc = 0.f;
           for (int k = 0; k < PB; ++k) sacc += dr[k];
           acc1[(hc + hh) * (width + 1) + width] += sacc;
         }
       }
-      for (int e = tid; e < out_ch * hn; e += PB) {
+      for (int e = tid; e < out_ch * hn; e += PBT) {
         const int o = e / hn, hh = e - o * hn;
         const float *dr = du_s + o * PB;
         const float *gr = g_s + hh * (PB + 1);
@@ -325,22 +329,32 @@ __global__ void __launch_bounds__(PB)
         acc2[o * (hidden + 1) + hc + hh] += s;
       }
     }
-    for (int o = tid; o < out_ch; o += PB) {
+    for (int o = tid; o < out_ch; o += PBT) {
       float s = 0.f;
       for (int k = 0; k < PB; ++k) s += du_s[o * PB + k];
       acc2[o * (hidden + 1) + hidden] += s;
     }
-    if (valid) {
+    // the two halves' dv meet in the dh_s / g_s region (free after the last
+    // chunk's reductions; it holds CMAX x PB floats)
+    __syncthreads();
+    float *dvx = dh_s;
+    if (half == 1) {
 #pragma unroll
       for (int c = 0; c < CMAX; ++c)
-        if (c < width) dv[(b * width + c) * N + n] = from_f<T>(dvr[c]);
+        if (c < width) dvx[c * PB + pt] = dvr[c];
+    }
+    __syncthreads();
+    if (half == 0 && valid) {
+#pragma unroll
+      for (int c = 0; c < CMAX; ++c)
+        if (c < width) dv[(b * width + c) * N + n] = from_f<T>(dvr[c] + dvx[c * PB + pt]);
     }
   }
   __syncthreads();
   const long long stride = (long long)hidden * (width + 1) + (long long)out_ch * (hidden + 1);
   float *dst = partial + blockIdx.x * stride;
-  for (int e = tid; e < hidden * (width + 1); e += PB) dst[e] = acc1[e];
-  for (int e = tid; e < out_ch * (hidden + 1); e += PB) dst[hidden * (width + 1) + e] = acc2[e];
+  for (int e = tid; e < hidden * (width + 1); e += PBT) dst[e] = acc1[e];
+  for (int e = tid; e < out_ch * (hidden + 1); e += PBT) dst[hidden * (width + 1) + e] = acc2[e];
 }
 
 // Lift adjoint: per-CTA partials of dP|dp ([width][in+1]).
@@ -500,7 +514,7 @@ static cudaError_t proj_bwd_t(const Launch &L, const Geom &g, int width, int hid
   const size_t smem = proj_bwd_layout(width, hidden, out_ch).total;
   auto kern = k_proj_bwd<T, CMAX>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  kern<<<grid, PB, smem, L.stream>>>((const T *)v, (const T *)du, (const T *)Q1, (const T *)q1,
+  kern<<<grid, PBT, smem, L.stream>>>((const T *)v, (const T *)du, (const T *)Q1, (const T *)q1,
                                      (const T *)Q2, (T *)dv, partial, g.B, g.N, width, hidden,
                                      out_ch);
   return cudaGetLastError();
