@@ -46,7 +46,21 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="bound on the CPU-oracle sample of the fno arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (smaller cases for profiler captures)")
     return ap.parse_args()
+
+
+def resolve_workload(args):
+    import dataclasses
+
+    from fourier_neural_spectral_fno_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    if args.batch is not None:
+        if args.batch < 1:
+            raise SystemExit("--batch must be >= 1")
+        wl = dataclasses.replace(wl, batch=args.batch)
+    return wl
 
 
 # --------------------------------------------------------------------------
@@ -274,7 +288,7 @@ def cpu_baseline(wl, inp, seconds):
 
 def run_reference(args, dist):
     from fourier_neural_spectral_fno_b200 import synth
-    wl = synth.WORKLOADS[args.workload]
+    wl = resolve_workload(args)
     if dist.rank != 0:
         return
     inp = synth.make_network_inputs(wl)
@@ -304,7 +318,7 @@ def run_fno(args, dist):
 
     from fourier_neural_spectral_fno_b200 import capi, synth
 
-    wl = synth.WORKLOADS[args.workload]
+    wl = resolve_workload(args)
     torch.cuda.set_device(dist.local)
     dev = torch.device("cuda", dist.local)
     capi.load()

@@ -16,6 +16,35 @@ namespace {
 
 constexpr int EP_FWD_PTS = 256;
 constexpr int EP_BWD_PTS = 128;
+constexpr int EP_BATCH = 8;   // 16-byte loads a thread keeps in flight per array
+
+// the 16 / sizeof(T) storage elements of a 16-byte chunk, as floats
+template <typename T> __device__ __forceinline__ void unpack16(const uint4 &v, float *f);
+template <> __device__ __forceinline__ void unpack16<float>(const uint4 &v, float *f) {
+  f[0] = __uint_as_float(v.x);
+  f[1] = __uint_as_float(v.y);
+  f[2] = __uint_as_float(v.z);
+  f[3] = __uint_as_float(v.w);
+}
+template <> __device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4 &v, float *f) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+template <> __device__ __forceinline__ void unpack16<__half>(const uint4 &v, float *f) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __half2 h;
+    memcpy(&h, &w[i], 4);
+    const float2 t = __half22float2(h);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
 
 __host__ __device__ inline size_t align16(size_t v) { return (v + 15) & ~(size_t)15; }
 
@@ -111,6 +140,14 @@ __global__ void __launch_bounds__(PTS) k_epilogue(EpiArgs a, Geom g) {
 #pragma unroll
     for (int m = 0; m < IB; ++m) accw[k][m] = 0.f;
 
+  // 16-byte vector loads: aligned bases and rows whose length is a multiple of
+  // the chunk (every chunk then lies wholly inside or wholly past the end)
+  const bool u_vec = a.U != nullptr && mL % 2 == 0 &&
+                     (reinterpret_cast<uintptr_t>(a.U) & 15) == 0;
+  const bool io_vec = MODE == EPI_BLOCK_BWD && SN % (16 / (int)sizeof(T)) == 0 &&
+                      ((reinterpret_cast<uintptr_t>(a.x) | reinterpret_cast<uintptr_t>(a.dy) |
+                        (a.act ? reinterpret_cast<uintptr_t>(a.pre) : 0)) & 15) == 0;
+
   for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
     const long long slab = tile / tiles_per_slab;
     const long long p0 = (tile - slab * tiles_per_slab) * (long long)PTS;
@@ -121,6 +158,33 @@ __global__ void __launch_bounds__(PTS) k_epilogue(EpiArgs a, Geom g) {
     const int nr = r_last - r_first + 1;
     __syncthreads();  // previous tile is done with U / dz_s / x_s
     // slab-axis inverse for the rows of this tile: U[row][k][c]
+    if (u_vec) {
+      // precomputed slab inverse: the tile's rows of one channel are nr * mL
+      // consecutive values; 16-byte chunks (two modes), a batch in flight
+      const int h = nr * mL / 2, nu = Cs * h;
+      for (int e0 = tid; e0 < nu; e0 += EP_BATCH * PTS) {
+        float4 v[EP_BATCH];
+#pragma unroll
+        for (int m = 0; m < EP_BATCH; ++m) {
+          const int e = e0 + m * PTS;
+          if (e < nu) {
+            const int c = e / h, kk = e - c * h;
+            const float4 *src = reinterpret_cast<const float4 *>(
+                a.U + (((b * Cs + c) * O + outer) * (long long)S + r_first) * mL);
+            v[m] = __ldg(src + kk);
+          }
+        }
+#pragma unroll
+        for (int m = 0; m < EP_BATCH; ++m) {
+          const int e = e0 + m * PTS;
+          if (e < nu) {
+            const int c = e / h, kk = e - c * h;
+            U[(2 * kk) * Csp + c] = make_float2(v[m].x, v[m].y);
+            U[(2 * kk + 1) * Csp + c] = make_float2(v[m].z, v[m].w);
+          }
+        }
+      }
+    } else
     for (int e = tid; e < nr * mL * Cs; e += PTS) {
       const int k = e % mL;
       const int rest = e / mL;
@@ -144,7 +208,53 @@ __global__ void __launch_bounds__(PTS) k_epilogue(EpiArgs a, Geom g) {
     const long long base_o = (b * Co * O + outer) * SN + pt;  // + o * O * SN
     const long long base_i = (b * Ci * O + outer) * SN + pt;  // + i * O * SN
     const long long cstride = (long long)O * SN;
-    if (MODE == EPI_BLOCK_BWD) {
+    if (MODE == EPI_BLOCK_BWD && io_vec) {
+      // dz = dy * GELU'(pre) and x of the tile from 16-byte chunks of VEC
+      // consecutive points of one channel; a batch of chunks of all three
+      // arrays in flight per thread, points past the end read as zeros
+      constexpr int VEC = 16 / sizeof(T), CPR = PTS / VEC;
+      const T *dy = reinterpret_cast<const T *>(a.dy);
+      const T *pre = reinterpret_cast<const T *>(a.pre);
+      const int ndz = Co * CPR, nxc = Ci * CPR, nmax = ndz > nxc ? ndz : nxc;
+      const long long bo = (b * Co * O + outer) * SN + p0, bi = (b * Ci * O + outer) * SN + p0;
+      for (int c0 = tid; c0 < nmax; c0 += EP_BATCH * PTS) {
+        uint4 vd[EP_BATCH], vp[EP_BATCH], vx[EP_BATCH];
+#pragma unroll
+        for (int m = 0; m < EP_BATCH; ++m) {
+          const int c = c0 + m * PTS;
+          const int row = c / CPR, q = c - row * CPR;
+          const bool in = p0 + q * VEC < SN;
+          vd[m] = vp[m] = vx[m] = make_uint4(0u, 0u, 0u, 0u);
+          if (in && c < ndz) {
+            const long long off = bo + row * cstride + q * VEC;
+            vd[m] = __ldg(reinterpret_cast<const uint4 *>(dy + off));
+            if (a.act) vp[m] = __ldg(reinterpret_cast<const uint4 *>(pre + off));
+          }
+          if (in && c < nxc)
+            vx[m] = __ldg(reinterpret_cast<const uint4 *>(x + bi + row * cstride + q * VEC));
+        }
+#pragma unroll
+        for (int m = 0; m < EP_BATCH; ++m) {
+          const int c = c0 + m * PTS;
+          const int row = c / CPR, q = c - row * CPR;
+          if (c < ndz) {
+            float d[VEC], pv[VEC];
+            unpack16<T>(vd[m], d);
+            unpack16<T>(vp[m], pv);
+            float *dst = dz_s + row * (PTS + 1) + q * VEC;
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) dst[i] = a.act ? d[i] * gelu_grad_f(pv[i]) : d[i];
+          }
+          if (c < nxc) {
+            float xv[VEC];
+            unpack16<T>(vx[m], xv);
+            float *dst = x_s + row * (PTS + 1) + q * VEC;
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) dst[i] = xv[i];
+          }
+        }
+      }
+    } else if (MODE == EPI_BLOCK_BWD) {
       const T *dy = reinterpret_cast<const T *>(a.dy);
       const T *pre = reinterpret_cast<const T *>(a.pre);
       for (int o = 0; o < Co; ++o) {
