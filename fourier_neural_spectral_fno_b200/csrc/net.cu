@@ -174,7 +174,10 @@ __host__ __device__ inline ProjBwdLayout proj_bwd_layout(int width, int hidden, 
   l.Q1s = off; off += sizeof(float) * (size_t)hidden * l.ld;
   l.q1s = off; off += sizeof(float) * hidden;
   l.Q2s = off; off += sizeof(float) * (size_t)out_ch * hidden;
-  l.vs = off; off += sizeof(float) * (size_t)(width + 1) * (PB + 1);
+  // v rows: width channels, the ones row, and pad rows up to a multiple of 4
+  // (read only by dQ1 blocks whose entries are discarded)
+  const int vrows = ((width + 3) & ~3) > width + 1 ? ((width + 3) & ~3) : width + 1;
+  l.vs = off; off += sizeof(float) * (size_t)vrows * (PB + 1);
   l.dus = off; off += sizeof(float) * (size_t)out_ch * PB;
   l.dhs = off; off += sizeof(float) * (size_t)HC * PB;
   l.gs = off; off += sizeof(float) * (size_t)HC * (PB + 1);
@@ -246,17 +249,19 @@ __global__ void __launch_bounds__(PBT)
         float dh = 0.f, gz = 0.f;
         if (h < hidden && valid) {
           const float4 *qp = reinterpret_cast<const float4 *>(Q1s + h * ld);
-          float z = q1s[h];
+          // four independent partial sums keep the FMA pipe busy
+          float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
 #pragma unroll
           for (int c4 = 0; c4 < CMAX / 4; ++c4) {
             if (4 * c4 < width) {
               const float4 q = qp[c4];
-              z = fmaf(q.x, vr[4 * c4], z);
-              z = fmaf(q.y, vr[4 * c4 + 1], z);
-              z = fmaf(q.z, vr[4 * c4 + 2], z);
-              z = fmaf(q.w, vr[4 * c4 + 3], z);
+              z0 = fmaf(q.x, vr[4 * c4], z0);
+              z1 = fmaf(q.y, vr[4 * c4 + 1], z1);
+              z2 = fmaf(q.z, vr[4 * c4 + 2], z2);
+              z3 = fmaf(q.w, vr[4 * c4 + 3], z3);
             }
           }
+          const float z = q1s[h] + ((z0 + z1) + (z2 + z3));
           float gp;
           gelu_and_grad_f(z, gz, gp);
           float dg = 0.f;
@@ -286,19 +291,24 @@ __global__ void __launch_bounds__(PBT)
         constexpr int HB = 4, CB = 4;
         const int ncb = (width + CB - 1) / CB;
         const int nblk = ((hn + HB - 1) / HB) * ncb;
+        // (dh rows past the chunk are zeros; v pad rows only reach discarded
+        // entries, so the loads need no guards)
         for (int blk = tid; blk < nblk; blk += PBT) {
           const int hb = blk / ncb, cb = blk - hb * ncb;
+          const float *dp = dh_s + hb * HB * PB;
+          const float *vp = v_s + cb * CB * (PB + 1);
           float acc[HB][CB];
 #pragma unroll
           for (int i = 0; i < HB; ++i)
 #pragma unroll
             for (int j = 0; j < CB; ++j) acc[i][j] = 0.f;
+#pragma unroll 4
           for (int k = 0; k < PB; ++k) {
             float dv4[HB], v4[CB];
 #pragma unroll
-            for (int i = 0; i < HB; ++i) dv4[i] = hb * HB + i < hn ? dh_s[(hb * HB + i) * PB + k] : 0.f;
+            for (int i = 0; i < HB; ++i) dv4[i] = dp[i * PB + k];
 #pragma unroll
-            for (int j = 0; j < CB; ++j) v4[j] = cb * CB + j < width ? v_s[(cb * CB + j) * (PB + 1) + k] : 0.f;
+            for (int j = 0; j < CB; ++j) v4[j] = vp[j * (PB + 1) + k];
 #pragma unroll
             for (int i = 0; i < HB; ++i)
 #pragma unroll
@@ -311,22 +321,33 @@ __global__ void __launch_bounds__(PBT)
               if (hb * HB + i < hn && cb * CB + j < width)
                 acc1[(hc + hb * HB + i) * (width + 1) + cb * CB + j] += acc[i][j];
         }
-        // bias column: dq1[h] = sum_p dh[h][p]
-        for (int hh = tid; hh < hn; hh += PBT) {
-          const float *dr = dh_s + hh * PB;
-          float sacc = 0.f;
-          for (int k = 0; k < PB; ++k) sacc += dr[k];
-          acc1[(hc + hh) * (width + 1) + width] += sacc;
+        // bias column dq1[h] = sum_p dh[h][p] and dQ2[o][h] = sum_p du[o][p]
+        // g[h][p], on the highest threads (idle during the dQ1 blocks), four
+        // partial sums each
+        for (int e = PBT - 1 - tid; e < hn + out_ch * hn; e += PBT) {
+          float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+          if (e < hn) {
+            const float *dr = dh_s + e * PB;
+            for (int k = 0; k < PB; k += 4) {
+              s0 += dr[k];
+              s1 += dr[k + 1];
+              s2 += dr[k + 2];
+              s3 += dr[k + 3];
+            }
+            acc1[(hc + e) * (width + 1) + width] += (s0 + s1) + (s2 + s3);
+          } else {
+            const int o = (e - hn) / hn, hh = e - hn - o * hn;
+            const float *dr = du_s + o * PB;
+            const float *gr = g_s + hh * (PB + 1);
+            for (int k = 0; k < PB; k += 4) {
+              s0 = fmaf(dr[k], gr[k], s0);
+              s1 = fmaf(dr[k + 1], gr[k + 1], s1);
+              s2 = fmaf(dr[k + 2], gr[k + 2], s2);
+              s3 = fmaf(dr[k + 3], gr[k + 3], s3);
+            }
+            acc2[o * (hidden + 1) + hc + hh] += (s0 + s1) + (s2 + s3);
+          }
         }
-      }
-      for (int e = tid; e < out_ch * hn; e += PBT) {
-        const int o = e / hn, hh = e - o * hn;
-        const float *dr = du_s + o * PB;
-        const float *gr = g_s + hh * (PB + 1);
-        float s = 0.f;
-#pragma unroll 8
-        for (int k = 0; k < PB; ++k) s = fmaf(dr[k], gr[k], s);
-        acc2[o * (hidden + 1) + hc + hh] += s;
       }
     }
     for (int o = tid; o < out_ch; o += PBT) {
