@@ -55,7 +55,14 @@ def resolve_workload(args):
     import dataclasses
 
     from fourier_neural_spectral_fno_b200 import synth
+    if args.workload not in synth.WORKLOADS:
+        raise SystemExit(f"unknown workload {args.workload!r}; one of: "
+                         + ", ".join(synth.WORKLOAD_ORDER))
     wl = synth.WORKLOADS[args.workload]
+    if wl.kind != "network":
+        nets = [n for n in synth.WORKLOAD_ORDER if synth.WORKLOADS[n].kind == "network"]
+        raise SystemExit(f"workload {args.workload!r} is a single-block parity case; bench.py "
+                         "times network workloads: " + ", ".join(nets))
     if args.batch is not None:
         if args.batch < 1:
             raise SystemExit("--batch must be >= 1")
