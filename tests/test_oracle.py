@@ -223,6 +223,31 @@ def test_adjoint_identity(grid, modes):
     np.testing.assert_allclose(lhs, rhs, rtol=1e-12)
 
 
+@pytest.mark.parametrize("grid,modes", [((8, 6), (3, 3)), ((5, 4, 6), (2, 1, 2))])
+def test_kept_mode_storage_order_single_modes(grid, modes):
+    """Storage order of K from single-mode inputs: on a non-last axis the kept
+    rows are the positive block 0..m-1 and then the negative block -m..-1
+    (= N-m..N-1), row-major over the axes.  x = cos(theta(k*, n)) has the
+    spectrum (N/2)(delta(k*) + delta(-k*)); with k*_last >= 1 only k* is kept,
+    so exactly one stored entry is N/2 and it sits at k*'s slot."""
+    d = len(grid)
+    n_total = int(np.prod(grid))
+    # signed wavenumbers of each axis in the documented storage order
+    rows = [list(range(m)) + list(range(-m, 0)) for m in modes[:-1]] + [list(range(modes[-1]))]
+    shape = tuple(len(r) for r in rows)
+    idx = np.indices(grid)
+    for slot in np.ndindex(*shape):
+        k_signed = [rows[j][slot[j]] for j in range(d)]
+        if k_signed[-1] == 0:
+            continue
+        phase = sum(2 * np.pi * k_signed[j] * idx[j] / grid[j] for j in range(d))
+        x = np.cos(phase)[None, None]
+        got = O.truncated_dft(x, modes).ravel()
+        expect = np.zeros(len(got), complex)
+        expect[np.ravel_multi_index(slot, shape)] = n_total / 2
+        np.testing.assert_allclose(got, expect, atol=1e-9, err_msg=str(k_signed))
+
+
 def test_mode_weights_odd_and_even_last_axis():
     np.testing.assert_array_equal(O.mode_weights((8,), (5,)), [1, 2, 2, 2, 1])
     np.testing.assert_array_equal(O.mode_weights((9,), (5,)), [1, 2, 2, 2, 2])
