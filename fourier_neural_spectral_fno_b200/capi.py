@@ -44,7 +44,7 @@ EXPORTED = (
     "fno_net_workspace_size", "fno_net_saves_size", "fno_spectral_conv_fwd",
     "fno_spectral_conv_bwd", "fno_block_fwd", "fno_block_bwd", "fno_forward", "fno_backward",
     "fno_mse", "fno_profile_enable", "fno_profile_read", "fno_set_tensor_cores",
-    "fno_device_error", "fno_spectral_conv_fwd_noalloc",
+    "fno_device_error", "fno_spectral_conv_fwd_noalloc", "fno_adam_step",
 )
 
 FNO_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -126,6 +126,9 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "fno_spectral_conv_fwd_noalloc": (i, [bd, vp, vp, vp, vp, vp]),
         "fno_device_error": (i, [i]),
         "fno_profile_read": (i, [ctypes.POINTER(KernelStat), i]),
+        "fno_adam_step": (i, [ctypes.c_int64, vp, vp, vp, vp, vp, i, i, ctypes.c_float,
+                              ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_float,
+                              ctypes.c_float, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -342,3 +345,24 @@ def fno_spectral_conv_fwd_noalloc(desc, x, R, y, xhat_save=None, stream=None):
     _check(load().fno_spectral_conv_fwd_noalloc(ctypes.byref(desc), _ptr(x), _ptr(R), _ptr(y),
                                                 _ptr(xhat_save), _stream(stream)))
     return y
+
+
+def _dtype_code_of(t) -> int:
+    import torch
+    codes = {torch.float32: FNO_F32, torch.float16: FNO_F16, torch.bfloat16: FNO_BF16}
+    if t.dtype not in codes:
+        raise ValueError(f"param_out dtype {t.dtype} is not a storage dtype")
+    return codes[t.dtype]
+
+
+def fno_adam_step(theta, m, v, grad, param_out, step: int, lr: float, beta1: float = 0.9,
+                  beta2: float = 0.999, eps: float = 1e-8, weight_decay: float = 0.0,
+                  grad_scale: float = 1.0, stream=None):
+    """One Adam step on the float32 master ``theta`` (with moments ``m``, ``v``)
+    fused with the copy into ``param_out`` (its torch dtype is the storage
+    dtype).  ``grad=None``: copy only; ``param_out=None``: update only."""
+    out_code = _dtype_code_of(param_out) if param_out is not None else FNO_F32
+    _check(load().fno_adam_step(theta.numel(), _ptr(theta), _ptr(m), _ptr(v), _ptr(grad),
+                                _ptr(param_out), out_code, int(step), float(lr), float(beta1),
+                                float(beta2), float(eps), float(weight_decay), float(grad_scale),
+                                _stream(stream)))

@@ -1,6 +1,7 @@
 // C ABI of the FNO library (include/fno.h): argument validation, workspace
 // layout and the launch sequence of each operation.  All arithmetic runs in
 // the kernels of transform.cu, mix.cu, epilogue.cu and net.cu.
+#include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
@@ -753,6 +754,48 @@ int fno_mse(int64_t n, int dtype, const void *u, const void *target, float *loss
   OPTIONAL_PTR(du, "du");
   Launch L = make_launch(stream);
   FNO_TRY(launch_mse(L, n, dtype, u, target, loss, du), "mse");
+  g_err[0] = 0;
+  return FNO_OK;
+}
+
+int fno_adam_step(int64_t n, float *theta, float *m, float *v, const float *grad,
+                  void *param_out, int out_dtype, int step, float lr, float beta1, float beta2,
+                  float eps, float weight_decay, float grad_scale, fno_stream_t stream) {
+  if (n < 1) return fail(FNO_ERR_INVALID_ARG, "n %lld < 1", (long long)n);
+  REQUIRE_PTR(theta, "theta");
+  OPTIONAL_PTR(param_out, "param_out");
+  if (param_out && (out_dtype < FNO_F32 || out_dtype > FNO_BF16))
+    return fail(FNO_ERR_INVALID_ARG, "out_dtype %d unknown", out_dtype);
+  AdamCoef c{};
+  if (grad) {
+    REQUIRE_PTR(grad, "grad");
+    REQUIRE_PTR(m, "m");
+    REQUIRE_PTR(v, "v");
+    if (step < 1) return fail(FNO_ERR_INVALID_ARG, "step %d < 1", step);
+    if (!(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f))
+      return fail(FNO_ERR_INVALID_ARG, "betas (%g, %g) not in [0, 1)", beta1, beta2);
+    if (!(eps > 0.f) || !isfinite(eps)) return fail(FNO_ERR_INVALID_ARG, "eps %g <= 0", eps);
+    if (!(lr >= 0.f) || !isfinite(lr)) return fail(FNO_ERR_INVALID_ARG, "lr %g < 0", lr);
+    if (!(weight_decay >= 0.f) || !isfinite(weight_decay))
+      return fail(FNO_ERR_INVALID_ARG, "weight_decay %g < 0", weight_decay);
+    if (!isfinite(grad_scale)) return fail(FNO_ERR_INVALID_ARG, "grad_scale is not finite");
+    c.lr = lr;
+    c.beta1 = beta1;
+    c.beta2 = beta2;
+    c.one_minus_beta1 = (float)(1.0 - (double)beta1);
+    c.one_minus_beta2 = (float)(1.0 - (double)beta2);
+    c.inv_bc1 = (float)(1.0 / (1.0 - pow((double)beta1, (double)step)));
+    c.inv_bc2 = (float)(1.0 / (1.0 - pow((double)beta2, (double)step)));
+    c.eps = eps;
+    c.lr_wd = (float)((double)lr * (double)weight_decay);
+    c.grad_scale = grad_scale;
+  } else if (!param_out) {
+    return fail(FNO_ERR_INVALID_ARG, "neither grad nor param_out given: nothing to do");
+  }
+  Launch L = make_launch(stream);
+  FNO_TRY(launch_adam(L, n, theta, grad ? m : nullptr, grad ? v : nullptr, grad, param_out,
+                      out_dtype, c),
+          "adam");
   g_err[0] = 0;
   return FNO_OK;
 }

@@ -162,4 +162,14 @@ cudaError_t launch_lift_bwd(const Launch &L, const Geom &g, int dtype, int in_ch
 cudaError_t launch_mse(const Launch &L, long long n, int dtype, const void *u, const void *t,
                        float *loss, void *du);
 
+// Adam on float32 master weights fused with their storage-dtype copy
+// (optim.cu).  g == nullptr: copy only; out == nullptr: update only.
+struct AdamCoef {
+  float lr, beta1, beta2, one_minus_beta1, one_minus_beta2;
+  float inv_bc1, inv_bc2;   // 1 / (1 - beta^t)
+  float eps, lr_wd, grad_scale;
+};
+cudaError_t launch_adam(const Launch &L, long long n, float *theta, float *m, float *v,
+                        const float *g, void *out, int out_dtype, const AdamCoef &c);
+
 }  // namespace fno

@@ -262,6 +262,28 @@ int fno_backward(const fno_net_desc *desc, const void *a, const fno_params *para
 int fno_mse(int64_t n, int dtype, const void *u, const void *target, float *loss, void *du,
             fno_stream_t stream);
 
+/* One optimiser step of the training loop over n float32 master weights, fused
+ * with the copy the next forward reads.  Adam (Kingma and Ba, "Adam: A Method
+ * for Stochastic Optimization", Algorithm 1) with decoupled weight decay
+ * (Loshchilov and Hutter, "Decoupled Weight Decay Regularization"); the copy's
+ * dtype carries the precision schedule of [MPTRAIN] (mixed, then full
+ * precision):
+ *   g = grad * grad_scale;  m = beta1 m + (1 - beta1) g;  v = beta2 v + (1 - beta2) g^2
+ *   theta -= lr (m / (1 - beta1^step)) / (sqrt(v / (1 - beta2^step)) + eps)
+ *            + lr weight_decay theta
+ *   param_out = theta rounded to out_dtype (round to nearest even)
+ * theta, m, v [n] float32 device, updated in place; grad [n] float32 device;
+ * param_out [n] device in out_dtype (enum fno_dtype), may be NULL.  grad NULL
+ * copies theta to param_out without an update (m, v, step and the
+ * hyper-parameters are then ignored).  step >= 1 is the 1-based step number;
+ * 0 <= beta < 1, eps > 0, lr >= 0, weight_decay >= 0.  Pointers 16-byte
+ * aligned; param_out overlaps none of theta, m, v, grad.  A flat buffer
+ * holding all of fno_params (each parameter at a 16-byte aligned offset) is
+ * updated in one call. */
+int fno_adam_step(int64_t n, float *theta, float *m, float *v, const float *grad,
+                  void *param_out, int out_dtype, int step, float lr, float beta1, float beta2,
+                  float eps, float weight_decay, float grad_scale, fno_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -40,6 +40,18 @@ Readings (where the pages are silent):
 4. tanh pre-activation feeds the spectral branch only; the 1x1 path sees raw x.
 5. Complex gradient convention: ``dZ = dL/dRe Z + i dL/dIm Z``.
 
+Training loop (the precision-scheduling step of [MPTRAIN]): the summary page
+says training may move from mixed to full precision part-way through.  It fixes
+neither the optimiser nor the switch point; the readings are
+
+6. Optimiser: Adam (Kingma and Ba, "Adam: A Method for Stochastic
+   Optimization", Algorithm 1) on float32 master weights, with optional
+   decoupled weight decay (Loshchilov and Hutter, "Decoupled Weight Decay
+   Regularization"); the step runs on the master copy and the next forward
+   reads it rounded to that step's storage dtype.
+7. Schedule: a list of (first step, storage dtype) phases; by default the first
+   half of the steps in half precision, then float32.
+
 Parity pins: ``tests/test_oracle.py`` (closed forms, invariants, brute force,
 library DFT, finite differences, hand-derived fixtures under ``tests/golden``).
 """
@@ -321,3 +333,117 @@ def mse(u, target):
     """``L = mean((u - t)^2)`` over every element and ``dL/du = 2 (u - t) / numel``."""
     diff = np.asarray(u, np.float64) - np.asarray(target, np.float64)
     return float(np.mean(diff * diff)), 2.0 * diff / diff.size
+
+
+# --------------------------------------------------------------------------
+# training loop with a precision schedule (readings 6 and 7)
+# --------------------------------------------------------------------------
+
+def round_to_storage(x, dtype: str) -> np.ndarray:
+    """Round to the storage dtype (round to nearest, ties to even); float64 out."""
+    x = np.asarray(x, np.float64)
+    if dtype == "f32":
+        return x.astype(np.float32).astype(np.float64)
+    if dtype == "f16":
+        return x.astype(np.float16).astype(np.float64)
+    if dtype == "bf16":
+        bits = x.astype(np.float32).view(np.uint32).astype(np.uint64)
+        keep = bits >> 16                      # the upper 16 bits survive
+        rest = bits & 0xFFFF                   # the dropped half
+        up = (rest > 0x8000) | ((rest == 0x8000) & (keep & 1 == 1))
+        keep = keep + up.astype(np.uint64)
+        return ((keep << 16) & 0xFFFFFFFF).astype(np.uint32).view(np.float32).astype(np.float64)
+    raise ValueError(dtype)
+
+
+def adam_update(theta, m, v, g, t: int, lr: float, beta1: float = 0.9, beta2: float = 0.999,
+                eps: float = 1e-8, weight_decay: float = 0.0):
+    """One Adam step at step number ``t`` (1-based), reading 6.
+
+    ``m = b1 m + (1 - b1) g``; ``v = b2 v + (1 - b2) g^2``;
+    ``theta -= lr (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps) + lr wd theta``.
+    Returns ``(theta, m, v)``.
+    """
+    theta = np.asarray(theta, np.float64)
+    g = np.asarray(g, np.float64)
+    m = beta1 * np.asarray(m, np.float64) + (1.0 - beta1) * g
+    v = beta2 * np.asarray(v, np.float64) + (1.0 - beta2) * g * g
+    m_hat = m / (1.0 - beta1 ** t)
+    v_hat = v / (1.0 - beta2 ** t)
+    theta = theta - lr * m_hat / (np.sqrt(v_hat) + eps) - lr * weight_decay * theta
+    return theta, m, v
+
+
+def dtype_at(phases, step: int) -> str:
+    """Storage dtype of ``step`` under ``phases`` = [(first step, dtype), ...] (reading 7)."""
+    current = None
+    for start, dtype in phases:
+        if start <= step:
+            current = dtype
+    if current is None:
+        raise ValueError("no phase covers step %d" % step)
+    return current
+
+
+_PARAM_KEYS = ("P", "p", "Q1", "q1", "Q2", "q2")
+_LAYER_KEYS = ("R", "W", "b")
+
+
+def _map_params(fn, *trees):
+    out = {}
+    for key in _PARAM_KEYS:
+        out[key] = fn(*[t[key] for t in trees])
+    for key in _LAYER_KEYS:
+        out[key] = [fn(*xs) for xs in zip(*[t[key] for t in trees])]
+    return out
+
+
+def _round_param(x, dtype):
+    x = np.asarray(x)
+    if np.iscomplexobj(x):
+        return round_to_storage(x.real, dtype) + 1j * round_to_storage(x.imag, dtype)
+    return round_to_storage(x, dtype)
+
+
+def train(a, target, params, modes, phases, steps: int, lr: float, beta1: float = 0.9,
+          beta2: float = 0.999, eps: float = 1e-8, weight_decay: float = 0.0, flags: int = 0):
+    """``steps`` Adam steps of the network on one batch under a precision schedule.
+
+    Step ``t`` (0-based) reads the master parameters and the inputs rounded to
+    ``dtype_at(phases, t)``, takes the MSE gradient of :func:`forward` there and
+    applies :func:`adam_update` (step number ``t + 1``) to the float64 master
+    copy.  Complex weights are updated as (re, im) pairs.  Returns
+    ``(master params, losses)``.
+    """
+    master = _map_params(lambda x: np.array(x, dtype=np.complex128 if np.iscomplexobj(x)
+                                            else np.float64), params)
+    mom = _map_params(np.zeros_like, master)      # complex weights: (re, im) moments
+    vel = _map_params(np.zeros_like, master)
+    losses = []
+    for t in range(steps):
+        dt = dtype_at(phases, t)
+        q = _map_params(lambda x: _round_param(x, dt), master)
+        a_q, t_q = round_to_storage(a, dt), round_to_storage(target, dt)
+        u, saves = forward(a_q, q, modes, flags, save=True)
+        loss, du = mse(u, t_q)
+        losses.append(loss)
+        grads = backward(a_q, q, saves, du, modes, flags)
+
+        def upd(th, mm, vv, gg, step=t + 1):
+            if np.iscomplexobj(th):   # real and imaginary parts are separate parameters
+                re = adam_update(th.real, mm.real, vv.real, np.real(gg), step, lr, beta1, beta2,
+                                 eps, weight_decay)
+                im = adam_update(th.imag, mm.imag, vv.imag, np.imag(gg), step, lr, beta1, beta2,
+                                 eps, weight_decay)
+                return re[0] + 1j * im[0], re[1] + 1j * im[1], re[2] + 1j * im[2]
+            return adam_update(th, mm, vv, gg, step, lr, beta1, beta2, eps, weight_decay)
+
+        new = {}
+        for key in _PARAM_KEYS:
+            new[key] = upd(master[key], mom[key], vel[key], grads[key])
+        for key in _LAYER_KEYS:
+            new[key] = [upd(*xs) for xs in zip(master[key], mom[key], vel[key], grads[key])]
+        master = {k: ([x[0] for x in v] if isinstance(v, list) else v[0]) for k, v in new.items()}
+        mom = {k: ([x[1] for x in v] if isinstance(v, list) else v[1]) for k, v in new.items()}
+        vel = {k: ([x[2] for x in v] if isinstance(v, list) else v[2]) for k, v in new.items()}
+    return master, losses

@@ -160,6 +160,28 @@ def test_network_validation(lib):
     assert lib.fno_mse(0, 0, 256, 256, 256, None, None) == capi.FNO_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("args,word", [
+    # n, theta, m, v, grad, out, out_dtype, step, lr, beta1, beta2, eps, wd, scale
+    ((0, 256, 256, 256, 256, 256, 2, 1, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1.0), "n 0"),
+    ((8, None, 256, 256, 256, 256, 2, 1, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1.0), "theta"),
+    ((8, 0x108, 256, 256, 256, 256, 2, 1, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1.0), "aligned"),
+    ((8, 256, None, 256, 256, 256, 2, 1, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1.0), "m is NULL"),
+    ((8, 256, 256, None, 256, 256, 2, 1, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1.0), "v is NULL"),
+    ((8, 256, 256, 256, 256, 256, 2, 0, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1.0), "step 0"),
+    ((8, 256, 256, 256, 256, 256, 2, 1, 1e-3, 1.0, 0.999, 1e-8, 0.0, 1.0), "betas"),
+    ((8, 256, 256, 256, 256, 256, 2, 1, 1e-3, 0.9, 0.999, 0.0, 0.0, 1.0), "eps"),
+    ((8, 256, 256, 256, 256, 256, 2, 1, -1.0, 0.9, 0.999, 1e-8, 0.0, 1.0), "lr"),
+    ((8, 256, 256, 256, 256, 256, 2, 1, 1e-3, 0.9, 0.999, 1e-8, -0.1, 1.0), "weight_decay"),
+    ((8, 256, 256, 256, 256, 256, 7, 1, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1.0), "out_dtype"),
+    ((8, 256, None, None, None, None, 2, 1, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1.0), "nothing to do"),
+    ((8, 256, 256, 256, 256, 0x208, 2, 1, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1.0), "param_out"),
+])
+def test_adam_step_validation(lib, args, word):
+    """Every rejected argument fails before anything is enqueued (no GPU needed)."""
+    assert lib.fno_adam_step(*args, None) == capi.FNO_ERR_INVALID_ARG
+    assert word in capi.last_error()
+
+
 def test_missing_library_raises(tmp_path):
     with pytest.raises(capi.FnoError):
         capi.load(str(tmp_path / "libfno.so"))

@@ -389,3 +389,109 @@ def test_bf16_rounding_is_round_to_nearest_even():
     vals = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.0 + 2 ** -9, -2.5])
     out = synth.quantize(vals, "bf16")
     np.testing.assert_array_equal(out, [1.0, 1.0, 1.0 + 2 ** -6, 1.0, -2.5])
+
+
+# --------------------------------------------------------------------------
+# training loop: Adam, storage rounding, precision schedule
+# --------------------------------------------------------------------------
+
+def test_adam_hand_derived_two_steps():
+    g = _load("adam_two_steps_hand.json")
+    theta, m, v = np.array([g["theta0"]]), np.zeros(1), np.zeros(1)
+    for t, grad in enumerate(g["grads"], start=1):
+        theta, m, v = O.adam_update(theta, m, v, np.array([grad]), t, g["lr"], g["beta1"],
+                                    g["beta2"], g["eps"])
+        np.testing.assert_allclose(m, [g["m"][t - 1]], rtol=1e-14)
+        np.testing.assert_allclose(v, [g["v"][t - 1]], rtol=1e-14)
+        np.testing.assert_allclose(theta, [g["theta"][t - 1]], rtol=1e-14)
+
+
+@pytest.mark.parametrize("grad", [3.0, -0.5, 1e-6, -2e-7])
+def test_adam_constant_gradient_closed_form(grad):
+    """With a constant gradient the bias-corrected moments are exactly g and g^2,
+    so every step moves theta by lr g / (|g| + eps); eps matters for tiny g."""
+    lr, eps, steps = 0.05, 1e-8, 7
+    theta, m, v = np.array([0.3]), np.zeros(1), np.zeros(1)
+    for t in range(1, steps + 1):
+        theta, m, v = O.adam_update(theta, m, v, np.array([grad]), t, lr, 0.9, 0.999, eps)
+    expect = 0.3 - steps * lr * grad / (abs(grad) + eps)
+    np.testing.assert_allclose(theta, [expect], rtol=1e-12)
+
+
+def test_adam_decoupled_weight_decay_closed_form():
+    """A zero gradient leaves both moments at zero; decoupled decay alone shrinks
+    theta by (1 - lr wd) per step."""
+    lr, wd = 0.01, 0.5
+    theta, m, v = np.array([2.0, -1.0]), np.zeros(2), np.zeros(2)
+    for t in range(1, 6):
+        theta, m, v = O.adam_update(theta, m, v, np.zeros(2), t, lr, weight_decay=wd)
+    np.testing.assert_allclose(theta, np.array([2.0, -1.0]) * (1 - lr * wd) ** 5, rtol=1e-14)
+    assert not m.any() and not v.any()
+
+
+def test_adam_converges_on_a_quadratic():
+    rng = np.random.default_rng(13)
+    curv = rng.uniform(0.5, 5.0, 16)
+    centre = rng.standard_normal(16)
+    theta, m, v = np.zeros(16), np.zeros(16), np.zeros(16)
+    for t in range(1, 3001):
+        theta, m, v = O.adam_update(theta, m, v, curv * (theta - centre), t, 0.01)
+    np.testing.assert_allclose(theta, centre, atol=1e-3)
+
+
+def test_round_to_storage_ties_to_even():
+    vals = [1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.0 + 2 ** -9, -2.5, 1.0 + 2 ** -8 + 2 ** -20]
+    np.testing.assert_array_equal(O.round_to_storage(vals, "bf16"),
+                                  [1.0, 1.0, 1.0 + 2 ** -6, 1.0, -2.5, 1.0 + 2 ** -7])
+    np.testing.assert_array_equal(O.round_to_storage([1.0 + 2 ** -11, 1.0 + 3 * 2 ** -11], "f16"),
+                                  [1.0, 1.0 + 2 ** -9])
+    np.testing.assert_array_equal(O.round_to_storage([1.0 + 2 ** -24], "f32"), [1.0])
+
+
+def test_precision_schedule_phases():
+    phases = [(0, "bf16"), (4, "f32")]
+    assert [O.dtype_at(phases, t) for t in range(6)] == ["bf16"] * 4 + ["f32"] * 2
+    assert O.dtype_at([(0, "f16")], 1000) == "f16"
+    with pytest.raises(ValueError):
+        O.dtype_at([(2, "f32")], 0)
+
+
+def test_train_first_step_is_adam_first_step():
+    """The loop's first step moves every parameter component by lr g / (|g| + eps),
+    g the network gradient at the starting point (Adam's first step in closed form)."""
+    grid, modes = (8, 6), (2, 2)
+    wl = synth.Workload("tiny", "network", "f32", 2, grid, modes, 4, in_ch=3, hidden=5,
+                        n_layers=2, backward=True)
+    inp = synth.make_network_inputs(wl)
+    a, params, t = inp["a"], inp["params"], inp["target"]
+    lr, eps = 1e-2, 1e-8
+    new, losses = O.train(a, t, params, modes, [(0, "f32")], 1, lr, eps=eps)
+    q = {k: ([O.round_to_storage(x.real, "f32") + 1j * O.round_to_storage(x.imag, "f32")
+              if np.iscomplexobj(x) else O.round_to_storage(x, "f32") for x in v]
+             if isinstance(v, list) else O.round_to_storage(v, "f32")) for k, v in params.items()}
+    a_q, t_q = O.round_to_storage(a, "f32"), O.round_to_storage(t, "f32")
+    u, saves = O.forward(a_q, q, modes, save=True)
+    loss, du = O.mse(u, t_q)
+    assert losses == [loss]
+    grads = O.backward(a_q, q, saves, du, modes)
+
+    def step(g):
+        return lr * g / (np.abs(g) + eps)
+
+    for key in ("P", "p", "Q1", "q1", "Q2", "q2"):
+        np.testing.assert_allclose(new[key], params[key] - step(grads[key]), rtol=1e-12, atol=1e-15)
+    for l in range(2):
+        np.testing.assert_allclose(new["W"][l], params["W"][l] - step(grads["W"][l]), rtol=1e-12)
+        r = params["R"][l]
+        expect = (r.real - step(grads["R"][l].real)) + 1j * (r.imag - step(grads["R"][l].imag))
+        np.testing.assert_allclose(new["R"][l], expect, rtol=1e-12)
+
+
+def test_train_loss_decreases_across_a_precision_switch():
+    grid, modes = (8, 6), (2, 2)
+    wl = synth.Workload("tiny", "network", "bf16", 2, grid, modes, 4, in_ch=3, hidden=5,
+                        n_layers=2, backward=True)
+    inp = synth.make_network_inputs(wl)
+    _, losses = O.train(inp["a"], inp["target"], inp["params"], modes, [(0, "bf16"), (3, "f32")],
+                        6, 1e-2)
+    assert all(b < a for a, b in zip(losses, losses[1:]))

@@ -127,7 +127,49 @@ def _mutants(fo):
         diff = np.asarray(u, np.float64) - np.asarray(target, np.float64)
         return float(np.mean(diff * diff)), diff / diff.size
 
+    def adam(variant):
+        def f(theta, m, v, g, t, lr, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0):
+            theta = np.asarray(theta, np.float64)
+            g = np.asarray(g, np.float64)
+            if variant == "coupled_decay":       # L2 term folded into the gradient
+                g = g + weight_decay * theta
+            m = beta1 * np.asarray(m, np.float64) + (1.0 - beta1) * g
+            v = beta2 * np.asarray(v, np.float64) + (1.0 - beta2) * g * g
+            if variant == "no_bias_correction":
+                m_hat, v_hat = m, v
+            else:
+                m_hat, v_hat = m / (1.0 - beta1 ** t), v / (1.0 - beta2 ** t)
+            if variant == "eps_inside_sqrt":
+                denom = np.sqrt(v_hat + eps)
+            else:
+                denom = np.sqrt(v_hat) + eps
+            decay = 0.0 if variant == "coupled_decay" else lr * weight_decay * theta
+            return theta - lr * m_hat / denom - decay, m, v
+        return f
+
+    def bf16_truncating(x, dtype):              # bf16 rounding by truncation
+        if dtype != "bf16":
+            return orig_round(x, dtype)
+        bits = np.asarray(x, np.float64).astype(np.float32).view(np.uint32)
+        return (bits & np.uint32(0xFFFF0000)).view(np.float32).astype(np.float64)
+
+    orig_round = fo.round_to_storage
+
+    def dtype_at_late(phases, step):            # a phase starts one step late
+        current = None
+        for start, dtype in phases:
+            if start < step or start == 0:
+                current = dtype
+        if current is None:
+            raise ValueError("no phase covers step %d" % step)
+        return current
+
     return {
+        "adam_no_bias_correction": {"adam_update": adam("no_bias_correction")},
+        "adam_eps_inside_sqrt": {"adam_update": adam("eps_inside_sqrt")},
+        "adam_coupled_decay": {"adam_update": adam("coupled_decay")},
+        "bf16_truncating": {"round_to_storage": bf16_truncating},
+        "schedule_phase_late": {"dtype_at": dtype_at_late},
         "dft_sign": {"truncated_dft": dft_sign},
         "inverse_sign": {"inverse_sum": inverse_sign},
         "inverse_unscaled": {"mode_weights": weights_times_n},
@@ -166,7 +208,8 @@ MUTANT_NAMES = [
     "ck_nyquist_doubled", "negative_block_reversed", "mix_conj_r", "tanh_preact_ignored",
     "gelu_tanh_approx", "gelu_grad_cdf_only", "dr_no_conj", "dxhat_no_conj", "dyhat_unweighted",
     "tanh_grad_missing", "db_dropped", "skip_grad_dropped", "dq2_from_preactivation",
-    "lift_bias_dropped", "mse_half_gradient",
+    "lift_bias_dropped", "mse_half_gradient", "adam_no_bias_correction", "adam_eps_inside_sqrt",
+    "adam_coupled_decay", "bf16_truncating", "schedule_phase_late",
 ]
 
 
