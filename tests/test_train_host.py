@@ -202,3 +202,69 @@ def test_trainer_f32_with_fake_library_matches_oracle_loop(monkeypatch):
     for key in ("R", "W", "b"):
         for l in range(2):
             np.testing.assert_allclose(got[key][l], ref[key][l], rtol=1e-5, atol=1e-6)
+
+
+def _free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _dp_trainer_worker(rank, world, port, out_dir):
+    import os
+
+    import torch.distributed as dist
+
+    from fourier_neural_spectral_fno_b200 import train as T
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        grid, modes = (8, 6), (2, 2)
+        wl = synth.Workload("tiny", "network", "f32", 4, grid, modes, 4, in_ch=3, hidden=5,
+                            n_layers=2, backward=True)
+        inp = synth.make_network_inputs(wl)
+        T.capi = _FakeLibrary(modes)
+        tr = T.Trainer(grid, modes, 3, 4, inp["params"], T.PrecisionSchedule([(0, "f32")]),
+                       hidden=5, n_layers=2, lr=1e-2, eps=1.0, device="cpu",
+                       process_group=dist.group.WORLD)
+        lo, hi = rank * 2, rank * 2 + 2          # equal shards of the batch of 4
+        a = torch.from_numpy(np.asarray(inp["a"][lo:hi], np.float32))
+        t = torch.from_numpy(np.asarray(inp["target"][lo:hi], np.float32))
+        for _ in range(2):
+            tr.step(a, t)
+        np.save(os.path.join(out_dir, f"master{rank}.npy"), tr.master.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_trainer_data_parallel_matches_full_batch(tmp_path, monkeypatch):
+    """Two gloo ranks with half the batch each, gradient all-reduce and the
+    1/world scale in the optimiser: the same weights as one rank on the whole
+    batch (the gradient of the global-mean MSE).  eps = 1 makes the step
+    close to linear in the gradient, so a wrong gradient scale shows (Adam
+    with a small eps would hide it)."""
+    import torch.multiprocessing as mp
+
+    from fourier_neural_spectral_fno_b200 import train as T
+    world = 2
+    mp.start_processes(_dp_trainer_worker, args=(world, _free_port(), str(tmp_path)),
+                       nprocs=world, start_method="spawn", join=True)
+    m0, m1 = np.load(tmp_path / "master0.npy"), np.load(tmp_path / "master1.npy")
+    np.testing.assert_array_equal(m0, m1)     # every rank holds the same weights
+    grid, modes = (8, 6), (2, 2)
+    wl = synth.Workload("tiny", "network", "f32", 4, grid, modes, 4, in_ch=3, hidden=5,
+                        n_layers=2, backward=True)
+    inp = synth.make_network_inputs(wl)
+    monkeypatch.setattr(T, "capi", _FakeLibrary(modes))
+    tr = T.Trainer(grid, modes, 3, 4, inp["params"], T.PrecisionSchedule([(0, "f32")]), hidden=5,
+                   n_layers=2, lr=1e-2, eps=1.0, device="cpu")
+    a = torch.from_numpy(np.asarray(inp["a"], np.float32))
+    t = torch.from_numpy(np.asarray(inp["target"], np.float32))
+    start = tr.master.numpy().copy()
+    for _ in range(2):
+        tr.step(a, t)
+    moved = np.abs(tr.master.numpy() - start).max()
+    assert moved > 1e-4                            # the steps are not negligible
+    np.testing.assert_allclose(m0, tr.master.numpy(), rtol=1e-5, atol=1e-3 * moved)
