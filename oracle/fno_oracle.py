@@ -447,3 +447,24 @@ def train(a, target, params, modes, phases, steps: int, lr: float, beta1: float 
         mom = {k: ([x[1] for x in v] if isinstance(v, list) else v[1]) for k, v in new.items()}
         vel = {k: ([x[2] for x in v] if isinstance(v, list) else v[2]) for k, v in new.items()}
     return master, losses
+
+
+# --------------------------------------------------------------------------
+# factorised spectral weights (TFNO, [MPTRAIN] summary; CP reading)
+# --------------------------------------------------------------------------
+
+def cp_weights(lam, a, b, c) -> np.ndarray:
+    """``R[i, o, k] = sum_r lam[r] a[i, r] b[o, r] c[k, r]``: a rank-r CP weight.
+
+    The summary page names TFNO (factorised spectral weights) without the
+    factorisation; the canonical polyadic form is the reading.  Complex factors
+    allowed.  Returns ``[Ci, Co, |K|]`` complex128.
+    """
+    return np.einsum("r,ir,or,kr->iok", np.asarray(lam, np.complex128),
+                     np.asarray(a, np.complex128), np.asarray(b, np.complex128),
+                     np.asarray(c, np.complex128))
+
+
+def spectral_conv_fwd_cp(x, lam, a, b, c, modes, flags: int = 0):
+    """:func:`spectral_conv_fwd` with the CP weight :func:`cp_weights` (definition)."""
+    return spectral_conv_fwd(x, cp_weights(lam, a, b, c), modes, flags)

@@ -1,4 +1,5 @@
-"""Planted mistakes in the CPU oracle: each must make a pin in test_oracle.py fail.
+"""Planted mistakes in the CPU oracle: each must make a pin fail (test_oracle.py,
+test_contraction.py).
 
 Every mutant below is a plausible slip in one step of the oracle: a sign, a
 conjugation, a normalisation, a mode weight, a mode order, a dropped term or a
@@ -21,7 +22,8 @@ import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-PINS = os.path.join(ROOT, "tests", "test_oracle.py")
+PINS = [os.path.join(ROOT, "tests", "test_oracle.py"),
+        os.path.join(ROOT, "tests", "test_contraction.py")]
 
 
 def _mutants(fo):
@@ -164,7 +166,18 @@ def _mutants(fo):
             raise ValueError("no phase covers step %d" % step)
         return current
 
+    def cp_factor_conjugated(lam, a, b, c):     # conj(c) in the CP weight
+        return np.einsum("r,ir,or,kr->iok", np.asarray(lam, np.complex128),
+                         np.asarray(a, np.complex128), np.asarray(b, np.complex128),
+                         np.conj(np.asarray(c, np.complex128)))
+
+    def cp_lambda_dropped(lam, a, b, c):        # CP weights without lam
+        return np.einsum("ir,or,kr->iok", np.asarray(a, np.complex128),
+                         np.asarray(b, np.complex128), np.asarray(c, np.complex128))
+
     return {
+        "cp_factor_conjugated": {"cp_weights": cp_factor_conjugated},
+        "cp_lambda_dropped": {"cp_weights": cp_lambda_dropped},
         "adam_no_bias_correction": {"adam_update": adam("no_bias_correction")},
         "adam_eps_inside_sqrt": {"adam_update": adam("eps_inside_sqrt")},
         "adam_coupled_decay": {"adam_update": adam("coupled_decay")},
@@ -209,7 +222,8 @@ MUTANT_NAMES = [
     "gelu_tanh_approx", "gelu_grad_cdf_only", "dr_no_conj", "dxhat_no_conj", "dyhat_unweighted",
     "tanh_grad_missing", "db_dropped", "skip_grad_dropped", "dq2_from_preactivation",
     "lift_bias_dropped", "mse_half_gradient", "adam_no_bias_correction", "adam_eps_inside_sqrt",
-    "adam_coupled_decay", "bf16_truncating", "schedule_phase_late",
+    "adam_coupled_decay", "bf16_truncating", "schedule_phase_late", "cp_factor_conjugated",
+    "cp_lambda_dropped",
 ]
 
 
@@ -252,4 +266,4 @@ def test_every_planted_mistake_fails_a_pin(name):
 
 if __name__ == "__main__":
     _apply(sys.argv[1])
-    sys.exit(pytest.main([PINS, "-q", "-x", "-p", "no:cacheprovider"]))
+    sys.exit(pytest.main(PINS + ["-q", "-x", "-p", "no:cacheprovider"]))
