@@ -220,7 +220,9 @@ def kernel_source_sha(tag: str) -> str:
              "proj_fwd": "net.cu", "fwd_transform_tc": "transform_tc.cu",
              "epi_block_fwd_tc": "epilogue_tc.cu", "inv_slab": "epilogue_tc.cu",
              "proj_fwd_tc": "net_tc.cu", "epi_block_fwd_pipe": "epilogue_pipe.cu",
-             "fwd_transform_pipe": "transform_pipe.cu", "proj_fwd_pipe": "proj_pipe.cu"}
+             "fwd_transform_pipe": "transform_pipe.cu", "proj_fwd_pipe": "proj_pipe.cu",
+             "epi_block_bwd": "epilogue.cu", "proj_bwd": "net.cu",
+             "fwd_transform_tc_dz": "transform_tc.cu", "fwd_transform_dz": "transform.cu"}
     path = os.path.join(ROOT, "fourier_neural_spectral_fno_b200", "csrc", files.get(tag, ""))
     if not os.path.isfile(path):
         return ""
@@ -238,6 +240,62 @@ def measured_traffic(tag: str, wl):
     if rec.get("source_sha") != kernel_source_sha(tag):
         return None
     return rec.get("bytes_per_launch")
+
+
+FP32_LANES_PER_SM = 128      # FP32 FMA lanes per SM: 4 sub-partitions x 32
+FALLBACK_SMS = 148
+FALLBACK_SM_MHZ = 1965.0
+
+
+def alu_peak_tflops(n_sms: int):
+    """FP32 CUDA-core peak: 2 FLOP per FMA x FMA lanes x SMs x maximum SM clock
+    (the clock from MEASURED_PEAKS.json, else the B200's 1965 MHz)."""
+    try:
+        mhz = float(json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["sm_max_mhz"])
+        src = "derived: measured max SM clock"
+    except Exception:
+        mhz, src = FALLBACK_SM_MHZ, "derived: nominal max SM clock"
+    return 2.0 * FP32_LANES_PER_SM * n_sms * mhz * 1e6 / 1e12, src
+
+
+def algorithmic_flops(tag: str, wl) -> float:
+    """FP32 FLOPs per launch of the CUDA-core kernels whose bound is arithmetic
+    (0 for the others): each contraction's multiply-adds, two FLOPs apiece."""
+    pts = wl.batch * wl.points
+    c, m_l, h = wl.width, wl.modes[-1], wl.hidden
+    table = {
+        # last-axis inverse of dxhat (a complex multiply-add per mode and channel: 4 FLOPs),
+        # dx = W^T dz and dW = dz x^T (2 FLOPs per channel pair each)
+        "epi_block_bwd": pts * (4 * m_l * c + 4 * c * c),
+        # hidden layer recomputed (Q1 v), dv = Q1^T dh, dQ1 = dh v^T, dQ2 = du g^T
+        "proj_bwd": pts * (6 * h * c + 2 * h * wl.out_ch),
+    }
+    return float(table.get(tag, 0.0))
+
+
+def roofline_record(dom: str, avg_ms: float, wl, n_sms: int) -> dict:
+    """The roofline object of the dominant kernel: against the FP32 CUDA-core
+    peak for the arithmetic-bound CUDA-core kernels, else against the measured
+    HBM copy bandwidth."""
+    alg = algorithmic_bytes(dom, wl)
+    hbm, hbm_src = hbm_peak()
+    gbs = alg / (avg_ms / 1e3) / 1e9 if alg else None
+    flops = algorithmic_flops(dom, wl)
+    if flops:
+        peak, src = alu_peak_tflops(n_sms)
+        achieved = flops / (avg_ms / 1e3) / 1e12
+        return {"kernel": dom, "bound": "alu", "achieved": achieved, "peak": peak,
+                "peak_source": f"{src} x {FP32_LANES_PER_SM} FP32 lanes x {n_sms} SMs x 2",
+                "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": measured_traffic(dom, wl), "avg_launch_ms": avg_ms,
+                "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": alg,
+                "hbm_view": {"achieved": gbs, "peak": hbm, "unit": "GB/s",
+                             "frac": (gbs / hbm) if gbs else None}}
+    return {"kernel": dom, "bound": "hbm", "achieved": gbs, "peak": hbm,
+            "peak_source": f"{hbm_src} (MEASURED_PEAKS.json hbm_gbs, copy)",
+            "unit": "GB/s", "frac": (gbs / hbm) if gbs else None,
+            "traffic": measured_traffic(dom, wl), "avg_launch_ms": avg_ms,
+            "algorithmic_bytes_per_launch": alg}
 
 
 def hbm_peak():
@@ -419,14 +477,8 @@ def run_fno(args, dist):
     stats = capi.fno_profile_read()
     dom = max(stats, key=lambda t: stats[t]["total_ms"])
     avg_ms = stats[dom]["total_ms"] / stats[dom]["launches"]
-    peak, peak_src = hbm_peak()
-    alg = algorithmic_bytes(dom, wl)
-    achieved = alg / (avg_ms / 1e3) / 1e9 if alg else None
-    roofline = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak,
-                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, copy)",
-                "unit": "GB/s", "frac": (achieved / peak) if achieved else None,
-                "traffic": measured_traffic(dom, wl), "avg_launch_ms": avg_ms,
-                "algorithmic_bytes_per_launch": alg}
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    roofline = roofline_record(dom, avg_ms, wl, n_sms)
     per_step = {t: round(v["total_ms"] / args.steps, 4) for t, v in sorted(
         stats.items(), key=lambda kv: -kv[1]["total_ms"])}
 

@@ -62,3 +62,39 @@ def test_workload_selection_errors(args, msg):
     p = _run(["--impl", "reference", "--steps", "1", "--warmup", "0"] + args, timeout=120)
     assert p.returncode != 0
     assert msg in p.stderr
+
+
+def _bench_module():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_under_test", BENCH)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_roofline_alu_for_cuda_core_backward():
+    from fourier_neural_spectral_fno_b200 import synth
+    bench = _bench_module()
+    wl = synth.WORKLOADS["fno2d_bf16_train_b32_w64_256sq_m24"]
+    rec = bench.roofline_record("epi_block_bwd", 2.5, wl, 148)
+    # per point: 4 m_L C (inverse of dxhat) + 4 C^2 (dx and dW) FLOPs over B N points
+    flops = 32 * 65536 * (4 * 24 * 64 + 4 * 64 * 64)
+    assert rec["bound"] == "alu" and rec["unit"] == "TFLOP/s"
+    assert rec["algorithmic_flops_per_launch"] == flops
+    assert rec["achieved"] == pytest.approx(flops / 2.5e-3 / 1e12)
+    assert rec["peak"] == pytest.approx(2 * 128 * 148 * 1965e6 / 1e12)
+    assert rec["frac"] == pytest.approx(rec["achieved"] / rec["peak"])
+    assert rec["hbm_view"]["unit"] == "GB/s" and rec["hbm_view"]["achieved"] > 0
+
+
+def test_roofline_hbm_for_the_forward_pipeline():
+    from fourier_neural_spectral_fno_b200 import synth
+    bench = _bench_module()
+    wl = synth.WORKLOADS["fno2d_f32_b16_w32_256sq_m16"]
+    rec = bench.roofline_record("epi_block_fwd_pipe", 0.1, wl, 148)
+    act = 16 * 32 * 65536 * 4
+    spec = 16 * 32 * 16 * 32 * 8
+    assert rec["bound"] == "hbm" and rec["unit"] == "GB/s"
+    assert rec["algorithmic_bytes_per_launch"] == 2 * act + spec
+    assert rec["achieved"] == pytest.approx((2 * act + spec) / 0.1e-3 / 1e9)
+    assert rec["peak"] == pytest.approx(6541.8)
