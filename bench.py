@@ -243,7 +243,6 @@ def measured_traffic(tag: str, wl):
 
 
 FP32_LANES_PER_SM = 128      # FP32 FMA lanes per SM: 4 sub-partitions x 32
-FALLBACK_SMS = 148
 FALLBACK_SM_MHZ = 1965.0
 
 
