@@ -8,7 +8,7 @@ source file it was built from (bench.py ignores a record whose source changed).
 
     ncu -i report.ncu-rep --page raw --csv > raw.csv
     python -m fourier_neural_spectral_fno_b200.profile_traffic raw.csv \
-        fno2d_f32_b16_w32_256sq_m16
+        fno2d_f32_b16_w32_256sq_m16 [--scale S] [--only tag,...]
 """
 
 from __future__ import annotations
@@ -17,6 +17,7 @@ import csv
 import hashlib
 import json
 import os
+import re
 import sys
 from collections import defaultdict
 
@@ -36,7 +37,14 @@ KERNELS = {
     "k_fwd_finish": ("fwd_finish", "transform.cu"),
     "k_lift4": ("lift", "net.cu"),
     "k_lift": ("lift", "net.cu"),
+    "k_proj_bwd": ("proj_bwd", "net.cu"),
+    "k_lift_bwd": ("lift_bwd", "net.cu"),
 }
+
+# k_epilogue<T, MODE, ...>: the timing tag follows the epilogue mode
+EPILOGUE_TAGS = {"0": "epi_spec", "1": "epi_block_fwd", "2": "epi_spec_bwd", "3": "epi_block_bwd"}
+
+UNIT_SCALE = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
 
 
 def source_sha(fname: str) -> str:
@@ -44,8 +52,21 @@ def source_sha(fname: str) -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
+_KERNEL_RE = re.compile(r"\b(k_\w+)\s*(?:<([^()]*)>)?")
+
+
 def _kernel_key(name: str):
-    base = name.split("(")[0].split("<")[0].split("::")[-1].strip()
+    """(timing tag, source file) of a kernel name as ncu prints it, or None.
+    The name's namespaces vary between ncu pages; the kernel is the first
+    identifier that starts with ``k_``."""
+    m = _KERNEL_RE.search(name.split("(")[0])
+    if not m:
+        return None
+    base, targs = m.group(1), m.group(2)
+    if base == "k_epilogue":
+        args = [t.strip() for t in (targs or "").split(",")]
+        tag = EPILOGUE_TAGS.get(args[1]) if len(args) > 1 else None
+        return (tag, "epilogue.cu") if tag else None
     return KERNELS.get(base)
 
 
@@ -63,29 +84,41 @@ def parse(csv_path: str):
             wr = float(r[col["dram__bytes_write.sum"]])
         except (KeyError, ValueError):
             continue
-        unit = rows[1][col["dram__bytes_read.sum"]]
-        scale = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}.get(unit, 1.0)
+        units = rows[1]
         a = acc[key]
-        a[0] += rd * scale
-        a[1] += wr * scale
+        a[0] += rd * UNIT_SCALE.get(units[col["dram__bytes_read.sum"]], 1.0)
+        a[1] += wr * UNIT_SCALE.get(units[col["dram__bytes_write.sum"]], 1.0)
         a[2] += 1
     return acc
 
 
 def main(argv) -> int:
-    if len(argv) != 3:
-        print(__doc__)
-        return 2
-    acc = parse(argv[1])
+    import argparse
+    ap = argparse.ArgumentParser(description=__doc__,
+                                 formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("csv")
+    ap.add_argument("workload")
+    ap.add_argument("--scale", type=float, default=1.0,
+                    help="units of the workload's launch per unit of the captured launch "
+                         "(a capture of a smaller batch, when traffic grows in proportion)")
+    ap.add_argument("--only", default="", help="comma-separated timing tags to record")
+    args = ap.parse_args(argv[1:])
+    acc = parse(args.csv)
+    only = {t for t in args.only.split(",") if t}
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         data = json.load(open(path))
     except Exception:
         data = {}
-    wl = data.setdefault(argv[2], {})
+    wl = data.setdefault(args.workload, {})
     for (tag, src), (rd, wr, n) in sorted(acc.items()):
+        if only and tag not in only:
+            continue
+        rd, wr = rd * args.scale, wr * args.scale
         wl[tag] = {"bytes_per_launch": (rd + wr) / n, "read_bytes": rd / n,
                    "write_bytes": wr / n, "launches": n, "source_sha": source_sha(src)}
+        if args.scale != 1.0:
+            wl[tag]["scaled_from_capture_by"] = args.scale
         print(f"{tag:22s} {src:18s} read {rd / n / 1e6:8.1f} MB  write {wr / n / 1e6:8.1f} MB")
     with open(path, "w") as f:
         json.dump(data, f, indent=1)
