@@ -214,6 +214,27 @@ class Trainer:
         """The float32 master weights as a NumPy float64 dict (R complex)."""
         return self.layout.unpack(self.master)
 
+    def state_dict(self) -> Dict[str, object]:
+        """Everything a resumed run needs: master weights, Adam moments, step
+        count, schedule and hyper-parameters (tensors copied to the host)."""
+        return {"master": self.master.detach().cpu().clone(), "m": self.m.detach().cpu().clone(),
+                "v": self.v.detach().cpu().clone(), "step": self.step_count,
+                "phases": list(self.schedule.phases), "lr": self.lr, "betas": tuple(self.betas),
+                "eps": self.eps, "weight_decay": self.weight_decay, "slots": self.layout.total}
+
+    def load_state_dict(self, state: Dict[str, object]) -> None:
+        """Resume from :meth:`state_dict` (same network shape)."""
+        if int(state["slots"]) != self.layout.total:
+            raise ValueError("checkpoint is of a different network shape")
+        self.master.copy_(state["master"])
+        self.m.copy_(state["m"])
+        self.v.copy_(state["v"])
+        self.step_count = int(state["step"])
+        self.schedule = PrecisionSchedule(state["phases"])
+        self.lr, self.betas = float(state["lr"]), tuple(state["betas"])
+        self.eps, self.weight_decay = float(state["eps"]), float(state["weight_decay"])
+        self.dtype, self.weights = None, None     # the next step copies the master afresh
+
     # ------------------------------------------------------------------- step
     def step(self, a, target):
         """One step on a batch: ``a`` [B][in][grid], ``target`` [B][out][grid]

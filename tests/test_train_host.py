@@ -268,3 +268,42 @@ def test_trainer_data_parallel_matches_full_batch(tmp_path, monkeypatch):
     moved = np.abs(tr.master.numpy() - start).max()
     assert moved > 1e-4                            # the steps are not negligible
     np.testing.assert_allclose(m0, tr.master.numpy(), rtol=1e-5, atol=1e-3 * moved)
+
+
+def test_trainer_resume_from_state_dict(monkeypatch):
+    """Two steps, a checkpoint, a fresh trainer that loads it and two more steps
+    end where four uninterrupted steps end (across the precision switch)."""
+    from fourier_neural_spectral_fno_b200 import train as T
+    grid, modes = (8, 6), (2, 2)
+    wl = synth.Workload("tiny", "network", "bf16", 2, grid, modes, 4, in_ch=3, hidden=5,
+                        n_layers=2, backward=True)
+    inp = synth.make_network_inputs(wl)
+    monkeypatch.setattr(T, "capi", _FakeLibrary(modes))
+    sched = [(0, "bf16"), (2, "f32")]
+    a = torch.from_numpy(np.asarray(inp["a"], np.float32))
+    t = torch.from_numpy(np.asarray(inp["target"], np.float32))
+
+    def trainer():
+        return T.Trainer(grid, modes, 3, 4, inp["params"], T.PrecisionSchedule(sched), hidden=5,
+                         n_layers=2, lr=1e-2, weight_decay=0.05, device="cpu")
+
+    straight = trainer()
+    for _ in range(4):
+        straight.step(a, t)
+    first = trainer()
+    for _ in range(2):
+        first.step(a, t)
+    state = first.state_dict()
+    resumed = T.Trainer(grid, modes, 3, 4, {**inp["params"]}, T.PrecisionSchedule([(0, "f32")]),
+                        hidden=5, n_layers=2, device="cpu")
+    resumed.load_state_dict(state)
+    assert resumed.step_count == 2 and resumed.schedule.phases == sched
+    for _ in range(2):
+        resumed.step(a, t)
+    assert torch.equal(resumed.master, straight.master)
+    assert torch.equal(resumed.m, straight.m) and torch.equal(resumed.v, straight.v)
+    with pytest.raises(ValueError):
+        T.Trainer(grid, modes, 3, 4, synth.make_network_inputs(
+            synth.Workload("w", "network", "f32", 2, grid, modes, 5, in_ch=3, hidden=5,
+                           n_layers=2, backward=True))["params"], T.PrecisionSchedule([(0, "f32")]),
+            hidden=5, n_layers=2, device="cpu").load_state_dict(state)
