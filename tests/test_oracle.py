@@ -59,6 +59,19 @@ def test_golden_2d_block():
     np.testing.assert_allclose(y.reshape(2, 2), g["y_spec"], atol=1e-12)
 
 
+def test_golden_network_composition():
+    g = _load("network_scalar_hand.json")
+    grid, modes = tuple(g["grid"]), tuple(g["modes"])
+    nk = O.num_modes(grid, modes)
+    params = {"P": np.array([[g["P"]]]), "p": np.array([g["p"]]),
+              "R": [np.zeros((1, 1, nk), complex)], "W": [np.array([[g["W"]]])],
+              "b": [np.array([g["b"]])], "Q1": np.array([[g["Q1"]]]), "q1": np.array([g["q1"]]),
+              "Q2": np.array([[g["Q2"]]]), "q2": np.array([g["q2"]])}
+    a = np.full((1, 1) + grid, g["a"])
+    np.testing.assert_allclose(O.forward(a, params, modes), np.full((1, 1) + grid, g["u"]),
+                               rtol=1e-14)
+
+
 def test_gelu_against_normal_table():
     g = _load("normal_cdf_table.json")
     z = np.array(g["z"])

@@ -175,7 +175,14 @@ def _mutants(fo):
         return np.einsum("ir,or,kr->iok", np.asarray(a, np.complex128),
                          np.asarray(b, np.complex128), np.asarray(c, np.complex128))
 
+    def projection_without_gelu(v, q1_mat, q1_vec, q2_mat, q2_vec):   # hidden layer linear
+        v = np.asarray(v, np.float64)
+        d = v.ndim - 2
+        h = fo._pointwise(q1_mat, v) + fo._bcast(q1_vec, d)
+        return fo._pointwise(q2_mat, h) + fo._bcast(q2_vec, d)
+
     return {
+        "projection_without_gelu": {"projection": projection_without_gelu},
         "cp_factor_conjugated": {"cp_weights": cp_factor_conjugated},
         "cp_lambda_dropped": {"cp_weights": cp_lambda_dropped},
         "adam_no_bias_correction": {"adam_update": adam("no_bias_correction")},
@@ -223,7 +230,7 @@ MUTANT_NAMES = [
     "tanh_grad_missing", "db_dropped", "skip_grad_dropped", "dq2_from_preactivation",
     "lift_bias_dropped", "mse_half_gradient", "adam_no_bias_correction", "adam_eps_inside_sqrt",
     "adam_coupled_decay", "bf16_truncating", "schedule_phase_late", "cp_factor_conjugated",
-    "cp_lambda_dropped",
+    "cp_lambda_dropped", "projection_without_gelu",
 ]
 
 
