@@ -185,3 +185,33 @@ def test_adam_step_validation(lib, args, word):
 def test_missing_library_raises(tmp_path):
     with pytest.raises(capi.FnoError):
         capi.load(str(tmp_path / "libfno.so"))
+
+
+@pytest.mark.parametrize("kw,word", [
+    ({"step": 0}, "step 0"),
+    ({"beta1": 1.5}, "betas (1.5"),
+    ({"beta2": -0.5}, "-0.5)"),
+    ({"eps": -1.0}, "eps -1"),
+    ({"lr": -2.0}, "lr -2"),
+    ({"weight_decay": -3.0}, "weight_decay -3"),
+    ({"grad_scale": float("inf")}, "grad_scale"),
+])
+def test_adam_binding_passes_each_argument_in_place(lib, kw, word):
+    """The binding's marshalling, checked through the library's validation,
+    which runs before anything touches a device (host buffers suffice)."""
+    import torch
+    t = torch.zeros(16)
+    args = dict(step=1, lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0,
+                grad_scale=1.0)
+    args.update(kw)
+    with pytest.raises(capi.FnoError) as e:
+        capi.fno_adam_step(t, t.clone(), t.clone(), t.clone(), torch.zeros(16, dtype=torch.bfloat16),
+                           stream=0, **args)
+    assert e.value.code == capi.FNO_ERR_INVALID_ARG and word in str(e.value)
+
+
+def test_adam_binding_rejects_a_non_storage_dtype(lib):
+    import torch
+    t = torch.zeros(8)
+    with pytest.raises(ValueError):
+        capi.fno_adam_step(t, t, t, t, torch.zeros(8, dtype=torch.float64), 1, 1e-3, stream=0)
