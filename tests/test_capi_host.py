@@ -215,3 +215,30 @@ def test_adam_binding_rejects_a_non_storage_dtype(lib):
     t = torch.zeros(8)
     with pytest.raises(ValueError):
         capi.fno_adam_step(t, t, t, t, torch.zeros(8, dtype=torch.float64), 1, 1e-3, stream=0)
+
+
+_WRAPPERS = {
+    "fno_spectral_conv_fwd": ["x", "R", "y", "xhat_save"],
+    "fno_spectral_conv_bwd": ["x", "xhat_save", "R", "dy", "dx", "dR"],
+    "fno_block_fwd": ["x", "R", "W", "b", "y", "pre_save", "xhat_save"],
+    "fno_block_bwd": ["x", "R", "W", "pre_save", "xhat_save", "dy", "dx", "dR", "dW", "db"],
+}
+
+
+@pytest.mark.parametrize("fn,arg", [(f, a) for f, args in _WRAPPERS.items() for a in args])
+def test_block_bindings_pass_each_pointer_in_place(lib, fn, arg):
+    """A misaligned buffer in one argument of a binding must be reported under
+    that argument's name by the library (validation runs before any device
+    work, so host buffers suffice)."""
+    import torch
+    d = capi.block_desc(2, 4, 4, (16, 16), (4, 4))
+
+    def buf(misaligned=False):
+        t = torch.zeros(1 << 14)
+        return t[1:] if misaligned else t
+
+    kwargs = {name: buf(name == arg) for name in _WRAPPERS[fn]}
+    with pytest.raises(capi.FnoError) as e:
+        getattr(capi, fn)(d, **kwargs, stream=0)
+    assert e.value.code == capi.FNO_ERR_INVALID_ARG
+    assert f": {arg} is not 16-byte aligned" in str(e.value)
