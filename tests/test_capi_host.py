@@ -242,3 +242,34 @@ def test_block_bindings_pass_each_pointer_in_place(lib, fn, arg):
         getattr(capi, fn)(d, **kwargs, stream=0)
     assert e.value.code == capi.FNO_ERR_INVALID_ARG
     assert f": {arg} is not 16-byte aligned" in str(e.value)
+
+
+@pytest.mark.parametrize("which,arg,msg", [
+    ("fwd", "a", "a"), ("fwd", "u", "u"), ("fwd", "saves", "saves"),
+    ("fwd", "P", "P"), ("fwd", "q1", "q1"), ("fwd", "Q2", "Q2"), ("fwd", "R", "R[l]"),
+    ("fwd", "W", "W[l]"), ("fwd", "b", "b[l]"),
+    ("bwd", "a", "a"), ("bwd", "saves", "saves"), ("bwd", "du", "du"),
+    ("bwd", "gP", "dP"), ("bwd", "gq2", "dq2"),
+])
+def test_network_bindings_pass_each_pointer_in_place(lib, which, arg, msg):
+    import torch
+    d = capi.net_desc(2, (16, 16), (4, 4), 3, 8, hidden=16, n_layers=2)
+
+    def buf(misaligned=False):
+        t = torch.zeros(1 << 14)
+        return t[1:] if misaligned else t
+
+    keys = ("P", "p", "Q1", "q1", "Q2", "q2")
+    params = {k: buf(arg == k) for k in keys}
+    params.update({k: [buf(arg == k), buf()] for k in ("R", "W", "b")})
+    with pytest.raises(capi.FnoError) as e:
+        if which == "fwd":
+            capi.fno_forward(d, buf(arg == "a"), capi.make_params(params), buf(arg == "u"),
+                             buf(arg == "saves"), stream=0)
+        else:
+            grads = {k: buf(arg == "g" + k) for k in keys}
+            grads.update({k: [buf(), buf()] for k in ("R", "W", "b")})
+            capi.fno_backward(d, buf(arg == "a"), capi.make_params(params), buf(arg == "saves"),
+                              buf(arg == "du"), capi.make_grads(grads), stream=0)
+    assert e.value.code == capi.FNO_ERR_INVALID_ARG
+    assert f": {msg} is not 16-byte aligned" in str(e.value)
