@@ -177,6 +177,8 @@ bool g_prof_on = false;
 
 __device__ int g_fno_device_error;   // set by kernels whose bounded waits expire
 
+std::mutex g_err_word_mu;
+
 int *device_error_word() {
   static int *addr[64] = {nullptr};
   int dev = 0;
@@ -184,6 +186,7 @@ int *device_error_word() {
     cudaGetLastError();
     return nullptr;
   }
+  std::lock_guard<std::mutex> lk(g_err_word_mu);   // first calls may race from several threads
   if (!addr[dev]) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_fno_device_error) != cudaSuccess) {

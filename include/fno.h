@@ -213,7 +213,9 @@ int fno_spectral_conv_fwd(const fno_block_desc *desc, const void *x, const void 
  *     array are rejected with FNO_ERR_WORKSPACE and a message naming both sizes.
  *   - The first call on each device looks up the array's device address (a
  *     host-side lookup that requires that device to be current).  Make that first
- *     call before any stream capture.
+ *     call before any stream capture.  The address is kept for the life of the
+ *     process, so cudaDeviceReset on that device after the first call is not
+ *     supported (the kept address would then be stale).
  *   - All calls share the one array, which keeps whatever the last call left in
  *     it; every scratch byte this operation reads it has first written, so
  *     nothing needs clearing.  Calls whose work overlaps on the GPU (concurrent

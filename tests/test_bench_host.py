@@ -97,4 +97,4 @@ def test_roofline_hbm_for_the_forward_pipeline():
     assert rec["bound"] == "hbm" and rec["unit"] == "GB/s"
     assert rec["algorithmic_bytes_per_launch"] == 2 * act + spec
     assert rec["achieved"] == pytest.approx((2 * act + spec) / 0.1e-3 / 1e9)
-    assert rec["peak"] == pytest.approx(6541.8)
+    assert rec["peak"] == pytest.approx(bench.hbm_peak()[0])   # measured copy peak, else fallback

@@ -64,7 +64,9 @@ def test_block2d_f32_b4_w20_64sq_m12_forward_and_backward():
     dx, dr, dw, db = empty(x.shape), empty((wl.width, wl.width, k, 2)), empty((wl.width, wl.width)), \
         empty((wl.width,))
     capi.fno_block_bwd(d, dev(x), dev_complex(r), dev(w), pre, xh, dev(dy), dx, dr, dw, db)
-    dx_ref, dr_ref, dw_ref, db_ref = O.block_bwd(x, r, w, host(pre), xh_ref, dy, wl.modes)
+    # the oracle's backward takes its own forward's pre-activation, rounded to float32
+    dx_ref, dr_ref, dw_ref, db_ref = O.block_bwd(x, r, w, synth.quantize(pre_ref, "f32"), xh_ref,
+                                                 dy, wl.modes)
     assert_close(host(dx), dx_ref, TOL["f32"], "dx")
     assert_close(host_complex(dr), dr_ref, TOL["f32"], "dR")
     assert_close(host(dw), dw_ref, TOL["f32"], "dW")
@@ -102,47 +104,40 @@ def test_fno2d_forward_is_batch_independent():
 # --------------------------------------------------------------------------
 
 def test_block2d_f16tanh_b8_w64_512sq_m32_forward_backward():
+    """Whole batch against the oracle: y and dx of every sample, and the
+    batch-summed dR, dW and db against the oracle's (its per-sample backward
+    passes summed).  Both backward passes take the same saved pre-activation,
+    the oracle's, rounded to float16."""
     wl = synth.WORKLOADS["block2d_f16tanh_b8_w64_512sq_m32"]
     inp = synth.make_block_inputs(wl)
     x, r, w, b, dy = inp["x"], inp["R"], inp["W"], inp["b"], inp["dy"]
     fl = capi.FNO_TANH_PREACT
-    C, k = wl.width, capi.num_modes(wl.grid, wl.modes)
-    rd, wd, bd = dev_complex(r, "f16"), dev(w, "f16"), dev(b, "f16")
-
-    def run(lo, hi):
-        n = hi - lo
-        d = capi.block_desc(n, C, C, wl.grid, wl.modes, "f16", fl)
-        xd, dyd = dev(x[lo:hi], "f16"), dev(dy[lo:hi], "f16")
-        y, pre = empty((n, C) + wl.grid, "f16"), empty((n, C) + wl.grid, "f16")
-        xh = empty((n, C, k, 2))
-        capi.fno_block_fwd(d, xd, rd, wd, bd, y, pre, xh)
-        dx = empty((n, C) + wl.grid, "f16")
-        dr, dw, db = empty((C, C, k, 2)), empty((C, C)), empty((C,))
-        capi.fno_block_bwd(d, xd, rd, wd, pre, xh, dyd, dx, dr, dw, db)
-        return y, pre, dx, dr, dw, db
-
-    y, pre, dx, dr, dw, db = run(0, wl.batch)
-    # per-sample outputs against the oracle (samples 0 and 7)
-    for s in (0, wl.batch - 1):
+    C, k, B = wl.width, capi.num_modes(wl.grid, wl.modes), wl.batch
+    d = capi.block_desc(B, C, C, wl.grid, wl.modes, "f16", fl)
+    xd, rd, wd, bd = dev(x, "f16"), dev_complex(r, "f16"), dev(w, "f16"), dev(b, "f16")
+    y, pre = empty((B, C) + wl.grid, "f16"), empty((B, C) + wl.grid, "f16")
+    capi.fno_block_fwd(d, xd, rd, wd, bd, y, pre)
+    yh = host(y)
+    pre_q = np.empty(x.shape)
+    dx_ref = np.empty(x.shape)
+    dr_ref, dw_ref, db_ref = 0, 0, 0
+    for s in range(B):
         y_ref, pre_ref, xh_ref = O.block_fwd(x[s:s + 1], r, w, b, wl.modes, O.TANH_PREACT)
-        assert_close(host(y)[s:s + 1], y_ref, TOL["f16"], f"y[{s}]")
-        pre_q = host(pre)[s:s + 1]
-        dx_ref, dr_ref, dw_ref, db_ref = O.block_bwd(x[s:s + 1], r, w, pre_q, xh_ref, dy[s:s + 1],
-                                                     wl.modes, O.TANH_PREACT)
-        assert_close(host(dx)[s:s + 1], dx_ref, TOL["f16"], f"dx[{s}]")
-        if s == 0:
-            _, _, _, dr0, dw0, db0 = run(0, 1)
-            assert_close(host_complex(dr0), dr_ref, TOL["f16"], "dR (sample 0)")
-            assert_close(host(dw0), dw_ref, TOL["f16"], "dW (sample 0)")
-            assert_close(host(db0), db_ref, TOL["f16"], "db (sample 0)")
-    # batch-summed weight gradients equal the sum of single-sample gradients
-    acc = [0, 0, 0]
-    for s in range(wl.batch):
-        _, _, _, drs, dws, dbs = run(s, s + 1)
-        acc = [acc[0] + host_complex(drs), acc[1] + host(dws), acc[2] + host(dbs)]
-    assert_close(host_complex(dr), acc[0], 1e-4, "dR = sum of per-sample dR")
-    assert_close(host(dw), acc[1], 1e-4, "dW = sum of per-sample dW")
-    assert_close(host(db), acc[2], 1e-4, "db = sum of per-sample db")
+        assert_close(yh[s:s + 1], y_ref, TOL["f16"], f"y[{s}]")
+        pre_q[s:s + 1] = synth.quantize(pre_ref, "f16")
+        dxs, drs, dws, dbs = O.block_bwd(x[s:s + 1], r, w, pre_q[s:s + 1], xh_ref, dy[s:s + 1],
+                                         wl.modes, O.TANH_PREACT)
+        dx_ref[s:s + 1] = dxs
+        dr_ref, dw_ref, db_ref = dr_ref + drs, dw_ref + dws, db_ref + dbs
+    dx = empty((B, C) + wl.grid, "f16")
+    dr, dw, db = empty((C, C, k, 2)), empty((C, C)), empty((C,))
+    capi.fno_block_bwd(d, xd, rd, wd, dev(pre_q, "f16"), None, dev(dy, "f16"), dx, dr, dw, db)
+    dxh = host(dx)
+    for s in range(B):
+        assert_close(dxh[s:s + 1], dx_ref[s:s + 1], TOL["f16"], f"dx[{s}]")
+    assert_close(host_complex(dr), dr_ref, TOL["f16"], "dR (batch of 8)")
+    assert_close(host(dw), dw_ref, TOL["f16"], "dW (batch of 8)")
+    assert_close(host(db), db_ref, TOL["f16"], "db (batch of 8)")
 
 
 # --------------------------------------------------------------------------
@@ -217,22 +212,32 @@ def test_fno2d_bf16_train_b32_w64_256sq_m24_step():
     for s in (0, wl.batch - 1):
         u_ref = O.forward(a[s:s + 1], p, wl.modes)
         assert_close(uh[s:s + 1], u_ref, TOL["bf16"], f"u[{s}]")
-    # gradients of sample 0 (its slice of the full-batch du) against the oracle
-    du0 = du[0:1].clone()
-    _, _, _, g0 = step(0, 1, du0)
+    # gradients of sample 0 against the oracle, both sides fed the oracle's
+    # cotangent: dL/du of the full-batch MSE restricted to sample 0, in bfloat16
     u_ref, sv_ref = O.forward(a[0:1], p, wl.modes, save=True)
-    g_ref = O.backward(a[0:1], p, sv_ref, host(du0), wl.modes)
+    du0_ref = synth.quantize(2.0 * (u_ref - tgt[0:1]) / tgt.size, "bf16")
+    _, _, _, g0 = step(0, 1, dev(du0_ref, "bf16"))
+    g_ref = O.backward(a[0:1], p, sv_ref, du0_ref, wl.modes)
     for key in ("P", "p", "Q1", "q1", "Q2", "q2"):
         assert_close(host(g0[key]), g_ref[key], TOL["bf16"], f"d{key} (sample 0)")
     for l in range(wl.n_layers):
         assert_close(host_complex(g0["R"][l]), g_ref["R"][l], TOL["bf16"], f"dR[{l}] (sample 0)")
         assert_close(host(g0["W"][l]), g_ref["W"][l], TOL["bf16"], f"dW[{l}] (sample 0)")
-    # full-batch gradients equal the sum of single-sample gradients
+        assert_close(host(g0["b"][l]), g_ref["b"][l], TOL["bf16"], f"db[{l}] (sample 0)")
+
+    # every full-batch gradient equals the sum of the single-sample gradients
+    # taken with the same cotangent (each sample is independent)
+    def flat(g):
+        out = [(k, host(g[k])) for k in ("P", "p", "Q1", "q1", "Q2", "q2")]
+        for l in range(wl.n_layers):
+            out += [(f"R[{l}]", host_complex(g["R"][l])), (f"W[{l}]", host(g["W"][l])),
+                    (f"b[{l}]", host(g["b"][l]))]
+        return out
+
     acc = None
     for s in range(wl.batch):
         _, _, _, gs = step(s, s + 1, du[s:s + 1].clone())
-        flat = [host(gs[k]) for k in ("P", "Q1", "Q2")] + [host(x) for x in gs["W"]]
-        acc = flat if acc is None else [x + y for x, y in zip(acc, flat)]
-    full = [host(g[k]) for k in ("P", "Q1", "Q2")] + [host(x) for x in g["W"]]
-    for i, (x, y) in enumerate(zip(full, acc)):
-        assert_close(x, y, 1e-4, f"gradient {i}: full batch = sum of samples")
+        fs = flat(gs)
+        acc = fs if acc is None else [(k, x + y) for (k, x), (_, y) in zip(acc, fs)]
+    for (k, x), (_, y) in zip(flat(g), acc):
+        assert_close(x, y, 1e-4, f"d{k}: full batch = sum of samples")

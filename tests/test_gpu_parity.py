@@ -156,8 +156,10 @@ def test_block_bwd_wide_channels_f32():
     assert_close(host(y), y_ref, 1e-5, "y")
     k = capi.num_modes(grid, modes)
     dx, dr, dw, db = empty((3, 64) + grid), empty((64, 48, k, 2)), empty((48, 64)), empty((48,))
-    capi.fno_block_bwd(d, dev(x), dev_complex(r), dev(w), pre, None, dev(dy), dx, dr, dw, db)
-    dx_ref, dr_ref, dw_ref, db_ref = O.block_bwd(x, r, w, host(pre), xh_ref, dy, modes)
+    # both sides take the same saved pre-activation: the oracle's, rounded to float32
+    pre_q = synth.quantize(pre_ref, "f32")
+    capi.fno_block_bwd(d, dev(x), dev_complex(r), dev(w), dev(pre_q), None, dev(dy), dx, dr, dw, db)
+    dx_ref, dr_ref, dw_ref, db_ref = O.block_bwd(x, r, w, pre_q, xh_ref, dy, modes)
     assert_close(host(dx), dx_ref, 1e-5, "dx")
     assert_close(host_complex(dr), dr_ref, 1e-5, "dR")
     assert_close(host(dw), dw_ref, 1e-5, "dW")
@@ -206,7 +208,7 @@ def test_network_forward_backward_mse(grid, modes, dtype):
     gd = grads_like(params)
     capi.fno_backward(d, a_d, cp, saves, du, capi.make_grads(gd))
     g_ref = O.backward(a, params, sv, host(du), modes)
-    tol = TOL[dtype] if dtype != "f32" else 2e-5
+    tol = TOL[dtype]
     for key in ("P", "p", "Q1", "q1", "Q2", "q2"):
         assert_close(host(gd[key]), g_ref[key], tol, key)
     for key in ("R", "W", "b"):

@@ -11,6 +11,7 @@ refused."""
 
 import numpy as np
 import pytest
+import torch
 
 from fourier_neural_spectral_fno_b200 import capi, synth
 
@@ -38,6 +39,9 @@ def test_noalloc_matches_workspace_entry_point_twice(grid, modes, dtype):
         capi.fno_spectral_conv_fwd_noalloc(d, x, r, y, xh)
         assert_close(host(y), host(y_ref), TOL[dtype], f"y (call {call})")
         assert_close(host_complex(xh), host_complex(xh_ref), TOL[dtype], f"xhat (call {call})")
+        # the same kernels run on the same inputs, so the results are identical
+        assert torch.equal(y, y_ref), f"y differs bitwise (call {call})"
+        assert torch.equal(xh, xh_ref), f"xhat differs bitwise (call {call})"
 
 
 def test_noalloc_rejects_problems_beyond_the_scratch():
