@@ -48,6 +48,10 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiler captures)")
+    ap.add_argument("--kernel-path", type=int, choices=(0, 1, 2, 3), default=1,
+                    help="library kernel selection (fno_set_tensor_cores): 1 default, "
+                         "3 tensor-core DFT-matrix pipelines, 2 tensor cores without "
+                         "pipelines, 0 CUDA cores")
     return ap.parse_args()
 
 
@@ -179,7 +183,8 @@ def workload_config(wl, n_gpus):
             "blocks": wl.n_layers, "storage": wl.dtype,
             "l2": "flushed between timed steps (512 MiB write outside the step events)",
             "step": ("training: forward + MSE + backward" +
-                     (" + NCCL gradient all-reduce" if n_gpus > 1 else "")
+                     (" + per-group NCCL gradient all-reduce overlapping the backward"
+                      if n_gpus > 1 else "") + " + Adam step"
                      if wl.backward and wl.kind == "network" else "forward"),
             "parallelism": (f"dp{n_gpus} (batch-sharded" +
                             (", gradient all-reduce)" if wl.backward and wl.kind == "network"
@@ -195,8 +200,11 @@ def algorithmic_bytes(tag: str, wl) -> float:
         k *= 2 * m
     spec = wl.batch * wl.width * k * 8
     r = wl.width * wl.width * k * 2 * s
+    u_bytes = wl.batch * wl.width * wl.points // wl.grid[-1] * wl.modes[-1] * 8
     table = {
         "fwd_transform": act + spec,                 # read x, write spectrum
+        "fwd_fft": act + spec,
+        "spec_mid": spec + r + u_bytes,              # read spectrum and R, write U
         "epi_block_fwd": 2 * act + spec,             # read x, write y, read spectrum
         "mix_fwd": 2 * spec + r,
         "lift": wl.batch * wl.in_ch * wl.points * s + act,
@@ -222,7 +230,9 @@ def kernel_source_sha(tag: str) -> str:
              "proj_fwd_tc": "net_tc.cu", "epi_block_fwd_pipe": "epilogue_pipe.cu",
              "fwd_transform_pipe": "transform_pipe.cu", "proj_fwd_pipe": "proj_pipe.cu",
              "epi_block_bwd": "epilogue.cu", "proj_bwd": "net.cu",
-             "fwd_transform_tc_dz": "transform_tc.cu", "fwd_transform_dz": "transform.cu"}
+             "fwd_transform_tc_dz": "transform_tc.cu", "fwd_transform_dz": "transform.cu",
+             "fwd_fft": "transform_fft.cu", "fwd_fft_dz": "transform_fft.cu",
+             "spec_mid": "spec_mid.cu"}
     path = os.path.join(ROOT, "fourier_neural_spectral_fno_b200", "csrc", files.get(tag, ""))
     if not os.path.isfile(path):
         return ""
@@ -295,6 +305,38 @@ def roofline_record(dom: str, avg_ms: float, wl, n_sms: int) -> dict:
             "unit": "GB/s", "frac": (gbs / hbm) if gbs else None,
             "traffic": measured_traffic(dom, wl), "avg_launch_ms": avg_ms,
             "algorithmic_bytes_per_launch": alg}
+
+
+NON_BLOCK_TAGS = ("lift", "proj_fwd", "proj_fwd_tc", "proj_fwd_pipe")
+
+
+def block_roofline_record(stats: dict, steps: int, wl) -> dict:
+    """The spectral block as a whole (forward workloads): its algorithmic HBM
+    bytes (x read once, y written once, R read once) over the summed device time
+    of every kernel that belongs to the blocks, per block, against the measured
+    copy bandwidth; ncu DRAM bytes per block where every block kernel has a
+    current capture."""
+    s = 4 if wl.dtype == "f32" else 2
+    k = wl.modes[-1]
+    for m in wl.modes[:-1]:
+        k *= 2 * m
+    alg = 2 * wl.batch * wl.width * wl.points * s + wl.width * wl.width * k * 2 * s
+    tags = [t for t in stats if t not in NON_BLOCK_TAGS]
+    ms = sum(stats[t]["total_ms"] for t in tags) / steps / wl.n_layers
+    hbm, src = hbm_peak()
+    gbs = alg / (ms / 1e3) / 1e9
+    traffic = 0.0
+    for t in tags:
+        per_launch = measured_traffic(t, wl)
+        if per_launch is None:
+            traffic = None
+            break
+        traffic += per_launch * stats[t]["launches"] / steps / wl.n_layers
+    return {"scope": "one spectral block (all its kernels)", "bound": "hbm", "achieved": gbs,
+            "peak": hbm, "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs, copy)",
+            "unit": "GB/s", "frac": gbs / hbm, "block_ms": ms,
+            "algorithmic_bytes_per_block": float(alg), "traffic": traffic,
+            "kernels": sorted(tags)}
 
 
 def hbm_peak():
@@ -386,6 +428,7 @@ def run_fno(args, dist):
     torch.cuda.set_device(dist.local)
     dev = torch.device("cuda", dist.local)
     capi.load()
+    capi.fno_set_tensor_cores(args.kernel_path)
 
     inp = synth.make_network_inputs(wl)
     tdt = torch.float32 if wl.dtype == "f32" else (torch.float16 if wl.dtype == "f16" else torch.bfloat16)
@@ -404,45 +447,39 @@ def run_fno(args, dist):
     a = up(inp["a"])
     u = torch.empty((wl.batch, wl.out_ch) + wl.grid, dtype=tdt, device=dev)
     train = wl.backward and wl.kind == "network"
-    ws_bytes = capi.fno_net_workspace_size(desc, capi.FNO_OP_NET_FWD)
-    if train:
-        ws_bytes = max(ws_bytes, capi.fno_net_workspace_size(desc, capi.FNO_OP_NET_BWD))
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    ws = None if train else torch.empty(capi.fno_net_workspace_size(desc, capi.FNO_OP_NET_FWD),
+                                        dtype=torch.uint8, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     if train:
-        # forward (keeping the saves), MSE against the target, backward into
-        # float32 gradients; with several ranks the gradients are summed by one
-        # NCCL all-reduce (the cotangent carries the global-mean scaling)
-        from fourier_neural_spectral_fno_b200 import dp
-        saves = torch.empty(capi.fno_net_saves_size(desc), dtype=torch.uint8, device=dev)
-        target = up(inp["target"])
-        loss = torch.empty(1, dtype=torch.float32, device=dev)
-        du = torch.empty_like(u)
-        grads = {k: ([torch.empty(np.shape(x) + ((2,) if np.iscomplexobj(x) else ()),
-                                  dtype=torch.float32, device=dev) for x in v]
-                     if isinstance(v, list) else
-                     torch.empty(np.shape(v), dtype=torch.float32, device=dev))
-                 for k, v in inp["params"].items()}
-        cg = capi.make_grads(grads)
-        scale = dp.mse_scale(u.numel(), u.numel() * dist.world)
+        # one training step of the library's Trainer: forward (keeping the
+        # saves), MSE against the target, backward into the flat float32
+        # gradient, with several ranks the per-group NCCL all-reduces that
+        # overlap the backward, and the fused Adam step that writes the next
+        # step's weights
+        import torch.distributed as tdist
 
-        def step():
-            capi.fno_forward(desc, a, cp, u, saves, ws, stream)
-            capi.fno_mse(u, target, loss, du, wl.dtype, stream)
-            if scale != 1.0:
-                du.mul_(scale)
-            capi.fno_backward(desc, a, cp, saves, du, cg, ws, stream)
-            if dist.world > 1:
-                dp.allreduce_grads(grads)
+        from fourier_neural_spectral_fno_b200 import train as fno_train
+        target = up(inp["target"])
+        trainer = fno_train.Trainer(
+            wl.grid, wl.modes, wl.in_ch, wl.width, inp["params"],
+            fno_train.PrecisionSchedule([(0, wl.dtype)]), hidden=wl.hidden,
+            out_channels=wl.out_ch, n_layers=wl.n_layers,
+            flags=capi.FNO_TANH_PREACT if wl.tanh else 0, lr=1e-4, device=dev,
+            process_group=tdist.group.WORLD if dist.world > 1 else None)
+        loss = torch.empty(1, dtype=torch.float32, device=dev)
+
+        def step(a_in=a, t_in=target, u_out=None, loss_out=loss):
+            loss_out.copy_(trainer.step(a_in, t_in))
     else:
-        def step():
-            capi.fno_forward(desc, a, cp, u, None, ws, stream)
+        target = loss = None
+
+        def step(a_in=a, t_in=None, u_out=u, loss_out=None):
+            capi.fno_forward(desc, a_in, cp, u_out, None, ws, stream)
 
     for _ in range(args.warmup):
         step()
-    launches = capi.last_launch_count()
     torch.cuda.synchronize()
 
     # ---- timed region: K steps, events around each step, L2 flushed between
@@ -474,14 +511,21 @@ def run_fno(args, dist):
     torch.cuda.synchronize()
     capi.fno_profile_enable(False)
     stats = capi.fno_profile_read()
+    launches = sum(v["launches"] for v in stats.values()) // args.steps   # the library's kernels
     dom = max(stats, key=lambda t: stats[t]["total_ms"])
     avg_ms = stats[dom]["total_ms"] / stats[dom]["launches"]
     n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
     roofline = roofline_record(dom, avg_ms, wl, n_sms)
+    if not train:
+        roofline["block"] = block_roofline_record(stats, args.steps, wl)
     per_step = {t: round(v["total_ms"] / args.steps, 4) for t, v in sorted(
         stats.items(), key=lambda kv: -kv[1]["total_ms"])}
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers.  Every step
+    # copies its inputs from pinned host memory and the host reads its result;
+    # two buffer slots let step i+1's input copy and step i's result copy run on
+    # a copy stream while the compute stream works (the stream order still
+    # makes each step wait for its own inputs).
     ins = [a, target] if train else [a]            # the step's inputs
     out = loss if train else u                     # the step's result the host reads
     ins_host = []
@@ -489,30 +533,60 @@ def run_fno(args, dist):
         h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
         h.copy_(t.cpu())
         ins_host.append(h)
-    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    e_steps = max(3, min(args.steps, 20))
+    slots = []
     for _ in range(2):
-        for t, h in zip(ins, ins_host):
-            t.copy_(h, non_blocking=True)
-        step()
-        out_host.copy_(out, non_blocking=True)
+        sl = {"ins": [torch.empty_like(t) for t in ins], "out": torch.empty_like(out),
+              "host": torch.empty(out.shape, dtype=out.dtype, pin_memory=True),
+              "in_ev": torch.cuda.Event(), "done_ev": torch.cuda.Event(),
+              "out_ev": torch.cuda.Event()}
+        slots.append(sl)
+    copy_stream = torch.cuda.Stream(device=dev)
+
+    def e2e_step(i):
+        sl = slots[i & 1]
+        with torch.cuda.stream(copy_stream):
+            if i >= 2:
+                copy_stream.wait_event(sl["out_ev"])    # slot free: step i-2 fully done
+            for t, h in zip(sl["ins"], ins_host):
+                t.copy_(h, non_blocking=True)
+            sl["in_ev"].record(copy_stream)
+        stream.wait_event(sl["in_ev"])
+        if train:
+            step(sl["ins"][0], sl["ins"][1], None, sl["out"])
+        else:
+            step(sl["ins"][0], None, sl["out"], None)
+        sl["done_ev"].record(stream)
+        with torch.cuda.stream(copy_stream):
+            copy_stream.wait_event(sl["done_ev"])
+            sl["host"].copy_(sl["out"], non_blocking=True)
+            sl["out_ev"].record(copy_stream)
+
+    def host_read(i):
+        sl = slots[i & 1]
+        sl["out_ev"].synchronize()
+        return float(sl["host"].view(-1)[0])        # the host reads the step's result
+
+    e_steps = max(3, min(args.steps, 20))
+    for i in range(2):
+        e2e_step(i)
+        host_read(i)
     torch.cuda.synchronize()
     dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(e_steps):
-        for t, h in zip(ins, ins_host):
-            t.copy_(h, non_blocking=True)
-        step()
-        out_host.copy_(out, non_blocking=True)
-        stream.synchronize()
-        float(out_host.view(-1)[0])           # the host reads the step's result
-    e1.record()
+    e0.record(copy_stream)
+    for i in range(e_steps):
+        e2e_step(i)
+        if i >= 1:
+            host_read(i - 1)
+    host_read(e_steps - 1)
+    e1.record(copy_stream)
     torch.cuda.synchronize()
     e_ms = dist.max(e0.elapsed_time(e1) / e_steps)
     e2e = {"value": dist.world * wl.batch / (e_ms / 1e3), "unit": "samples/s",
            "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in ins),
-           "d2h_bytes_per_step": out.numel() * out.element_size(), "ms_per_step": e_ms}
+           "d2h_bytes_per_step": out.numel() * out.element_size(), "ms_per_step": e_ms,
+           "copies": "pinned host buffers; H2D and D2H on a copy stream overlapping the "
+                     "neighbouring steps' compute (two buffer slots)"}
 
     clocks = clk.summary()
     cpu = None
@@ -524,7 +598,8 @@ def run_fno(args, dist):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                 "region_ms_per_step_incl_flush": region_ms / args.steps,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": wl.dtype, "data": "synthetic", "config": workload_config(wl, dist.world),
+                "dtype": wl.dtype, "data": "synthetic",
+                "config": dict(workload_config(wl, dist.world), kernel_path=args.kernel_path),
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches * args.steps, "launches_per_step": launches,
                 "clocks": clocks, "kernels_ms_per_step": per_step}

@@ -45,8 +45,10 @@ EXPORTED = (
     "fno_spectral_conv_bwd", "fno_block_fwd", "fno_block_bwd", "fno_forward", "fno_backward",
     "fno_mse", "fno_profile_enable", "fno_profile_read", "fno_set_tensor_cores",
     "fno_device_error", "fno_spectral_conv_fwd_noalloc", "fno_adam_step",
+    "fno_backward_ready", "fno_spectral_conv_fwd_cp", "fno_block_fwd_cp",
 )
 
+FNO_MAX_CP_RANK = 32
 FNO_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -120,10 +122,15 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "fno_forward": (i, [nd, vp, ctypes.POINTER(Params), vp, vp, vp, sz, vp]),
         "fno_backward": (i, [nd, vp, ctypes.POINTER(Params), vp, vp, ctypes.POINTER(Grads), vp,
                              sz, vp]),
+        "fno_backward_ready": (i, [nd, vp, ctypes.POINTER(Params), vp, vp,
+                                   ctypes.POINTER(Grads), vp, sz, vp,
+                                   ctypes.POINTER(ctypes.c_void_p), i]),
         "fno_mse": (i, [ctypes.c_int64, i, vp, vp, vp, vp, vp]),
         "fno_profile_enable": (i, [i]),
         "fno_set_tensor_cores": (i, [i]),
         "fno_spectral_conv_fwd_noalloc": (i, [bd, vp, vp, vp, vp, vp]),
+        "fno_spectral_conv_fwd_cp": (i, [bd, i, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "fno_block_fwd_cp": (i, [bd, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "fno_device_error": (i, [i]),
         "fno_profile_read": (i, [ctypes.POINTER(KernelStat), i]),
         "fno_adam_step": (i, [ctypes.c_int64, vp, vp, vp, vp, vp, i, i, ctypes.c_float,
@@ -260,6 +267,26 @@ def fno_block_fwd(desc, x, R, W, b, y, pre_save=None, xhat_save=None, ws=None, s
     return y
 
 
+def fno_spectral_conv_fwd_cp(desc, rank, x, lam, A, B, C, y, xhat_save=None, ws=None,
+                             stream=None):
+    """Spectral forward with CP-factorised weights (factors [..][rank][2])."""
+    ws, nb = _workspace(fno_workspace_size(desc, FNO_OP_SPECTRAL_FWD), x.device, ws)
+    _check(load().fno_spectral_conv_fwd_cp(ctypes.byref(desc), int(rank), _ptr(x), _ptr(lam),
+                                           _ptr(A), _ptr(B), _ptr(C), _ptr(y), _ptr(xhat_save),
+                                           _ptr(ws), nb, _stream(stream)))
+    return y
+
+
+def fno_block_fwd_cp(desc, rank, x, lam, A, B, C, W, b, y, pre_save=None, xhat_save=None,
+                     ws=None, stream=None):
+    """Block forward with CP-factorised weights (factors [..][rank][2])."""
+    ws, nb = _workspace(fno_workspace_size(desc, FNO_OP_BLOCK_FWD), x.device, ws)
+    _check(load().fno_block_fwd_cp(ctypes.byref(desc), int(rank), _ptr(x), _ptr(lam), _ptr(A),
+                                   _ptr(B), _ptr(C), _ptr(W), _ptr(b), _ptr(y), _ptr(pre_save),
+                                   _ptr(xhat_save), _ptr(ws), nb, _stream(stream)))
+    return y
+
+
 def fno_block_bwd(desc, x, R, W, pre_save, xhat_save, dy, dx, dR, dW, db, ws=None, stream=None):
     ws, nb = _workspace(fno_workspace_size(desc, FNO_OP_BLOCK_BWD), x.device, ws)
     _check(load().fno_block_bwd(ctypes.byref(desc), _ptr(x), _ptr(R), _ptr(W), _ptr(pre_save),
@@ -298,10 +325,25 @@ def fno_forward(desc, a, params: Params, u, saves=None, ws=None, stream=None):
     return u
 
 
-def fno_backward(desc, a, params: Params, saves, du, grads: Grads, ws=None, stream=None):
+def fno_backward(desc, a, params: Params, saves, du, grads: Grads, ws=None, stream=None,
+                 ready=None):
+    """``ready``: optional list of n_layers + 2 ``torch.cuda.Event`` that the
+    backward records as each gradient group becomes final (fno_backward_ready):
+    the projection's, then the layers' from the last to the first, then the lift's."""
     ws, nb = _workspace(fno_net_workspace_size(desc, FNO_OP_NET_BWD), a.device, ws)
-    _check(load().fno_backward(ctypes.byref(desc), _ptr(a), ctypes.byref(params), _ptr(saves),
-                               _ptr(du), ctypes.byref(grads), _ptr(ws), nb, _stream(stream)))
+    if ready is None:
+        _check(load().fno_backward(ctypes.byref(desc), _ptr(a), ctypes.byref(params), _ptr(saves),
+                                   _ptr(du), ctypes.byref(grads), _ptr(ws), nb, _stream(stream)))
+        return
+    handles = []
+    for ev in ready:
+        if ev.cuda_event == 0:      # torch creates the event lazily, on its first record
+            ev.record()
+        handles.append(ev.cuda_event)
+    arr = (ctypes.c_void_p * len(handles))(*handles)
+    _check(load().fno_backward_ready(ctypes.byref(desc), _ptr(a), ctypes.byref(params),
+                                     _ptr(saves), _ptr(du), ctypes.byref(grads), _ptr(ws), nb,
+                                     _stream(stream), arr, len(handles)))
     return grads
 
 
@@ -326,12 +368,14 @@ def fno_profile_read(max_kernels: int = 64) -> Dict[str, Dict[str, float]]:
 
 
 def fno_set_tensor_cores(mode) -> int:
-    """Kernel selection: 1 / True = tcgen05 kernels with the TMA pipelines where
-    shapes allow, 2 = tcgen05 kernels without the pipelines, 0 / False = the
-    CUDA-core kernels.  Returns the previous setting."""
+    """Kernel selection: 1 / True = the default kernels (pruned-FFT transform
+    and fused spectral middle on the CUDA cores, tcgen05 TMA pipelines for the
+    epilogue and projection) where shapes allow, 3 = tcgen05 TMA pipelines
+    throughout (dense DFT-matrix transform), 2 = tcgen05 kernels without the
+    pipelines, 0 / False = the CUDA-core kernels.  Returns the previous setting."""
     m = int(mode)
-    if m not in (0, 1, 2):
-        raise ValueError("tensor-core mode must be 0, 1 or 2")
+    if m not in (0, 1, 2, 3):
+        raise ValueError("kernel mode must be 0, 1, 2 or 3")
     return int(load().fno_set_tensor_cores(m))
 
 

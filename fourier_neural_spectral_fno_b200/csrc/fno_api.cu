@@ -205,20 +205,31 @@ Launch make_launch(fno_stream_t s) {
   return L;
 }
 
+// u_ready: U (ws + w.u) already holds the spectrum inverted along the slab
+// axis (launch_spec_mid), so no slab-axis inverse is launched here.
 cudaError_t run_epilogue(const Launch &L, const Geom &g, int dtype, int mode, const EpiArgs &a,
-                         unsigned char *ws, const BlockWs &w) {
+                         unsigned char *ws, const BlockWs &w, bool u_ready = false) {
   float2 *U = reinterpret_cast<float2 *>(ws + w.u);
   // channels of the spectrum being inverted: Ci for the backward modes (dxhat)
   const int cs = (mode == EPI_SPEC_BWD || mode == EPI_BLOCK_BWD) ? a.Ci : a.Co;
-  if (L.tc == 1 && epi_pipe_supported(g, dtype, mode, a.Ci, a.Co, a.x, U)) {
-    cudaError_t e = launch_inv_slab(L, g, cs, a.Z, U);
-    if (e != cudaSuccess) return e;
+  if ((L.tc == 1 || L.tc == 3) && epi_pipe_supported(g, dtype, mode, a.Ci, a.Co, a.x, U)) {
+    if (!u_ready) {
+      cudaError_t e = launch_inv_slab(L, g, cs, a.Z, U);
+      if (e != cudaSuccess) return e;
+    }
     return launch_epi_pipe(L, g, dtype, mode, a, U);
   }
   if (L.tc && epi_tc_supported(g, dtype, mode, a.Ci, a.Co)) {
-    cudaError_t e = launch_inv_slab(L, g, cs, a.Z, U);
-    if (e != cudaSuccess) return e;
+    if (!u_ready) {
+      cudaError_t e = launch_inv_slab(L, g, cs, a.Z, U);
+      if (e != cudaSuccess) return e;
+    }
     return launch_epilogue_tc(L, g, dtype, mode, a, U);
+  }
+  if (u_ready) {
+    EpiArgs b = a;
+    b.U = U;
+    return launch_epilogue(L, g, dtype, mode, b);
   }
   if (mode == EPI_BLOCK_BWD && g.S > 1) {
     // the block backward reads the slab-axis inverse once per row instead of
@@ -236,9 +247,11 @@ cudaError_t run_epilogue(const Launch &L, const Geom &g, int dtype, int mode, co
 // block-level building blocks (validated arguments)
 // ---------------------------------------------------------------------------
 
+// cp (optional): CP-factorised weights of the given rank in place of R
 int run_forward(const Launch &L, const Geom &g, int dtype, unsigned flags, int Ci, int Co,
                 const void *x, const void *R, const void *W, const void *b, void *y, void *pre,
-                float *xhat_save, unsigned char *ws, int epi_mode) {
+                float *xhat_save, unsigned char *ws, int epi_mode, const CpFactors *cp = nullptr,
+                int rank = 0) {
   const BlockWs w = block_ws(g, Ci, Co, epi_mode == EPI_SPEC ? FNO_OP_SPECTRAL_FWD : FNO_OP_BLOCK_FWD);
   float2 *zpart = reinterpret_cast<float2 *>(ws + w.zpart);
   float2 *xhat = xhat_save ? reinterpret_cast<float2 *>(xhat_save)
@@ -247,7 +260,15 @@ int run_forward(const Launch &L, const Geom &g, int dtype, unsigned flags, int C
   FNO_TRY(launch_fwd_transform(L, g, dtype, (flags & FNO_TANH_PREACT) ? LOAD_TANH : LOAD_PLAIN,
                                Ci, x, nullptr, zpart, xhat),
           "forward transform");
-  FNO_TRY(launch_mix_fwd(L, g, dtype, Ci, Co, xhat, R, yhat), "mixing");
+  // 2D grids on the default path: mixing and the slab-axis inverse in one launch
+  const bool mid = !cp && L.tc == 1 && spec_mid_supported(g);
+  if (cp)
+    FNO_TRY(launch_mix_cp(L, g, dtype, Ci, Co, rank, xhat, *cp, yhat), "factorised mixing");
+  else if (mid)
+    FNO_TRY(launch_spec_mid(L, g, dtype, Ci, Co, xhat, R, reinterpret_cast<float2 *>(ws + w.u)),
+            "mixing and slab-axis inverse");
+  else
+    FNO_TRY(launch_mix_fwd(L, g, dtype, Ci, Co, xhat, R, yhat), "mixing");
   const float2 *Z = yhat;
   if (g.QO > 1) {
     float2 *zexp = reinterpret_cast<float2 *>(ws + w.zexp);
@@ -265,7 +286,7 @@ int run_forward(const Launch &L, const Geom &g, int dtype, unsigned flags, int C
   a.Co = Co;
   a.act = !(flags & FNO_NO_ACT);
   a.tanh_pre = (flags & FNO_TANH_PREACT) ? 1 : 0;
-  FNO_TRY(run_epilogue(L, g, dtype, epi_mode, a, ws, w), "epilogue");
+  FNO_TRY(run_epilogue(L, g, dtype, epi_mode, a, ws, w, mid), "epilogue");
   return FNO_OK;
 }
 
@@ -452,7 +473,7 @@ int fno_last_launch_count(void) { return g_launches; }
 
 int fno_set_tensor_cores(int enable) {
   const int prev = g_use_tc;
-  g_use_tc = enable == 2 ? 2 : enable ? 1 : 0;
+  g_use_tc = (enable == 2 || enable == 3) ? enable : enable ? 1 : 0;
   return prev;
 }
 
@@ -601,6 +622,69 @@ int fno_block_fwd(const fno_block_desc *desc, const void *x, const void *R, cons
   return rc;
 }
 
+static int check_cp(const fno_block_desc *desc, const Geom &g, int rank, const void *lam,
+                    const void *A, const void *B, const void *C) {
+  if (rank < 1) return fail(FNO_ERR_INVALID_ARG, "rank %d < 1", rank);
+  if (rank > kMaxCpRank)
+    return fail(FNO_ERR_UNSUPPORTED, "rank %d exceeds %d", rank, kMaxCpRank);
+  REQUIRE_PTR(lam, "lam");
+  REQUIRE_PTR(A, "A");
+  REQUIRE_PTR(B, "B");
+  REQUIRE_PTR(C, "C");
+  const size_t smem = sizeof(float2) * (size_t)(desc->cin + desc->cout) * kMaxCpRank;
+  if (smem > kSmemLimit) return fail(FNO_ERR_UNSUPPORTED, "factor staging needs %zu B", smem);
+  (void)g;
+  return FNO_OK;
+}
+
+int fno_spectral_conv_fwd_cp(const fno_block_desc *desc, int rank, const void *x, const void *lam,
+                             const void *A, const void *B, const void *C, void *y,
+                             float *xhat_save, void *ws, size_t ws_bytes, fno_stream_t stream) {
+  Geom g;
+  int rc = check_block(desc, &g);
+  if (rc) return rc;
+  if ((rc = check_smem(g, desc->cin, desc->cout, FNO_OP_SPECTRAL_FWD))) return rc;
+  if ((rc = check_cp(desc, g, rank, lam, A, B, C))) return rc;
+  REQUIRE_PTR(x, "x");
+  REQUIRE_PTR(y, "y");
+  OPTIONAL_PTR(xhat_save, "xhat_save");
+  const size_t need = block_ws(g, desc->cin, desc->cout, FNO_OP_SPECTRAL_FWD).total;
+  if (ws_bytes < need) return fail(FNO_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, need);
+  REQUIRE_PTR(ws, "ws");
+  Launch L = make_launch(stream);
+  const CpFactors f{lam, A, B, C};
+  rc = run_forward(L, g, desc->dtype, desc->flags, desc->cin, desc->cout, x, nullptr, nullptr,
+                   nullptr, y, nullptr, xhat_save, (unsigned char *)ws, EPI_SPEC, &f, rank);
+  if (!rc) g_err[0] = 0;
+  return rc;
+}
+
+int fno_block_fwd_cp(const fno_block_desc *desc, int rank, const void *x, const void *lam,
+                     const void *A, const void *B, const void *C, const void *W, const void *b,
+                     void *y, void *pre_save, float *xhat_save, void *ws, size_t ws_bytes,
+                     fno_stream_t stream) {
+  Geom g;
+  int rc = check_block(desc, &g);
+  if (rc) return rc;
+  if ((rc = check_smem(g, desc->cin, desc->cout, FNO_OP_BLOCK_FWD))) return rc;
+  if ((rc = check_cp(desc, g, rank, lam, A, B, C))) return rc;
+  REQUIRE_PTR(x, "x");
+  REQUIRE_PTR(W, "W");
+  REQUIRE_PTR(b, "b");
+  REQUIRE_PTR(y, "y");
+  OPTIONAL_PTR(pre_save, "pre_save");
+  OPTIONAL_PTR(xhat_save, "xhat_save");
+  const size_t need = block_ws(g, desc->cin, desc->cout, FNO_OP_BLOCK_FWD).total;
+  if (ws_bytes < need) return fail(FNO_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, need);
+  REQUIRE_PTR(ws, "ws");
+  Launch L = make_launch(stream);
+  const CpFactors f{lam, A, B, C};
+  rc = run_forward(L, g, desc->dtype, desc->flags, desc->cin, desc->cout, x, nullptr, W, b, y,
+                   pre_save, xhat_save, (unsigned char *)ws, EPI_BLOCK_FWD, &f, rank);
+  if (!rc) g_err[0] = 0;
+  return rc;
+}
+
 int fno_block_bwd(const fno_block_desc *desc, const void *x, const void *R, const void *W,
                   const void *pre_save, const float *xhat_save, const void *dy, void *dx,
                   float *dR, float *dW, float *db, void *ws, size_t ws_bytes,
@@ -684,9 +768,22 @@ int fno_forward(const fno_net_desc *desc, const void *a, const fno_params *param
 int fno_backward(const fno_net_desc *desc, const void *a, const fno_params *params,
                  const void *saves, const void *du, fno_grads *grads, void *ws, size_t ws_bytes,
                  fno_stream_t stream) {
+  return fno_backward_ready(desc, a, params, saves, du, grads, ws, ws_bytes, stream, nullptr, 0);
+}
+
+int fno_backward_ready(const fno_net_desc *desc, const void *a, const fno_params *params,
+                       const void *saves, const void *du, fno_grads *grads, void *ws,
+                       size_t ws_bytes, fno_stream_t stream, fno_event_t *ready, int n_ready) {
   Geom g;
   int rc = check_net(desc, &g);
   if (rc) return rc;
+  if (ready || n_ready) {
+    if (!ready || n_ready != desc->n_layers + 2)
+      return fail(FNO_ERR_INVALID_ARG, "ready needs n_layers + 2 = %d events (got %d%s)",
+                  desc->n_layers + 2, n_ready, ready ? "" : ", array NULL");
+    for (int j = 0; j < n_ready; ++j)
+      if (!ready[j]) return fail(FNO_ERR_INVALID_ARG, "ready[%d] is NULL", j);
+  }
   REQUIRE_PTR(a, "a");
   if (!params) return fail(FNO_ERR_INVALID_ARG, "params is NULL");
   if (!grads) return fail(FNO_ERR_INVALID_ARG, "grads is NULL");
@@ -730,12 +827,14 @@ int fno_backward(const fno_net_desc *desc, const void *a, const fno_params *para
   FNO_TRY(launch_reduce_rows(L, partial, np, pstride, (long long)hidden * (width + 1), outc,
                              hidden, grads->Q2, grads->q2),
           "dQ2 reduction");
+  if (ready) FNO_TRY(cudaEventRecord(ready[0], L.stream), "recording ready[0]");
   for (int l = nl - 1; l >= 0; --l) {
     rc = run_backward(L, g, desc->dtype, desc->flags, width, width, sv + sm.x(l),
                       reinterpret_cast<const float *>(sv + sm.xh(l)), params->R[l], params->W[l],
                       sv + sm.pre(l), dv[(l + 1) & 1], dv[l & 1], grads->R[l], grads->W[l],
                       grads->b[l], wsb + w.block, true);
     if (rc) return rc;
+    if (ready) FNO_TRY(cudaEventRecord(ready[nl - l], L.stream), "recording a layer's ready event");
   }
   FNO_TRY(launch_lift_bwd(L, g, desc->dtype, desc->in_channels, width, a, dv[0], partial),
           "lift backward");
@@ -743,6 +842,7 @@ int fno_backward(const fno_net_desc *desc, const void *a, const fno_params *para
   FNO_TRY(launch_reduce_rows(L, partial, nl2, (long long)width * (desc->in_channels + 1), 0, width,
                              desc->in_channels, grads->P, grads->p),
           "dP reduction");
+  if (ready) FNO_TRY(cudaEventRecord(ready[nl + 1], L.stream), "recording ready[L + 1]");
   g_err[0] = 0;
   return FNO_OK;
 }

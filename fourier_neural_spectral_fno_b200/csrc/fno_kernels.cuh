@@ -35,7 +35,10 @@ struct Launch {
   cudaStream_t stream;
   int *count;       // incremented per kernel launch
   int num_sms;
-  int tc;           // 1: tensor-core kernels + TMA pipelines, 2: without pipelines, 0: none
+  int tc;           // 1: default (pruned-FFT transform and fused spectral middle on CUDA
+                    //    cores, tcgen05 TMA pipelines for the epilogue and projection);
+                    // 3: tcgen05 TMA pipelines throughout (dense DFT-matrix transform);
+                    // 2: tcgen05 without the pipelines; 0: CUDA cores only
   int *err;         // device error word (bounded waits that expired)
 };
 
@@ -68,6 +71,29 @@ cudaError_t launch_s1_tc(const Launch &L, const Geom &g, int dtype, int load_mod
 bool fwd_pipe_supported(const Geom &g, int dtype, int load_mode, const void *in0);
 cudaError_t launch_fwd_pipe(const Launch &L, const Geom &g, int dtype, int load_mode,
                             long long C, const void *in0, float2 *zpart);
+
+// pruned radix-16 FFT transform on the CUDA cores (transform_fft.cu): one
+// thread-block cluster per plane writes out[plane][QS][mL] (for 2D grids that
+// is xhat itself; for 3D the outer axis is still to be contracted)
+bool fwd_fft_supported(const Geom &g, const void *in0, const void *in1, int load_mode);
+cudaError_t launch_fwd_fft(const Launch &L, const Geom &g, int dtype, int load_mode, long long C,
+                           const void *in0, const void *in1, float2 *out);
+
+// 2D spectral middle (spec_mid.cu): mixing + slab-axis inverse in one launch,
+// U[b][o][S][mL] = sum_q ((c_k/N) sum_i xhat[b,i,q,k] R[i,o,q,k]) exp(+i kq n)
+bool spec_mid_supported(const Geom &g);
+cudaError_t launch_spec_mid(const Launch &L, const Geom &g, int dtype, int Ci, int Co,
+                            const float2 *xhat, const void *R, float2 *U);
+
+// CP-factorised weights (mix_cp.cu): R[i,o,k] = sum_r lam[r] A[i,r] B[o,r] C[k,r],
+// factors complex (re, im) in the storage dtype: lam [rank], A [Ci][rank],
+// B [Co][rank], C [K][rank]; yhat as launch_mix_fwd writes it
+constexpr int kMaxCpRank = 32;
+struct CpFactors {
+  const void *lam, *A, *B, *C;
+};
+cudaError_t launch_mix_cp(const Launch &L, const Geom &g, int dtype, int Ci, int Co, int rank,
+                          const float2 *xhat, const CpFactors &f, float2 *yhat);
 
 // ---- mixing (S3) -----------------------------------------------------------
 // yhat[b,o,k] = (c_k / N) sum_i xhat[b,i,k] R[i,o,k]

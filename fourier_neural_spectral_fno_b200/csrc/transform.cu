@@ -263,7 +263,14 @@ cudaError_t launch_fwd_transform(const Launch &L, const Geom &g, int dtype, int 
   const long long planes = g.B * C * g.O;
   int nb;
   cudaError_t err;
-  if (L.tc == 1 && fwd_pipe_supported(g, dtype, load_mode, in0)) {
+  if (L.tc == 1 && fwd_fft_supported(g, in0, in1, load_mode)) {
+    // the cluster writes whole plane spectra: 2D grids are done, 3D grids
+    // still contract the outer axis (one "band")
+    if (g.QO == 1) return launch_fwd_fft(L, g, dtype, load_mode, C, in0, in1, xhat);
+    err = launch_fwd_fft(L, g, dtype, load_mode, C, in0, in1, zpart);
+    if (err != cudaSuccess) return err;
+    nb = 1;
+  } else if ((L.tc == 1 || L.tc == 3) && fwd_pipe_supported(g, dtype, load_mode, in0)) {
     nb = s1_tc_bands(g);
     err = launch_fwd_pipe(L, g, dtype, load_mode, C, in0, zpart);
     if (err != cudaSuccess) return err;

@@ -13,8 +13,10 @@ All weights live in flat device buffers with one 16-byte aligned slot per
 parameter: the float32 master copy, the Adam moments, the float32 gradient
 that ``fno_backward`` writes, and the copy in the current storage dtype that
 the forward reads.  A step is forward, MSE and backward in that step's
-dtype, an optional all-reduce of the flat gradient (data parallelism over the
-batch), then one fused ``fno_adam_step`` launch that updates the master copy
+dtype, the all-reduce of the gradient (data parallelism over the batch: one
+collective per gradient group, started as soon as the backward has finished
+the group, so that it overlaps the backward of the earlier layers), then one
+fused ``fno_adam_step`` launch that updates the master copy
 and writes the next step's weights in the next step's dtype.
 
 Host logic only: every arithmetic step runs in ``libfno.so``; torch provides
@@ -79,18 +81,21 @@ class PrecisionSchedule:
 class ParamLayout:
     """Slots of the network's parameters in one flat buffer.
 
-    Order: P, p, R[0..L-1], W[0..L-1], b[0..L-1], Q1, q1, Q2, q2, with the
-    shapes of ``fno_params`` (R as [width][width][|K|][2] (re, im)).  Every
-    slot starts at a multiple of ``ALIGN`` elements; the gaps stay zero.
+    Order: P, p, then per layer R[l], W[l], b[l], then Q1, q1, Q2, q2, with
+    the shapes of ``fno_params`` (R as [width][width][|K|][2] (re, im)).  Every
+    slot starts at a multiple of ``ALIGN`` elements; the gaps stay zero.  The
+    parameters of each gradient group the backward finishes together (the
+    projection, each layer, the lift) are one contiguous range, so each group's
+    all-reduce is one collective on a view of the flat gradient.
     """
 
     def __init__(self, in_channels: int, width: int, hidden: int, out_channels: int,
                  n_layers: int, n_modes: int):
         self.n_layers = n_layers
         entries = [("P", None, (width, in_channels)), ("p", None, (width,))]
-        entries += [("R", l, (width, width, n_modes, 2)) for l in range(n_layers)]
-        entries += [("W", l, (width, width)) for l in range(n_layers)]
-        entries += [("b", l, (width,)) for l in range(n_layers)]
+        for l in range(n_layers):
+            entries += [("R", l, (width, width, n_modes, 2)), ("W", l, (width, width)),
+                        ("b", l, (width,))]
         entries += [("Q1", None, (hidden, width)), ("q1", None, (hidden,)),
                     ("Q2", None, (out_channels, hidden)), ("q2", None, (out_channels,))]
         self.slots = []
@@ -100,6 +105,24 @@ class ParamLayout:
             self.slots.append((key, layer, shape, off, size))
             off += (size + ALIGN - 1) // ALIGN * ALIGN
         self.total = off
+
+    def _start(self, key: str, layer=None) -> int:
+        for k, l, _, off, _ in self.slots:
+            if k == key and l == layer:
+                return off
+        raise KeyError(key)
+
+    def buckets(self) -> List[Tuple[int, int]]:
+        """[lo, hi) element ranges of the gradient groups in the order the
+        backward finishes them (fno_backward_ready): the projection, the layers
+        from the last to the first, the lift.  Together they tile [0, total)."""
+        L = self.n_layers
+        starts = [self._start("R", l) for l in range(L)] + [self._start("Q1")]
+        out = [(starts[L], self.total)]
+        for l in range(L - 1, -1, -1):
+            out.append((starts[l], starts[l + 1]))
+        out.append((0, starts[0]))
+        return out
 
     def views(self, flat) -> Dict[str, object]:
         """Per-parameter views of ``flat`` (lists for R, W, b)."""
@@ -177,6 +200,9 @@ class Trainer:
         self.dtype: Optional[str] = None
         self.weights = None
         self._bufs: Dict[Tuple[str, int], Dict[str, object]] = {}
+        self._buckets = self.layout.buckets()
+        self._ready = None        # per-group events and the collective stream (CUDA, world > 1)
+        self._comm = None
 
     # ---------------------------------------------------------------- helpers
     def _desc(self, dtype: str, batch: int):
@@ -235,6 +261,22 @@ class Trainer:
         self.eps, self.weight_decay = float(state["eps"]), float(state["weight_decay"])
         self.dtype, self.weights = None, None     # the next step copies the master afresh
 
+    def _allreduce_buckets(self) -> None:
+        """Sum every gradient group over the process group, one collective per
+        group in the order the backward finishes them (on CUDA: on the
+        collective stream, each after its group's ready event)."""
+        import torch
+        import torch.distributed as dist
+        if self._ready is None:
+            for lo, hi in self._buckets:
+                dist.all_reduce(self.grad[lo:hi], group=self.pg)
+            return
+        for (lo, hi), ev in zip(self._buckets, self._ready):
+            self._comm.wait_event(ev)
+            with torch.cuda.stream(self._comm):
+                dist.all_reduce(self.grad[lo:hi], group=self.pg)
+        torch.cuda.current_stream(self.device).wait_stream(self._comm)
+
     # ------------------------------------------------------------------- step
     def step(self, a, target):
         """One step on a batch: ``a`` [B][in][grid], ``target`` [B][out][grid]
@@ -252,13 +294,26 @@ class Trainer:
         cg = capi.make_grads(self.layout.views(self.grad))
         capi.fno_forward(d, a_s, cp, b["u"], b["saves"], ws=b["ws_fwd"])
         capi.fno_mse(b["u"], t_s, b["loss"], b["du"], dtype=dt)
-        capi.fno_backward(d, a_s, cp, b["saves"], b["du"], cg, ws=b["ws_bwd"])
         scale = 1.0
+        world = 1
         if self.pg is not None:
             import torch.distributed as dist
             world = dist.get_world_size(self.pg)
+        if world > 1 and self.device.type == "cuda":
+            # each gradient group's all-reduce starts on the collective stream as
+            # soon as the backward has finished that group, overlapping the
+            # backward of the earlier layers
+            if self._ready is None:
+                self._ready = [torch.cuda.Event() for _ in self._buckets]
+                self._comm = torch.cuda.Stream(device=self.device)
+            capi.fno_backward(d, a_s, cp, b["saves"], b["du"], cg, ws=b["ws_bwd"],
+                              ready=self._ready)
+            self._allreduce_buckets()
+            scale = 1.0 / world
+        else:
+            capi.fno_backward(d, a_s, cp, b["saves"], b["du"], cg, ws=b["ws_bwd"])
             if world > 1:
-                dist.all_reduce(self.grad, group=self.pg)
+                self._allreduce_buckets()
                 scale = 1.0 / world
         self.step_count += 1
         nxt = self.schedule.dtype_at(self.step_count)

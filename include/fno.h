@@ -62,6 +62,7 @@ extern "C" {
 #endif
 
 typedef struct CUstream_st *fno_stream_t; /* identical to cudaStream_t */
+typedef struct CUevent_st *fno_event_t;   /* identical to cudaEvent_t */
 
 enum fno_status {
   FNO_OK = 0,
@@ -151,11 +152,14 @@ const char *fno_version(void);
 /* Number of kernel launches the last successful call on this thread enqueued. */
 int fno_last_launch_count(void);
 
-/* Kernel selection: 1 (default) uses the tcgen05 tensor-core kernels wherever
- * the shape allows them, including the warp-specialised TMA pipelines; 2 uses
- * the tensor-core kernels without the TMA pipelines; 0 forces the CUDA-core
- * kernels everywhere.  All are complete implementations; the switch exists to
- * compare them.  Process-wide; returns the previous setting. */
+/* Kernel selection.  1 (default): the pruned radix-16 FFT transform and the
+ * fused mixing + slab-axis inverse on the CUDA cores, with the warp-specialised
+ * tcgen05 TMA pipelines for the epilogue and the projection, wherever the shape
+ * allows each; 3: the tcgen05 TMA pipelines throughout, the transform as a
+ * dense DFT-matrix contraction on the tensor cores; 2: the tensor-core kernels
+ * without the TMA pipelines; 0: the CUDA-core kernels everywhere.  All are
+ * complete implementations; the switch exists to compare them.  Process-wide;
+ * any other nonzero value means 1; returns the previous setting. */
 int fno_set_tensor_cores(int enable);
 
 /* Synchronises the current device and reads the library's device error word,
@@ -225,6 +229,23 @@ int fno_spectral_conv_fwd(const fno_block_desc *desc, const void *x, const void 
 int fno_spectral_conv_fwd_noalloc(const fno_block_desc *desc, const void *x, const void *R,
                                   void *y, float *xhat_save, fno_stream_t stream);
 
+/* Factorised spectral weights (TFNO of [MPTRAIN], summary): the weight is the
+ * rank-`rank` CP tensor R[i,o,k] = sum_r lam[r] A[i,r] B[o,r] C[k,r] and is
+ * never formed; the mixing contracts xhat with A over i, multiplies by C and
+ * contracts with lam B over r (the order the greedy planner picks at low
+ * rank).  Factors are complex, (re, im) interleaved in the storage dtype:
+ * lam [rank][2], A [Ci][rank][2], B [Co][rank][2], C [|K|][rank][2], K in the
+ * order of R.  1 <= rank <= FNO_MAX_CP_RANK.  Workspace, other arguments,
+ * results and errors are those of fno_spectral_conv_fwd / fno_block_fwd. */
+#define FNO_MAX_CP_RANK 32
+int fno_spectral_conv_fwd_cp(const fno_block_desc *desc, int rank, const void *x, const void *lam,
+                             const void *A, const void *B, const void *C, void *y,
+                             float *xhat_save, void *ws, size_t ws_bytes, fno_stream_t stream);
+int fno_block_fwd_cp(const fno_block_desc *desc, int rank, const void *x, const void *lam,
+                     const void *A, const void *B, const void *C, const void *W, const void *b,
+                     void *y, void *pre_save, float *xhat_save, void *ws, size_t ws_bytes,
+                     fno_stream_t stream);
+
 /* Adjoint of fno_spectral_conv_fwd.  Inputs: x (needed for tanh'), xhat_save
  * from the forward (may be NULL: then it is recomputed from x), R, dy
  * [B][Co][grid].  Outputs: dx [B][Ci][grid] (storage dtype),
@@ -258,6 +279,23 @@ int fno_forward(const fno_net_desc *desc, const void *a, const fno_params *param
 int fno_backward(const fno_net_desc *desc, const void *a, const fno_params *params,
                  const void *saves, const void *du, fno_grads *grads, void *ws,
                  size_t ws_bytes, fno_stream_t stream);
+
+/* fno_backward that also reports when each group of gradients is final, for
+ * data parallelism whose gradient all-reduce overlaps the rest of the backward
+ * ("Efficient multi-GPU distributed training strategies for neural operator
+ * networks", key methods: all-reduce data parallelism).  The backward finishes
+ * the groups in this order and records ready[j] (cudaEventRecord on `stream`)
+ * right after group j's last kernel:
+ *   ready[0]                 dQ1, dq1, dQ2, dq2 (projection)
+ *   ready[1 + j], j < L      dR, dW, db of layer L - 1 - j (L = n_layers)
+ *   ready[L + 1]             dP, dp (lift)
+ * The events belong to the caller (created by it, any flags); n_ready must be
+ * n_layers + 2.  A caller that makes a second stream wait on ready[j] can start
+ * group j's all-reduce there while the backward of the earlier layers runs.
+ * Arguments, results and errors are otherwise those of fno_backward. */
+int fno_backward_ready(const fno_net_desc *desc, const void *a, const fno_params *params,
+                       const void *saves, const void *du, fno_grads *grads, void *ws,
+                       size_t ws_bytes, fno_stream_t stream, fno_event_t *ready, int n_ready);
 
 /* Mean-squared error over n elements: *loss = mean((u - t)^2) (float32,
  * device), du = 2 (u - t) / n (storage dtype).  du may be NULL. */

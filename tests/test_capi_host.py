@@ -273,3 +273,42 @@ def test_network_bindings_pass_each_pointer_in_place(lib, which, arg, msg):
                               buf(arg == "du"), capi.make_grads(grads), stream=0)
     assert e.value.code == capi.FNO_ERR_INVALID_ARG
     assert f": {msg} is not 16-byte aligned" in str(e.value)
+
+
+def test_factorised_forward_validation(lib):
+    d = capi.block_desc(2, 4, 4, (16, 16), (4, 4))
+    need = capi.fno_workspace_size(d, capi.FNO_OP_BLOCK_FWD)
+    f = lib.fno_block_fwd_cp
+    ok = dict(x=256, lam=256, A=256, B=256, C=256, W=256, b=256, y=256)
+
+    def call(rank, **kw):
+        a = dict(ok, **kw)
+        return f(ctypes.byref(d), rank, a["x"], a["lam"], a["A"], a["B"], a["C"], a["W"], a["b"],
+                 a["y"], None, None, 256, need, None)
+    assert call(0) == capi.FNO_ERR_INVALID_ARG and "rank" in capi.last_error()
+    assert call(capi.FNO_MAX_CP_RANK + 1) == capi.FNO_ERR_UNSUPPORTED
+    for name in ("lam", "A", "B", "C"):
+        assert call(4, **{name: None}) == capi.FNO_ERR_INVALID_ARG
+        assert name in capi.last_error()
+        assert call(4, **{name: 0x1008}) == capi.FNO_ERR_INVALID_ARG
+    g = lib.fno_spectral_conv_fwd_cp
+    assert g(ctypes.byref(d), 4, 256, 256, 256, 256, 256, 256, None, 256, 1,
+             None) == capi.FNO_ERR_WORKSPACE
+
+
+def test_backward_ready_validation(lib):
+    d = capi.net_desc(2, (16, 16), (4, 4), 3, 8, 16, 1, 2)
+    need = capi.fno_net_workspace_size(d, capi.FNO_OP_NET_BWD)
+    params, grads = capi.Params(), capi.Grads()
+    evs = (ctypes.c_void_p * 4)(*([0x100] * 4))
+    f = lib.fno_backward_ready
+    # wrong count, NULL array with a count, and a NULL event are refused up front
+    assert f(ctypes.byref(d), 256, ctypes.byref(params), 256, 256, ctypes.byref(grads), 256, need,
+             None, evs, 3) == capi.FNO_ERR_INVALID_ARG
+    assert "n_layers + 2" in capi.last_error()
+    assert f(ctypes.byref(d), 256, ctypes.byref(params), 256, 256, ctypes.byref(grads), 256, need,
+             None, None, 4) == capi.FNO_ERR_INVALID_ARG
+    evs[2] = None
+    assert f(ctypes.byref(d), 256, ctypes.byref(params), 256, 256, ctypes.byref(grads), 256, need,
+             None, evs, 4) == capi.FNO_ERR_INVALID_ARG
+    assert "ready[2]" in capi.last_error()

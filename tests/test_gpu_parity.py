@@ -39,14 +39,25 @@ SHAPES = [
     ((256, 96), (16, 12)),
     ((384, 128), (10, 16)),
     ((4, 128, 64), (2, 8, 8)),
+    # shapes the pruned-FFT transform takes (last axis 64, 128, 256 or 512 with
+    # at most 32 modes): ragged slab bands, several-CTA clusters, the fused
+    # spectral middle (slab axis a multiple of 16) and its fallback
+    ((40, 256), (7, 16)),
+    ((48, 512), (9, 32)),
+    ((272, 64), (30, 5)),
+    ((1100, 64), (3, 8)),
+    ((96, 128), (20, 24)),
+    ((6, 32, 128), (3, 4, 9)),
 ]
 
 
-@pytest.fixture(autouse=True, params=[1, 2, 0], ids=["tc", "tc_nopipe", "cudacore"])
+@pytest.fixture(autouse=True, params=[1, 3, 2, 0], ids=["default", "tc_dft", "tc_nopipe", "cudacore"])
 def kernel_path(request):
-    """Every parity test runs on the tcgen05 kernels with the TMA pipelines,
-    on the tcgen05 kernels without them (where the shape allows either) and on
-    the CUDA-core kernels; no bounded device wait may expire."""
+    """Every parity test runs on the default kernels (pruned-FFT transform and
+    fused spectral middle, tcgen05 epilogue pipeline), on the tcgen05 TMA
+    pipelines with the dense DFT-matrix transform, on the tcgen05 kernels
+    without pipelines (where the shape allows each) and on the CUDA-core
+    kernels; no bounded device wait may expire."""
     capi.fno_set_tensor_cores(request.param)
     yield request.param
     capi.fno_device_error(clear=True)
@@ -217,6 +228,21 @@ def test_network_forward_backward_mse(grid, modes, dtype):
             assert_close(got, g_ref[key][l], tol, f"{key}[{l}]")
 
 
+def test_default_path_launches_three_kernels_per_block():
+    """On a 2D grid the default path runs a block forward as the pruned-FFT
+    transform, the fused spectral middle and the epilogue."""
+    grid, modes = (256, 256), (16, 16)
+    x, r, w, b, _ = _block_inputs(grid, modes, 2, 8, 8, "f32")
+    d = capi.block_desc(2, 8, 8, grid, modes)
+    y = empty((2, 8) + grid)
+    prev = capi.fno_set_tensor_cores(1)
+    try:
+        capi.fno_block_fwd(d, dev(x), dev_complex(r), dev(w), dev(b), y)
+        assert capi.last_launch_count() == 3
+    finally:
+        capi.fno_set_tensor_cores(prev)
+
+
 def test_launch_count_is_reported(kernel_path):
     grid, modes = (16, 12), (4, 5)
     x, r, w, b, _ = _block_inputs(grid, modes, 2, 3, 3, "f32")
@@ -247,3 +273,43 @@ def test_block_gelu_elementwise(grid, modes):
     big = np.abs(ref) > 0.1
     assert np.max(err[big] / np.abs(ref[big])) < 2e-6
     assert np.max(err[~big]) < 3e-7
+
+
+def _cp_inputs(grid, modes, rank, ci, co, dtype, seed):
+    rng = np.random.default_rng(seed)
+    k = capi.num_modes(grid, modes)
+
+    def cplx(*shape):
+        return synth.quantize_complex(rng.uniform(-1, 1, shape) + 1j * rng.uniform(-1, 1, shape),
+                                      dtype)
+    lam = cplx(rank)
+    a, b, c = cplx(ci, rank), cplx(co, rank), cplx(k, rank)
+    return lam, a, b, c
+
+
+@pytest.mark.parametrize("grid,modes", [((64, 64), (10, 12)), ((15, 9), (5, 5)),
+                                        ((256, 256), (16, 16)), ((6, 10, 12), (2, 3, 4))])
+@pytest.mark.parametrize("rank", [1, 5, 16, 32])
+@pytest.mark.parametrize("dtype,flags", [("f32", 0), ("f16", 1), ("bf16", 0)])
+def test_factorised_weights_forward(grid, modes, rank, dtype, flags):
+    """CP-factorised weights against the oracle's dense reconstruction: the
+    spectral forward (spectral_conv_fwd_cp) and the block forward (block_fwd
+    with R = cp_weights)."""
+    b_, ci, co = 2, 6, 5
+    x, _, w, b, _ = _block_inputs(grid, modes, b_, ci, co, dtype, seed=7)
+    lam, a, bf, c = _cp_inputs(grid, modes, rank, ci, co, dtype, seed=8)
+    d = capi.block_desc(b_, ci, co, grid, modes, dtype, flags)
+    k = capi.num_modes(grid, modes)
+    dv = [dev_complex(v, dtype) for v in (lam, a, bf, c)]
+    y = empty((b_, co) + grid, dtype)
+    xh = empty((b_, ci, k, 2))
+    capi.fno_spectral_conv_fwd_cp(d, rank, dev(x, dtype), *dv, y, xh)
+    y_ref, xh_ref = O.spectral_conv_fwd_cp(x, lam, a, bf, c, modes, oracle_flags(flags))
+    assert_close(host_complex(xh), xh_ref, TOL[dtype], "xhat")
+    assert_close(host(y), y_ref, TOL[dtype], "y (spectral)")
+    yb, pre = empty((b_, co) + grid, dtype), empty((b_, co) + grid, dtype)
+    capi.fno_block_fwd_cp(d, rank, dev(x, dtype), *dv, dev(w, dtype), dev(b, dtype), yb, pre)
+    yb_ref, pre_ref, _ = O.block_fwd(x, O.cp_weights(lam, a, bf, c), w, b, modes,
+                                     oracle_flags(flags))
+    assert_close(host(pre), pre_ref, TOL[dtype], "pre (block)")
+    assert_close(host(yb), yb_ref, TOL[dtype], "y (block)")

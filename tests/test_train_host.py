@@ -41,8 +41,32 @@ def test_layout_slots_are_aligned_and_disjoint():
         assert size == int(np.prod(shape))
         prev_end = off + size
     assert lay.total >= prev_end and lay.total % ALIGN == 0
-    assert [k for k, *_ in lay.slots] == ["P", "p"] + ["R"] * 3 + ["W"] * 3 + ["b"] * 3 + \
+    assert [k for k, *_ in lay.slots] == ["P", "p"] + ["R", "W", "b"] * 3 + \
         ["Q1", "q1", "Q2", "q2"]
+    assert [l for _, l, *_ in lay.slots] == [None, None, 0, 0, 0, 1, 1, 1, 2, 2, 2] + [None] * 4
+
+
+def test_layout_buckets_follow_the_backward_and_tile_the_buffer():
+    lay = ParamLayout(3, 6, 9, 2, 3, 40)
+    bk = lay.buckets()
+    assert len(bk) == 3 + 2
+    assert sorted(bk) == sorted(set(bk))
+    # contiguous tiling of [0, total)
+    edges = sorted(bk)
+    assert edges[0][0] == 0 and edges[-1][1] == lay.total
+    assert all(a[1] == b[0] for a, b in zip(edges, edges[1:]))
+    # projection first, then layers 2, 1, 0, then the lift
+    start = {(k, l): off for k, l, _, off, _ in lay.slots}
+    assert bk[0] == (start[("Q1", None)], lay.total)
+    assert bk[1][0] == start[("R", 2)] and bk[3][0] == start[("R", 0)]
+    assert bk[-1] == (0, start[("R", 0)])
+    # each bucket holds exactly its group's slots
+    for (lo, hi), keys in zip(bk, [{"Q1", "q1", "Q2", "q2"}, {2}, {1}, {0}, {"P", "p"}]):
+        inside = {(k, l) for k, l, _, off, size in lay.slots if lo <= off and off + size <= hi}
+        if isinstance(next(iter(keys)), int):
+            assert inside == {(k, next(iter(keys))) for k in ("R", "W", "b")}
+        else:
+            assert inside == {(k, None) for k in keys}
 
 
 def test_layout_pack_unpack_round_trip():
@@ -60,7 +84,8 @@ def test_layout_pack_unpack_round_trip():
             np.testing.assert_array_equal(back[key][l], np.asarray(params[key][l]).astype(
                 np.complex64 if key == "R" else np.float32))
     views = lay.views(flat)
-    assert tuple(views["R"][1].shape) == (6, 6, lay.slots[3][2][2], 2)
+    n_modes = next(shape for k, l, shape, *_ in lay.slots if (k, l) == ("R", 1))[2]
+    assert tuple(views["R"][1].shape) == (6, 6, n_modes, 2)
     # gaps between slots stay zero
     used = np.zeros(lay.total, bool)
     for *_, off, size in lay.slots:
