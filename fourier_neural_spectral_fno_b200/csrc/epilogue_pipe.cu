@@ -77,14 +77,16 @@ __host__ __device__ inline size_t alg(size_t v, size_t a) { return (v + a - 1) /
 // lo rows), the last-axis twiddles, the bias, mbarriers.
 struct PipeGeom {
   int Rt, nvar, KS, KSp, KXp, KA, NP, DC, cs_cols, ax_cols;
-  int NA, NS;
+  int NA, NS, NB;
   int col_spec, col_x, used_cols, cols;
-  uint32_t sbo, x_bytes, u_bytes;
+  uint32_t sbo, sbo_s, x_bytes, u_bytes;
   size_t uoff, stage, bhalf, bbuf, b, tw, bias, bar, tbase, total;
 };
 
+// img: the spectral half of B arrives prebuilt per grid row (the slab-axis
+// inverse writes it in the operand layout), so the B buffer holds W alone
 __host__ __device__ inline PipeGeom pipe_geom(const Geom &g, bool has_x, int Ci, int Co, int eb,
-                                              bool tf32) {
+                                              bool tf32, bool img = false) {
   PipeGeom e;
   e.Rt = g.NL >= ROWS ? 1 : ROWS / g.NL;
   e.nvar = g.NL >= ROWS ? g.NL / ROWS : 1;
@@ -102,21 +104,24 @@ __host__ __device__ inline PipeGeom pipe_geom(const Geom &g, bool has_x, int Ci,
   e.used_cols = e.col_x + e.NA * e.ax_cols;
   e.cols = 32;
   while (e.cols < e.used_cols && e.cols < 1024) e.cols *= 2;
-  e.sbo = (uint32_t)(e.KA * eb / 16) * 128u;
+  const int kb = img ? e.KXp : e.KA;            // K of the B buffer
+  e.sbo = (uint32_t)(kb * eb / 16) * 128u;
+  e.sbo_s = (uint32_t)(e.KSp * eb / 16) * 128u;  // the prebuilt spectral image
   e.x_bytes = has_x ? (uint32_t)(Ci * ROWS * eb) : 0u;
-  e.u_bytes = (uint32_t)(Co * e.KS * 4);
+  e.u_bytes = img ? (uint32_t)(e.DC * e.KSp * eb) : (uint32_t)(Co * e.KS * 4);
   e.uoff = alg(e.x_bytes, 128);
   e.stage = alg(e.uoff + e.u_bytes, 1024);
-  e.bhalf = (size_t)e.NP * e.KA * eb;
+  e.bhalf = (size_t)e.NP * kb * eb;
   e.bbuf = alg((tf32 ? 2 : 1) * e.bhalf, 1024);
-  const size_t fixed = e.NA * e.bbuf + alg(sizeof(float2) * g.NL, 128) + sizeof(float) * 64 +
+  e.NB = img ? 1 : e.NA;                         // W is constant: one buffer
+  const size_t fixed = e.NB * e.bbuf + alg(sizeof(float2) * g.NL, 128) + sizeof(float) * 64 +
                        sizeof(uint64_t) * (2 * MAX_STAGES + 6) + 16;
   const size_t room = kSmemMax > fixed ? kSmemMax - fixed : 0;
   const size_t ns = room / e.stage;
   e.NS = (int)(ns < (size_t)MAX_STAGES ? ns : (size_t)MAX_STAGES);
   size_t off = 0;
   off += (size_t)(e.NS > 0 ? e.NS : 0) * e.stage;
-  e.b = off; off += e.NA * e.bbuf;
+  e.b = off; off += e.NB * e.bbuf;
   e.tw = off; off = alg(off + sizeof(float2) * g.NL, 128);
   e.bias = off; off += sizeof(float) * 64;
   e.bar = off; off += sizeof(uint64_t) * (2 * MAX_STAGES + 6);
@@ -184,6 +189,7 @@ __device__ __forceinline__ void stage16(uint32_t col, uint32_t lo_off, const flo
 struct PipeArgs {
   const void *W, *bias;
   void *out, *pre_out;
+  const unsigned char *img;   // prebuilt spectral B images per grid row (IMG), else NULL
   int *err;
   int Ci, Co, act;
 };
@@ -224,14 +230,14 @@ __device__ __forceinline__ void cursor_next(Cursor &c, int Rt, const Geom &g) {
   }
 }
 
-template <typename T, bool HAS_X, int CX>
+template <typename T, bool HAS_X, int CX, bool IMG>
 __global__ void __launch_bounds__(THREADS, 1)
     k_epi_pipe(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmu,
                PipeArgs a, Geom g) {
   using K = PKind<T>;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int Ci = a.Ci, Co = a.Co;
-  const PipeGeom e = pipe_geom(g, HAS_X, Ci, Co, K::EB, K::tf32);
+  const PipeGeom e = pipe_geom(g, HAS_X, Ci, Co, K::EB, K::tf32, IMG);
   unsigned char *bbase = smem + e.b;
   float2 *twL = reinterpret_cast<float2 *>(smem + e.tw);
   float *bias_s = reinterpret_cast<float *>(smem + e.bias);
@@ -252,7 +258,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (tid == 0) {
     for (int s = 0; s < MAX_STAGES; ++s) {
       tc::mbar_init(&full[s], 1);
-      tc::mbar_init(&empty[s], NCONV);
+      // IMG: the MMAs read the stage itself, so the epilogue warps free it
+      // once a tile's MMAs are complete; else the staging warps after copying
+      tc::mbar_init(&empty[s], IMG ? NEPI : NCONV);
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&aready[i], NCONV);
@@ -263,19 +271,19 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   if (warp == WARP_TMA && lane == 0) {
     if (HAS_X) tma::prefetch_map(&tmx);
-    tma::prefetch_map(&tmu);
+    if (!IMG) tma::prefetch_map(&tmu);
   }
   build_twiddles(twL, NL);
-  for (size_t i = (size_t)tid * 16; i < e.NA * e.bbuf; i += THREADS * 16)
+  for (size_t i = (size_t)tid * 16; i < e.NB * e.bbuf; i += THREADS * 16)
     *reinterpret_cast<uint4 *>(bbase + i) = make_uint4(0, 0, 0, 0);
   __syncthreads();
-  if (HAS_X) {  // W in columns [KSp, KSp + Ci) of every B buffer; bias
+  if (HAS_X) {  // W in columns [KSp, KSp + Ci) of every B buffer (IMG: [0, Ci)); bias
     const T *W = reinterpret_cast<const T *>(a.W);
     for (int i = tid; i < Co * Ci; i += THREADS) {
       const int o = i / Ci, c = i - o * Ci;
       const float w = to_f<T>(W[i]);
-      const uint32_t off = boff(o, e.KSp + c, K::EB, e.sbo);
-      for (int nb = 0; nb < e.NA; ++nb) bstore1<T>(bbase + nb * e.bbuf, e.bhalf, off, w);
+      const uint32_t off = boff(o, (IMG ? 0 : e.KSp) + c, K::EB, e.sbo);
+      for (int nb = 0; nb < e.NB; ++nb) bstore1<T>(bbase + nb * e.bbuf, e.bhalf, off, w);
     }
   }
   {
@@ -310,7 +318,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           unsigned char *st = smem + (size_t)s * e.stage;
           if (HAS_X)
             tma::load_4d(st, &tmx, &full[s], c.row0 * NL + c.n0, c.outer, 0, (int)c.b);
-          tma::load_4d(st + e.uoff, &tmu, &full[s], c.row0 * 2 * mL, c.outer, 0, (int)c.b);
+          if (IMG)
+            tma::load_bulk(st + e.uoff,
+                           a.img + ((c.b * g.O + c.outer) * g.S + c.row0) * (size_t)e.u_bytes,
+                           e.u_bytes, &full[s]);
+          else
+            tma::load_4d(st + e.uoff, &tmu, &full[s], c.row0 * 2 * mL, c.outer, 0, (int)c.b);
         }
         __syncwarp();
         cursor_next(c, e.Rt, g);
@@ -345,13 +358,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         // one thread issues; operands advance by constants (tf32: the A_hi and
         // A_lo products of each K step, both against [B_hi; B_lo])
         if (lane == 0) {
-          uint64_t bd = ab ? bdesc1 : bdesc0;
+          // IMG: the spectral steps read this tile's ring stage, the x steps W
+          uint64_t bd = IMG ? tc::smem_desc_kmajor(
+                                  tc::smem_u32(smem + (size_t)(j % e.NS) * e.stage + e.uoff), 128,
+                                  e.sbo_s)
+                            : (ab ? bdesc1 : bdesc0);
           uint32_t acol = tbase + e.col_spec + variant * e.cs_cols;
           uint32_t lo = lo_spec;
           for (int s = 0; s < ns + nx; ++s) {
             if (s == ns) {
               acol = tbase + e.col_x + ab * e.ax_cols;
               lo = lo_x;
+              if (IMG) bd = bdesc0;
             }
             if (K::tf32) {
               tc::mma_tf32_ts(d, acol, bd, idesc, s > 0 ? 1u : 0u);
@@ -448,8 +466,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!__all_sync(0xffffffffu, ok)) break;      // warp-uniform exit
       tc::fence_after_sync();
       const unsigned char *st = smem + (size_t)s * e.stage;
-      // B spectral block: U rows -> K-major core matrices
-      if (slots_fit) {
+      // B spectral block: U rows -> K-major core matrices (IMG: prebuilt)
+      if (IMG) {
+      } else if (slots_fit) {
         const float *us = reinterpret_cast<const float *>(st + e.uoff);
         unsigned char *bh = bbase + ab * e.bbuf;
         float4 v[MAXSLOT];
@@ -494,7 +513,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       __syncwarp();
-      if (lane == 0) tma::arrive(&empty[s]);            // the stage may be refilled
+      if (!IMG && lane == 0) tma::arrive(&empty[s]);    // the stage may be refilled
       tc::tmem_wait_st();
       tc::fence_proxy_async_smem();
       tc::fence_before_sync();
@@ -514,6 +533,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int j = 0; j < ntl; ++j) {
       if (!__all_sync(0xffffffffu, tc::mbar_wait(&mdone[j & 1], (j >> 1) & 1, a.err))) break;
       tc::fence_after_sync();
+      if (IMG && lane == 0) tma::arrive(&empty[j % e.NS]);   // tile j's MMAs are done with it
       const uint32_t dcol = arow + (uint32_t)((j & 1) * e.DC);
       float v[GPH][16];
 #pragma unroll
@@ -579,14 +599,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-template <typename T, bool HAS_X>
+template <typename T, bool HAS_X, bool IMG>
 cudaError_t launch_pipe_t(const Launch &L, const Geom &g, const PipeArgs &a, const void *x,
                           const float2 *U) {
   using K = PKind<T>;
-  const PipeGeom e = pipe_geom(g, HAS_X, a.Ci, a.Co, K::EB, K::tf32);
+  const PipeGeom e = pipe_geom(g, HAS_X, a.Ci, a.Co, K::EB, K::tf32, IMG);
   const long long SN = (long long)g.S * g.NL;
   CUtensorMap tmx, tmu;
   memset(&tmx, 0, sizeof(tmx));
+  memset(&tmu, 0, sizeof(tmu));
   if (HAS_X) {
     const uint64_t dims[4] = {(uint64_t)SN, (uint64_t)g.O, (uint64_t)a.Ci, (uint64_t)g.B};
     const uint64_t str[3] = {(uint64_t)SN * K::EB, (uint64_t)g.O * SN * K::EB,
@@ -594,7 +615,7 @@ cudaError_t launch_pipe_t(const Launch &L, const Geom &g, const PipeArgs &a, con
     const uint32_t box[4] = {(uint32_t)ROWS, 1u, (uint32_t)a.Ci, 1u};
     if (!encode_tmap_4d(&tmx, K::tmap, x, dims, str, box)) return cudaErrorInvalidValue;
   }
-  {
+  if (!IMG) {
     const uint64_t row = (uint64_t)g.S * 2 * g.mL;   // floats of one (b, o, outer) slab
     const uint64_t dims[4] = {row, (uint64_t)g.O, (uint64_t)a.Co, (uint64_t)g.B};
     const uint64_t str[3] = {row * 4, (uint64_t)g.O * row * 4, (uint64_t)a.Co * g.O * row * 4};
@@ -609,10 +630,17 @@ cudaError_t launch_pipe_t(const Launch &L, const Geom &g, const PipeArgs &a, con
     kern<<<grid, THREADS, e.total, L.stream>>>(tmx, tmu, a, g);
   };
   const int cmax = a.Co > a.Ci ? a.Co : a.Ci;
-  if (cmax <= 16) go(k_epi_pipe<T, HAS_X, 16>);
-  else if (cmax <= 32) go(k_epi_pipe<T, HAS_X, 32>);
-  else go(k_epi_pipe<T, HAS_X, 64>);
+  if (cmax <= 16) go(k_epi_pipe<T, HAS_X, 16, IMG>);
+  else if (cmax <= 32) go(k_epi_pipe<T, HAS_X, 32, IMG>);
+  else go(k_epi_pipe<T, HAS_X, 64, IMG>);
   return cudaGetLastError();
+}
+
+template <typename T, bool HAS_X>
+cudaError_t launch_pipe_img(const Launch &L, const Geom &g, const PipeArgs &a, const void *x,
+                            const float2 *U) {
+  return a.img ? launch_pipe_t<T, HAS_X, true>(L, g, a, x, U)
+               : launch_pipe_t<T, HAS_X, false>(L, g, a, x, U);
 }
 
 }  // namespace
@@ -635,6 +663,18 @@ bool epi_pipe_supported(const Geom &g, int dtype, int mode, int Ci, int Co, cons
   return true;
 }
 
+bool epi_img_supported(const Geom &g, int dtype, int mode, int Ci, int Co) {
+  if (mode != EPI_SPEC && mode != EPI_BLOCK_FWD) return false;
+  if (g.d != 2 || g.NL < ROWS || Co % 16 != 0 || (2 * g.mL) % 16 != 0) return false;
+  const bool tf32 = dtype == DT_F32;
+  const PipeGeom e = pipe_geom(g, mode == EPI_BLOCK_FWD, Ci, Co, tf32 ? 4 : 2, tf32, true);
+  return e.NS >= 2 && e.total <= kSmemMax && e.KS == e.KSp;
+}
+
+size_t epi_img_row_bytes(int dtype, int Co, int mL) {
+  return (size_t)(dtype == DT_F32 ? 2 * Co : Co) * 2 * mL * (dtype == DT_F32 ? 4 : 2);
+}
+
 cudaError_t launch_epi_pipe(const Launch &L, const Geom &g, int dtype, int mode,
                             const EpiArgs &ea, const float2 *U) {
   PipeArgs a{};
@@ -646,18 +686,19 @@ cudaError_t launch_epi_pipe(const Launch &L, const Geom &g, int dtype, int mode,
   a.Ci = ea.Ci;
   a.Co = ea.Co;
   a.act = ea.act;
+  a.img = ea.img;
   const bool has_x = mode == EPI_BLOCK_FWD;
   launch_begin(L);
   cudaError_t err;
   if (dtype == DT_F32)
-    err = has_x ? launch_pipe_t<float, true>(L, g, a, ea.x, U)
-                : launch_pipe_t<float, false>(L, g, a, ea.x, U);
+    err = has_x ? launch_pipe_img<float, true>(L, g, a, ea.x, U)
+                : launch_pipe_img<float, false>(L, g, a, ea.x, U);
   else if (dtype == DT_F16)
-    err = has_x ? launch_pipe_t<__half, true>(L, g, a, ea.x, U)
-                : launch_pipe_t<__half, false>(L, g, a, ea.x, U);
+    err = has_x ? launch_pipe_img<__half, true>(L, g, a, ea.x, U)
+                : launch_pipe_img<__half, false>(L, g, a, ea.x, U);
   else
-    err = has_x ? launch_pipe_t<__nv_bfloat16, true>(L, g, a, ea.x, U)
-                : launch_pipe_t<__nv_bfloat16, false>(L, g, a, ea.x, U);
+    err = has_x ? launch_pipe_img<__nv_bfloat16, true>(L, g, a, ea.x, U)
+                : launch_pipe_img<__nv_bfloat16, false>(L, g, a, ea.x, U);
   launch_end(L, has_x ? "epi_block_fwd_pipe" : "epi_spec_pipe");
   return err;
 }

@@ -116,7 +116,7 @@ int check_block(const fno_block_desc *d, Geom *g) {
 
 // Workspace map of a block operation.
 struct BlockWs {
-  size_t zpart, xhat, yhat, zexp, u, dxhat, partial, total;
+  size_t zpart, xhat, yhat, zexp, tw, u, img, dxhat, partial, total;
 };
 
 BlockWs block_ws(const Geom &g, int Ci, int Co, int op) {
@@ -135,8 +135,13 @@ BlockWs block_ws(const Geom &g, int Ci, int Co, int op) {
   off += al(cplx * (size_t)(g.B * Cmax * g.K));
   w.zexp = off;
   off += al(inv_expand_bytes(g, Cmax));
+  w.tw = off;                         // slab-axis twiddles of the 2D spectral middle
+  off += al(spec_mid_table_bytes(g));
   w.u = off;                          // spectrum inverted along the slab axis
   off += al(inv_slab_bytes(g, Cmax));
+  w.img = off;                        // or, per grid row, the epilogue's B operand image
+  if (op == FNO_OP_SPECTRAL_FWD || op == FNO_OP_BLOCK_FWD)
+    off += al(g.d == 2 ? (size_t)g.B * g.S * epi_img_row_bytes(DT_F32, Co, g.mL) : 0);
   w.dxhat = off;
   w.partial = off;
   if (op == FNO_OP_SPECTRAL_BWD || op == FNO_OP_BLOCK_BWD) {
@@ -261,11 +266,18 @@ int run_forward(const Launch &L, const Geom &g, int dtype, unsigned flags, int C
                                Ci, x, nullptr, zpart, xhat),
           "forward transform");
   // 2D grids on the default path: mixing and the slab-axis inverse in one launch
-  const bool mid = !cp && L.tc == 1 && spec_mid_supported(g);
+  const bool mid = !cp && L.tc == 1 && spec_mid_supported(g, Ci, Co);
+  // the slab-axis inverse writes the epilogue's B operand directly where the
+  // pipelined epilogue takes it
+  const bool img = mid && epi_img_supported(g, dtype, epi_mode, Ci, Co) &&
+                   epi_pipe_supported(g, dtype, epi_mode, Ci, Co, x, ws + w.u);
   if (cp)
     FNO_TRY(launch_mix_cp(L, g, dtype, Ci, Co, rank, xhat, *cp, yhat), "factorised mixing");
   else if (mid)
-    FNO_TRY(launch_spec_mid(L, g, dtype, Ci, Co, xhat, R, reinterpret_cast<float2 *>(ws + w.u)),
+    FNO_TRY(launch_spec_mid(L, g, dtype, Ci, Co, xhat, R, yhat,
+                            reinterpret_cast<float2 *>(ws + w.tw),
+                            reinterpret_cast<float2 *>(ws + w.u), img ? ws + w.img : nullptr,
+                            epi_mode == EPI_BLOCK_FWD ? b : nullptr),
             "mixing and slab-axis inverse");
   else
     FNO_TRY(launch_mix_fwd(L, g, dtype, Ci, Co, xhat, R, yhat), "mixing");
@@ -286,6 +298,7 @@ int run_forward(const Launch &L, const Geom &g, int dtype, unsigned flags, int C
   a.Co = Co;
   a.act = !(flags & FNO_NO_ACT);
   a.tanh_pre = (flags & FNO_TANH_PREACT) ? 1 : 0;
+  a.img = img ? ws + w.img : nullptr;
   FNO_TRY(run_epilogue(L, g, dtype, epi_mode, a, ws, w, mid), "epilogue");
   return FNO_OK;
 }

@@ -79,11 +79,25 @@ bool fwd_fft_supported(const Geom &g, const void *in0, const void *in1, int load
 cudaError_t launch_fwd_fft(const Launch &L, const Geom &g, int dtype, int load_mode, long long C,
                            const void *in0, const void *in1, float2 *out);
 
-// 2D spectral middle (spec_mid.cu): mixing + slab-axis inverse in one launch,
-// U[b][o][S][mL] = sum_q ((c_k/N) sum_i xhat[b,i,q,k] R[i,o,q,k]) exp(+i kq n)
-bool spec_mid_supported(const Geom &g);
+// the same transform with whole planes per persistent CTA (transform_plane.cu):
+// rows streamed by bulk async copies, slab axis as a pruned FFT on chip;
+// writes out[plane][QS][mL] like launch_fwd_fft
+bool fwd_plane_supported(const Geom &g, int dtype, const void *in0, const void *in1,
+                         int load_mode);
+cudaError_t launch_fwd_plane(const Launch &L, const Geom &g, int dtype, int load_mode, long long C,
+                             const void *in0, const void *in1, float2 *out);
+
+// 2D spectral middle (spec_mid.cu): mixing into yhat (as launch_mix_fwd),
+// then the slab-axis inverse as a pruned FFT into
+// U[b][o][S][mL] = sum_q yhat[b,o,q,k] exp(+2 pi i kq n / S); two launches
+// twr: workspace for the slab-axis twiddle table (spec_mid_table_bytes)
+bool spec_mid_supported(const Geom &g, int Ci, int Co);
+size_t spec_mid_table_bytes(const Geom &g);
+// img (optional): write the epilogue's B images (epi_img_supported) instead of
+// U, with bias (may be NULL) folded in
 cudaError_t launch_spec_mid(const Launch &L, const Geom &g, int dtype, int Ci, int Co,
-                            const float2 *xhat, const void *R, float2 *U);
+                            const float2 *xhat, const void *R, float2 *yhat, float2 *twr,
+                            float2 *U, unsigned char *img, const void *bias);
 
 // CP-factorised weights (mix_cp.cu): R[i,o,k] = sum_r lam[r] A[i,r] B[o,r] C[k,r],
 // factors complex (re, im) in the storage dtype: lam [rank], A [Ci][rank],
@@ -124,6 +138,8 @@ struct EpiArgs {
   float *partial;   // bwd: per-CTA partial sums of dW/db, [grid][Co][Ci+1]
   const float2 *U;  // optional: the spectrum already inverted along the slab axis,
                     // [B][Cs][O][S][mL] (launch_inv_slab); NULL: computed per tile
+  const unsigned char *img;  // optional (pipelined forward epilogue): per grid row the
+                             // spectral half of the B operand, prebuilt (launch_spec_mid)
   int Ci, Co;
   int act, tanh_pre;
 };
@@ -143,6 +159,12 @@ bool epi_pipe_supported(const Geom &g, int dtype, int mode, int Ci, int Co, cons
                         const void *U);
 cudaError_t launch_epi_pipe(const Launch &L, const Geom &g, int dtype, int mode,
                             const EpiArgs &a, const float2 *U);
+// the prebuilt-image form (a.img): 2D, last axis >= 128, Co % 16 == 0, 2 mL % 16 == 0.
+// One image per (sample, grid row): the K-major no-swizzle core-matrix layout of
+// the B operand rows o (float32: tf32 high parts in rows [0, Co), low parts in
+// [Co, 2 Co)) by columns 2k (re), 2k + 1 (im), bias folded into column 0
+bool epi_img_supported(const Geom &g, int dtype, int mode, int Ci, int Co);
+size_t epi_img_row_bytes(int dtype, int Co, int mL);
 size_t epi_partial_bytes(const Geom &g, int Ci, int Co, int num_sms);
 cudaError_t launch_epilogue(const Launch &L, const Geom &g, int dtype, int mode,
                             const EpiArgs &a);

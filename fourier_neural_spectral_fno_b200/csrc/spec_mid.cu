@@ -1,20 +1,22 @@
-// The block's spectral middle for 2D grids in one launch: per-mode channel
-// mixing (step S3) followed by the inverse transform along the slab axis (the
-// first half of S4), producing U, the spectrum inverted along the slab axis,
-// that the fused epilogue contracts with the last-axis basis.
+// The block's spectral middle for 2D grids: per-mode channel mixing (step S3)
+// and the inverse transform along the slab axis (the first half of S4), as
+// two launches that each read their inputs from HBM or L2 once.
 //
-//   yhat[b,o,q,k] = (c_k / N) sum_i xhat[b,i,q,k] R[i,o,q,k]
-//   U[b,o,n,k]    = sum_q yhat[b,o,q,k] exp(+2 pi i kq(q) n / S)
+//   yhat[b,o,q,k] = (c_k / N) sum_i xhat[b,i,q,k] R[i,o,q,k]      (k_mix_modes)
+//   U[b,o,n,k]    = sum_q yhat[b,o,q,k] exp(+2 pi i kq(q) n / S)    (k_inv_slab_fft)
 //
-// A CTA owns 4 samples x 4 output channels x 4 last-axis modes and every
-// slab-axis mode q, so the inverse of each (b, o, k) column has all its inputs
-// in shared memory.  The inverse is a pruned radix-16 FFT: with S = 16 Q and
-// n = Q a + r,
+// k_mix_modes: a CTA owns a group of consecutive modes and four samples; it
+// stages their xhat and every weight of those modes in shared memory (eight
+// loads in flight per thread), then forms all (b, o) products from there.
+//
+// k_inv_slab_fft: a CTA owns one (b, o) slab.  The inverse is a pruned
+// radix-16 FFT: with S = 16 Q and n = Q a + r,
 //   U[Q a + r] = sum_p exp(+2 pi i p a / 16) V_r[p],
 //   V_r[p]     = sum_{kq = p (mod 16)} yhat[kq] exp(+2 pi i kq r / S),
-// i.e. the kept wavenumbers are folded by residue into sixteen bins (at most
-// a few per bin), then one register FFT16 per (column, r) expands them to
-// sixteen grid rows.
+// i.e. the kept wavenumbers (signed, in [-mS, mS)) are folded by residue into
+// sixteen bins of at most four, then one register FFT16 per (r, k) expands
+// them to sixteen grid rows; consecutive threads take consecutive k, so every
+// row of U is written by one coalesced store.
 #include "fft16.cuh"
 #include "fno_common.cuh"
 #include "fno_kernels.cuh"
@@ -23,153 +25,267 @@ namespace fno {
 
 namespace {
 
-constexpr int SM_THREADS = 256;
-constexpr int SM_BG = 4, SM_OG = 4, SM_KG = 4;
-constexpr int SM_NCOL = SM_BG * SM_OG * SM_KG;
+constexpr int MM_THREADS = 256;
+constexpr int MM_BS = 4;                        // samples per CTA
+constexpr size_t MM_R_STAGE = 64 * 1024;        // staged weights per CTA
+constexpr int IS_THREADS = 256;
 constexpr int SM_MAXQS = 64;
-constexpr int SM_MAXPER = 8;   // kept slab-axis modes per residue mod 16
 
-struct MidPlan {
-  size_t ys, twr, slots, total;
-};
-
-__host__ __device__ inline MidPlan mid_plan(int QS, int S) {
-  MidPlan p{};
-  size_t off = 0;
-  p.ys = off; off += sizeof(float2) * SM_NCOL * (size_t)(QS + 1);
-  p.twr = off; off += sizeof(float2) * (size_t)QS * (S / 16);
-  p.slots = off; off += sizeof(int) * 16 * (SM_MAXPER + 1);
-  p.total = off;
-  return p;
+// modes per CTA: 4 (whole 32-byte sectors of the mode-contiguous rows) unless
+// the staged weights would exceed MM_R_STAGE
+int mix_modes_group(int Ci, int Co) {
+  int mg = 4;
+  while (mg > 1 && sizeof(float2) * (size_t)Ci * Co * mg > MM_R_STAGE) mg /= 2;
+  return sizeof(float2) * (size_t)Ci * Co * mg > MM_R_STAGE ? 0 : mg;
 }
 
-template <typename T>
-__global__ void __launch_bounds__(SM_THREADS)
-    k_spec_mid(const float2 *__restrict__ xhat, const T *__restrict__ R, float2 *__restrict__ U,
-               long long B, int Ci, int Co, int S, int mS, int QS, int mL, int NL, float inv_n) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  const MidPlan pl = mid_plan(QS, S);
-  float2 *ys = reinterpret_cast<float2 *>(smem + pl.ys);     // [col][QS + 1]
-  float2 *twr = reinterpret_cast<float2 *>(smem + pl.twr);   // [slot][Qp]
-  int *slot_cnt = reinterpret_cast<int *>(smem + pl.slots);  // [16]
-  int *slot_tab = slot_cnt + 16;                             // [16][SM_MAXPER]
-  const int tid = threadIdx.x;
-  const int Qp = S / 16;
-  const long long K = (long long)QS * mL;
-  const int k0 = blockIdx.x * SM_KG, o0 = blockIdx.y * SM_OG;
-  const long long b0 = (long long)blockIdx.z * SM_BG;
-  const int QSp = QS + 1;
+// hi = x rounded to tf32 (nearest), lo = x - hi rounded to tf32: the
+// operand split of the float32 tensor-core path
+__device__ __forceinline__ void tc_split(float x, uint32_t &hi, uint32_t &lo) {
+  uint32_t h, l;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(x));
+  const float rem = x - __uint_as_float(h);
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(l) : "f"(rem));
+  hi = h;
+  lo = l;
+}
 
-  // twiddles exp(+2 pi i kq(slot) r / S) and the slots of each residue
-  for (int e = tid; e < QS * Qp; e += SM_THREADS) {
-    const int slot = e / Qp, r = e - slot * Qp;
-    const int kq = kept_k(slot, mS, S);
-    double sn, cs;
-    sincospi(2.0 * (double)mulmod(kq, r, S) / S, &sn, &cs);
-    twr[e] = make_float2((float)cs, (float)sn);
-  }
-  if (tid < 16) {
-    int c = 0;
-    for (int slot = 0; slot < QS; ++slot)
-      if ((kept_k(slot, mS, S) & 15) == tid) slot_tab[tid * SM_MAXPER + c++] = slot;
-    slot_cnt[tid] = c;
-  }
-
-  // ---- mixing: task = (position (q, kk), output-channel pair)
-  const int npos = QS * SM_KG;
-  for (int task = tid; task < npos * (SM_OG / 2); task += SM_THREADS) {
-    const int pos = task % npos, op = task / npos;
-    const int q = pos / SM_KG, kk = pos - q * SM_KG, k = k0 + kk;
-    const int oa = o0 + 2 * op;
-    float2 acc[SM_BG][2];
+// global load of 8 values per thread before any is stored: the staging keeps
+// eight loads in flight instead of one
+template <typename F>
+__device__ __forceinline__ void stage8(float2 *dst, int n, F load) {
+  for (int base = threadIdx.x; base < n; base += 8 * MM_THREADS) {
+    float2 v[8];
 #pragma unroll
-    for (int bb = 0; bb < SM_BG; ++bb) acc[bb][0] = acc[bb][1] = make_float2(0.f, 0.f);
-    if (k < mL) {
-      const long long qk = (long long)q * mL + k;
-      const bool va = oa < Co, vb = oa + 1 < Co;
-#pragma unroll 4
-      for (int i = 0; i < Ci; ++i) {
-        const float2 ra = va ? ldc<T>(R + 2 * (((long long)i * Co + oa) * K + qk)) : make_float2(0.f, 0.f);
-        const float2 rb = vb ? ldc<T>(R + 2 * (((long long)i * Co + oa + 1) * K + qk)) : make_float2(0.f, 0.f);
-#pragma unroll
-        for (int bb = 0; bb < SM_BG; ++bb) {
-          if (b0 + bb < B) {
-            const float2 xv = __ldg(xhat + ((b0 + bb) * Ci + i) * K + qk);
-            cfma(acc[bb][0], xv, ra);
-            cfma(acc[bb][1], xv, rb);
-          }
-        }
-      }
+    for (int u = 0; u < 8; ++u) {
+      const int e = base + u * MM_THREADS;
+      v[u] = e < n ? load(e) : make_float2(0.f, 0.f);
     }
-    const float w = k < mL ? mode_weight(k, NL, inv_n) : 0.f;
 #pragma unroll
-    for (int bb = 0; bb < SM_BG; ++bb)
-#pragma unroll
-      for (int oo = 0; oo < 2; ++oo) {
-        const int col = (bb * SM_OG + 2 * op + oo) * SM_KG + kk;
-        ys[col * QSp + q] = make_float2(w * acc[bb][oo].x, w * acc[bb][oo].y);
-      }
+    for (int u = 0; u < 8; ++u) {
+      const int e = base + u * MM_THREADS;
+      if (e < n) dst[e] = v[u];
+    }
   }
-  __syncthreads();
+}
 
-  // ---- inverse along the slab axis: task = (column, r), column fastest
-  for (int task = tid; task < SM_NCOL * Qp; task += SM_THREADS) {
-    const int col = task % SM_NCOL, r = task / SM_NCOL;
-    const int kk = col % SM_KG, bo = col / SM_KG;
-    const int ol = bo % SM_OG, bb = bo / SM_OG;
-    const long long b = b0 + bb;
-    const int o = o0 + ol, k = k0 + kk;
-    const float2 *y = ys + col * QSp;
+template <typename T, int MG>
+__global__ void __launch_bounds__(MM_THREADS)
+    k_mix_modes(const float2 *__restrict__ xhat, const T *__restrict__ R, float2 *__restrict__ yhat,
+                float2 *__restrict__ twr, int B, int Ci, int Co, int K, int mL, int NL,
+                float inv_n, int S, int mS, int QS) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  float2 *xs = reinterpret_cast<float2 *>(smem);     // [MM_BS][Ci][MG]
+  float2 *rs = xs + (size_t)MM_BS * Ci * MG;         // [Ci][Co][MG]
+  const int m0 = blockIdx.x * MG, b0 = blockIdx.y * MM_BS;
+  const int mg = min(MG, K - m0), nb = min(MM_BS, B - b0);
+  const int tid = threadIdx.x;
+  if (blockIdx.x == 0 && blockIdx.y == 0) {
+    // the slab-axis inverse's twiddles exp(+2 pi i kq(slot) r / S), [slot][S/16]
+    const int Qp = S / 16;
+    for (int e = tid; e < QS * Qp; e += MM_THREADS) {
+      const int slot = e / Qp, r = e - slot * Qp;
+      float sn, cs;
+      sincospif(2.0f * (float)mulmod(kept_k(slot, mS, S), r, S) / (float)S, &sn, &cs);
+      twr[e] = make_float2(cs, sn);
+    }
+  }
+  const float2 *xsrc = xhat + (size_t)b0 * Ci * K + m0;
+  stage8(xs, nb * Ci * MG, [&](int e) {
+    const int row = e / MG, m = e % MG;                  // MG is a power of two
+    return m < mg ? __ldg(xsrc + (size_t)row * K + m) : make_float2(0.f, 0.f);
+  });
+  const T *rsrc = R + 2 * (size_t)m0;
+  stage8(rs, Ci * Co * MG, [&](int e) {
+    const int row = e / MG, m = e % MG;
+    return m < mg ? ldc<T>(rsrc + 2 * ((size_t)row * K + m)) : make_float2(0.f, 0.f);
+  });
+  __syncthreads();
+  // output (b, o, m), m fastest: the weight reads of a warp are contiguous;
+  // the (b, o) pair advances by a constant stride per thread
+  const int m = tid % MG;
+  const int bo_step = MM_THREADS / MG;
+  const float w = m < mg ? mode_weight((m0 + m) % mL, NL, inv_n) : 0.f;
+  int b = 0, o = tid / MG;
+  while (o >= Co) { o -= Co; ++b; }
+  const int db = bo_step / Co, dob = bo_step % Co;
+  for (; b < nb;) {
+    const float2 *xp = xs + (size_t)b * Ci * MG + m;
+    const float2 *rp = rs + (size_t)o * MG + m;
+    const size_t rstep = (size_t)Co * MG;
+    float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
+    int i = 0;
+    for (; i + 1 < Ci; i += 2) {
+      cfma(s0, xp[(size_t)i * MG], rp[i * rstep]);
+      cfma(s1, xp[(size_t)(i + 1) * MG], rp[(i + 1) * rstep]);
+    }
+    if (i < Ci) cfma(s0, xp[(size_t)i * MG], rp[i * rstep]);
+    if (m < mg)
+      yhat[((size_t)(b0 + b) * Co + o) * K + m0 + m] =
+          make_float2(w * (s0.x + s1.x), w * (s0.y + s1.y));
+    b += db;
+    o += dob;
+    if (o >= Co) { o -= Co; ++b; }
+  }
+}
+
+// byte offset of B-operand element (row n, column c) in a K-major no-swizzle
+// image of `sbo`-byte 8-row groups (the tcgen05 core-matrix layout)
+__device__ __forceinline__ uint32_t img_off(int n, int c, int eb, uint32_t sbo) {
+  const int cb = c * eb;
+  return (uint32_t)(n >> 3) * sbo + (uint32_t)(cb >> 4) * 128u + (uint32_t)(n & 7) * 16u +
+         (uint32_t)(cb & 15);
+}
+
+// NDM: the kept wavenumbers of residue p (mod 16) are among p + 16 d,
+// d in [-NDM, NDM) (NDM = 1 for mS <= 16, 2 for mS <= 32); FULL: mS = 16 NDM,
+// so every candidate is kept and no test is needed.
+// IMG 0: write U; 1: float32 B images (tf32 high / low rows); 2 / 3: float16 /
+// bfloat16 B images (the epilogue's operand layout, bias folded into column 0)
+template <int NDM, bool FULL, int IMG, typename TB>
+__global__ void __launch_bounds__(IS_THREADS)
+    k_inv_slab_fft(const float2 *__restrict__ yhat, const float2 *__restrict__ twr_g,
+                   float2 *__restrict__ U, unsigned char *__restrict__ img,
+                   const TB *__restrict__ bias, int S, int mS, int QS, int mL, int Co) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int Qp = S / 16;
+  float2 *ys = reinterpret_cast<float2 *>(smem);      // [QS][mL]
+  float2 *twr = ys + (size_t)QS * mL;                  // [slot][Qp]
+  const size_t slab = blockIdx.x;
+  const int tid = threadIdx.x;
+  const float2 *src = yhat + slab * QS * mL;
+  for (int e = tid; e < QS * mL; e += IS_THREADS) ys[e] = __ldg(src + e);
+  for (int e = tid; e < QS * Qp; e += IS_THREADS) twr[e] = __ldg(twr_g + e);
+  __syncthreads();
+  float2 *dst = U + slab * (size_t)S * mL;
+  constexpr int EB = IMG == 1 ? 4 : 2;
+  const int b = (int)(slab / Co), o = (int)(slab - (size_t)b * Co);
+  const uint32_t sbo = (uint32_t)(2 * mL * EB / 16) * 128u;
+  const size_t row_bytes = (size_t)(IMG == 1 ? 2 * Co : Co) * 2 * mL * EB;
+  const float bias_o = (IMG && bias) ? to_f<TB>(bias[o]) : 0.f;
+  int k = tid % mL, r = tid / mL;                        // task = r mL + k
+  const int dr = IS_THREADS / mL, dk = IS_THREADS % mL;
+  for (; r < Qp;) {
     float2 v[16];
 #pragma unroll
     for (int p = 0; p < 16; ++p) {
-      float2 s = make_float2(0.f, 0.f);
-      const int n = slot_cnt[p];
-      for (int e = 0; e < n; ++e) {
-        const int slot = slot_tab[p * SM_MAXPER + e];
-        cfma(s, y[slot], twr[slot * Qp + r]);
+      float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int d = -NDM; d < NDM; ++d) {
+        const int kq = p + 16 * d;            // signed wavenumber
+        if (FULL || (kq >= -mS && kq < mS)) {
+          const int slot = kq >= 0 ? kq : kq + QS;
+          cfma(acc, ys[slot * mL + k], twr[slot * Qp + r]);
+        }
       }
-      v[p] = s;
+      v[p] = acc;
     }
     fft::fft16<+1>(v);
-    if (b < B && o < Co && k < mL) {
-      float2 *dst = U + ((b * Co + o) * (long long)S + r) * mL + k;
+    if (IMG == 0) {
+      float2 *d = dst + (size_t)r * mL + k;
 #pragma unroll
-      for (int a = 0; a < 16; ++a) dst[(long long)a * Qp * mL] = v[a];
+      for (int a = 0; a < 16; ++a) d[(size_t)a * Qp * mL] = v[a];
+    } else {
+      const uint32_t hi = img_off(o, 2 * k, EB, sbo);
+      unsigned char *base = img + ((size_t)b * S + r) * row_bytes;
+#pragma unroll
+      for (int a = 0; a < 16; ++a) {
+        float2 u = v[a];
+        if (k == 0) u.x += bias_o;
+        unsigned char *row = base + (size_t)a * Qp * row_bytes;
+        if (IMG == 1) {
+          uint32_t hx, lx, hy, ly;
+          tc_split(u.x, hx, lx);
+          tc_split(u.y, hy, ly);
+          *reinterpret_cast<uint2 *>(row + hi) = make_uint2(hx, hy);
+          *reinterpret_cast<uint2 *>(row + img_off(Co + o, 2 * k, EB, sbo)) = make_uint2(lx, ly);
+        } else if (IMG == 2) {
+          *reinterpret_cast<__half2 *>(row + hi) = __floats2half2_rn(u.x, u.y);
+        } else {
+          *reinterpret_cast<__nv_bfloat162 *>(row + hi) = __floats2bfloat162_rn(u.x, u.y);
+        }
+      }
     }
+    r += dr;
+    k += dk;
+    if (k >= mL) { k -= mL; ++r; }
   }
 }
 
 }  // namespace
 
-bool spec_mid_supported(const Geom &g) {
+size_t spec_mid_table_bytes(const Geom &g) {
+  return g.d == 2 ? sizeof(float2) * (size_t)g.QS * (g.S / 16) : 0;
+}
+
+bool spec_mid_supported(const Geom &g, int Ci, int Co) {
   if (g.d != 2 || g.QO != 1) return false;
   if (g.S % 16 != 0 || g.QS > SM_MAXQS) return false;
-  // residues hold at most ceil(QS / 16) + 1 kept modes
-  if ((g.QS + 15) / 16 + 1 > SM_MAXPER) return false;
-  if (g.B > 65535LL * SM_BG) return false;
-  return mid_plan(g.QS, g.S).total <= 200 * 1024;
+  if (g.B * (long long)g.K * kMaxWidth > (1LL << 31)) return false;
+  if (mix_modes_group(Ci, Co) < 1) return false;
+  if ((g.B + MM_BS - 1) / MM_BS > 65535) return false;
+  const size_t inv = sizeof(float2) * ((size_t)g.QS * g.mL + (size_t)g.QS * (g.S / 16));
+  return inv <= 200 * 1024;
 }
 
 cudaError_t launch_spec_mid(const Launch &L, const Geom &g, int dtype, int Ci, int Co,
-                            const float2 *xhat, const void *R, float2 *U) {
-  const MidPlan p = mid_plan(g.QS, g.S);
-  dim3 grid((unsigned)((g.mL + SM_KG - 1) / SM_KG), (unsigned)((Co + SM_OG - 1) / SM_OG),
-            (unsigned)((g.B + SM_BG - 1) / SM_BG));
+                            const float2 *xhat, const void *R, float2 *yhat, float2 *twr,
+                            float2 *U, unsigned char *img, const void *bias) {
+  const int mg = mix_modes_group(Ci, Co);
+  const size_t smem = sizeof(float2) * ((size_t)MM_BS * Ci + (size_t)Ci * Co) * mg;
+  dim3 grid((unsigned)((g.K + mg - 1) / mg), (unsigned)((g.B + MM_BS - 1) / MM_BS));
   launch_begin(L);
   auto go = [&](auto kern, const auto *r) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)p.total);
+                                         (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, SM_THREADS, p.total, L.stream>>>(xhat, r, U, g.B, Ci, Co, g.S, g.mS, g.QS, g.mL,
-                                                  g.NL, g.inv_n);
+    kern<<<grid, MM_THREADS, smem, L.stream>>>(xhat, r, yhat, twr, (int)g.B, Ci, Co, (int)g.K,
+                                               g.mL, g.NL, g.inv_n, g.S, g.mS, g.QS);
     return cudaGetLastError();
   };
+  auto by_mg = [&](auto k4, auto k2, auto k1, const auto *r) {
+    return mg == 4 ? go(k4, r) : mg == 2 ? go(k2, r) : go(k1, r);
+  };
   cudaError_t e;
-  if (dtype == DT_F32) e = go(k_spec_mid<float>, (const float *)R);
-  else if (dtype == DT_F16) e = go(k_spec_mid<__half>, (const __half *)R);
-  else e = go(k_spec_mid<__nv_bfloat16>, (const __nv_bfloat16 *)R);
-  launch_end(L, "spec_mid");
+  if (dtype == DT_F32)
+    e = by_mg(k_mix_modes<float, 4>, k_mix_modes<float, 2>, k_mix_modes<float, 1>,
+              (const float *)R);
+  else if (dtype == DT_F16)
+    e = by_mg(k_mix_modes<__half, 4>, k_mix_modes<__half, 2>, k_mix_modes<__half, 1>,
+              (const __half *)R);
+  else
+    e = by_mg(k_mix_modes<__nv_bfloat16, 4>, k_mix_modes<__nv_bfloat16, 2>,
+              k_mix_modes<__nv_bfloat16, 1>, (const __nv_bfloat16 *)R);
+  launch_end(L, "mix_modes");
+  if (e != cudaSuccess) return e;
+
+  const size_t smem2 = sizeof(float2) * ((size_t)g.QS * g.mL + (size_t)g.QS * (g.S / 16));
+  const unsigned slabs = (unsigned)(g.B * Co);
+  launch_begin(L);
+  auto go2 = [&](auto kern, const auto *bp) {
+    cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)smem2);
+    if (e2 != cudaSuccess) return e2;
+    kern<<<slabs, IS_THREADS, smem2, L.stream>>>(yhat, twr, U, img, bp, g.S, g.mS, g.QS, g.mL,
+                                                 Co);
+    return cudaGetLastError();
+  };
+  // by the kept set of the slab axis, then by output form
+  auto by_out = [&](auto k0, auto k1, auto k2, auto k3) {
+    if (!img) return go2(k0, (const float *)nullptr);
+    if (dtype == DT_F32) return go2(k1, (const float *)bias);
+    if (dtype == DT_F16) return go2(k2, (const __half *)bias);
+    return go2(k3, (const __nv_bfloat16 *)bias);
+  };
+#define FNO_INV_SLAB(NDM, FULL)                                                           \
+  by_out(k_inv_slab_fft<NDM, FULL, 0, float>, k_inv_slab_fft<NDM, FULL, 1, float>,         \
+         k_inv_slab_fft<NDM, FULL, 2, __half>, k_inv_slab_fft<NDM, FULL, 3, __nv_bfloat16>)
+  if (g.mS == 16) e = FNO_INV_SLAB(1, true);
+  else if (g.mS == 32) e = FNO_INV_SLAB(2, true);
+  else if (g.mS > 16) e = FNO_INV_SLAB(2, false);
+  else e = FNO_INV_SLAB(1, false);
+#undef FNO_INV_SLAB
+  launch_end(L, img ? "inv_slab_img" : "inv_slab_fft");
   return e;
 }
 

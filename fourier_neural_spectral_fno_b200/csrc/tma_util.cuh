@@ -32,6 +32,18 @@ __device__ __forceinline__ void load_4d(void *dst, const CUtensorMap *map, uint6
       : "memory");
 }
 
+// Untiled bulk copy of `bytes` contiguous bytes from global into shared memory
+// (both addresses 16-byte aligned, bytes a multiple of 16), completed as
+// transaction bytes on `mbar`.
+__device__ __forceinline__ void load_bulk(void *dst, const void *src, uint32_t bytes,
+                                          uint64_t *mbar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          tc::smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(tc::smem_u32(mbar))
+      : "memory");
+}
+
 __device__ __forceinline__ void prefetch_map(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -263,9 +263,14 @@ cudaError_t launch_fwd_transform(const Launch &L, const Geom &g, int dtype, int 
   const long long planes = g.B * C * g.O;
   int nb;
   cudaError_t err;
-  if (L.tc == 1 && fwd_fft_supported(g, in0, in1, load_mode)) {
-    // the cluster writes whole plane spectra: 2D grids are done, 3D grids
-    // still contract the outer axis (one "band")
+  if (L.tc == 1 && fwd_plane_supported(g, dtype, in0, in1, load_mode)) {
+    // whole plane spectra: 2D grids are done, 3D grids still contract the
+    // outer axis (one "band")
+    if (g.QO == 1) return launch_fwd_plane(L, g, dtype, load_mode, C, in0, in1, xhat);
+    err = launch_fwd_plane(L, g, dtype, load_mode, C, in0, in1, zpart);
+    if (err != cudaSuccess) return err;
+    nb = 1;
+  } else if (L.tc == 1 && fwd_fft_supported(g, in0, in1, load_mode)) {
     if (g.QO == 1) return launch_fwd_fft(L, g, dtype, load_mode, C, in0, in1, xhat);
     err = launch_fwd_fft(L, g, dtype, load_mode, C, in0, in1, zpart);
     if (err != cudaSuccess) return err;
