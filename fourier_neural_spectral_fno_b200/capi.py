@@ -45,7 +45,7 @@ EXPORTED = (
     "fno_spectral_conv_bwd", "fno_block_fwd", "fno_block_bwd", "fno_forward", "fno_backward",
     "fno_mse", "fno_profile_enable", "fno_profile_read", "fno_set_tensor_cores",
     "fno_device_error", "fno_spectral_conv_fwd_noalloc", "fno_adam_step",
-    "fno_backward_ready", "fno_spectral_conv_fwd_cp", "fno_block_fwd_cp",
+    "fno_backward_ready", "fno_spectral_conv_fwd_cp", "fno_block_fwd_cp", "fno_set_wait_limit",
 )
 
 FNO_MAX_CP_RANK = 32
@@ -132,6 +132,7 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "fno_spectral_conv_fwd_cp": (i, [bd, i, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "fno_block_fwd_cp": (i, [bd, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "fno_device_error": (i, [i]),
+        "fno_set_wait_limit": (i, [i]),
         "fno_profile_read": (i, [ctypes.POINTER(KernelStat), i]),
         "fno_adam_step": (i, [ctypes.c_int64, vp, vp, vp, vp, vp, i, i, ctypes.c_float,
                               ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_float,
@@ -368,15 +369,27 @@ def fno_profile_read(max_kernels: int = 64) -> Dict[str, Dict[str, float]]:
 
 
 def fno_set_tensor_cores(mode) -> int:
-    """Kernel selection: 1 / True = the default kernels (pruned-FFT transform
-    and fused spectral middle on the CUDA cores, tcgen05 TMA pipelines for the
-    epilogue and projection) where shapes allow, 3 = tcgen05 TMA pipelines
-    throughout (dense DFT-matrix transform), 2 = tcgen05 kernels without the
-    pipelines, 0 / False = the CUDA-core kernels.  Returns the previous setting."""
+    """Kernel selection: 1 / True = the default kernels (per shape the faster
+    design as measured: the streaming pruned-FFT transform, mixing and pruned
+    slab-axis inverse on the CUDA cores, tcgen05 TMA pipelines for the epilogue
+    and projection), 4 = the default with the clustered FFT transform, 3 =
+    tcgen05 TMA pipelines throughout (dense DFT-matrix transform), 2 = tcgen05
+    kernels without the pipelines, 0 / False = the CUDA-core kernels.  Returns
+    the previous setting."""
     m = int(mode)
-    if m not in (0, 1, 2, 3):
-        raise ValueError("kernel mode must be 0, 1, 2 or 3")
+    if m not in (0, 1, 2, 3, 4):
+        raise ValueError("kernel mode must be 0, 1, 2, 3 or 4")
     return int(load().fno_set_tensor_cores(m))
+
+
+def fno_set_wait_limit(spins: int) -> int:
+    """Bound every tensor-core pipeline wait to ``spins`` suspended polls
+    (default 131072, about two seconds); returns the previous bound.  A test
+    hook: 0 makes waits give up after one probe (results then invalid)."""
+    prev = int(load().fno_set_wait_limit(int(spins)))
+    if prev < 0:
+        _check(prev)
+    return prev
 
 
 def fno_device_error(clear: bool = True) -> None:

@@ -11,6 +11,7 @@
 
 #include "fno.h"
 #include "fno_kernels.cuh"
+#include "tc_util.cuh"
 
 using namespace fno;
 
@@ -180,7 +181,9 @@ std::vector<ProfRec> g_prof;   // event pool; the first g_prof_used entries are 
 size_t g_prof_used = 0;
 bool g_prof_on = false;
 
-__device__ int g_fno_device_error;   // set by kernels whose bounded waits expire
+// [0]: set by kernels whose bounded waits expire; [1]: the wait limit they use
+// (suspended polls per wait, fno_set_wait_limit)
+__device__ int g_fno_device_error[2] = {0, FNO_DEFAULT_WAIT_SPINS};
 
 std::mutex g_err_word_mu;
 
@@ -210,6 +213,14 @@ Launch make_launch(fno_stream_t s) {
   return L;
 }
 
+// The slab-axis inverse U = E_S Z: the pruned FFT on the default paths where
+// the shape allows it, else the dense sum.
+cudaError_t invert_slab(const Launch &L, const Geom &g, long long C, const float2 *Z, float2 *U) {
+  if ((L.tc == 1 || L.tc == 4) && inv_slab_fft_supported(g))
+    return launch_inv_slab_fft(L, g, C, Z, U);
+  return launch_inv_slab(L, g, C, Z, U);
+}
+
 // u_ready: U (ws + w.u) already holds the spectrum inverted along the slab
 // axis (launch_spec_mid), so no slab-axis inverse is launched here.
 cudaError_t run_epilogue(const Launch &L, const Geom &g, int dtype, int mode, const EpiArgs &a,
@@ -217,16 +228,16 @@ cudaError_t run_epilogue(const Launch &L, const Geom &g, int dtype, int mode, co
   float2 *U = reinterpret_cast<float2 *>(ws + w.u);
   // channels of the spectrum being inverted: Ci for the backward modes (dxhat)
   const int cs = (mode == EPI_SPEC_BWD || mode == EPI_BLOCK_BWD) ? a.Ci : a.Co;
-  if ((L.tc == 1 || L.tc == 3) && epi_pipe_supported(g, dtype, mode, a.Ci, a.Co, a.x, U)) {
+  if ((L.tc == 1 || L.tc == 3 || L.tc == 4) && epi_pipe_supported(g, dtype, mode, a.Ci, a.Co, a.x, U)) {
     if (!u_ready) {
-      cudaError_t e = launch_inv_slab(L, g, cs, a.Z, U);
+      cudaError_t e = invert_slab(L, g, cs, a.Z, U);
       if (e != cudaSuccess) return e;
     }
     return launch_epi_pipe(L, g, dtype, mode, a, U);
   }
   if (L.tc && epi_tc_supported(g, dtype, mode, a.Ci, a.Co)) {
     if (!u_ready) {
-      cudaError_t e = launch_inv_slab(L, g, cs, a.Z, U);
+      cudaError_t e = invert_slab(L, g, cs, a.Z, U);
       if (e != cudaSuccess) return e;
     }
     return launch_epilogue_tc(L, g, dtype, mode, a, U);
@@ -239,7 +250,7 @@ cudaError_t run_epilogue(const Launch &L, const Geom &g, int dtype, int mode, co
   if (mode == EPI_BLOCK_BWD && g.S > 1) {
     // the block backward reads the slab-axis inverse once per row instead of
     // recomputing it in every tile
-    cudaError_t e = launch_inv_slab(L, g, cs, a.Z, U);
+    cudaError_t e = invert_slab(L, g, cs, a.Z, U);
     if (e != cudaSuccess) return e;
     EpiArgs b = a;
     b.U = U;
@@ -266,10 +277,11 @@ int run_forward(const Launch &L, const Geom &g, int dtype, unsigned flags, int C
                                Ci, x, nullptr, zpart, xhat),
           "forward transform");
   // 2D grids on the default path: mixing and the slab-axis inverse in one launch
-  const bool mid = !cp && L.tc == 1 && spec_mid_supported(g, Ci, Co);
+  const bool mid = !cp && (L.tc == 1 || L.tc == 4) && spec_mid_supported(g, Ci, Co);
   // the slab-axis inverse writes the epilogue's B operand directly where the
   // pipelined epilogue takes it
   const bool img = mid && epi_img_supported(g, dtype, epi_mode, Ci, Co) &&
+                   spec_mid_img_supported(g, Co) &&
                    epi_pipe_supported(g, dtype, epi_mode, Ci, Co, x, ws + w.u);
   if (cp)
     FNO_TRY(launch_mix_cp(L, g, dtype, Ci, Co, rank, xhat, *cp, yhat), "factorised mixing");
@@ -486,7 +498,7 @@ int fno_last_launch_count(void) { return g_launches; }
 
 int fno_set_tensor_cores(int enable) {
   const int prev = g_use_tc;
-  g_use_tc = (enable == 2 || enable == 3) ? enable : enable ? 1 : 0;
+  g_use_tc = (enable >= 2 && enable <= 4) ? enable : enable ? 1 : 0;
   return prev;
 }
 
@@ -504,6 +516,19 @@ int fno_device_error(int clear) {
   if (v) return fail(FNO_ERR_TIMEOUT, "a bounded device-side wait expired (results invalid)");
   g_err[0] = 0;
   return FNO_OK;
+}
+
+int fno_set_wait_limit(int spins) {
+  if (spins < 0) return fail(FNO_ERR_INVALID_ARG, "wait limit %d < 0", spins);
+  int *p = device_error_word();
+  if (!p) return fail(FNO_ERR_CUDA, "no CUDA device");
+  int prev = 0;
+  cudaError_t e = cudaMemcpy(&prev, p + 1, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the wait limit");
+  e = cudaMemcpy(p + 1, &spins, sizeof(int), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "setting the wait limit");
+  g_err[0] = 0;
+  return prev;
 }
 
 int fno_profile_enable(int on) {

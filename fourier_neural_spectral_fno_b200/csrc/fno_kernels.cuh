@@ -35,8 +35,10 @@ struct Launch {
   cudaStream_t stream;
   int *count;       // incremented per kernel launch
   int num_sms;
-  int tc;           // 1: default (pruned-FFT transform and fused spectral middle on CUDA
-                    //    cores, tcgen05 TMA pipelines for the epilogue and projection);
+  int tc;           // 1: default (pruned-FFT transform, mixing and pruned slab-axis
+                    //    inverse on CUDA cores where each is measured faster, tcgen05
+                    //    TMA pipelines for the epilogue and projection);
+                    // 4: as 1 with the clustered FFT transform;
                     // 3: tcgen05 TMA pipelines throughout (dense DFT-matrix transform);
                     // 2: tcgen05 without the pipelines; 0: CUDA cores only
   int *err;         // device error word (bounded waits that expired)
@@ -90,8 +92,14 @@ cudaError_t launch_fwd_plane(const Launch &L, const Geom &g, int dtype, int load
 // 2D spectral middle (spec_mid.cu): mixing into yhat (as launch_mix_fwd),
 // then the slab-axis inverse as a pruned FFT into
 // U[b][o][S][mL] = sum_q yhat[b,o,q,k] exp(+2 pi i kq n / S); two launches
+// the pruned slab-axis inverse alone (the backward's dxhat), same output as
+// launch_inv_slab: U[b][c][S][mL]
+bool inv_slab_fft_supported(const Geom &g);
+cudaError_t launch_inv_slab_fft(const Launch &L, const Geom &g, long long C, const float2 *Z,
+                                float2 *U);
 // twr: workspace for the slab-axis twiddle table (spec_mid_table_bytes)
 bool spec_mid_supported(const Geom &g, int Ci, int Co);
+bool spec_mid_img_supported(const Geom &g, int Co);   // the image-writing inverse fits
 size_t spec_mid_table_bytes(const Geom &g);
 // img (optional): write the epilogue's B images (epi_img_supported) instead of
 // U, with bias (may be NULL) folded in

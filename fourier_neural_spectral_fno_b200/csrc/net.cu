@@ -496,7 +496,7 @@ static cudaError_t proj_fwd_t(const Launch &L, const Geom &g, int width, int hid
 cudaError_t launch_proj_fwd(const Launch &L, const Geom &g, int dtype, int width, int hidden,
                             int out_ch, const void *v, const void *Q1, const void *q1,
                             const void *Q2, const void *q2, void *u) {
-  if ((L.tc == 1 || L.tc == 3) && proj_pipe_supported(g, dtype, width, hidden, out_ch, v))
+  if ((L.tc == 1 || L.tc == 3 || L.tc == 4) && proj_pipe_supported(g, dtype, width, hidden, out_ch, v))
     return launch_proj_pipe(L, g, dtype, width, hidden, out_ch, v, Q1, q1, Q2, q2, u);
   if (L.tc && proj_tc_supported(g, dtype, width, hidden, out_ch))
     return launch_proj_fwd_tc(L, g, dtype, width, hidden, out_ch, v, Q1, q1, Q2, q2, u);

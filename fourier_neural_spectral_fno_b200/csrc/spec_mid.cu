@@ -109,17 +109,18 @@ __global__ void __launch_bounds__(MM_THREADS)
   int b = 0, o = tid / MG;
   while (o >= Co) { o -= Co; ++b; }
   const int db = bo_step / Co, dob = bo_step % Co;
+  const int rstep = Co * MG;
   for (; b < nb;) {
-    const float2 *xp = xs + (size_t)b * Ci * MG + m;
-    const float2 *rp = rs + (size_t)o * MG + m;
-    const size_t rstep = (size_t)Co * MG;
+    const float2 *xp = xs + b * Ci * MG + m;
+    const float2 *rp = rs + o * MG + m;
     float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
     int i = 0;
+#pragma unroll 4
     for (; i + 1 < Ci; i += 2) {
-      cfma(s0, xp[(size_t)i * MG], rp[i * rstep]);
-      cfma(s1, xp[(size_t)(i + 1) * MG], rp[(i + 1) * rstep]);
+      cfma(s0, xp[i * MG], rp[i * rstep]);
+      cfma(s1, xp[(i + 1) * MG], rp[(i + 1) * rstep]);
     }
-    if (i < Ci) cfma(s0, xp[(size_t)i * MG], rp[i * rstep]);
+    if (i < Ci) cfma(s0, xp[i * MG], rp[i * rstep]);
     if (m < mg)
       yhat[((size_t)(b0 + b) * Co + o) * K + m0 + m] =
           make_float2(w * (s0.x + s1.x), w * (s0.y + s1.y));
@@ -139,14 +140,12 @@ __device__ __forceinline__ uint32_t img_off(int n, int c, int eb, uint32_t sbo) 
 
 // NDM: the kept wavenumbers of residue p (mod 16) are among p + 16 d,
 // d in [-NDM, NDM) (NDM = 1 for mS <= 16, 2 for mS <= 32); FULL: mS = 16 NDM,
-// so every candidate is kept and no test is needed.
-// IMG 0: write U; 1: float32 B images (tf32 high / low rows); 2 / 3: float16 /
-// bfloat16 B images (the epilogue's operand layout, bias folded into column 0)
-template <int NDM, bool FULL, int IMG, typename TB>
+// so every candidate is kept and no test is needed.  twr_g: the twiddle table
+// of the mixing kernel, or NULL to build it here.
+template <int NDM, bool FULL>
 __global__ void __launch_bounds__(IS_THREADS)
     k_inv_slab_fft(const float2 *__restrict__ yhat, const float2 *__restrict__ twr_g,
-                   float2 *__restrict__ U, unsigned char *__restrict__ img,
-                   const TB *__restrict__ bias, int S, int mS, int QS, int mL, int Co) {
+                   float2 *__restrict__ U, int S, int mS, int QS, int mL) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int Qp = S / 16;
   float2 *ys = reinterpret_cast<float2 *>(smem);      // [QS][mL]
@@ -155,14 +154,18 @@ __global__ void __launch_bounds__(IS_THREADS)
   const int tid = threadIdx.x;
   const float2 *src = yhat + slab * QS * mL;
   for (int e = tid; e < QS * mL; e += IS_THREADS) ys[e] = __ldg(src + e);
-  for (int e = tid; e < QS * Qp; e += IS_THREADS) twr[e] = __ldg(twr_g + e);
+  if (twr_g) {
+    for (int e = tid; e < QS * Qp; e += IS_THREADS) twr[e] = __ldg(twr_g + e);
+  } else {   // no table from the mixing kernel: build it here
+    for (int e = tid; e < QS * Qp; e += IS_THREADS) {
+      const int slot = e / Qp, rr = e - slot * Qp;
+      float sn, cs;
+      sincospif(2.0f * (float)mulmod(kept_k(slot, mS, S), rr, S) / (float)S, &sn, &cs);
+      twr[e] = make_float2(cs, sn);
+    }
+  }
   __syncthreads();
   float2 *dst = U + slab * (size_t)S * mL;
-  constexpr int EB = IMG == 1 ? 4 : 2;
-  const int b = (int)(slab / Co), o = (int)(slab - (size_t)b * Co);
-  const uint32_t sbo = (uint32_t)(2 * mL * EB / 16) * 128u;
-  const size_t row_bytes = (size_t)(IMG == 1 ? 2 * Co : Co) * 2 * mL * EB;
-  const float bias_o = (IMG && bias) ? to_f<TB>(bias[o]) : 0.f;
   int k = tid % mL, r = tid / mL;                        // task = r mL + k
   const int dr = IS_THREADS / mL, dk = IS_THREADS % mL;
   for (; r < Qp;) {
@@ -181,38 +184,125 @@ __global__ void __launch_bounds__(IS_THREADS)
       v[p] = acc;
     }
     fft::fft16<+1>(v);
-    if (IMG == 0) {
-      float2 *d = dst + (size_t)r * mL + k;
+    float2 *d = dst + (size_t)r * mL + k;
 #pragma unroll
-      for (int a = 0; a < 16; ++a) d[(size_t)a * Qp * mL] = v[a];
-    } else {
-      const uint32_t hi = img_off(o, 2 * k, EB, sbo);
-      unsigned char *base = img + ((size_t)b * S + r) * row_bytes;
-#pragma unroll
-      for (int a = 0; a < 16; ++a) {
-        float2 u = v[a];
-        if (k == 0) u.x += bias_o;
-        unsigned char *row = base + (size_t)a * Qp * row_bytes;
-        if (IMG == 1) {
-          uint32_t hx, lx, hy, ly;
-          tc_split(u.x, hx, lx);
-          tc_split(u.y, hy, ly);
-          *reinterpret_cast<uint2 *>(row + hi) = make_uint2(hx, hy);
-          *reinterpret_cast<uint2 *>(row + img_off(Co + o, 2 * k, EB, sbo)) = make_uint2(lx, ly);
-        } else if (IMG == 2) {
-          *reinterpret_cast<__half2 *>(row + hi) = __floats2half2_rn(u.x, u.y);
-        } else {
-          *reinterpret_cast<__nv_bfloat162 *>(row + hi) = __floats2bfloat162_rn(u.x, u.y);
-        }
-      }
-    }
+    for (int a = 0; a < 16; ++a) d[(size_t)a * Qp * mL] = v[a];
     r += dr;
     k += dk;
     if (k >= mL) { k -= mL; ++r; }
   }
 }
 
+// The same inverse writing the epilogue's B images: a CTA owns eight
+// consecutive output channels (one 8-row group of the operand's core matrices)
+// and a quarter of the r's, and thread t takes channel t % 8 and mode
+// (t / 8) % mL, so that the sixteen-byte rows of the core matrices of one grid
+// row leave a warp as one contiguous 256-byte store (the (re, im) pairs of two
+// modes of eight channels).  IMG 1: float32 images (tf32 high parts in rows
+// [0, Co), low parts in [Co, 2 Co)); 2 / 3: float16 / bfloat16 images; the
+// bias is folded into column 0.
+constexpr int IMG_RSPLIT = 4;
+template <int NDM, bool FULL, int IMG, typename TB>
+__global__ void __launch_bounds__(IS_THREADS)
+    k_inv_slab_img(const float2 *__restrict__ yhat, const float2 *__restrict__ twr_g,
+                   unsigned char *__restrict__ img, const TB *__restrict__ bias, int S, int mS,
+                   int QS, int mL, int Co) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int Qp = S / 16;
+  float2 *ys = reinterpret_cast<float2 *>(smem);      // [slot][k][8 channels]
+  float2 *twr = ys + (size_t)QS * mL * 8;              // [slot][Qp]
+  const int groups = Co / 8;
+  const int b = blockIdx.x / groups, o0 = (blockIdx.x - b * groups) * 8;
+  const int tid = threadIdx.x;
+  for (int e = tid; e < 8 * QS * mL; e += IS_THREADS) {
+    const int oo = e / (QS * mL), sk = e - oo * (QS * mL);
+    ys[sk * 8 + oo] = __ldg(yhat + ((size_t)b * Co + o0 + oo) * QS * mL + sk);
+  }
+  for (int e = tid; e < QS * Qp; e += IS_THREADS) twr[e] = __ldg(twr_g + e);
+  __syncthreads();
+  constexpr int EB = IMG == 1 ? 4 : 2;
+  const uint32_t sbo = (uint32_t)(2 * mL * EB / 16) * 128u;
+  const size_t row_bytes = (size_t)(IMG == 1 ? 2 * Co : Co) * 2 * mL * EB;
+  const int oo = tid & 7;
+  const int o = o0 + oo;
+  const float bias_o = bias ? to_f<TB>(bias[o]) : 0.f;
+  const int per_r = 8 * mL;
+  const int r_lo = blockIdx.y * ((Qp + IMG_RSPLIT - 1) / IMG_RSPLIT);
+  const int r_hi = min(Qp, r_lo + (Qp + IMG_RSPLIT - 1) / IMG_RSPLIT);
+  for (int task = tid; task < (r_hi - r_lo) * per_r; task += IS_THREADS) {
+    const int r = r_lo + task / per_r, k = (task / 8) % mL;
+    float2 v[16];
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+      float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int d = -NDM; d < NDM; ++d) {
+        const int kq = p + 16 * d;
+        if (FULL || (kq >= -mS && kq < mS)) {
+          const int slot = kq >= 0 ? kq : kq + QS;
+          cfma(acc, ys[(slot * mL + k) * 8 + oo], twr[slot * Qp + r]);
+        }
+      }
+      v[p] = acc;
+    }
+    fft::fft16<+1>(v);
+    const uint32_t hi = img_off(o, 2 * k, EB, sbo);
+    const uint32_t lo = IMG == 1 ? img_off(Co + o, 2 * k, EB, sbo) : 0u;
+    unsigned char *base = img + ((size_t)b * S + r) * row_bytes;
+#pragma unroll
+    for (int a = 0; a < 16; ++a) {
+      float2 u = v[a];
+      if (k == 0) u.x += bias_o;
+      unsigned char *row = base + (size_t)a * Qp * row_bytes;
+      if (IMG == 1) {
+        uint32_t hx, lx, hy, ly;
+        tc_split(u.x, hx, lx);
+        tc_split(u.y, hy, ly);
+        *reinterpret_cast<uint2 *>(row + hi) = make_uint2(hx, hy);
+        *reinterpret_cast<uint2 *>(row + lo) = make_uint2(lx, ly);
+      } else if (IMG == 2) {
+        *reinterpret_cast<__half2 *>(row + hi) = __floats2half2_rn(u.x, u.y);
+      } else {
+        *reinterpret_cast<__nv_bfloat162 *>(row + hi) = __floats2bfloat162_rn(u.x, u.y);
+      }
+    }
+  }
+}
+
 }  // namespace
+
+bool inv_slab_fft_supported(const Geom &g) {
+  if (g.d != 2 || g.QO != 1 || g.S % 16 != 0 || g.QS > SM_MAXQS) return false;
+  const size_t inv = sizeof(float2) * ((size_t)g.QS * g.mL + (size_t)g.QS * (g.S / 16));
+  return inv <= 200 * 1024;
+}
+
+cudaError_t launch_inv_slab_fft(const Launch &L, const Geom &g, long long C, const float2 *Z,
+                                float2 *U) {
+  const size_t smem2 = sizeof(float2) * ((size_t)g.QS * g.mL + (size_t)g.QS * (g.S / 16));
+  const unsigned slabs = (unsigned)(g.B * C);
+  launch_begin(L);
+  auto go2 = [&](auto kern) {
+    cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)smem2);
+    if (e2 != cudaSuccess) return e2;
+    kern<<<slabs, IS_THREADS, smem2, L.stream>>>(Z, nullptr, U, g.S, g.mS, g.QS, g.mL);
+    return cudaGetLastError();
+  };
+  cudaError_t e;
+  if (g.mS == 16) e = go2(k_inv_slab_fft<1, true>);
+  else if (g.mS == 32) e = go2(k_inv_slab_fft<2, true>);
+  else if (g.mS > 16) e = go2(k_inv_slab_fft<2, false>);
+  else e = go2(k_inv_slab_fft<1, false>);
+  launch_end(L, "inv_slab_fft");
+  return e;
+}
+
+bool spec_mid_img_supported(const Geom &g, int Co) {
+  if (Co % 8 != 0) return false;
+  const size_t smem = sizeof(float2) * ((size_t)8 * g.QS * g.mL + (size_t)g.QS * (g.S / 16));
+  return smem <= 200 * 1024;
+}
 
 size_t spec_mid_table_bytes(const Geom &g) {
   return g.d == 2 ? sizeof(float2) * (size_t)g.QS * (g.S / 16) : 0;
@@ -259,32 +349,46 @@ cudaError_t launch_spec_mid(const Launch &L, const Geom &g, int dtype, int Ci, i
   launch_end(L, "mix_modes");
   if (e != cudaSuccess) return e;
 
-  const size_t smem2 = sizeof(float2) * ((size_t)g.QS * g.mL + (size_t)g.QS * (g.S / 16));
-  const unsigned slabs = (unsigned)(g.B * Co);
   launch_begin(L);
-  auto go2 = [&](auto kern, const auto *bp) {
-    cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          (int)smem2);
-    if (e2 != cudaSuccess) return e2;
-    kern<<<slabs, IS_THREADS, smem2, L.stream>>>(yhat, twr, U, img, bp, g.S, g.mS, g.QS, g.mL,
-                                                 Co);
-    return cudaGetLastError();
-  };
-  // by the kept set of the slab axis, then by output form
-  auto by_out = [&](auto k0, auto k1, auto k2, auto k3) {
-    if (!img) return go2(k0, (const float *)nullptr);
-    if (dtype == DT_F32) return go2(k1, (const float *)bias);
-    if (dtype == DT_F16) return go2(k2, (const __half *)bias);
-    return go2(k3, (const __nv_bfloat16 *)bias);
-  };
-#define FNO_INV_SLAB(NDM, FULL)                                                           \
-  by_out(k_inv_slab_fft<NDM, FULL, 0, float>, k_inv_slab_fft<NDM, FULL, 1, float>,         \
-         k_inv_slab_fft<NDM, FULL, 2, __half>, k_inv_slab_fft<NDM, FULL, 3, __nv_bfloat16>)
-  if (g.mS == 16) e = FNO_INV_SLAB(1, true);
-  else if (g.mS == 32) e = FNO_INV_SLAB(2, true);
-  else if (g.mS > 16) e = FNO_INV_SLAB(2, false);
-  else e = FNO_INV_SLAB(1, false);
-#undef FNO_INV_SLAB
+  if (!img) {
+    const size_t smem2 = sizeof(float2) * ((size_t)g.QS * g.mL + (size_t)g.QS * (g.S / 16));
+    const unsigned slabs = (unsigned)(g.B * Co);
+    auto go2 = [&](auto kern) {
+      cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            (int)smem2);
+      if (e2 != cudaSuccess) return e2;
+      kern<<<slabs, IS_THREADS, smem2, L.stream>>>(yhat, twr, U, g.S, g.mS, g.QS, g.mL);
+      return cudaGetLastError();
+    };
+    if (g.mS == 16) e = go2(k_inv_slab_fft<1, true>);
+    else if (g.mS == 32) e = go2(k_inv_slab_fft<2, true>);
+    else if (g.mS > 16) e = go2(k_inv_slab_fft<2, false>);
+    else e = go2(k_inv_slab_fft<1, false>);
+  } else {
+    const size_t smem3 =
+        sizeof(float2) * ((size_t)8 * g.QS * g.mL + (size_t)g.QS * (g.S / 16));
+    dim3 grid3((unsigned)(g.B * (Co / 8)), IMG_RSPLIT);
+    auto go3 = [&](auto kern, const auto *bp) {
+      cudaError_t e3 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            (int)smem3);
+      if (e3 != cudaSuccess) return e3;
+      kern<<<grid3, IS_THREADS, smem3, L.stream>>>(yhat, twr, img, bp, g.S, g.mS, g.QS, g.mL, Co);
+      return cudaGetLastError();
+    };
+    auto by_out = [&](auto k1, auto k2, auto k3) {
+      if (dtype == DT_F32) return go3(k1, (const float *)bias);
+      if (dtype == DT_F16) return go3(k2, (const __half *)bias);
+      return go3(k3, (const __nv_bfloat16 *)bias);
+    };
+#define FNO_INV_IMG(NDM, FULL)                                                      \
+  by_out(k_inv_slab_img<NDM, FULL, 1, float>, k_inv_slab_img<NDM, FULL, 2, __half>, \
+         k_inv_slab_img<NDM, FULL, 3, __nv_bfloat16>)
+    if (g.mS == 16) e = FNO_INV_IMG(1, true);
+    else if (g.mS == 32) e = FNO_INV_IMG(2, true);
+    else if (g.mS > 16) e = FNO_INV_IMG(2, false);
+    else e = FNO_INV_IMG(1, false);
+#undef FNO_INV_IMG
+  }
   launch_end(L, img ? "inv_slab_img" : "inv_slab_fft");
   return e;
 }

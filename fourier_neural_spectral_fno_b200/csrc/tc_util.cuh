@@ -177,11 +177,15 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *mbar, uint32_t par
   return ok != 0;
 }
 // Bounded wait: returns false (and sets *err) if the phase did not complete
-// within about two seconds (2^17 suspensions of at most 16 us each, plus a
-// first unhinted probe so that completed phases return at once).
+// within `err[1]` suspended polls of at most 16 us each (the library's wait
+// limit, 2^17 by default: about two seconds), after a first unhinted probe so
+// that completed phases return at once.  err == NULL (the drains before a CTA
+// exits) always allows the default limit.
+#define FNO_DEFAULT_WAIT_SPINS (1 << 17)
 __device__ __forceinline__ bool mbar_wait(uint64_t *mbar, uint32_t parity, int *err) {
   if (mbar_try_wait(mbar, parity)) return true;
-  for (int i = 0; i < (1 << 17); ++i)
+  const int limit = err ? *(reinterpret_cast<volatile int *>(err) + 1) : FNO_DEFAULT_WAIT_SPINS;
+  for (int i = 0; i < limit; ++i)
     if (mbar_try_wait_sleep(mbar, parity, 16384u)) return true;
   if (err) atomicExch(err, 1);
   return false;

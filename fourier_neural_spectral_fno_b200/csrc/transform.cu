@@ -263,19 +263,19 @@ cudaError_t launch_fwd_transform(const Launch &L, const Geom &g, int dtype, int 
   const long long planes = g.B * C * g.O;
   int nb;
   cudaError_t err;
-  if (L.tc == 1 && fwd_plane_supported(g, dtype, in0, in1, load_mode)) {
-    // whole plane spectra: 2D grids are done, 3D grids still contract the
-    // outer axis (one "band")
-    if (g.QO == 1) return launch_fwd_plane(L, g, dtype, load_mode, C, in0, in1, xhat);
-    err = launch_fwd_plane(L, g, dtype, load_mode, C, in0, in1, zpart);
-    if (err != cudaSuccess) return err;
-    nb = 1;
-  } else if (L.tc == 1 && fwd_fft_supported(g, in0, in1, load_mode)) {
+  // Default path, chosen by the per-stage measurement of both designs on the
+  // workloads' shapes: the streaming pruned FFT for 2D grids; the tensor-core
+  // DFT contraction for 3D grids and wherever the streaming kernel does not
+  // fit (the clustered FFT kernel is measured slower than either and is kept
+  // for kernel path 4 only).
+  if (L.tc == 1 && g.d == 2 && fwd_plane_supported(g, dtype, in0, in1, load_mode)) {
+    return launch_fwd_plane(L, g, dtype, load_mode, C, in0, in1, xhat);
+  } else if (L.tc == 4 && fwd_fft_supported(g, in0, in1, load_mode)) {
     if (g.QO == 1) return launch_fwd_fft(L, g, dtype, load_mode, C, in0, in1, xhat);
     err = launch_fwd_fft(L, g, dtype, load_mode, C, in0, in1, zpart);
     if (err != cudaSuccess) return err;
     nb = 1;
-  } else if ((L.tc == 1 || L.tc == 3) && fwd_pipe_supported(g, dtype, load_mode, in0)) {
+  } else if ((L.tc == 1 || L.tc == 3 || L.tc == 4) && fwd_pipe_supported(g, dtype, load_mode, in0)) {
     nb = s1_tc_bands(g);
     err = launch_fwd_pipe(L, g, dtype, load_mode, C, in0, zpart);
     if (err != cudaSuccess) return err;

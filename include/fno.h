@@ -152,14 +152,17 @@ const char *fno_version(void);
 /* Number of kernel launches the last successful call on this thread enqueued. */
 int fno_last_launch_count(void);
 
-/* Kernel selection.  1 (default): the pruned radix-16 FFT transform and the
- * fused mixing + slab-axis inverse on the CUDA cores, with the warp-specialised
- * tcgen05 TMA pipelines for the epilogue and the projection, wherever the shape
- * allows each; 3: the tcgen05 TMA pipelines throughout, the transform as a
- * dense DFT-matrix contraction on the tensor cores; 2: the tensor-core kernels
- * without the TMA pipelines; 0: the CUDA-core kernels everywhere.  All are
- * complete implementations; the switch exists to compare them.  Process-wide;
- * any other nonzero value means 1; returns the previous setting. */
+/* Kernel selection.  1 (default): per shape the design measured faster: the
+ * truncated transform as a streaming pruned radix-16 FFT on the CUDA cores
+ * (2D grids) or a dense DFT-matrix contraction on the tensor cores (3D grids,
+ * and shapes the streaming kernel does not take), the mixing and a pruned
+ * slab-axis inverse on the CUDA cores, the warp-specialised tcgen05 TMA
+ * pipelines for the epilogue and the projection; 4: as 1 with the transform
+ * as a clustered pruned FFT; 3: the tcgen05 TMA pipelines throughout with the
+ * dense DFT-matrix transform; 2: the tensor-core kernels without the TMA
+ * pipelines; 0: the CUDA-core kernels everywhere.  All are complete
+ * implementations; the switch exists to compare them.  Process-wide; any
+ * other nonzero value means 1; returns the previous setting. */
 int fno_set_tensor_cores(int enable);
 
 /* Synchronises the current device and reads the library's device error word,
@@ -167,6 +170,16 @@ int fno_set_tensor_cores(int enable);
  * pipeline expires (its results are then invalid).  Returns FNO_OK or
  * FNO_ERR_TIMEOUT; clear != 0 resets the word. */
 int fno_device_error(int clear);
+
+/* Bound of every wait of the tensor-core pipelines on the current device, in
+ * suspended polls of at most about 16 us (default 131072, about two seconds);
+ * returns the previous bound, or a negative error.  A test hook: with 0 each
+ * wait gives up after one probe, so a kernel whose roles are not already in
+ * step records FNO_ERR_TIMEOUT (fno_device_error) and leaves invalid results;
+ * its waits before leaving the GPU (for copies and MMAs already in flight)
+ * keep the default bound.  Synchronises the device; restore the default
+ * before normal work. */
+int fno_set_wait_limit(int spins);
 
 /* Per-kernel timing.  fno_profile_enable(1) starts a recording: from then on
  * every kernel the library launches (on any thread) is bracketed by a pair of

@@ -312,3 +312,8 @@ def test_backward_ready_validation(lib):
     assert f(ctypes.byref(d), 256, ctypes.byref(params), 256, 256, ctypes.byref(grads), 256, need,
              None, evs, 4) == capi.FNO_ERR_INVALID_ARG
     assert "ready[2]" in capi.last_error()
+
+
+def test_wait_limit_rejects_negative_values(lib):
+    assert lib.fno_set_wait_limit(-1) == capi.FNO_ERR_INVALID_ARG
+    assert "wait limit" in capi.last_error()

@@ -51,11 +51,13 @@ SHAPES = [
 ]
 
 
-@pytest.fixture(autouse=True, params=[1, 3, 2, 0], ids=["default", "tc_dft", "tc_nopipe", "cudacore"])
+@pytest.fixture(autouse=True, params=[1, 4, 3, 2, 0],
+                ids=["default", "fft_cluster", "tc_dft", "tc_nopipe", "cudacore"])
 def kernel_path(request):
-    """Every parity test runs on the default kernels (pruned-FFT transform and
-    fused spectral middle, tcgen05 epilogue pipeline), on the tcgen05 TMA
-    pipelines with the dense DFT-matrix transform, on the tcgen05 kernels
+    """Every parity test runs on the default kernels (streaming pruned-FFT
+    transform, mixing and pruned slab-axis inverse, tcgen05 epilogue
+    pipeline), on the default with the clustered FFT transform, on the tcgen05
+    TMA pipelines with the dense DFT-matrix transform, on the tcgen05 kernels
     without pipelines (where the shape allows each) and on the CUDA-core
     kernels; no bounded device wait may expire."""
     capi.fno_set_tensor_cores(request.param)
@@ -251,7 +253,7 @@ def test_launch_count_is_reported(kernel_path):
     capi.fno_block_fwd(d, dev(x), dev_complex(r), dev(w), dev(b), y)
     # transform, finish, mix, epilogue; the default path inverts the slab axis
     # in a launch of its own
-    assert capi.last_launch_count() == (5 if kernel_path == 1 else 4)
+    assert capi.last_launch_count() == (5 if kernel_path in (1, 4) else 4)
 
 
 @pytest.mark.parametrize("grid,modes", [((64, 64), (10, 12)), ((256, 128), (16, 20)), ((15, 9), (5, 5))])

@@ -29,8 +29,14 @@ def test_mbarrier_waits_only_in_the_bounded_helper():
     # the bounded wait: a fixed number of suspended attempts, then the error word
     body = helper[helper.index("bool mbar_wait("):]
     body = body[:body.index("\n}\n")]
-    assert re.search(r"for \(.*<\s*\(1u? << 17\)", body) or "1 << 17" in body or "131072" in body
+    # a loop bounded by the library's wait limit (err[1], set by fno_set_wait_limit)
+    # or, for the drains (err == NULL), by the default of 2^17 suspended polls
+    assert re.search(r"for \(int i = 0; i < limit; \+\+i\)", body)
+    assert "err ?" in body and "FNO_DEFAULT_WAIT_SPINS" in body
+    assert re.search(r"#define FNO_DEFAULT_WAIT_SPINS \(1 << 17\)", helper)
     assert "err" in body
+    api = srcs["fno_api.cu"]
+    assert re.search(r"g_fno_device_error\[2\] = \{0, FNO_DEFAULT_WAIT_SPINS\}", api)
 
 
 def test_no_deliberate_traps():
