@@ -200,11 +200,14 @@ def algorithmic_bytes(tag: str, wl) -> float:
         k *= 2 * m
     spec = wl.batch * wl.width * k * 8
     r = wl.width * wl.width * k * 2 * s
-    u_bytes = wl.batch * wl.width * wl.points // wl.grid[-1] * wl.modes[-1] * 8
+    rows = wl.batch * wl.points // wl.grid[-1]       # (sample, grid row) pairs
+    img = rows * (2 if wl.dtype == "f32" else 1) * wl.width * 2 * wl.modes[-1] * s
     table = {
         "fwd_transform": act + spec,                 # read x, write spectrum
         "fwd_fft": act + spec,
-        "spec_mid": spec + r + u_bytes,              # read spectrum and R, write U
+        "fwd_plane": act + spec,
+        "fwd_plane_dz": 2 * act + spec,
+        "inv_slab_img": spec + img,                  # read yhat, write the B images
         "epi_block_fwd": 2 * act + spec,             # read x, write y, read spectrum
         "mix_fwd": 2 * spec + r,
         "lift": wl.batch * wl.in_ch * wl.points * s + act,
@@ -232,7 +235,8 @@ def kernel_source_sha(tag: str) -> str:
              "epi_block_bwd": "epilogue.cu", "proj_bwd": "net.cu",
              "fwd_transform_tc_dz": "transform_tc.cu", "fwd_transform_dz": "transform.cu",
              "fwd_fft": "transform_fft.cu", "fwd_fft_dz": "transform_fft.cu",
-             "spec_mid": "spec_mid.cu"}
+             "fwd_plane": "transform_plane.cu", "fwd_plane_dz": "transform_plane.cu",
+             "inv_slab_img": "spec_mid.cu", "inv_slab_fft": "spec_mid.cu"}
     path = os.path.join(ROOT, "fourier_neural_spectral_fno_b200", "csrc", files.get(tag, ""))
     if not os.path.isfile(path):
         return ""

@@ -10,13 +10,15 @@
 // stream through the SM, so HBM traffic, staging, MMAs and the GELU epilogue
 // of consecutive tiles overlap.
 //
-//   warp 13       TMA producer: x tile [Ci][128] and U rows [Co][Rt 2 mL] of
+//   warp 17       TMA producer: x tile [Ci][128] and U rows [Co][Rt 2 mL] of
 //                 tile j into ring stage j % NS (mbarrier transaction count)
-//   warps 0-3     staging: U -> B operand (smem, K-major core matrices,
+//   warps 0-7     staging: U -> B operand (smem, K-major core matrices,
 //                 tf32 hi/lo split, bias folded into the k = 0 column), x ->
-//                 A operand (TMEM, one lane per point); double-buffered
-//   warp 12       one thread issues the MMAs of tile j into D buffer j % 2
-//   warps 4-11    epilogue: D -> registers, bias already in, optional pre
+//                 A operand (TMEM, one lane per point); double-buffered; two
+//                 warps per TMEM lane quarter, each owning half of the x
+//                 channel groups and of the B chunks
+//   warp 16       one thread issues the MMAs of tile j into D buffer j % 2
+//   warps 8-15    epilogue: D -> registers, bias already in, optional pre
 //                 store, GELU, coalesced y stores; two warps per TMEM lane
 //                 quarter, each owning half of the channel groups
 //
@@ -38,10 +40,10 @@ namespace fno {
 namespace {
 
 constexpr int ROWS = 128;                  // points per tile = TMEM lanes
-constexpr int NCONV = 4;                   // staging warps
+constexpr int NCONV = 8;                   // staging warps (two per TMEM lane quarter)
 constexpr int NEPI = 8;                    // epilogue warps
-constexpr int WARP_MMA = NCONV + NEPI;     // 12
-constexpr int WARP_TMA = WARP_MMA + 1;     // 13
+constexpr int WARP_MMA = NCONV + NEPI;     // 16
+constexpr int WARP_TMA = WARP_MMA + 1;     // 17
 constexpr int THREADS = (WARP_TMA + 1) * 32;
 constexpr int MAX_STAGES = 6;
 constexpr size_t kSmemMax = 227 * 1024;
@@ -390,14 +392,17 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp < NCONV) {
     // ---------------------------------------------------------- staging
-    const int t = tid;                                  // point / TMEM lane
-    const uint32_t arow = tbase + ((uint32_t)(warp * 32) << 16);
+    // two warps per TMEM lane quarter: point t, and half `shalf` of the x
+    // channel groups and of the B chunks
+    const int t = tid & (ROWS - 1);                     // point / TMEM lane
+    const int shalf = tid / ROWS;
+    const uint32_t arow = tbase + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t lo_spec = K::tf32 ? (uint32_t)e.KSp : 0u;
     const uint32_t lo_x = K::tf32 ? (uint32_t)e.KXp : 0u;
     // resident spectral A block per variant: row t = point n0 + t (NL >= 128)
     // or point t of the Rt rows (NL < 128): (cos, -sin)(2 pi k n / NL) in the
     // slot of the point's row, zeros elsewhere
-    for (int v = 0; v < e.nvar; ++v) {
+    for (int v = 0; v < (shalf == 0 ? e.nvar : 0); ++v) {
       const int n = e.Rt > 1 ? t % NL : v * ROWS + t;
       const int rl = e.Rt > 1 ? t / NL : 0;
       const uint32_t c0v = arow + e.col_spec + v * e.cs_cols;
@@ -433,19 +438,20 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int nchunk = rup(Co, 8) * njb;
     const int two_ml = 2 * mL;
     // This thread's chunks of the B spectral block are the same for every
-    // tile: chunk i = t + 128 m.  Chunk order walks 8-row groups diagonally so a
+    // tile: chunk i = tid + 256 m.  Chunk order walks 8-row groups diagonally so a
     // quarter warp touches 8 distinct 16-byte bank groups on both the read and
     // the write side.  Packed per slot: source float index (low 16 bits), B byte
     // offset (high 16 bits); bias_mask bit m: add the bias (k = 0 real column).
-    constexpr int MAXSLOT = 8;
+    constexpr int MAXSLOT = 4;
+    constexpr int NSTG = NCONV * 32;
     uint32_t slot[MAXSLOT];
     float slot_bias[MAXSLOT];
-    const bool slots_fit = nchunk <= MAXSLOT * ROWS && e.bhalf <= 65536;
+    const bool slots_fit = nchunk <= MAXSLOT * NSTG && e.bhalf <= 65536;
 #pragma unroll
     for (int m = 0; m < MAXSLOT; ++m) {
       slot[m] = 0xffffffffu;
       slot_bias[m] = 0.f;
-      const int i = t + ROWS * m;
+      const int i = tid + NSTG * m;
       if (slots_fit && i < nchunk) {
         const int o8 = i / (8 * njb), rem = i - o8 * 8 * njb;
         const int ol = rem & 7, jrot = rem >> 3;
@@ -486,7 +492,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       } else {
         const float *us = reinterpret_cast<const float *>(st + e.uoff);
         unsigned char *bh = bbase + ab * e.bbuf;
-        for (int i = t; i < nchunk; i += ROWS) {
+        for (int i = tid; i < nchunk; i += NSTG) {
           const int o8 = i / (8 * njb), rem = i - o8 * 8 * njb;
           const int ol = rem & 7, jrot = rem >> 3;
           const int jb = (jrot + ol) % njb;
@@ -503,7 +509,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t xc = arow + e.col_x + ab * e.ax_cols;
 #pragma unroll
         for (int c0 = 0; c0 < CX; c0 += 16) {
-          if (c0 < e.KXp) {
+          if (c0 < e.KXp && ((c0 >> 4) & 1) == shalf) {
             float vals[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)

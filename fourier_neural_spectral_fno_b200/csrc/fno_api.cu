@@ -117,7 +117,7 @@ int check_block(const fno_block_desc *d, Geom *g) {
 
 // Workspace map of a block operation.
 struct BlockWs {
-  size_t zpart, xhat, yhat, zexp, tw, u, img, dxhat, partial, total;
+  size_t zpart, xhat, yhat, zexp, u, img, dxhat, partial, total;
 };
 
 BlockWs block_ws(const Geom &g, int Ci, int Co, int op) {
@@ -136,8 +136,6 @@ BlockWs block_ws(const Geom &g, int Ci, int Co, int op) {
   off += al(cplx * (size_t)(g.B * Cmax * g.K));
   w.zexp = off;
   off += al(inv_expand_bytes(g, Cmax));
-  w.tw = off;                         // slab-axis twiddles of the 2D spectral middle
-  off += al(spec_mid_table_bytes(g));
   w.u = off;                          // spectrum inverted along the slab axis
   off += al(inv_slab_bytes(g, Cmax));
   w.img = off;                        // or, per grid row, the epilogue's B operand image
@@ -287,7 +285,6 @@ int run_forward(const Launch &L, const Geom &g, int dtype, unsigned flags, int C
     FNO_TRY(launch_mix_cp(L, g, dtype, Ci, Co, rank, xhat, *cp, yhat), "factorised mixing");
   else if (mid)
     FNO_TRY(launch_spec_mid(L, g, dtype, Ci, Co, xhat, R, yhat,
-                            reinterpret_cast<float2 *>(ws + w.tw),
                             reinterpret_cast<float2 *>(ws + w.u), img ? ws + w.img : nullptr,
                             epi_mode == EPI_BLOCK_FWD ? b : nullptr),
             "mixing and slab-axis inverse");

@@ -89,23 +89,21 @@ bool fwd_plane_supported(const Geom &g, int dtype, const void *in0, const void *
 cudaError_t launch_fwd_plane(const Launch &L, const Geom &g, int dtype, int load_mode, long long C,
                              const void *in0, const void *in1, float2 *out);
 
-// 2D spectral middle (spec_mid.cu): mixing into yhat (as launch_mix_fwd),
-// then the slab-axis inverse as a pruned FFT into
-// U[b][o][S][mL] = sum_q yhat[b,o,q,k] exp(+2 pi i kq n / S); two launches
+// 2D spectral middle (spec_mid.cu): mixing into yhat (launch_mix_fwd), then
+// the slab-axis inverse as a pruned FFT into
+// U[b][o][S][mL] = sum_q yhat[b,o,q,k] exp(+2 pi i kq n / S); two launches.
+// img (optional): write the epilogue's B images (epi_img_supported and
+// spec_mid_img_supported) instead of U, with bias (may be NULL) folded in
+bool spec_mid_supported(const Geom &g, int Ci, int Co);
+bool spec_mid_img_supported(const Geom &g, int Co);
+cudaError_t launch_spec_mid(const Launch &L, const Geom &g, int dtype, int Ci, int Co,
+                            const float2 *xhat, const void *R, float2 *yhat, float2 *U,
+                            unsigned char *img, const void *bias);
 // the pruned slab-axis inverse alone (the backward's dxhat), same output as
 // launch_inv_slab: U[b][c][S][mL]
 bool inv_slab_fft_supported(const Geom &g);
 cudaError_t launch_inv_slab_fft(const Launch &L, const Geom &g, long long C, const float2 *Z,
                                 float2 *U);
-// twr: workspace for the slab-axis twiddle table (spec_mid_table_bytes)
-bool spec_mid_supported(const Geom &g, int Ci, int Co);
-bool spec_mid_img_supported(const Geom &g, int Co);   // the image-writing inverse fits
-size_t spec_mid_table_bytes(const Geom &g);
-// img (optional): write the epilogue's B images (epi_img_supported) instead of
-// U, with bias (may be NULL) folded in
-cudaError_t launch_spec_mid(const Launch &L, const Geom &g, int dtype, int Ci, int Co,
-                            const float2 *xhat, const void *R, float2 *yhat, float2 *twr,
-                            float2 *U, unsigned char *img, const void *bias);
 
 // CP-factorised weights (mix_cp.cu): R[i,o,k] = sum_r lam[r] A[i,r] B[o,r] C[k,r],
 // factors complex (re, im) in the storage dtype: lam [rank], A [Ci][rank],

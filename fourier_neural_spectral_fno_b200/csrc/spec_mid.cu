@@ -1,22 +1,21 @@
-// The block's spectral middle for 2D grids: per-mode channel mixing (step S3)
-// and the inverse transform along the slab axis (the first half of S4), as
-// two launches that each read their inputs from HBM or L2 once.
+// The block's spectral middle for 2D grids: after the per-mode mixing (step
+// S3, k_mix_fwd in mix.cu), the inverse transform along the slab axis (the
+// first half of S4) as a pruned radix-16 FFT,
 //
-//   yhat[b,o,q,k] = (c_k / N) sum_i xhat[b,i,q,k] R[i,o,q,k]      (k_mix_modes)
-//   U[b,o,n,k]    = sum_q yhat[b,o,q,k] exp(+2 pi i kq(q) n / S)    (k_inv_slab_fft)
+//   U[b,o,n,k] = sum_q yhat[b,o,q,k] exp(+2 pi i kq(q) n / S).
 //
-// k_mix_modes: a CTA owns a group of consecutive modes and four samples; it
-// stages their xhat and every weight of those modes in shared memory (eight
-// loads in flight per thread), then forms all (b, o) products from there.
-//
-// k_inv_slab_fft: a CTA owns one (b, o) slab.  The inverse is a pruned
-// radix-16 FFT: with S = 16 Q and n = Q a + r,
+// With S = 16 Q and n = Q a + r,
 //   U[Q a + r] = sum_p exp(+2 pi i p a / 16) V_r[p],
 //   V_r[p]     = sum_{kq = p (mod 16)} yhat[kq] exp(+2 pi i kq r / S),
 // i.e. the kept wavenumbers (signed, in [-mS, mS)) are folded by residue into
 // sixteen bins of at most four, then one register FFT16 per (r, k) expands
-// them to sixteen grid rows; consecutive threads take consecutive k, so every
-// row of U is written by one coalesced store.
+// them to sixteen grid rows.
+//
+// k_inv_slab_fft writes U (one CTA per (b, o) slab, consecutive threads on
+// consecutive k, so every row of U leaves as one coalesced store);
+// k_inv_slab_img writes, per (sample, grid row), the spectral half of the
+// pipelined epilogue's tcgen05 B operand directly in its shared-memory layout,
+// so the epilogue fetches it with one bulk copy and builds nothing.
 #include "fft16.cuh"
 #include "fno_common.cuh"
 #include "fno_kernels.cuh"
@@ -25,19 +24,8 @@ namespace fno {
 
 namespace {
 
-constexpr int MM_THREADS = 256;
-constexpr int MM_BS = 4;                        // samples per CTA
-constexpr size_t MM_R_STAGE = 64 * 1024;        // staged weights per CTA
 constexpr int IS_THREADS = 256;
 constexpr int SM_MAXQS = 64;
-
-// modes per CTA: 4 (whole 32-byte sectors of the mode-contiguous rows) unless
-// the staged weights would exceed MM_R_STAGE
-int mix_modes_group(int Ci, int Co) {
-  int mg = 4;
-  while (mg > 1 && sizeof(float2) * (size_t)Ci * Co * mg > MM_R_STAGE) mg /= 2;
-  return sizeof(float2) * (size_t)Ci * Co * mg > MM_R_STAGE ? 0 : mg;
-}
 
 // hi = x rounded to tf32 (nearest), lo = x - hi rounded to tf32: the
 // operand split of the float32 tensor-core path
@@ -50,86 +38,6 @@ __device__ __forceinline__ void tc_split(float x, uint32_t &hi, uint32_t &lo) {
   lo = l;
 }
 
-// global load of 8 values per thread before any is stored: the staging keeps
-// eight loads in flight instead of one
-template <typename F>
-__device__ __forceinline__ void stage8(float2 *dst, int n, F load) {
-  for (int base = threadIdx.x; base < n; base += 8 * MM_THREADS) {
-    float2 v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int e = base + u * MM_THREADS;
-      v[u] = e < n ? load(e) : make_float2(0.f, 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int e = base + u * MM_THREADS;
-      if (e < n) dst[e] = v[u];
-    }
-  }
-}
-
-template <typename T, int MG>
-__global__ void __launch_bounds__(MM_THREADS)
-    k_mix_modes(const float2 *__restrict__ xhat, const T *__restrict__ R, float2 *__restrict__ yhat,
-                float2 *__restrict__ twr, int B, int Ci, int Co, int K, int mL, int NL,
-                float inv_n, int S, int mS, int QS) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  float2 *xs = reinterpret_cast<float2 *>(smem);     // [MM_BS][Ci][MG]
-  float2 *rs = xs + (size_t)MM_BS * Ci * MG;         // [Ci][Co][MG]
-  const int m0 = blockIdx.x * MG, b0 = blockIdx.y * MM_BS;
-  const int mg = min(MG, K - m0), nb = min(MM_BS, B - b0);
-  const int tid = threadIdx.x;
-  if (blockIdx.x == 0 && blockIdx.y == 0) {
-    // the slab-axis inverse's twiddles exp(+2 pi i kq(slot) r / S), [slot][S/16]
-    const int Qp = S / 16;
-    for (int e = tid; e < QS * Qp; e += MM_THREADS) {
-      const int slot = e / Qp, r = e - slot * Qp;
-      float sn, cs;
-      sincospif(2.0f * (float)mulmod(kept_k(slot, mS, S), r, S) / (float)S, &sn, &cs);
-      twr[e] = make_float2(cs, sn);
-    }
-  }
-  const float2 *xsrc = xhat + (size_t)b0 * Ci * K + m0;
-  stage8(xs, nb * Ci * MG, [&](int e) {
-    const int row = e / MG, m = e % MG;                  // MG is a power of two
-    return m < mg ? __ldg(xsrc + (size_t)row * K + m) : make_float2(0.f, 0.f);
-  });
-  const T *rsrc = R + 2 * (size_t)m0;
-  stage8(rs, Ci * Co * MG, [&](int e) {
-    const int row = e / MG, m = e % MG;
-    return m < mg ? ldc<T>(rsrc + 2 * ((size_t)row * K + m)) : make_float2(0.f, 0.f);
-  });
-  __syncthreads();
-  // output (b, o, m), m fastest: the weight reads of a warp are contiguous;
-  // the (b, o) pair advances by a constant stride per thread
-  const int m = tid % MG;
-  const int bo_step = MM_THREADS / MG;
-  const float w = m < mg ? mode_weight((m0 + m) % mL, NL, inv_n) : 0.f;
-  int b = 0, o = tid / MG;
-  while (o >= Co) { o -= Co; ++b; }
-  const int db = bo_step / Co, dob = bo_step % Co;
-  const int rstep = Co * MG;
-  for (; b < nb;) {
-    const float2 *xp = xs + b * Ci * MG + m;
-    const float2 *rp = rs + o * MG + m;
-    float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
-    int i = 0;
-#pragma unroll 4
-    for (; i + 1 < Ci; i += 2) {
-      cfma(s0, xp[i * MG], rp[i * rstep]);
-      cfma(s1, xp[(i + 1) * MG], rp[(i + 1) * rstep]);
-    }
-    if (i < Ci) cfma(s0, xp[i * MG], rp[i * rstep]);
-    if (m < mg)
-      yhat[((size_t)(b0 + b) * Co + o) * K + m0 + m] =
-          make_float2(w * (s0.x + s1.x), w * (s0.y + s1.y));
-    b += db;
-    o += dob;
-    if (o >= Co) { o -= Co; ++b; }
-  }
-}
-
 // byte offset of B-operand element (row n, column c) in a K-major no-swizzle
 // image of `sbo`-byte 8-row groups (the tcgen05 core-matrix layout)
 __device__ __forceinline__ uint32_t img_off(int n, int c, int eb, uint32_t sbo) {
@@ -140,12 +48,11 @@ __device__ __forceinline__ uint32_t img_off(int n, int c, int eb, uint32_t sbo) 
 
 // NDM: the kept wavenumbers of residue p (mod 16) are among p + 16 d,
 // d in [-NDM, NDM) (NDM = 1 for mS <= 16, 2 for mS <= 32); FULL: mS = 16 NDM,
-// so every candidate is kept and no test is needed.  twr_g: the twiddle table
-// of the mixing kernel, or NULL to build it here.
+// so every candidate is kept and no test is needed.
 template <int NDM, bool FULL>
 __global__ void __launch_bounds__(IS_THREADS)
-    k_inv_slab_fft(const float2 *__restrict__ yhat, const float2 *__restrict__ twr_g,
-                   float2 *__restrict__ U, int S, int mS, int QS, int mL) {
+    k_inv_slab_fft(const float2 *__restrict__ yhat, float2 *__restrict__ U, int S, int mS,
+                   int QS, int mL) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int Qp = S / 16;
   float2 *ys = reinterpret_cast<float2 *>(smem);      // [QS][mL]
@@ -154,15 +61,11 @@ __global__ void __launch_bounds__(IS_THREADS)
   const int tid = threadIdx.x;
   const float2 *src = yhat + slab * QS * mL;
   for (int e = tid; e < QS * mL; e += IS_THREADS) ys[e] = __ldg(src + e);
-  if (twr_g) {
-    for (int e = tid; e < QS * Qp; e += IS_THREADS) twr[e] = __ldg(twr_g + e);
-  } else {   // no table from the mixing kernel: build it here
-    for (int e = tid; e < QS * Qp; e += IS_THREADS) {
-      const int slot = e / Qp, rr = e - slot * Qp;
-      float sn, cs;
-      sincospif(2.0f * (float)mulmod(kept_k(slot, mS, S), rr, S) / (float)S, &sn, &cs);
-      twr[e] = make_float2(cs, sn);
-    }
+  for (int e = tid; e < QS * Qp; e += IS_THREADS) {   // exp(+2 pi i kq(slot) r / S)
+    const int slot = e / Qp, rr = e - slot * Qp;
+    float sn, cs;
+    sincospif(2.0f * (float)mulmod(kept_k(slot, mS, S), rr, S) / (float)S, &sn, &cs);
+    twr[e] = make_float2(cs, sn);
   }
   __syncthreads();
   float2 *dst = U + slab * (size_t)S * mL;
@@ -204,8 +107,7 @@ __global__ void __launch_bounds__(IS_THREADS)
 constexpr int IMG_RSPLIT = 4;
 template <int NDM, bool FULL, int IMG, typename TB>
 __global__ void __launch_bounds__(IS_THREADS)
-    k_inv_slab_img(const float2 *__restrict__ yhat, const float2 *__restrict__ twr_g,
-                   unsigned char *__restrict__ img, const TB *__restrict__ bias, int S, int mS,
+    k_inv_slab_img(const float2 *__restrict__ yhat, unsigned char *__restrict__ img, const TB *__restrict__ bias, int S, int mS,
                    int QS, int mL, int Co) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int Qp = S / 16;
@@ -218,7 +120,12 @@ __global__ void __launch_bounds__(IS_THREADS)
     const int oo = e / (QS * mL), sk = e - oo * (QS * mL);
     ys[sk * 8 + oo] = __ldg(yhat + ((size_t)b * Co + o0 + oo) * QS * mL + sk);
   }
-  for (int e = tid; e < QS * Qp; e += IS_THREADS) twr[e] = __ldg(twr_g + e);
+  for (int e = tid; e < QS * Qp; e += IS_THREADS) {
+    const int slot = e / Qp, rr = e - slot * Qp;
+    float sn, cs;
+    sincospif(2.0f * (float)mulmod(kept_k(slot, mS, S), rr, S) / (float)S, &sn, &cs);
+    twr[e] = make_float2(cs, sn);
+  }
   __syncthreads();
   constexpr int EB = IMG == 1 ? 4 : 2;
   const uint32_t sbo = (uint32_t)(2 * mL * EB / 16) * 128u;
@@ -286,7 +193,7 @@ cudaError_t launch_inv_slab_fft(const Launch &L, const Geom &g, long long C, con
     cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           (int)smem2);
     if (e2 != cudaSuccess) return e2;
-    kern<<<slabs, IS_THREADS, smem2, L.stream>>>(Z, nullptr, U, g.S, g.mS, g.QS, g.mL);
+    kern<<<slabs, IS_THREADS, smem2, L.stream>>>(Z, U, g.S, g.mS, g.QS, g.mL);
     return cudaGetLastError();
   };
   cudaError_t e;
@@ -304,51 +211,21 @@ bool spec_mid_img_supported(const Geom &g, int Co) {
   return smem <= 200 * 1024;
 }
 
-size_t spec_mid_table_bytes(const Geom &g) {
-  return g.d == 2 ? sizeof(float2) * (size_t)g.QS * (g.S / 16) : 0;
-}
-
 bool spec_mid_supported(const Geom &g, int Ci, int Co) {
   if (g.d != 2 || g.QO != 1) return false;
   if (g.S % 16 != 0 || g.QS > SM_MAXQS) return false;
   if (g.B * (long long)g.K * kMaxWidth > (1LL << 31)) return false;
-  if (mix_modes_group(Ci, Co) < 1) return false;
-  if ((g.B + MM_BS - 1) / MM_BS > 65535) return false;
+  (void)Ci;
+  (void)Co;
   const size_t inv = sizeof(float2) * ((size_t)g.QS * g.mL + (size_t)g.QS * (g.S / 16));
   return inv <= 200 * 1024;
 }
 
 cudaError_t launch_spec_mid(const Launch &L, const Geom &g, int dtype, int Ci, int Co,
-                            const float2 *xhat, const void *R, float2 *yhat, float2 *twr,
-                            float2 *U, unsigned char *img, const void *bias) {
-  const int mg = mix_modes_group(Ci, Co);
-  const size_t smem = sizeof(float2) * ((size_t)MM_BS * Ci + (size_t)Ci * Co) * mg;
-  dim3 grid((unsigned)((g.K + mg - 1) / mg), (unsigned)((g.B + MM_BS - 1) / MM_BS));
-  launch_begin(L);
-  auto go = [&](auto kern, const auto *r) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    kern<<<grid, MM_THREADS, smem, L.stream>>>(xhat, r, yhat, twr, (int)g.B, Ci, Co, (int)g.K,
-                                               g.mL, g.NL, g.inv_n, g.S, g.mS, g.QS);
-    return cudaGetLastError();
-  };
-  auto by_mg = [&](auto k4, auto k2, auto k1, const auto *r) {
-    return mg == 4 ? go(k4, r) : mg == 2 ? go(k2, r) : go(k1, r);
-  };
-  cudaError_t e;
-  if (dtype == DT_F32)
-    e = by_mg(k_mix_modes<float, 4>, k_mix_modes<float, 2>, k_mix_modes<float, 1>,
-              (const float *)R);
-  else if (dtype == DT_F16)
-    e = by_mg(k_mix_modes<__half, 4>, k_mix_modes<__half, 2>, k_mix_modes<__half, 1>,
-              (const __half *)R);
-  else
-    e = by_mg(k_mix_modes<__nv_bfloat16, 4>, k_mix_modes<__nv_bfloat16, 2>,
-              k_mix_modes<__nv_bfloat16, 1>, (const __nv_bfloat16 *)R);
-  launch_end(L, "mix_modes");
+                            const float2 *xhat, const void *R, float2 *yhat, float2 *U,
+                            unsigned char *img, const void *bias) {
+  cudaError_t e = launch_mix_fwd(L, g, dtype, Ci, Co, xhat, R, yhat);
   if (e != cudaSuccess) return e;
-
   launch_begin(L);
   if (!img) {
     const size_t smem2 = sizeof(float2) * ((size_t)g.QS * g.mL + (size_t)g.QS * (g.S / 16));
@@ -357,7 +234,7 @@ cudaError_t launch_spec_mid(const Launch &L, const Geom &g, int dtype, int Ci, i
       cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             (int)smem2);
       if (e2 != cudaSuccess) return e2;
-      kern<<<slabs, IS_THREADS, smem2, L.stream>>>(yhat, twr, U, g.S, g.mS, g.QS, g.mL);
+      kern<<<slabs, IS_THREADS, smem2, L.stream>>>(yhat, U, g.S, g.mS, g.QS, g.mL);
       return cudaGetLastError();
     };
     if (g.mS == 16) e = go2(k_inv_slab_fft<1, true>);
@@ -372,7 +249,7 @@ cudaError_t launch_spec_mid(const Launch &L, const Geom &g, int dtype, int Ci, i
       cudaError_t e3 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             (int)smem3);
       if (e3 != cudaSuccess) return e3;
-      kern<<<grid3, IS_THREADS, smem3, L.stream>>>(yhat, twr, img, bp, g.S, g.mS, g.QS, g.mL, Co);
+      kern<<<grid3, IS_THREADS, smem3, L.stream>>>(yhat, img, bp, g.S, g.mS, g.QS, g.mL, Co);
       return cudaGetLastError();
     };
     auto by_out = [&](auto k1, auto k2, auto k3) {
