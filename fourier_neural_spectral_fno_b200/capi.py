@@ -34,6 +34,7 @@ FNO_NO_ACT = 2
 
 FNO_OP_SPECTRAL_FWD, FNO_OP_SPECTRAL_BWD, FNO_OP_BLOCK_FWD, FNO_OP_BLOCK_BWD = 0, 1, 2, 3
 FNO_OP_NET_FWD, FNO_OP_NET_BWD = 4, 5
+FNO_OP_SPECTRAL_BWD_CP, FNO_OP_BLOCK_BWD_CP = 6, 7
 
 FNO_MAX_DIMS = 3
 FNO_MAX_LAYERS = 16
@@ -46,6 +47,7 @@ EXPORTED = (
     "fno_mse", "fno_profile_enable", "fno_profile_read", "fno_set_tensor_cores",
     "fno_device_error", "fno_spectral_conv_fwd_noalloc", "fno_adam_step",
     "fno_backward_ready", "fno_spectral_conv_fwd_cp", "fno_block_fwd_cp", "fno_set_wait_limit",
+    "fno_spectral_conv_bwd_cp", "fno_block_bwd_cp",
 )
 
 FNO_MAX_CP_RANK = 32
@@ -131,6 +133,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "fno_spectral_conv_fwd_noalloc": (i, [bd, vp, vp, vp, vp, vp]),
         "fno_spectral_conv_fwd_cp": (i, [bd, i, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "fno_block_fwd_cp": (i, [bd, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "fno_spectral_conv_bwd_cp": (i, [bd, i] + [vp] * 13 + [sz, vp]),
+        "fno_block_bwd_cp": (i, [bd, i] + [vp] * 17 + [sz, vp]),
         "fno_device_error": (i, [i]),
         "fno_set_wait_limit": (i, [i]),
         "fno_profile_read": (i, [ctypes.POINTER(KernelStat), i]),
@@ -286,6 +290,28 @@ def fno_block_fwd_cp(desc, rank, x, lam, A, B, C, W, b, y, pre_save=None, xhat_s
                                    _ptr(B), _ptr(C), _ptr(W), _ptr(b), _ptr(y), _ptr(pre_save),
                                    _ptr(xhat_save), _ptr(ws), nb, _stream(stream)))
     return y
+
+
+def fno_spectral_conv_bwd_cp(desc, rank, x, lam, A, B, C, xhat_save, dy, dx, dlam, dA, dB, dC,
+                             ws=None, stream=None):
+    """Adjoint of :func:`fno_spectral_conv_fwd_cp`: dx and the factor gradients."""
+    ws, nb = _workspace(fno_workspace_size(desc, FNO_OP_SPECTRAL_BWD_CP), x.device, ws)
+    _check(load().fno_spectral_conv_bwd_cp(ctypes.byref(desc), int(rank), _ptr(x), _ptr(lam),
+                                           _ptr(A), _ptr(B), _ptr(C), _ptr(xhat_save), _ptr(dy),
+                                           _ptr(dx), _ptr(dlam), _ptr(dA), _ptr(dB), _ptr(dC),
+                                           _ptr(ws), nb, _stream(stream)))
+    return dx, dlam, dA, dB, dC
+
+
+def fno_block_bwd_cp(desc, rank, x, lam, A, B, C, W, pre_save, xhat_save, dy, dx, dlam, dA, dB,
+                     dC, dW, db, ws=None, stream=None):
+    """Adjoint of :func:`fno_block_fwd_cp`: dx, the factor gradients, dW and db."""
+    ws, nb = _workspace(fno_workspace_size(desc, FNO_OP_BLOCK_BWD_CP), x.device, ws)
+    _check(load().fno_block_bwd_cp(ctypes.byref(desc), int(rank), _ptr(x), _ptr(lam), _ptr(A),
+                                   _ptr(B), _ptr(C), _ptr(W), _ptr(pre_save), _ptr(xhat_save),
+                                   _ptr(dy), _ptr(dx), _ptr(dlam), _ptr(dA), _ptr(dB), _ptr(dC),
+                                   _ptr(dW), _ptr(db), _ptr(ws), nb, _stream(stream)))
+    return dx, dlam, dA, dB, dC, dW, db
 
 
 def fno_block_bwd(desc, x, R, W, pre_save, xhat_save, dy, dx, dR, dW, db, ws=None, stream=None):

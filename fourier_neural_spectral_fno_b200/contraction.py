@@ -18,8 +18,8 @@ page gives neither the factorisation nor the greedy rule; the readings are
   alone is myopic: it multiplies the small CP factors together first and so
   rebuilds the dense weight.)
 
-Host logic only.  A plan is a list of pairwise steps; executing them is the
-caller's business (the GPU path for factorised weights is not built yet).
+Host logic only.  A plan is a list of pairwise steps; the GPU mixing kernel for
+factorised weights contracts in the order this plan gives at low rank.
 """
 
 from __future__ import annotations

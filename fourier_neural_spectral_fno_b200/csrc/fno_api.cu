@@ -117,7 +117,7 @@ int check_block(const fno_block_desc *d, Geom *g) {
 
 // Workspace map of a block operation.
 struct BlockWs {
-  size_t zpart, xhat, yhat, zexp, u, img, dxhat, partial, total;
+  size_t zpart, xhat, yhat, zexp, u, img, dxhat, partial, rcp, drcp, cps, total;
 };
 
 BlockWs block_ws(const Geom &g, int Ci, int Co, int op) {
@@ -143,10 +143,22 @@ BlockWs block_ws(const Geom &g, int Ci, int Co, int op) {
     off += al(g.d == 2 ? (size_t)g.B * g.S * epi_img_row_bytes(DT_F32, Co, g.mL) : 0);
   w.dxhat = off;
   w.partial = off;
-  if (op == FNO_OP_SPECTRAL_BWD || op == FNO_OP_BLOCK_BWD) {
+  const bool cp = op == FNO_OP_SPECTRAL_BWD_CP || op == FNO_OP_BLOCK_BWD_CP;
+  const bool bwd = op == FNO_OP_SPECTRAL_BWD || op == FNO_OP_BLOCK_BWD || cp;
+  const bool block_bwd = op == FNO_OP_BLOCK_BWD || op == FNO_OP_BLOCK_BWD_CP;
+  if (bwd) {
     off += al(cplx * (size_t)(g.B * Ci * g.K));
     w.partial = off;
-    if (op == FNO_OP_BLOCK_BWD) off += al(sizeof(float) * (size_t)kPartialCTAs * Co * (Ci + 1));
+    if (block_bwd) off += al(sizeof(float) * (size_t)kPartialCTAs * Co * (Ci + 1));
+  }
+  w.rcp = w.drcp = w.cps = off;
+  if (cp) {   // the rebuilt weight (float32-sized), its gradient, the projection scratch
+    w.rcp = off;
+    off += al(sizeof(float2) * (size_t)Ci * Co * g.K);
+    w.drcp = off;
+    off += al(sizeof(float2) * (size_t)Ci * Co * g.K);
+    w.cps = off;
+    off += al(sizeof(float2) * (size_t)Ci * kMaxCpRank);
   }
   w.total = off;
   return w;
@@ -312,11 +324,14 @@ int run_forward(const Launch &L, const Geom &g, int dtype, unsigned flags, int C
   return FNO_OK;
 }
 
+// ws_op: the operation whose workspace map `ws` follows (the dense op, or its
+// factorised variant, whose map extends it)
 int run_backward(const Launch &L, const Geom &g, int dtype, unsigned flags, int Ci, int Co,
                  const void *x, const float *xhat_save, const void *R, const void *W,
                  const void *pre, const void *dy, void *dx, float *dR, float *dW, float *db,
-                 unsigned char *ws, bool block) {
-  const BlockWs w = block_ws(g, Ci, Co, block ? FNO_OP_BLOCK_BWD : FNO_OP_SPECTRAL_BWD);
+                 unsigned char *ws, bool block, int ws_op = -1) {
+  const BlockWs w = block_ws(g, Ci, Co,
+                             ws_op >= 0 ? ws_op : block ? FNO_OP_BLOCK_BWD : FNO_OP_SPECTRAL_BWD);
   float2 *zpart = reinterpret_cast<float2 *>(ws + w.zpart);
   const float2 *xhat = reinterpret_cast<const float2 *>(xhat_save);
   if (!xhat) {
@@ -564,7 +579,8 @@ int fno_profile_read(fno_kernel_stat *out, int max) {
 size_t fno_workspace_size(const fno_block_desc *desc, int op) {
   Geom g;
   if (check_block(desc, &g)) return 0;
-  if (op < FNO_OP_SPECTRAL_FWD || op > FNO_OP_BLOCK_BWD) {
+  if (op < FNO_OP_SPECTRAL_FWD || op > FNO_OP_BLOCK_BWD_CP || op == FNO_OP_NET_FWD ||
+      op == FNO_OP_NET_BWD) {
     fail(FNO_ERR_INVALID_ARG, "op %d is not a block op", op);
     return 0;
   }
@@ -718,6 +734,70 @@ int fno_block_fwd_cp(const fno_block_desc *desc, int rank, const void *x, const 
                    pre_save, xhat_save, (unsigned char *)ws, EPI_BLOCK_FWD, &f, rank);
   if (!rc) g_err[0] = 0;
   return rc;
+}
+
+static int bwd_cp(const fno_block_desc *desc, int rank, const void *x, const void *lam,
+                  const void *A, const void *B, const void *C, const void *W, const void *pre_save,
+                  const float *xhat_save, const void *dy, void *dx, float *dlam, float *dA,
+                  float *dB, float *dC, float *dW, float *db, void *ws, size_t ws_bytes,
+                  fno_stream_t stream, bool block) {
+  Geom g;
+  int rc = check_block(desc, &g);
+  if (rc) return rc;
+  const int op = block ? FNO_OP_BLOCK_BWD_CP : FNO_OP_SPECTRAL_BWD_CP;
+  if ((rc = check_smem(g, desc->cin, desc->cout, block ? FNO_OP_BLOCK_BWD : FNO_OP_SPECTRAL_BWD)))
+    return rc;
+  if ((rc = check_cp(desc, g, rank, lam, A, B, C))) return rc;
+  REQUIRE_PTR(x, "x");
+  REQUIRE_PTR(dy, "dy");
+  REQUIRE_PTR(dx, "dx");
+  REQUIRE_PTR(dlam, "dlam");
+  REQUIRE_PTR(dA, "dA");
+  REQUIRE_PTR(dB, "dB");
+  REQUIRE_PTR(dC, "dC");
+  OPTIONAL_PTR(xhat_save, "xhat_save");
+  if (block) {
+    REQUIRE_PTR(W, "W");
+    if (!(desc->flags & FNO_NO_ACT)) REQUIRE_PTR(pre_save, "pre_save");
+    REQUIRE_PTR(dW, "dW");
+    REQUIRE_PTR(db, "db");
+  }
+  const BlockWs w = block_ws(g, desc->cin, desc->cout, op);
+  if (ws_bytes < w.total) return fail(FNO_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, w.total);
+  REQUIRE_PTR(ws, "ws");
+  Launch L = make_launch(stream);
+  unsigned char *wsb = (unsigned char *)ws;
+  const CpFactors f{lam, A, B, C};
+  void *R = wsb + w.rcp;
+  float *dR = reinterpret_cast<float *>(wsb + w.drcp);
+  FNO_TRY(launch_cp_rebuild(L, g, desc->dtype, desc->cin, desc->cout, rank, f, R),
+          "factorised weight rebuild");
+  rc = run_backward(L, g, desc->dtype, desc->flags, desc->cin, desc->cout, x, xhat_save, R, W,
+                    pre_save, dy, dx, dR, dW, db, wsb, block, op);
+  if (rc) return rc;
+  FNO_TRY(launch_cp_grads(L, g, desc->dtype, desc->cin, desc->cout, rank, f, dR,
+                          reinterpret_cast<float *>(wsb + w.cps), dlam, dA, dB, dC),
+          "factor gradients");
+  g_err[0] = 0;
+  return FNO_OK;
+}
+
+int fno_spectral_conv_bwd_cp(const fno_block_desc *desc, int rank, const void *x,
+                             const void *lam, const void *A, const void *B, const void *C,
+                             const float *xhat_save, const void *dy, void *dx, float *dlam,
+                             float *dA, float *dB, float *dC, void *ws, size_t ws_bytes,
+                             fno_stream_t stream) {
+  return bwd_cp(desc, rank, x, lam, A, B, C, nullptr, nullptr, xhat_save, dy, dx, dlam, dA, dB,
+                dC, nullptr, nullptr, ws, ws_bytes, stream, false);
+}
+
+int fno_block_bwd_cp(const fno_block_desc *desc, int rank, const void *x, const void *lam,
+                     const void *A, const void *B, const void *C, const void *W,
+                     const void *pre_save, const float *xhat_save, const void *dy, void *dx,
+                     float *dlam, float *dA, float *dB, float *dC, float *dW, float *db, void *ws,
+                     size_t ws_bytes, fno_stream_t stream) {
+  return bwd_cp(desc, rank, x, lam, A, B, C, W, pre_save, xhat_save, dy, dx, dlam, dA, dB, dC, dW,
+                db, ws, ws_bytes, stream, true);
 }
 
 int fno_block_bwd(const fno_block_desc *desc, const void *x, const void *R, const void *W,

@@ -114,6 +114,16 @@ struct CpFactors {
 };
 cudaError_t launch_mix_cp(const Launch &L, const Geom &g, int dtype, int Ci, int Co, int rank,
                           const float2 *xhat, const CpFactors &f, float2 *yhat);
+// backward through the factors: the dense weight rebuilt in the storage dtype
+// (R [Ci][Co][K][2]) for the dense backward, then from its gradient dR
+// (float32 [Ci][Co][K][2]) the factor gradients (float32, (re, im)):
+// dlam [rank], dA [Ci][rank], dB [Co][rank], dC [K][rank]; scratch: Ci rank
+// complex floats
+cudaError_t launch_cp_rebuild(const Launch &L, const Geom &g, int dtype, int Ci, int Co, int rank,
+                              const CpFactors &f, void *R);
+cudaError_t launch_cp_grads(const Launch &L, const Geom &g, int dtype, int Ci, int Co, int rank,
+                            const CpFactors &f, const float *dR, float *scratch, float *dlam,
+                            float *dA, float *dB, float *dC);
 
 // ---- mixing (S3) -----------------------------------------------------------
 // yhat[b,o,k] = (c_k / N) sum_i xhat[b,i,k] R[i,o,k]

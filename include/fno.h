@@ -86,7 +86,9 @@ enum fno_op {
   FNO_OP_BLOCK_FWD = 2,
   FNO_OP_BLOCK_BWD = 3,
   FNO_OP_NET_FWD = 4,
-  FNO_OP_NET_BWD = 5
+  FNO_OP_NET_BWD = 5,
+  FNO_OP_SPECTRAL_BWD_CP = 6, /* fno_spectral_conv_bwd_cp */
+  FNO_OP_BLOCK_BWD_CP = 7     /* fno_block_bwd_cp */
 };
 
 #define FNO_MAX_DIMS 3
@@ -258,6 +260,28 @@ int fno_block_fwd_cp(const fno_block_desc *desc, int rank, const void *x, const 
                      const void *A, const void *B, const void *C, const void *W, const void *b,
                      void *y, void *pre_save, float *xhat_save, void *ws, size_t ws_bytes,
                      fno_stream_t stream);
+
+/* Adjoints of the factorised forwards.  The gradient of the dense weight,
+ * dR = sum_b conj(xhat) (c_k/N) DFT_K(dz), is formed as in the dense backward
+ * (on the weight rebuilt from the factors in the storage dtype), then projected
+ * onto the factors by the chain rule (the weight is holomorphic in each factor,
+ * so dz = sum dR conj(dR/dz) under the convention dz = dL/dRe z + i dL/dIm z):
+ *   dlam[r] = sum_{i,o,k} dR conj(A[i,r] B[o,r] C[k,r]),
+ *   dA[i,r] = sum_{o,k} dR conj(lam[r] B[o,r] C[k,r]),  likewise dB, dC.
+ * Outputs (float32, (re, im), overwritten): dlam [rank][2], dA [Ci][rank][2],
+ * dB [Co][rank][2], dC [|K|][rank][2]; dx (storage dtype), and for the block
+ * dW, db as fno_block_bwd.  Workspace: fno_workspace_size(desc,
+ * FNO_OP_SPECTRAL_BWD_CP or FNO_OP_BLOCK_BWD_CP). */
+int fno_spectral_conv_bwd_cp(const fno_block_desc *desc, int rank, const void *x,
+                             const void *lam, const void *A, const void *B, const void *C,
+                             const float *xhat_save, const void *dy, void *dx, float *dlam,
+                             float *dA, float *dB, float *dC, void *ws, size_t ws_bytes,
+                             fno_stream_t stream);
+int fno_block_bwd_cp(const fno_block_desc *desc, int rank, const void *x, const void *lam,
+                     const void *A, const void *B, const void *C, const void *W,
+                     const void *pre_save, const float *xhat_save, const void *dy, void *dx,
+                     float *dlam, float *dA, float *dB, float *dC, float *dW, float *db, void *ws,
+                     size_t ws_bytes, fno_stream_t stream);
 
 /* Adjoint of fno_spectral_conv_fwd.  Inputs: x (needed for tanh'), xhat_save
  * from the forward (may be NULL: then it is recomputed from x), R, dy

@@ -468,3 +468,30 @@ def cp_weights(lam, a, b, c) -> np.ndarray:
 def spectral_conv_fwd_cp(x, lam, a, b, c, modes, flags: int = 0):
     """:func:`spectral_conv_fwd` with the CP weight :func:`cp_weights` (definition)."""
     return spectral_conv_fwd(x, cp_weights(lam, a, b, c), modes, flags)
+
+
+def cp_factor_grads(d_r, lam, a, b, c):
+    """Gradients of the CP factors from the dense weight's gradient ``d_r``.
+
+    The weight ``R[i,o,k] = sum_r lam[r] a[i,r] b[o,r] c[k,r]`` is holomorphic in
+    each factor, so with the convention ``dz = dL/dRe z + i dL/dIm z`` the chain
+    rule gives ``dz = sum dR conj(dR/dz)``:
+    ``dlam[r] = sum_{iok} dR conj(a b c)``, ``da[i,r] = sum_{ok} dR conj(lam b c)``,
+    ``db[o,r] = sum_{ik} dR conj(lam a c)``, ``dc[k,r] = sum_{io} dR conj(lam a b)``.
+    Returns ``(dlam, da, db, dc)`` complex128.
+    """
+    d_r = np.asarray(d_r, np.complex128)
+    lam, a, b, c = (np.asarray(v, np.complex128) for v in (lam, a, b, c))
+    dlam = np.einsum("iok,ir,or,kr->r", d_r, np.conj(a), np.conj(b), np.conj(c))
+    da = np.einsum("iok,r,or,kr->ir", d_r, np.conj(lam), np.conj(b), np.conj(c))
+    db = np.einsum("iok,r,ir,kr->or", d_r, np.conj(lam), np.conj(a), np.conj(c))
+    dc = np.einsum("iok,r,ir,or->kr", d_r, np.conj(lam), np.conj(a), np.conj(b))
+    return dlam, da, db, dc
+
+
+def spectral_conv_bwd_cp(x, lam, a, b, c, xhat, dy, modes, flags: int = 0):
+    """Adjoint of :func:`spectral_conv_fwd_cp`: :func:`spectral_conv_bwd` on the
+    reconstructed weight, then :func:`cp_factor_grads`.
+    Returns ``(dx, dlam, da, db, dc)``."""
+    dx, d_r = spectral_conv_bwd(x, cp_weights(lam, a, b, c), xhat, dy, modes, flags)
+    return (dx,) + cp_factor_grads(d_r, lam, a, b, c)

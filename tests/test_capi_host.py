@@ -317,3 +317,44 @@ def test_backward_ready_validation(lib):
 def test_wait_limit_rejects_negative_values(lib):
     assert lib.fno_set_wait_limit(-1) == capi.FNO_ERR_INVALID_ARG
     assert "wait limit" in capi.last_error()
+
+
+def test_factorised_backward_validation(lib):
+    d = capi.block_desc(2, 4, 4, (16, 16), (4, 4))
+    need = capi.fno_workspace_size(d, capi.FNO_OP_BLOCK_BWD_CP)
+    assert need > capi.fno_workspace_size(d, capi.FNO_OP_BLOCK_BWD)
+    assert capi.fno_workspace_size(d, capi.FNO_OP_SPECTRAL_BWD_CP) > 0
+    f = lib.fno_block_bwd_cp
+    ok = dict(x=256, lam=256, A=256, B=256, C=256, W=256, pre=256, dy=256, dx=256, dlam=256,
+              dA=256, dB=256, dC=256, dW=256, db=256)
+
+    def call(rank, ws=need, **kw):
+        a = dict(ok, **kw)
+        return f(ctypes.byref(d), rank, a["x"], a["lam"], a["A"], a["B"], a["C"], a["W"],
+                 a["pre"], None, a["dy"], a["dx"], a["dlam"], a["dA"], a["dB"], a["dC"], a["dW"],
+                 a["db"], 256, ws, None)
+    assert call(0) == capi.FNO_ERR_INVALID_ARG
+    assert call(capi.FNO_MAX_CP_RANK + 1) == capi.FNO_ERR_UNSUPPORTED
+    for name in ("dlam", "dA", "dB", "dC", "dW", "db", "dx", "dy"):
+        assert call(4, **{name: None}) == capi.FNO_ERR_INVALID_ARG
+        assert name in capi.last_error()
+    assert call(4, ws=need - 1) == capi.FNO_ERR_WORKSPACE
+
+
+def _header_arities():
+    """Number of parameters of every function the header declares."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(fno_[a-z_0-9]+)\s*\(([^;{]*?)\)\s*;", text):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_the_header(lib):
+    """Every ctypes signature declares exactly the header's parameter count, so
+    no argument (the stream last of all) is ever passed with default conversion."""
+    arities = _header_arities()
+    assert set(arities) == set(capi.EXPORTED)
+    for name, n in arities.items():
+        assert len(getattr(lib, name).argtypes) == n, name

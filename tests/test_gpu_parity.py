@@ -317,3 +317,46 @@ def test_factorised_weights_forward(grid, modes, rank, dtype, flags):
                                      oracle_flags(flags))
     assert_close(host(pre), pre_ref, TOL[dtype], "pre (block)")
     assert_close(host(yb), yb_ref, TOL[dtype], "y (block)")
+
+
+@pytest.mark.parametrize("grid,modes", [((64, 64), (10, 12)), ((15, 9), (5, 5)),
+                                        ((256, 256), (16, 16)), ((6, 10, 12), (2, 3, 4))])
+@pytest.mark.parametrize("rank", [1, 7, 32])
+@pytest.mark.parametrize("dtype,flags", [("f32", 0), ("f32", 1), ("bf16", 0)])
+def test_factorised_weights_backward(grid, modes, rank, dtype, flags):
+    """Adjoints through the CP factors against the oracle: dx and the factor
+    gradients of the spectral convolution (spectral_conv_bwd_cp), and of the
+    block (block_bwd on cp_weights, then cp_factor_grads)."""
+    import torch
+    b_, ci, co = 2, 5, 6
+    x, _, w, b, dy = _block_inputs(grid, modes, b_, ci, co, dtype, seed=9)
+    fac = _cp_inputs(grid, modes, rank, ci, co, dtype, seed=10)
+    d = capi.block_desc(b_, ci, co, grid, modes, dtype, flags)
+    k = capi.num_modes(grid, modes)
+    dv = [dev_complex(v, dtype) for v in fac]
+    of = oracle_flags(flags)
+    _, xh_ref = O.spectral_conv_fwd_cp(x, *fac, modes, of)
+    outs = [empty((b_, ci) + grid, dtype), empty((rank, 2)), empty((ci, rank, 2)),
+            empty((co, rank, 2)), empty((k, rank, 2))]
+    capi.fno_spectral_conv_bwd_cp(d, rank, dev(x, dtype), *dv, dev_complex(xh_ref), dev(dy, dtype),
+                                  *outs)
+    ref = O.spectral_conv_bwd_cp(x, *fac, xh_ref, dy, modes, of)
+    assert_close(host(outs[0]), ref[0], TOL[dtype], "dx (spectral)")
+    for name, got, want in zip(("dlam", "dA", "dB", "dC"), outs[1:], ref[1:]):
+        assert_close(host_complex(got), want, TOL[dtype], name + " (spectral)")
+    # the block: the oracle forward's pre-activation, rounded to the storage dtype, on both sides
+    r_dense = O.cp_weights(*fac)
+    _, pre_ref, _ = O.block_fwd(x, r_dense, w, b, modes, of)
+    pre_q = synth.quantize(pre_ref, dtype)
+    outs = [empty((b_, ci) + grid, dtype), empty((rank, 2)), empty((ci, rank, 2)),
+            empty((co, rank, 2)), empty((k, rank, 2)), empty((co, ci)), empty((co,))]
+    capi.fno_block_bwd_cp(d, rank, dev(x, dtype), *dv, dev(w, dtype), dev(pre_q, dtype), None,
+                          dev(dy, dtype), *outs)
+    dx_ref, dr_ref, dw_ref, db_ref = O.block_bwd(x, r_dense, w, pre_q, xh_ref, dy, modes, of)
+    dfac = O.cp_factor_grads(dr_ref, *fac)
+    assert_close(host(outs[0]), dx_ref, TOL[dtype], "dx (block)")
+    for name, got, want in zip(("dlam", "dA", "dB", "dC"), outs[1:5], dfac):
+        assert_close(host_complex(got), want, TOL[dtype], name + " (block)")
+    assert_close(host(outs[5]), dw_ref, TOL[dtype], "dW (block)")
+    assert_close(host(outs[6]), db_ref, TOL[dtype], "db (block)")
+    del torch

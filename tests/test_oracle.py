@@ -304,6 +304,49 @@ def test_spectral_conv_bwd_finite_differences(flags):
     np.testing.assert_allclose(_fd_dir(loss_r, r, 1j * vr), np.sum(d_r.imag * vr), rtol=1e-6)
 
 
+@pytest.mark.parametrize("flags", [0, O.TANH_PREACT])
+def test_spectral_conv_bwd_cp_finite_differences(flags):
+    """Every CP factor's gradient (real and imaginary directions) and dx against
+    central differences of L = <spectral_conv_fwd_cp(x, factors), g>."""
+    grid, modes, rank = (8, 6), (2, 3), 3
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((2, 3) + grid)
+    n_k = O.num_modes(grid, modes)
+
+    def cplx(*shape):
+        return rng.standard_normal(shape) + 1j * rng.standard_normal(shape)
+    fac = [cplx(rank), cplx(3, rank), cplx(4, rank), cplx(n_k, rank)]
+    g = rng.standard_normal((2, 4) + grid)
+    _, xhat = O.spectral_conv_fwd_cp(x, *fac, modes, flags)
+    dx, *dfac = O.spectral_conv_bwd_cp(x, *fac, xhat, g, modes, flags)
+    loss_x = lambda xx: np.sum(O.spectral_conv_fwd_cp(xx, *fac, modes, flags)[0] * g)
+    v = rng.standard_normal(x.shape)
+    np.testing.assert_allclose(_fd_dir(loss_x, x, v), np.sum(dx * v), rtol=1e-6)
+    for j in range(4):
+        def loss_j(z, j=j):
+            f2 = list(fac)
+            f2[j] = z
+            return np.sum(O.spectral_conv_fwd_cp(x, *f2, modes, flags)[0] * g)
+        vj = rng.standard_normal(fac[j].shape)
+        np.testing.assert_allclose(_fd_dir(loss_j, fac[j], vj), np.sum(dfac[j].real * vj),
+                                   rtol=1e-5, atol=1e-9)
+        np.testing.assert_allclose(_fd_dir(loss_j, fac[j], 1j * vj), np.sum(dfac[j].imag * vj),
+                                   rtol=1e-5, atol=1e-9)
+
+
+def test_cp_factor_grads_of_a_rank_one_weight_by_hand():
+    """Rank 1 with unit factors: R = lam a b c everywhere, so each factor's
+    gradient is the sum of dR times the conjugate of the other three."""
+    d_r = np.arange(2 * 3 * 4).reshape(2, 3, 4) * (1 + 0.5j)
+    lam, a, b, c = np.array([2.0]), np.ones((2, 1)), np.ones((3, 1)) * 1j, np.ones((4, 1))
+    dlam, da, db, dc = O.cp_factor_grads(d_r, lam, a, b, c)
+    total = d_r.sum()
+    assert np.allclose(dlam, [total * (-1j)])             # conj(a b c) = -i
+    assert np.allclose(da[:, 0], d_r.sum(axis=(1, 2)) * 2 * (-1j))
+    assert np.allclose(db[:, 0], d_r.sum(axis=(0, 2)) * 2)
+    assert np.allclose(dc[:, 0], d_r.sum(axis=(0, 1)) * 2 * (-1j))
+
+
 @pytest.mark.parametrize("grid,modes,flags", [((8, 6), (2, 3), 0), ((8, 6), (2, 3), O.TANH_PREACT),
                                               ((4, 6, 5), (1, 2, 3), 0), ((10,), (4,), O.NO_ACT)])
 def test_block_bwd_finite_differences(grid, modes, flags):

@@ -175,6 +175,14 @@ def _mutants(fo):
         return np.einsum("ir,or,kr->iok", np.asarray(a, np.complex128),
                          np.asarray(b, np.complex128), np.asarray(c, np.complex128))
 
+    def cp_grads_unconjugated(d_r, lam, a, b, c):   # factor gradients without conj
+        d_r = np.asarray(d_r, np.complex128)
+        lam, a, b, c = (np.asarray(v, np.complex128) for v in (lam, a, b, c))
+        return (np.einsum("iok,ir,or,kr->r", d_r, a, b, c),
+                np.einsum("iok,r,or,kr->ir", d_r, lam, b, c),
+                np.einsum("iok,r,ir,kr->or", d_r, lam, a, c),
+                np.einsum("iok,r,ir,or->kr", d_r, lam, a, b))
+
     def projection_without_gelu(v, q1_mat, q1_vec, q2_mat, q2_vec):   # hidden layer linear
         v = np.asarray(v, np.float64)
         d = v.ndim - 2
@@ -185,6 +193,7 @@ def _mutants(fo):
         "projection_without_gelu": {"projection": projection_without_gelu},
         "cp_factor_conjugated": {"cp_weights": cp_factor_conjugated},
         "cp_lambda_dropped": {"cp_weights": cp_lambda_dropped},
+        "cp_grads_unconjugated": {"cp_factor_grads": cp_grads_unconjugated},
         "adam_no_bias_correction": {"adam_update": adam("no_bias_correction")},
         "adam_eps_inside_sqrt": {"adam_update": adam("eps_inside_sqrt")},
         "adam_coupled_decay": {"adam_update": adam("coupled_decay")},
@@ -230,7 +239,7 @@ MUTANT_NAMES = [
     "tanh_grad_missing", "db_dropped", "skip_grad_dropped", "dq2_from_preactivation",
     "lift_bias_dropped", "mse_half_gradient", "adam_no_bias_correction", "adam_eps_inside_sqrt",
     "adam_coupled_decay", "bf16_truncating", "schedule_phase_late", "cp_factor_conjugated",
-    "cp_lambda_dropped", "projection_without_gelu",
+    "cp_lambda_dropped", "cp_grads_unconjugated", "projection_without_gelu",
 ]
 
 
