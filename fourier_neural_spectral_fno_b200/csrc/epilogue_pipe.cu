@@ -232,6 +232,50 @@ __device__ __forceinline__ void cursor_next(Cursor &c, int Rt, const Geom &g) {
   }
 }
 
+// NSTEP K steps of the tile's MMA chain into D, unrolled: every operand is a
+// base plus a compile-time offset (8 TMEM columns of A, 256 bytes of B per
+// step).  acc_first: the first step accumulates onto D as well.
+template <typename K, int NSTEP>
+__device__ __forceinline__ void issue_exact(uint32_t d, uint32_t a, uint32_t lo, uint64_t b,
+                                            uint32_t idesc, bool acc_first) {
+#pragma unroll
+  for (int s = 0; s < NSTEP; ++s) {
+    const uint32_t acc = (acc_first || s > 0) ? 1u : 0u;
+    if (K::tf32) {
+      tc::mma_tf32_ts(d, a + 8 * s, b + (uint64_t)(16 * s), idesc, acc);
+      tc::mma_tf32_ts(d, a + lo + 8 * s, b + (uint64_t)(16 * s), idesc, 1u);
+    } else {
+      tc::mma_f16_ts(d, a + 8 * s, b + (uint64_t)(16 * s), idesc, acc);
+    }
+  }
+}
+
+// n K steps: the exact unrolled sequence for the common counts, else a plain
+// loop (no branch inside either)
+template <typename K>
+__device__ __forceinline__ void issue_steps(uint32_t d, uint32_t a, uint32_t lo, uint64_t b,
+                                            uint32_t idesc, int n, bool acc_first) {
+  switch (n) {
+    case 1: issue_exact<K, 1>(d, a, lo, b, idesc, acc_first); return;
+    case 2: issue_exact<K, 2>(d, a, lo, b, idesc, acc_first); return;
+    case 3: issue_exact<K, 3>(d, a, lo, b, idesc, acc_first); return;
+    case 4: issue_exact<K, 4>(d, a, lo, b, idesc, acc_first); return;
+    case 6: issue_exact<K, 6>(d, a, lo, b, idesc, acc_first); return;
+    case 8: issue_exact<K, 8>(d, a, lo, b, idesc, acc_first); return;
+    default: break;
+  }
+  if (n <= 0) return;
+  issue_exact<K, 1>(d, a, lo, b, idesc, acc_first);
+  for (int s = 1; s < n; ++s) {
+    if (K::tf32) {
+      tc::mma_tf32_ts(d, a + 8 * s, b + (uint64_t)(16 * s), idesc, 1u);
+      tc::mma_tf32_ts(d, a + lo + 8 * s, b + (uint64_t)(16 * s), idesc, 1u);
+    } else {
+      tc::mma_f16_ts(d, a + 8 * s, b + (uint64_t)(16 * s), idesc, 1u);
+    }
+  }
+}
+
 template <typename T, bool HAS_X, int CX, bool IMG>
 __global__ void __launch_bounds__(THREADS, 1)
     k_epi_pipe(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmu,
@@ -347,7 +391,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // 256 bytes (16 in descriptor units, no carry out of the 14-bit field)
       const uint64_t bdesc0 = tc::smem_desc_kmajor(tc::smem_u32(bbase), 128, e.sbo);
       const uint64_t bdesc1 =
-          tc::smem_desc_kmajor(tc::smem_u32(bbase + (e.NA - 1) * e.bbuf), 128, e.sbo);
+          tc::smem_desc_kmajor(tc::smem_u32(bbase + (e.NB - 1) * e.bbuf), 128, e.sbo);
       int j = 0;
       for (; j < ntl; ++j) {
         bool ok = tc::mbar_wait(&aready[j & 1], (j >> 1) & 1, a.err);
@@ -357,31 +401,21 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int variant = e.Rt > 1 ? 0 : c.n0 / ROWS;
         const int ab = e.NA == 2 ? (j & 1) : 0;
         const uint32_t d = tbase + (uint32_t)((j & 1) * e.DC);
-        // one thread issues; operands advance by constants (tf32: the A_hi and
-        // A_lo products of each K step, both against [B_hi; B_lo])
-        if (lane == 0) {
-          // IMG: the spectral steps read this tile's ring stage, the x steps W
-          uint64_t bd = IMG ? tc::smem_desc_kmajor(
-                                  tc::smem_u32(smem + (size_t)(j % e.NS) * e.stage + e.uoff), 128,
-                                  e.sbo_s)
-                            : (ab ? bdesc1 : bdesc0);
-          uint32_t acol = tbase + e.col_spec + variant * e.cs_cols;
-          uint32_t lo = lo_spec;
-          for (int s = 0; s < ns + nx; ++s) {
-            if (s == ns) {
-              acol = tbase + e.col_x + ab * e.ax_cols;
-              lo = lo_x;
-              if (IMG) bd = bdesc0;
-            }
-            if (K::tf32) {
-              tc::mma_tf32_ts(d, acol, bd, idesc, s > 0 ? 1u : 0u);
-              tc::mma_tf32_ts(d, acol + lo, bd, idesc, 1u);
-            } else {
-              tc::mma_f16_ts(d, acol, bd, idesc, s > 0 ? 1u : 0u);
-            }
-            acol += 8;
-            bd += 16;
-          }
+        // one elected thread issues the tile's K steps (tf32: the A_hi and A_lo
+        // products of each K step, both against [B_hi; B_lo]); one K step
+        // advances B by 256 bytes (16 in descriptor units, no carry out of the
+        // 14-bit field) and A by 8 TMEM columns
+        if (tc::elect_one()) {
+          // IMG: the spectral steps read this tile's ring stage, the x steps W;
+          // else both read the staged B buffer, the x steps after the spectral
+          const uint64_t bspec =
+              IMG ? tc::smem_desc_kmajor(
+                        tc::smem_u32(smem + (size_t)(j % e.NS) * e.stage + e.uoff), 128, e.sbo_s)
+                  : (ab ? bdesc1 : bdesc0);
+          const uint64_t bx = IMG ? bdesc0 : bspec + (uint64_t)(16 * ns);
+          issue_steps<K>(d, tbase + e.col_spec + variant * e.cs_cols, lo_spec, bspec, idesc, ns,
+                         false);
+          issue_steps<K>(d, tbase + e.col_x + ab * e.ax_cols, lo_x, bx, idesc, nx, true);
           tc::mma_commit(&mdone[j & 1]);
         }
         __syncwarp();

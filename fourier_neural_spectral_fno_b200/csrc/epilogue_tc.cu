@@ -350,9 +350,9 @@ __global__ void __launch_bounds__(EPI_THREADS) k_epi_tc(EpiTcArgs a, Geom g) {
     tc::fence_proxy_async_smem();
     tc::fence_before_sync();
     __syncthreads();
-    // (3) one thread issues the MMAs: spectral K steps then x K steps; for
-    // tf32 each K step is A_hi [B_hi; B_lo] + A_lo [B_hi; B_lo]
-    if (tid == 0) {
+    // (3) one elected thread of warp 0 issues the MMAs: spectral K steps then x
+    // K steps; for tf32 each K step is A_hi [B_hi; B_lo] + A_lo [B_hi; B_lo]
+    if ((tid >> 5) == 0 && tc::elect_one()) {
       tc::fence_after_sync();
       const uint32_t aspec = tbase + e.DC + variant * e.cs_cols;
       const uint32_t ax = tbase + e.x_col;

@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(TC_THREADS)
     tc::tmem_wait_st();
     tc::fence_before_sync();
     __syncthreads();
-    if (t == 0) {
+    if ((t >> 5) == 0 && tc::elect_one()) {   // one elected thread of warp 0
       tc::fence_after_sync();
       const int ns = e.Cp / K::KSTEP;
       uint64_t bh = bh0, bl = bl0;      // +256 bytes (16 units) per K step

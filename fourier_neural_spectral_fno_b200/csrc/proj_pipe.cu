@@ -150,6 +150,27 @@ __device__ __forceinline__ void stage16(uint32_t col, uint32_t lo_off, const flo
   }
 }
 
+// K steps [k0, k0 + NSTEP) of the hidden-layer chain (tf32: v_hi Q1_hi,
+// v_hi Q1_lo, v_lo Q1_hi per step); the first step of the chain (k0 = 0)
+// overwrites D.
+template <typename K, int NSTEP>
+__device__ __forceinline__ void proj_steps(uint32_t d, uint32_t a0, int cp, uint64_t bh0,
+                                           uint64_t bl0, uint32_t idesc, int k0) {
+#pragma unroll
+  for (int s = 0; s < NSTEP; ++s) {
+    const int ks = k0 + s;
+    const uint32_t acc = ks > 0 ? 1u : 0u;
+    const uint64_t bo = (uint64_t)(16 * ks);
+    if (K::tf32) {
+      tc::mma_tf32_ts(d, a0 + 8 * ks, bh0 + bo, idesc, acc);
+      tc::mma_tf32_ts(d, a0 + 8 * ks, bl0 + bo, idesc, 1u);
+      tc::mma_tf32_ts(d, a0 + (uint32_t)cp + 8 * ks, bh0 + bo, idesc, 1u);
+    } else {
+      tc::mma_f16_ts(d, a0 + 8 * ks, bh0 + bo, idesc, acc);
+    }
+  }
+}
+
 template <typename T, int CX>
 __global__ void __launch_bounds__(THREADS, 1)
     k_proj_pipe(const __grid_constant__ CUtensorMap tmv, ProjArgs a) {
@@ -287,21 +308,21 @@ __global__ void __launch_bounds__(THREADS, 1)
       const bool w = tc::mbar_wait(&aready[j & 1], (j >> 1) & 1, a.err);
       if (!__all_sync(0xffffffffu, w)) break;
       tc::fence_after_sync();
-      if (lane == 0) {
+      // one elected thread issues the K steps: the exact unrolled sequence for
+      // the common widths, else a plain loop (operands advance by 8 TMEM
+      // columns and 256 bytes of B per step)
+      if (tc::elect_one()) {
         const uint32_t d = tbase + (uint32_t)((j & 1) * e.HP);
-        uint32_t a0 = tbase + e.col_a + (j & 1) * e.ax_cols;
-        uint64_t bh = bh0, bl = bl0;
-        for (int ks = 0; ks < ns; ++ks) {
-          if (K::tf32) {
-            tc::mma_tf32_ts(d, a0, bh, idesc, ks > 0 ? 1u : 0u);
-            tc::mma_tf32_ts(d, a0, bl, idesc, 1u);
-            tc::mma_tf32_ts(d, a0 + e.Cp, bh, idesc, 1u);
-          } else {
-            tc::mma_f16_ts(d, a0, bh, idesc, ks > 0 ? 1u : 0u);
-          }
-          a0 += 8;
-          bh += 16;
-          bl += 16;
+        const uint32_t a0 = tbase + e.col_a + (j & 1) * e.ax_cols;
+        switch (ns) {
+          case 1: proj_steps<K, 1>(d, a0, e.Cp, bh0, bl0, idesc, 0); break;
+          case 2: proj_steps<K, 2>(d, a0, e.Cp, bh0, bl0, idesc, 0); break;
+          case 3: proj_steps<K, 3>(d, a0, e.Cp, bh0, bl0, idesc, 0); break;
+          case 4: proj_steps<K, 4>(d, a0, e.Cp, bh0, bl0, idesc, 0); break;
+          case 6: proj_steps<K, 6>(d, a0, e.Cp, bh0, bl0, idesc, 0); break;
+          case 8: proj_steps<K, 8>(d, a0, e.Cp, bh0, bl0, idesc, 0); break;
+          default:
+            for (int ks = 0; ks < ns; ++ks) proj_steps<K, 1>(d, a0, e.Cp, bh0, bl0, idesc, ks);
         }
         tc::mma_commit(&mdone[j & 1]);
       }

@@ -118,6 +118,21 @@ __host__ __device__ constexpr uint32_t instr_desc(int ab_format, int M, int N) {
 }
 constexpr int FMT_F16 = 0, FMT_BF16 = 1, FMT_TF32 = 2;
 
+// True in exactly one lane of the converged warp (elect.sync).  MMA issuers
+// enter their issue sequence through it with the whole warp present.  Measured
+// on B200: an MMA sequence issued this way, as a branch-free run of exactly the
+// needed steps (unrolled, or a plain loop), keeps up with the tensor core (34
+// cycles for M = 128, N = 64, K = 8 tf32); per-MMA branches in a lane-0 region
+// cost 130-220 cycles per MMA whatever N is, and a deep unroll with a
+// predicate on each step (sized for the largest count) about 130.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // D[tmem] (+)= A[tmem] * B[smem]  (issued by one thread)
 __device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                             uint32_t idesc, uint32_t accumulate) {

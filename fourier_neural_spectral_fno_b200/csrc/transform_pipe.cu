@@ -395,15 +395,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       const bool w = tc::mbar_wait(b2ready, jj & 1, a.err);
       if (!__all_sync(0xffffffffu, w)) return false;
       tc::fence_after_sync();
-      if (lane == 0) {
+      if (tc::elect_one()) {   // unrolled: bases plus compile-time offsets
         const uint32_t d2 = tbase + e.col_d2;
-        uint64_t bd = b2desc;
-        uint32_t acol = tbase + e.col_a2;
-        for (int ks = 0; ks < ROWS / 8; ++ks) {
-          tc::mma_tf32_ts(d2, acol, bd, id2, ks > 0 ? 1u : 0u);
-          acol += 8;
-          bd += 16;
-        }
+        const uint32_t acol = tbase + e.col_a2;
+#pragma unroll
+        for (int ks = 0; ks < ROWS / 8; ++ks)
+          tc::mma_tf32_ts(d2, acol + 8 * ks, b2desc + (uint64_t)(16 * ks), id2, ks > 0 ? 1u : 0u);
         tc::mma_commit(&s2done[jj & 1]);
       }
       __syncwarp();
@@ -420,21 +417,20 @@ __global__ void __launch_bounds__(THREADS, 1)
           break;
         }
         tc::fence_after_sync();
-        if (lane == 0) {
-          uint64_t ad = desc_sw128(tc::smem_u32(smem + (size_t)s * e.stage));
-          uint64_t bd = fdesc + (uint64_t)(c * 4 * 16);
+        if (tc::elect_one()) {
+          const uint64_t ad = desc_sw128(tc::smem_u32(smem + (size_t)s * e.stage));
+          const uint64_t bd = fdesc + (uint64_t)(c * 4 * 16);
           const uint32_t ahi = tbase + e.col_alo + (g % NABUF) * 64;
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
             const uint32_t acc = (c | ks) ? 1u : 0u;
+            // A: 32 bytes along K inside the swizzle atom; F: 256 bytes per K step
             if (K::tf32) {
-              tc::mma_tf32_ts(d1, ahi + ks * 8, bd, id1, acc);
-              tc::mma_tf32_ts(d1, ahi + 32 + ks * 8, bd, id1, 1u);
+              tc::mma_tf32_ts(d1, ahi + ks * 8, bd + (uint64_t)(16 * ks), id1, acc);
+              tc::mma_tf32_ts(d1, ahi + 32 + ks * 8, bd + (uint64_t)(16 * ks), id1, 1u);
             } else {
-              mma_ss(d1, ad, bd, id1, acc, false);
+              mma_ss(d1, ad + (uint64_t)(2 * ks), bd + (uint64_t)(16 * ks), id1, acc, false);
             }
-            ad += 2;     // 32 bytes along K inside the swizzle atom
-            bd += 16;    // 256 bytes: next K step of F
           }
           if (K::tf32) tc::mma_commit(&lofree[g % NABUF]);   // A buffer free
           else tc::mma_commit(&empty[s]);                 // stage free

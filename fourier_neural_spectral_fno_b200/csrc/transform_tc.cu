@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(TC_THREADS) k_s1_tc(S1Args a) {
       tc::tmem_wait_st();
       tc::fence_before_sync();
       __syncthreads();
-      if (t == 0) {
+      if ((t >> 5) == 0 && tc::elect_one()) {   // one elected thread of warp 0
         tc::fence_after_sync();
         const uint32_t a0 = tbase + A_COL0 + buf * ACOLS;
         // descriptors advance by constants (256 bytes = 16 units per K step)
