@@ -103,39 +103,44 @@ struct KeptIndex {
 // ---------------------------------------------------------------------------
 // activations
 // ---------------------------------------------------------------------------
-// erf(t) for t >= 0: Chebyshev least-squares fit on [0, 3.9] evaluated by
-// Horner's rule in x = (t - 1.95) / 1.95; 1 beyond 3.9 (1 - erf(3.9) = 3.5e-8).
-// Coefficients from fourier_neural_spectral_fno_b200/gen_erf_poly.py; the
-// float32 evaluation is within 6e-7 of erf (tests/test_gelu_poly.py).  It has
-// no branches, so the GELUs of a thread's channels interleave freely.
-__device__ __forceinline__ float erf_pos(float t) {
-  const float x = (fminf(t, 3.9f) - 1.95f) * 0.51282054f;
-  float a = 0.0026791077f;
-  a = fmaf(a, x, -0.0049660155f);
-  a = fmaf(a, x, -0.013497429f);
-  a = fmaf(a, x, 0.03540305f);
-  a = fmaf(a, x, 0.015209468f);
-  a = fmaf(a, x, -0.10800477f);
-  a = fmaf(a, x, 0.063275486f);
-  a = fmaf(a, x, 0.14825702f);
-  a = fmaf(a, x, -0.25860572f);
-  a = fmaf(a, x, 0.04010987f);
-  a = fmaf(a, x, 0.33213925f);
-  a = fmaf(a, x, -0.4308476f);
-  a = fmaf(a, x, 0.096189916f);
-  a = fmaf(a, x, 0.3598901f);
-  a = fmaf(a, x, -0.5448647f);
-  a = fmaf(a, x, 0.4110579f);
-  a = fmaf(a, x, -0.18670471f);
-  a = fmaf(a, x, 0.04910043f);
-  a = fmaf(a, x, 0.9941793f);
-  return t > 3.9f ? 1.0f : a;
+// erf by Hastings' approximation (Abramowitz and Stegun, Handbook of
+// Mathematical Functions, formula 7.1.28): for t >= 0
+//   erf t = 1 - (1 + a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5 + a6 t^6)^-16
+// with |error| <= 3e-7.  Horner's rule, four squarings and one approximate
+// reciprocal; a power that overflows gives erfc = 0.  No branches, so the
+// GELUs of a thread's channels interleave freely.
+constexpr float kErfA1 = 0.0705230784f, kErfA2 = 0.0422820123f, kErfA3 = 0.0092705272f,
+                kErfA4 = 0.0001520143f, kErfA5 = 0.0002765672f, kErfA6 = 0.0000430638f;
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
 }
 
-// standard normal CDF Phi(p) = (1 + erf(p / sqrt 2)) / 2
+// erfc(t) = 1 - erf(t) for t >= 0.  The power is carried as v = q - 1
+// (each squaring v <- v (v + 2)), so near t = 0, where q is close to 1, the
+// rounding of q is not raised to the 16th power: Phi = erfc / 2 is within
+// 2.5e-7 in float32 (the formula's own 1.3e-7 and the roundings).
+__device__ __forceinline__ float erfc_pos(float t) {
+  float u = fmaf(kErfA6, t, kErfA5);
+  u = fmaf(u, t, kErfA4);
+  u = fmaf(u, t, kErfA3);
+  u = fmaf(u, t, kErfA2);
+  u = fmaf(u, t, kErfA1);
+  u *= t;
+  u *= u + 2.0f;
+  u *= u + 2.0f;
+  u *= u + 2.0f;
+  u *= u + 2.0f;
+  return rcp_approx(1.0f + u);
+}
+
+// standard normal CDF Phi(p) = erfc(-p / sqrt 2) / 2: the tail half-erfc is
+// taken directly for p < 0, so small values keep their relative accuracy
 __device__ __forceinline__ float norm_cdf(float p) {
-  const float e = erf_pos(fabsf(p) * 0.70710678118654752440f);
-  return 0.5f + 0.5f * copysignf(e, p);
+  const float h = 0.5f * erfc_pos(fabsf(p) * 0.70710678118654752440f);
+  return p >= 0.0f ? 1.0f - h : h;
 }
 __device__ __forceinline__ float gelu_f(float p) { return p * norm_cdf(p); }
 // GELU and its derivative from one evaluation of the normal CDF
@@ -175,35 +180,30 @@ __device__ __forceinline__ f32x2 f2add(f32x2 a, f32x2 b) {
 }
 __device__ __forceinline__ f32x2 f2splat(float c) { return f2pack(c, c); }
 
-// GELU of two values at once: the erf polynomial of erf_pos on packed pairs.
-// |p| is clamped at 3.9 sqrt(2) (erf(3.9) = 1 - 3.5e-8) and the variable change
-// x = |p| / (1.95 sqrt 2) - 1 is one fused multiply-add.
+// GELU of two values at once, on packed pairs (the forward's activation):
+// formula 7.1.28 with 1 / sqrt 2 folded into the coefficients (a_k 2^(-k/2))
+// and q raised to the 16th power directly (four multiplies), then
+// w = (p / 2) erfc(|p| / sqrt 2) and GELU(p) = p - w (p >= 0) or w (p < 0).
+// The error of q^16 near p = 0 is scaled by p here: |GELU error| <= 4e-7
+// max(1, |p|) in float32.
 __device__ __forceinline__ void gelu2(float &a, float &b) {
-  const float ta = fminf(fabsf(a), 5.5154328f), tb = fminf(fabsf(b), 5.5154328f);
-  const f32x2 x = f2fma(f2pack(ta, tb), f2splat(0.36261886f), f2splat(-1.0f));
-  f32x2 e = f2splat(0.0026791077f);
-  e = f2fma(e, x, f2splat(-0.0049660155f));
-  e = f2fma(e, x, f2splat(-0.013497429f));
-  e = f2fma(e, x, f2splat(0.03540305f));
-  e = f2fma(e, x, f2splat(0.015209468f));
-  e = f2fma(e, x, f2splat(-0.10800477f));
-  e = f2fma(e, x, f2splat(0.063275486f));
-  e = f2fma(e, x, f2splat(0.14825702f));
-  e = f2fma(e, x, f2splat(-0.25860572f));
-  e = f2fma(e, x, f2splat(0.04010987f));
-  e = f2fma(e, x, f2splat(0.33213925f));
-  e = f2fma(e, x, f2splat(-0.4308476f));
-  e = f2fma(e, x, f2splat(0.096189916f));
-  e = f2fma(e, x, f2splat(0.3598901f));
-  e = f2fma(e, x, f2splat(-0.5448647f));
-  e = f2fma(e, x, f2splat(0.4110579f));
-  e = f2fma(e, x, f2splat(-0.18670471f));
-  e = f2fma(e, x, f2splat(0.04910043f));
-  e = f2fma(e, x, f2splat(0.9941793f));
-  float ea, eb;
-  f2unpack(e, ea, eb);
-  const f32x2 phi = f2fma(f2pack(copysignf(ea, a), copysignf(eb, b)), f2splat(0.5f), f2splat(0.5f));
-  f2unpack(f2mul(phi, f2pack(a, b)), a, b);
+  const f32x2 t = f2pack(fabsf(a), fabsf(b));
+  f32x2 q = f2fma(f2splat(5.38297490493278e-06f), t, f2splat(4.889063711743802e-05f));
+  q = f2fma(q, t, f2splat(3.8003574445610866e-05f));
+  q = f2fma(q, t, f2splat(0.0032776263542473316f));
+  q = f2fma(q, t, f2splat(0.02114100567996502f));
+  q = f2fma(q, t, f2splat(0.04986734688282013f));
+  q = f2fma(q, t, f2splat(1.0f));
+  q = f2mul(q, q);
+  q = f2mul(q, q);
+  q = f2mul(q, q);
+  q = f2mul(q, q);
+  float qa, qb, wa, wb;
+  f2unpack(q, qa, qb);
+  f2unpack(f2mul(f2pack(rcp_approx(qa), rcp_approx(qb)), f2mul(f2pack(a, b), f2splat(0.5f))), wa,
+           wb);
+  a = a >= 0.0f ? a - wa : wa;
+  b = b >= 0.0f ? b - wb : wb;
 }
 
 // weight c_k / N of last-axis mode k_l (1 on DC and Nyquist, else 2)

@@ -8,14 +8,14 @@
 // with Q2 on the CUDA cores.  Float32 storage: three tf32 passes (v_hi Q1_hi +
 // v_hi Q1_lo + v_lo Q1_hi); 16-bit storage: one kind::f16 pass.
 //
-//   warp 13      TMA producer: v tile [width][128] into ring stage j % NS
+//   warp 21      TMA producer: v tile [width][128] into ring stage j % NS
 //   warps 0-3    staging: v -> A operand in TMEM (tf32 head / remainder)
-//   warp 12      MMA issuer: tile j into D buffer j % 2; its one mbarrier wait
+//   warp 20      MMA issuer: tile j into D buffer j % 2; its one mbarrier wait
 //                per tile (aready) also means the D buffer is free, since the
 //                staging warps wait for the epilogue before arriving
-//   warps 4-11   epilogue: two warps per TMEM lane quarter, each taking half of
-//                the hidden units; the halves' Q2 partial sums meet in shared
-//                memory and one half stores u
+//   warps 4-19   epilogue: four warps per TMEM lane quarter, each taking a
+//                quarter of the hidden units; the quarters' Q2 partial sums
+//                meet in shared memory and the first quarter stores u
 // Every wait is a bounded mbarrier wait; exits are warp-uniform, and the
 // epilogue warps share one named barrier per tile.
 #include <string.h>
@@ -31,9 +31,10 @@ namespace {
 
 constexpr int ROWS = 128;
 constexpr int NCONV = 4;
-constexpr int NEPI = 8;
-constexpr int WARP_MMA = NCONV + NEPI;     // 12
-constexpr int WARP_TMA = WARP_MMA + 1;     // 13
+constexpr int NEPI = 16;                   // four per TMEM lane quarter
+constexpr int NPART = NEPI / 4;            // hidden-unit parts
+constexpr int WARP_MMA = NCONV + NEPI;     // 20
+constexpr int WARP_TMA = WARP_MMA + 1;     // 21
 constexpr int THREADS = (WARP_TMA + 1) * 32;
 constexpr int MAX_STAGES = 6;
 constexpr int kMaxOut = 4;
@@ -65,8 +66,10 @@ __host__ __device__ inline int rup(int v, int m) { return (v + m - 1) / m * m; }
 __host__ __device__ inline size_t alg(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Plan.  TMEM: two D buffers [0, 2 HP), then two A buffers (tf32: head and
-// remainder, 2 Cp columns each).  Shared memory: the ring (v tiles), B = Q1
-// (head block, then remainder block), q1, Q2, the half-sum exchange, barriers.
+// remainder, 2 Cp columns each).  HP is a multiple of 16 NPART, so every part
+// of the hidden units is whole 16-column groups.  Shared memory: the ring (v
+// tiles), B = Q1 (head block, then remainder block), q1, Q2, the part-sum
+// exchange, barriers.
 struct ProjGeom {
   int Cp, HP, ax_cols, col_a, used, NS;
   uint32_t sbo, x_bytes;
@@ -76,7 +79,7 @@ struct ProjGeom {
 __host__ __device__ inline ProjGeom proj_geom(int width, int hidden, int eb, bool tf32) {
   ProjGeom e;
   e.Cp = rup(width, 16);
-  e.HP = rup(hidden, 32);                 // two halves of whole 16-column groups
+  e.HP = rup(hidden, 16 * NPART);
   e.ax_cols = tf32 ? 2 * e.Cp : e.Cp / 2;
   e.col_a = 2 * e.HP;
   e.used = e.col_a + 2 * e.ax_cols;
@@ -85,7 +88,8 @@ __host__ __device__ inline ProjGeom proj_geom(int width, int hidden, int eb, boo
   e.stage = alg(e.x_bytes, 1024);
   e.bhalf = (size_t)e.HP * e.Cp * eb;
   const size_t fixed = alg((tf32 ? 2 : 1) * e.bhalf, 1024) + sizeof(float) * e.HP +
-                       sizeof(float) * kMaxOut * e.HP + sizeof(float) * 2 * kMaxOut * ROWS +
+                       sizeof(float) * kMaxOut * e.HP +
+                       sizeof(float) * 2 * (NPART - 1) * kMaxOut * ROWS +
                        sizeof(uint64_t) * (2 * MAX_STAGES + 8) + 16;
   const size_t room = kSmemMax > fixed ? kSmemMax - fixed : 0;
   const size_t ns = room / e.stage;
@@ -94,7 +98,7 @@ __host__ __device__ inline ProjGeom proj_geom(int width, int hidden, int eb, boo
   e.b = off; off = alg(off + (tf32 ? 2 : 1) * e.bhalf, 1024);
   e.q1 = off; off += sizeof(float) * e.HP;
   e.q2 = off; off += sizeof(float) * kMaxOut * e.HP;
-  e.red = off; off += sizeof(float) * 2 * kMaxOut * ROWS;
+  e.red = off; off += sizeof(float) * 2 * (NPART - 1) * kMaxOut * ROWS;
   off = alg(off, 8);
   e.bar = off; off += sizeof(uint64_t) * (2 * MAX_STAGES + 8);
   e.tbase = off; off += 16;
@@ -107,14 +111,15 @@ __host__ __device__ __forceinline__ uint32_t boff(int n, int k, int eb, uint32_t
   return (uint32_t)(n >> 3) * sbo + (kb >> 4) * 128 + (n & 7) * 16 + (kb & 15);
 }
 
-// named barrier over the eight epilogue warps
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// named barrier over the epilogue warps
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
+static_assert(NEPI * 32 == 512, "the named barriers count the epilogue threads");
 __device__ __forceinline__ bool epi_all(bool v) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.and.pred p, 1, 256, q;\n\t"
+      "bar.red.and.pred p, 1, 512, q;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(r)
       : "r"((uint32_t)v)
@@ -333,15 +338,35 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc::mbar_wait(fin, 0, nullptr);
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3, half = (warp - NCONV) >> 2;
+    const int q = warp & 3, part = (warp - NCONV) >> 2;
     const int t = q * 32 + lane;
     const uint32_t arow = tbase + ((uint32_t)(q * 32) << 16);
-    const int hbeg = half * (e.HP / 2), hend = hbeg + e.HP / 2;
+    const int hbeg = part * (e.HP / NPART), hend = hbeg + e.HP / NPART;
     T *u = reinterpret_cast<T *>(a.u);
     const T *q2 = reinterpret_cast<const T *>(a.q2);
     float q2b[kMaxOut];
 #pragma unroll
     for (int o = 0; o < kMaxOut; ++o) q2b[o] = o < out_ch ? to_f<T>(q2[o]) : 0.f;
+    // 16 hidden units h0.. of this point: + q1, GELU, into the Q2 sums
+    auto group = [&](const uint32_t (&dv)[16], int h0, float (&acc)[kMaxOut]) {
+#pragma unroll
+      for (int i = 0; i < 16; i += 4) {   // q1 / Q2 as 16-byte vectors
+        const float4 qa = *reinterpret_cast<const float4 *>(q1s + h0 + i);
+        float z0 = __uint_as_float(dv[i]) + qa.x;
+        float z1 = __uint_as_float(dv[i + 1]) + qa.y;
+        float z2 = __uint_as_float(dv[i + 2]) + qa.z;
+        float z3 = __uint_as_float(dv[i + 3]) + qa.w;
+        gelu2(z0, z1);
+        gelu2(z2, z3);
+#pragma unroll
+        for (int o = 0; o < kMaxOut; ++o) {
+          if (o < out_ch) {
+            const float4 qb = *reinterpret_cast<const float4 *>(q2s + o * e.HP + h0 + i);
+            acc[o] = fmaf(qb.w, z3, fmaf(qb.z, z2, fmaf(qb.y, z1, fmaf(qb.x, z0, acc[o]))));
+          }
+        }
+      }
+    };
     for (int j = 0; j < ntl; ++j) {
       if (!epi_all(tc::mbar_wait(&mdone[j & 1], (j >> 1) & 1, a.err))) break;
       tc::fence_after_sync();
@@ -349,45 +374,43 @@ __global__ void __launch_bounds__(THREADS, 1)
       float acc[kMaxOut];
 #pragma unroll
       for (int o = 0; o < kMaxOut; ++o) acc[o] = 0.f;
-      for (int h0 = hbeg; h0 < hend; h0 += 16) {
-        uint32_t dv[16];
-        tc::tmem_ld16(dcol + h0, dv);
+      // rounds of two 16-column groups: both loads in flight, one wait; the
+      // last round's wait frees the D buffer
+      for (int r0 = hbeg; r0 < hend; r0 += 32) {
+        const bool two = r0 + 16 < hend;            // warp-uniform
+        uint32_t dv0[16], dv1[16];
+        tc::tmem_ld16(dcol + r0, dv0);
+        if (two) tc::tmem_ld16(dcol + r0 + 16, dv1);
         tc::tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; i += 4) {   // q1 / Q2 as 16-byte vectors
-          const float4 qa = *reinterpret_cast<const float4 *>(q1s + h0 + i);
-          float z0 = __uint_as_float(dv[i]) + qa.x;
-          float z1 = __uint_as_float(dv[i + 1]) + qa.y;
-          float z2 = __uint_as_float(dv[i + 2]) + qa.z;
-          float z3 = __uint_as_float(dv[i + 3]) + qa.w;
-          gelu2(z0, z1);
-          gelu2(z2, z3);
-#pragma unroll
-          for (int o = 0; o < kMaxOut; ++o) {
-            if (o < out_ch) {
-              const float4 qb = *reinterpret_cast<const float4 *>(q2s + o * e.HP + h0 + i);
-              acc[o] = fmaf(qb.w, z3, fmaf(qb.z, z2, fmaf(qb.y, z1, fmaf(qb.x, z0, acc[o]))));
-            }
-          }
+        if (r0 + 32 >= hend) {
+          tc::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) tma::arrive(&dempty[j & 1]);
         }
+        group(dv0, r0, acc);
+        if (two) group(dv1, r0 + 16, acc);
       }
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) tma::arrive(&dempty[j & 1]);
-      float *rb = red + (j & 1) * kMaxOut * ROWS;
-      if (half == 1) {
+      // parts 1.. leave their sums in buffer j % 2; part 0 adds them and stores
+      float *rb = red + (j & 1) * (NPART - 1) * kMaxOut * ROWS;
+      if (part > 0) {
 #pragma unroll
         for (int o = 0; o < kMaxOut; ++o)
-          if (o < out_ch) rb[o * ROWS + t] = acc[o];
+          if (o < out_ch) rb[((part - 1) * kMaxOut + o) * ROWS + t] = acc[o];
       }
       epi_sync();
-      if (half == 0) {
+      if (part == 0) {
         const long long tile = t_begin + j;
         const long long b = tile / tpb;
         const long long n = (tile - b * tpb) * ROWS + t;
 #pragma unroll
-        for (int o = 0; o < kMaxOut; ++o)
-          if (o < out_ch) u[(b * out_ch + o) * N + n] = from_f<T>(acc[o] + rb[o * ROWS + t] + q2b[o]);
+        for (int o = 0; o < kMaxOut; ++o) {
+          if (o < out_ch) {
+            float v = acc[o] + q2b[o];
+#pragma unroll
+            for (int p2 = 0; p2 < NPART - 1; ++p2) v += rb[(p2 * kMaxOut + o) * ROWS + t];
+            u[(b * out_ch + o) * N + n] = from_f<T>(v);
+          }
+        }
       }
     }
   }

@@ -259,8 +259,12 @@ def test_launch_count_is_reported(kernel_path):
 @pytest.mark.parametrize("grid,modes", [((64, 64), (10, 12)), ((256, 128), (16, 20)), ((15, 9), (5, 5))])
 def test_block_gelu_elementwise(grid, modes):
     """With R = 0, W = I and b = 0 the block output is GELU(x) point by point,
-    which pins the kernels' GELU elementwise (not only in the L2 norm): within
-    3e-7 absolute and 2e-6 relative of the exact erf form wherever |GELU| > 0.1."""
+    which pins the kernels' GELU elementwise (not only in the L2 norm).  Their
+    erf is formula 7.1.28 of Abramowitz and Stegun (|error| <= 3e-7), so the
+    GELU adds at most |x| 1.5e-7; the pre-activation W x through the three tf32
+    passes is within 2^-23 |x| (the rounded remainder), and the float32
+    roundings add about 1.5e-7 |x|: within 5e-7 max(1, |x|) of the exact erf
+    form at every point."""
     b_, c = 2, 16
     n = int(np.prod(grid))
     x = np.linspace(-9.0, 9.0, b_ * c * n).reshape((b_, c) + tuple(grid))
@@ -274,9 +278,7 @@ def test_block_gelu_elementwise(grid, modes):
     got = host(y).astype(np.float64)
     ref = O.gelu(x.astype(np.float64))
     err = np.abs(got - ref)
-    big = np.abs(ref) > 0.1
-    assert np.max(err[big] / np.abs(ref[big])) < 2e-6
-    assert np.max(err[~big]) < 3e-7
+    assert np.max(err / np.maximum(np.abs(x), 1.0)) < 5e-7
 
 
 def _cp_inputs(grid, modes, rank, ci, co, dtype, seed):
