@@ -683,6 +683,471 @@ cudaError_t launch_pipe_img(const Launch &L, const Geom &g, const PipeArgs &a, c
                : launch_pipe_t<T, HAS_X, false>(L, g, a, x, U);
 }
 
+// ===========================================================================
+// Block backward (step S6, 16-bit storage) as a warp-specialised tcgen05
+// pipeline.  For a tile of 128 consecutive grid points p:
+//     dz[p, o] = dy[p, o] GELU'(pre[p, o])
+//     dx[p, i] = sum_j basis[p, j] Udx[i, j] + sum_o dz[p, o] W[o, i]
+//     dW[o, i] += sum_p dz[p, o] x[p, i],  db[o] += sum_p dz[p, o]
+// Udx is the spectrum of dxhat inverted along the slab axis (the slab-axis
+// inverse kernel), basis the last-axis inverse basis of the forward.  The dx
+// chain is the forward epilogue's GEMM with dz in place of x and W^T in place
+// of W; the dW chain reads the x tile straight from the ring stage (TMA with
+// 128-byte swizzle, the K-major layout the tensor core reads) against dz^T,
+// which the staging warps write to shared memory, and accumulates in a TMEM
+// accumulator that persists over all tiles of the CTA.  Sixteen rows of ones
+// after the x rows make the last sixteen accumulator columns db.
+//
+//   warp 17       TMA producer: x (two 64-point boxes, swizzled), dy, pre and
+//                 the Udx rows of tile j into ring stage j % NS
+//   warps 0-7     staging: dz -> A (TMEM) and dz^T -> A_dW (shared memory);
+//                 Udx rows -> the spectral columns of the dx B operand
+//   warp 16       MMA issuer: both chains of tile j; one commit frees the ring
+//                 stage, another signals D_dx full and the A/B buffers free
+//   warps 8-15    epilogue: D_dx -> dx; at the end, D_dW -> per-CTA partials
+// ===========================================================================
+constexpr int BW_NCONV = 8, BW_NEPI = 8;
+constexpr int BW_WARP_MMA = BW_NCONV + BW_NEPI;   // 16
+constexpr int BW_WARP_TMA = BW_WARP_MMA + 1;      // 17
+constexpr int BW_THREADS = (BW_WARP_TMA + 1) * 32;
+constexpr int BW_MAX_STAGES = 4;
+constexpr int BW_XBOX = 64;                       // points per swizzled x box (128 bytes)
+
+struct BwdGeom {
+  int Rt, nvar, KS, KSp, KA, NW, NS, NAW;
+  int col_dw, col_spec, col_z, used_cols, cols, cs_cols;
+  uint32_t sbo, sbo_w, bytes_tx;
+  size_t xbox, x_off, dy_off, pre_off, u_off, stage, bbuf, abuf, b, aw, tw, bar, tbase, total;
+};
+
+// 16-bit storage only (eb = 2); requires Ci % 16 == 0 and Co % 16 == 0
+__host__ __device__ inline BwdGeom bwd_geom(const Geom &g, int Ci, int Co, bool act) {
+  BwdGeom e;
+  e.Rt = g.NL >= ROWS ? 1 : ROWS / g.NL;
+  e.nvar = g.NL >= ROWS ? g.NL / ROWS : 1;
+  e.KS = e.Rt * 2 * g.mL;
+  e.KSp = rup(e.KS, 16);
+  e.KA = e.KSp + Co;                       // K of the dx chain: spectral, then dz
+  e.NW = Ci + 16;                          // N of the dW chain: x rows, then ones
+  e.cs_cols = e.KSp / 2;
+  e.col_dw = 2 * Ci;                       // two D_dx buffers first
+  e.col_spec = e.col_dw + rup(e.NW, 16);
+  e.col_z = e.col_spec + e.nvar * e.cs_cols;
+  e.used_cols = e.col_z + 2 * (Co / 2);
+  e.cols = 32;
+  while (e.cols < e.used_cols && e.cols < 1024) e.cols *= 2;
+  e.sbo = (uint32_t)(e.KA * 2 / 16) * 128u;
+  e.sbo_w = (uint32_t)(ROWS * 2 / 16) * 128u;
+  e.xbox = (size_t)e.NW * 128;             // one swizzled box: NW rows of 128 bytes
+  e.x_off = 0;
+  e.dy_off = alg(e.x_off + 2 * e.xbox, 1024);
+  e.pre_off = alg(e.dy_off + (size_t)Co * ROWS * 2, 128);
+  e.u_off = alg(e.pre_off + (act ? (size_t)Co * ROWS * 2 : 0), 128);
+  e.stage = alg(e.u_off + (size_t)Ci * e.KS * 4, 1024);
+  e.bytes_tx = (uint32_t)(2 * (size_t)Ci * 128 + (size_t)Co * ROWS * 2 * (act ? 2 : 1) +
+                          (size_t)Ci * e.KS * 4);
+  e.bbuf = alg((size_t)Ci * e.KA * 2, 1024);
+  e.abuf = (size_t)ROWS * ROWS * 2;        // dz^T: 128 rows (o, zero past Co) x 128 points
+  const size_t fixed_base = 2 * e.bbuf + alg(sizeof(float2) * g.NL, 128) +
+                            sizeof(uint64_t) * (2 * BW_MAX_STAGES + 6) + 16;
+  size_t room2 = 232448 > fixed_base + 2 * e.abuf ? 232448 - fixed_base - 2 * e.abuf : 0;
+  e.NAW = room2 / e.stage >= 2 ? 2 : 1;
+  const size_t room = 232448 > fixed_base + e.NAW * e.abuf ? 232448 - fixed_base - e.NAW * e.abuf : 0;
+  const size_t ns = room / e.stage;
+  e.NS = (int)(ns < (size_t)BW_MAX_STAGES ? ns : (size_t)BW_MAX_STAGES);
+  size_t off = (size_t)(e.NS > 0 ? e.NS : 0) * e.stage;
+  e.b = off; off += 2 * e.bbuf;
+  e.aw = off; off += e.NAW * e.abuf;
+  e.tw = off; off = alg(off + sizeof(float2) * g.NL, 128);
+  e.bar = off; off += sizeof(uint64_t) * (2 * BW_MAX_STAGES + 6);
+  e.tbase = off; off += 16;
+  e.total = off < 116 * 1024 ? 116 * 1024 : off;
+  return e;
+}
+
+// K-major, 128-byte swizzle descriptor (8-row groups 1024 bytes apart): the
+// layout a TMA box with a 128-byte inner extent and 128-byte swizzle writes
+__device__ __forceinline__ uint64_t desc_sw128_b(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// the dW chain of one tile: 8 K steps of 16 points; A = dz^T (no swizzle,
+// 256 bytes per step), B = the x boxes (32 bytes per step inside a 128-byte
+// swizzle atom, four steps per box)
+__device__ __forceinline__ void issue_dw(uint32_t d, uint64_t adesc, uint64_t xdesc0,
+                                         uint64_t xdesc1, uint32_t idesc, bool acc_first) {
+#pragma unroll
+  for (int s = 0; s < ROWS / 16; ++s) {
+    const uint64_t bd = (s < 4 ? xdesc0 : xdesc1) + (uint64_t)(2 * (s & 3));
+    tc::mma_f16_ss(d, adesc + (uint64_t)(16 * s), bd, idesc, (acc_first || s > 0) ? 1u : 0u);
+  }
+}
+
+template <typename T, int CX>
+__global__ void __launch_bounds__(BW_THREADS, 1)
+    k_epi_bwd_pipe(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmdy,
+                   const __grid_constant__ CUtensorMap tmpre,
+                   const __grid_constant__ CUtensorMap tmu, PipeArgs a, float *partial, Geom g) {
+  using K = PKind<T>;
+  static_assert(!PKind<T>::tf32, "16-bit storage only");
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const int Ci = a.Ci, Co = a.Co;
+  const bool act = a.act != 0;
+  const BwdGeom e = bwd_geom(g, Ci, Co, act);
+  unsigned char *bbase = smem + e.b;
+  unsigned char *awbase = smem + e.aw;
+  float2 *twL = reinterpret_cast<float2 *>(smem + e.tw);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + e.bar);
+  uint64_t *empty = full + BW_MAX_STAGES;
+  uint64_t *aready = empty + BW_MAX_STAGES;
+  uint64_t *mdone = aready + 2;
+  uint64_t *dempty = mdone + 2;
+  uint32_t *tbase_s = reinterpret_cast<uint32_t *>(smem + e.tbase);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int NL = g.NL, mL = g.mL;
+  const long long SN = (long long)g.S * NL;
+
+  if (warp == 0) {
+    tc::tmem_alloc(tbase_s, e.cols);
+    tc::tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int s = 0; s < BW_MAX_STAGES; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);       // the tile's MMA commit
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&aready[i], BW_NCONV);
+      tc::mbar_init(&mdone[i], 1);
+      tc::mbar_init(&dempty[i], BW_NEPI);
+    }
+    tma::fence_barrier_init();
+  }
+  if (warp == BW_WARP_TMA && lane == 0) {
+    tma::prefetch_map(&tmx);
+    tma::prefetch_map(&tmdy);
+    if (act) tma::prefetch_map(&tmpre);
+    tma::prefetch_map(&tmu);
+  }
+  build_twiddles(twL, NL);
+  // zero the B buffers and the dz^T buffers (rows past Co stay zero); the ones
+  // rows after the x rows of every box of every stage (any swizzle of ones is
+  // ones)
+  for (size_t i = (size_t)tid * 16; i < 2 * e.bbuf + e.NAW * e.abuf; i += BW_THREADS * 16)
+    *reinterpret_cast<uint4 *>(bbase + i) = make_uint4(0, 0, 0, 0);
+  {
+    const uint32_t one2 = PKind<T>::fmt == tc::FMT_BF16 ? 0x3F803F80u : 0x3C003C00u;
+    const int per_box = 16 * 128 / 16;      // 16-byte chunks of the ones rows of one box
+    for (int i = tid; i < e.NS * 2 * per_box; i += BW_THREADS) {
+      const int sb = i / per_box, c = i - sb * per_box;
+      unsigned char *dst = smem + (size_t)(sb >> 1) * e.stage + e.x_off + (size_t)(sb & 1) * e.xbox +
+                           (size_t)Ci * 128 + (size_t)c * 16;
+      *reinterpret_cast<uint4 *>(dst) = make_uint4(one2, one2, one2, one2);
+    }
+  }
+  __syncthreads();
+  {  // W^T in columns [KSp, KSp + Co) of both B buffers: B[n = i][k = KSp + o] = W[o][i]
+    const T *W = reinterpret_cast<const T *>(a.W);
+    for (int idx = tid; idx < Co * Ci; idx += BW_THREADS) {
+      const int o = idx / Ci, i = idx - o * Ci;
+      const uint32_t off = boff(i, e.KSp + o, 2, e.sbo);
+      for (int nb = 0; nb < 2; ++nb) *reinterpret_cast<T *>(bbase + nb * e.bbuf + off) = W[idx];
+    }
+  }
+  tc::fence_proxy_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = *tbase_s;
+
+  const int tps = (int)(SN / ROWS);
+  const long long ntiles = g.B * g.O * tps;
+  const long long per_cta = (ntiles + gridDim.x - 1) / gridDim.x;
+  const long long t_begin = blockIdx.x * per_cta;
+  const long long t_end = t_begin + per_cta < ntiles ? t_begin + per_cta : ntiles;
+  const int ntl = t_begin < t_end ? (int)(t_end - t_begin) : 0;
+
+  if (warp == BW_WARP_TMA) {
+    // ---------------------------------------------------------- TMA producer
+    Cursor c = cursor_at(t_begin, tps, g);
+    int j = 0;
+    for (; j < ntl; ++j) {
+      const int s = j % e.NS;
+      const bool ok = j < e.NS || tc::mbar_wait(&empty[s], ((j / e.NS) - 1) & 1, a.err);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      if (lane == 0) {
+        unsigned char *st = smem + (size_t)s * e.stage;
+        const int p0 = c.row0 * NL + c.n0;
+        tma::arrive_expect_tx(&full[s], e.bytes_tx);
+        tma::load_4d(st + e.x_off, &tmx, &full[s], p0, c.outer, 0, (int)c.b);
+        tma::load_4d(st + e.x_off + e.xbox, &tmx, &full[s], p0 + BW_XBOX, c.outer, 0, (int)c.b);
+        tma::load_4d(st + e.dy_off, &tmdy, &full[s], p0, c.outer, 0, (int)c.b);
+        if (act) tma::load_4d(st + e.pre_off, &tmpre, &full[s], p0, c.outer, 0, (int)c.b);
+        tma::load_4d(st + e.u_off, &tmu, &full[s], c.row0 * 2 * mL, c.outer, 0, (int)c.b);
+      }
+      __syncwarp();
+      cursor_next(c, e.Rt, g);
+    }
+    for (int jj = j - 1; jj >= 0 && jj >= j - e.NS; --jj)
+      tc::mbar_wait(&full[jj % e.NS], (jj / e.NS) & 1, nullptr);
+  } else if (warp == BW_WARP_MMA) {
+    // ---------------------------------------------------------- MMA issuer
+    Cursor c = cursor_at(t_begin, tps, g);
+    const uint32_t idx_desc = tc::instr_desc(K::fmt, ROWS, Ci);
+    const uint32_t idw_desc = tc::instr_desc(K::fmt, ROWS, e.NW);
+    const int nss = e.KSp / 16, nzs = Co / 16;
+    int j = 0;
+    for (; j < ntl; ++j) {
+      bool ok = tc::mbar_wait(&aready[j & 1], (j >> 1) & 1, a.err);
+      if (ok && j >= 2) ok = tc::mbar_wait(&dempty[j & 1], ((j - 2) >> 1) & 1, a.err);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc::fence_after_sync();
+      const int s = j % e.NS;
+      const int variant = e.Rt > 1 ? 0 : c.n0 / ROWS;
+      if (tc::elect_one()) {
+        const uint32_t d = tbase + (uint32_t)((j & 1) * Ci);
+        const uint64_t bdesc =
+            tc::smem_desc_kmajor(tc::smem_u32(bbase + (j & 1) * e.bbuf), 128, e.sbo);
+        // dx: spectral steps (resident basis A, Udx columns of B), then dz steps
+        issue_steps<K>(d, tbase + e.col_spec + variant * e.cs_cols, 0u, bdesc, idx_desc, nss,
+                       false);
+        issue_steps<K>(d, tbase + e.col_z + (j & 1) * (Co / 2), 0u,
+                       bdesc + (uint64_t)(16 * nss), idx_desc, nzs, true);
+        // dW, db: A = dz^T, B = the stage's x boxes and ones rows
+        const unsigned char *xs = smem + (size_t)s * e.stage + e.x_off;
+        issue_dw(tbase + e.col_dw,
+                 tc::smem_desc_kmajor(tc::smem_u32(awbase + (j % e.NAW) * e.abuf), 128, e.sbo_w),
+                 desc_sw128_b(tc::smem_u32(xs)), desc_sw128_b(tc::smem_u32(xs + e.xbox)),
+                 idw_desc, j > 0);
+        tc::mma_commit(&empty[s]);
+        tc::mma_commit(&mdone[j & 1]);
+      }
+      __syncwarp();
+      cursor_next(c, e.Rt, g);
+    }
+    if (j > 0) tc::mbar_wait(&mdone[(j - 1) & 1], ((j - 1) >> 1) & 1, nullptr);
+  } else if (warp < BW_NCONV) {
+    // ---------------------------------------------------------- staging
+    const int t = tid & (ROWS - 1);
+    const int shalf = tid / ROWS;
+    const uint32_t arow = tbase + ((uint32_t)((warp & 3) * 32) << 16);
+    // resident spectral A per variant, as in the forward (16-bit: two per column)
+    for (int v = 0; v < (shalf == 0 ? e.nvar : 0); ++v) {
+      const int n = e.Rt > 1 ? t % NL : v * ROWS + t;
+      const int rl = e.Rt > 1 ? t / NL : 0;
+      const uint32_t c0v = arow + e.col_spec + v * e.cs_cols;
+      int r = 0, k = 0, par = 0, idx = 0;
+      for (int c0 = 0; c0 < e.KSp; c0 += 16) {
+        float vals[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float val = 0.f;
+          if (c0 + i < e.KS) {
+            if (r == rl) {
+              const float2 w = twL[idx];
+              val = par ? -w.y : w.x;
+            }
+            if (par) {
+              ++k;
+              idx += n;
+              if (idx >= NL) idx -= NL;
+              if (k == mL) {
+                k = 0;
+                ++r;
+                idx = 0;
+              }
+            }
+            par ^= 1;
+          }
+          vals[i] = val;
+        }
+        stage16<T>(c0v + c0 / 2, 0u, vals);
+      }
+    }
+    const int njb = e.KS / 4;                 // 16-byte chunks of one Udx row
+    const int nchunk = Ci * njb;
+    constexpr int NSTG = BW_NCONV * 32;
+    for (int j = 0; j < ntl; ++j) {
+      const int s = j % e.NS;
+      const int ab = j & 1, aw = j % e.NAW;
+      bool ok = tc::mbar_wait(&full[s], (j / e.NS) & 1, a.err);
+      // A_dz / B buffer ab were last read by tile j - 2; dz^T buffer aw by tile j - NAW
+      if (ok && j >= 2) ok = tc::mbar_wait(&mdone[ab], ((j - 2) >> 1) & 1, a.err);
+      if (ok && e.NAW == 1 && j >= 1)
+        ok = tc::mbar_wait(&mdone[(j - 1) & 1], ((j - 1) >> 1) & 1, a.err);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc::fence_after_sync();
+      const unsigned char *st = smem + (size_t)s * e.stage;
+      // Udx rows -> B[n = i][k < KS], chunks of four K values
+      {
+        const float *us = reinterpret_cast<const float *>(st + e.u_off);
+        unsigned char *bh = bbase + ab * e.bbuf;
+        for (int i = tid; i < nchunk; i += NSTG) {
+          const int o8 = i / (8 * njb), rem = i - o8 * 8 * njb;
+          const int ol = rem & 7, jrot = rem >> 3;
+          const int jb = (jrot + ol) % njb;
+          const int ch = o8 * 8 + ol;
+          const float4 v = *reinterpret_cast<const float4 *>(us + ch * e.KS + 4 * jb);
+          bstore4<T>(bh, 0, boff(ch, 4 * jb, 2, e.sbo), v);
+        }
+      }
+      // dz = dy GELU'(pre): this half's 16-channel groups -> A (TMEM) and dz^T
+      {
+        const T *dys = reinterpret_cast<const T *>(st + e.dy_off);
+        const T *prs = reinterpret_cast<const T *>(st + e.pre_off);
+        const uint32_t zc = arow + e.col_z + ab * (Co / 2);
+        unsigned char *awb = awbase + aw * e.abuf;
+#pragma unroll
+        for (int c0 = 0; c0 < CX; c0 += 16) {
+          if (c0 < Co && ((c0 >> 4) & 1) == shalf) {
+            float vals[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float d = to_f<T>(dys[(c0 + i) * ROWS + t]);
+              vals[i] = act ? d * gelu_grad_f(to_f<T>(prs[(c0 + i) * ROWS + t])) : d;
+            }
+            stage16<T>(zc + c0 / 2, 0u, vals);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              *reinterpret_cast<T *>(awb + boff(c0 + i, t, 2, e.sbo_w)) = from_f<T>(vals[i]);
+          }
+        }
+      }
+      tc::tmem_wait_st();
+      tc::fence_proxy_async_smem();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tma::arrive(&aready[ab]);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue
+    const int q = warp & 3, half = (warp - BW_NCONV) >> 2;
+    const int t = q * 32 + lane;
+    const uint32_t arow = tbase + ((uint32_t)(q * 32) << 16);
+    const long long cstride = (long long)g.O * SN;
+    T *out = reinterpret_cast<T *>(a.out);
+    Cursor c = cursor_at(t_begin, tps, g);
+    int j = 0;
+    for (; j < ntl; ++j) {
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&mdone[j & 1], (j >> 1) & 1, a.err))) break;
+      tc::fence_after_sync();
+      const uint32_t dcol = arow + (uint32_t)((j & 1) * Ci);
+      constexpr int GPH = CX / 32 > 0 ? CX / 32 : 1;
+      float v[GPH][16];
+#pragma unroll
+      for (int gi = 0; gi < GPH; ++gi) {
+        const int c0 = (2 * gi + half) * 16;
+        if (c0 < Ci) {
+          uint32_t dv[16];
+          tc::tmem_ld16(dcol + c0, dv);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[gi][i] = __uint_as_float(dv[i]);
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tma::arrive(&dempty[j & 1]);
+      const long long ob = (c.b * Ci * g.O + c.outer) * SN + (long long)c.row0 * NL + c.n0 + t;
+#pragma unroll
+      for (int gi = 0; gi < GPH; ++gi) {
+        const int c0 = (2 * gi + half) * 16;
+        if (c0 < Ci) {
+          T *op = out + ob + (long long)c0 * cstride;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            *op = from_f<T>(v[gi][i]);
+            op += cstride;
+          }
+        }
+      }
+      cursor_next(c, e.Rt, g);
+    }
+    // all of the CTA's MMAs are complete once the last tile's mdone has been
+    // seen (or there were none): D_dW row o = lane t -> partial[cta][o][0..Ci]
+    const bool all_seen = __all_sync(0xffffffffu, j == ntl);
+    tc::fence_after_sync();
+    float *dst = partial + (long long)blockIdx.x * Co * (Ci + 1);
+    const bool row = t < Co;
+    for (int c0 = half * 16; c0 < e.NW; c0 += 32) {
+      uint32_t dv[16];
+      tc::tmem_ld16(arow + e.col_dw + c0, dv);
+      tc::tmem_wait_ld();
+      if (row && all_seen) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int col = c0 + i;
+          const float val = ntl > 0 ? __uint_as_float(dv[i]) : 0.f;
+          if (col < Ci) dst[t * (Ci + 1) + col] = val;
+          else if (col == Ci) dst[t * (Ci + 1) + Ci] = val;
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tbase, e.cols);
+  }
+}
+
+template <typename T>
+cudaError_t launch_bwd_pipe_t(const Launch &L, const Geom &g, const PipeArgs &a, const void *x,
+                              const void *dy, const void *pre, const float2 *U, float *partial,
+                              int *nparts) {
+  using K = PKind<T>;
+  const bool act = a.act != 0;
+  const BwdGeom e = bwd_geom(g, a.Ci, a.Co, act);
+  const long long SN = (long long)g.S * g.NL;
+  CUtensorMap tmx, tmdy, tmpre, tmu;
+  memset(&tmx, 0, sizeof(tmx));
+  memset(&tmdy, 0, sizeof(tmdy));
+  memset(&tmpre, 0, sizeof(tmpre));
+  memset(&tmu, 0, sizeof(tmu));
+  {
+    const uint64_t dims[4] = {(uint64_t)SN, (uint64_t)g.O, (uint64_t)a.Ci, (uint64_t)g.B};
+    const uint64_t str[3] = {(uint64_t)SN * 2, (uint64_t)g.O * SN * 2,
+                             (uint64_t)a.Ci * g.O * SN * 2};
+    const uint32_t box[4] = {(uint32_t)BW_XBOX, 1u, (uint32_t)a.Ci, 1u};
+    if (!encode_tmap_4d(&tmx, K::tmap, x, dims, str, box, true)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[4] = {(uint64_t)SN, (uint64_t)g.O, (uint64_t)a.Co, (uint64_t)g.B};
+    const uint64_t str[3] = {(uint64_t)SN * 2, (uint64_t)g.O * SN * 2,
+                             (uint64_t)a.Co * g.O * SN * 2};
+    const uint32_t box[4] = {(uint32_t)ROWS, 1u, (uint32_t)a.Co, 1u};
+    if (!encode_tmap_4d(&tmdy, K::tmap, dy, dims, str, box)) return cudaErrorInvalidValue;
+    if (act && !encode_tmap_4d(&tmpre, K::tmap, pre, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t row = (uint64_t)g.S * 2 * g.mL;
+    const uint64_t dims[4] = {row, (uint64_t)g.O, (uint64_t)a.Ci, (uint64_t)g.B};
+    const uint64_t str[3] = {row * 4, (uint64_t)g.O * row * 4, (uint64_t)a.Ci * g.O * row * 4};
+    const uint32_t box[4] = {(uint32_t)e.KS, 1u, (uint32_t)a.Ci, 1u};
+    if (!encode_tmap_4d(&tmu, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, U, dims, str, box))
+      return cudaErrorInvalidValue;
+  }
+  const long long ntiles = g.B * g.O * (SN / ROWS);
+  const int grid = (int)(ntiles < L.num_sms ? ntiles : L.num_sms);
+  *nparts = grid;
+  auto go = [&](auto kern) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)e.total);
+    kern<<<grid, BW_THREADS, e.total, L.stream>>>(tmx, tmdy, tmpre, tmu, a, partial, g);
+  };
+  const int cmax = a.Co > a.Ci ? a.Co : a.Ci;
+  if (cmax <= 16) go(k_epi_bwd_pipe<T, 16>);
+  else if (cmax <= 32) go(k_epi_bwd_pipe<T, 32>);
+  else go(k_epi_bwd_pipe<T, 64>);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 bool epi_pipe_supported(const Geom &g, int dtype, int mode, int Ci, int Co, const void *x,
@@ -740,6 +1205,41 @@ cudaError_t launch_epi_pipe(const Launch &L, const Geom &g, int dtype, int mode,
     err = has_x ? launch_pipe_img<__nv_bfloat16, true>(L, g, a, ea.x, U)
                 : launch_pipe_img<__nv_bfloat16, false>(L, g, a, ea.x, U);
   launch_end(L, has_x ? "epi_block_fwd_pipe" : "epi_spec_pipe");
+  return err;
+}
+
+
+bool epi_bwd_pipe_supported(const Geom &g, int dtype, int Ci, int Co, int tanh_pre,
+                            const void *x, const void *dy, const void *pre, int act,
+                            const void *U) {
+  if (dtype == DT_F32 || tanh_pre || g.d < 2) return false;
+  if (Ci % 16 != 0 || Co % 16 != 0 || Ci > 64 || Co > 64) return false;
+  if (!(g.NL % ROWS == 0 || ROWS % g.NL == 0)) return false;
+  const long long SN = (long long)g.S * g.NL;
+  if (SN % ROWS != 0 || SN > (1LL << 30) || g.B > (1LL << 30)) return false;
+  const BwdGeom e = bwd_geom(g, Ci, Co, act != 0);
+  if (e.KS % 4 != 0 || e.KS > 256 || e.used_cols > 512) return false;
+  if (e.NS < 2 || e.total > kSmemMax) return false;
+  const uintptr_t al = reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy) |
+                       reinterpret_cast<uintptr_t>(U) | (act ? reinterpret_cast<uintptr_t>(pre) : 0);
+  return (al & 15) == 0;
+}
+
+cudaError_t launch_epi_bwd_pipe(const Launch &L, const Geom &g, int dtype, const EpiArgs &ea,
+                                const float2 *U, int *nparts) {
+  PipeArgs a{};
+  a.W = ea.W;
+  a.out = ea.out;
+  a.err = L.err;
+  a.Ci = ea.Ci;
+  a.Co = ea.Co;
+  a.act = ea.act;
+  launch_begin(L);
+  cudaError_t err = dtype == DT_F16
+                        ? launch_bwd_pipe_t<__half>(L, g, a, ea.x, ea.dy, ea.pre, U, ea.partial, nparts)
+                        : launch_bwd_pipe_t<__nv_bfloat16>(L, g, a, ea.x, ea.dy, ea.pre, U,
+                                                           ea.partial, nparts);
+  launch_end(L, "epi_block_bwd_pipe");
   return err;
 }
 

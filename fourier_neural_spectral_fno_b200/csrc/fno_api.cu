@@ -233,11 +233,22 @@ cudaError_t invert_slab(const Launch &L, const Geom &g, long long C, const float
 
 // u_ready: U (ws + w.u) already holds the spectrum inverted along the slab
 // axis (launch_spec_mid), so no slab-axis inverse is launched here.
+// nparts (block backward): the number of per-CTA dW / db partials written
 cudaError_t run_epilogue(const Launch &L, const Geom &g, int dtype, int mode, const EpiArgs &a,
-                         unsigned char *ws, const BlockWs &w, bool u_ready = false) {
+                         unsigned char *ws, const BlockWs &w, bool u_ready = false,
+                         int *nparts = nullptr) {
   float2 *U = reinterpret_cast<float2 *>(ws + w.u);
   // channels of the spectrum being inverted: Ci for the backward modes (dxhat)
   const int cs = (mode == EPI_SPEC_BWD || mode == EPI_BLOCK_BWD) ? a.Ci : a.Co;
+  if (nparts) *nparts = epi_grid(g, EPI_BLOCK_BWD, L.num_sms);
+  if (mode == EPI_BLOCK_BWD && nparts && (L.tc == 1 || L.tc == 3 || L.tc == 4) &&
+      epi_bwd_pipe_supported(g, dtype, a.Ci, a.Co, a.tanh_pre, a.x, a.dy, a.pre, a.act, U)) {
+    if (!u_ready) {
+      cudaError_t e = invert_slab(L, g, cs, a.Z, U);
+      if (e != cudaSuccess) return e;
+    }
+    return launch_epi_bwd_pipe(L, g, dtype, a, U, nparts);
+  }
   if ((L.tc == 1 || L.tc == 3 || L.tc == 4) && epi_pipe_supported(g, dtype, mode, a.Ci, a.Co, a.x, U)) {
     if (!u_ready) {
       cudaError_t e = invert_slab(L, g, cs, a.Z, U);
@@ -367,9 +378,11 @@ int run_backward(const Launch &L, const Geom &g, int dtype, unsigned flags, int 
   a.tanh_pre = (flags & FNO_TANH_PREACT) ? 1 : 0;
   float *partial = reinterpret_cast<float *>(ws + w.partial);
   a.partial = partial;
-  FNO_TRY(run_epilogue(L, g, dtype, block ? EPI_BLOCK_BWD : EPI_SPEC_BWD, a, ws, w), "epilogue");
+  int nparts = 0;
+  FNO_TRY(run_epilogue(L, g, dtype, block ? EPI_BLOCK_BWD : EPI_SPEC_BWD, a, ws, w, false,
+                       &nparts),
+          "epilogue");
   if (block) {
-    const int nparts = epi_grid(g, EPI_BLOCK_BWD, L.num_sms);
     FNO_TRY(launch_reduce_rows(L, partial, nparts, (long long)Co * (Ci + 1), 0, Co, Ci, dW, db),
             "dW/db reduction");
   }

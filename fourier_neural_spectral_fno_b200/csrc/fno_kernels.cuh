@@ -181,6 +181,15 @@ cudaError_t launch_epi_pipe(const Launch &L, const Geom &g, int dtype, int mode,
 // [Co, 2 Co)) by columns 2k (re), 2k + 1 (im), bias folded into column 0
 bool epi_img_supported(const Geom &g, int dtype, int mode, int Ci, int Co);
 size_t epi_img_row_bytes(int dtype, int Co, int mL);
+// warp-specialised tcgen05 block backward (EPI_BLOCK_BWD), 16-bit storage, no
+// tanh pre-activation, d >= 2, Ci and Co multiples of 16: dx, and per-CTA
+// partials of dW / db in a.partial ([*nparts][Co][Ci + 1]); U = dxhat inverted
+// along the slab axis ([B][Ci][O][S][mL] float2)
+bool epi_bwd_pipe_supported(const Geom &g, int dtype, int Ci, int Co, int tanh_pre,
+                            const void *x, const void *dy, const void *pre, int act,
+                            const void *U);
+cudaError_t launch_epi_bwd_pipe(const Launch &L, const Geom &g, int dtype, const EpiArgs &a,
+                                const float2 *U, int *nparts);
 size_t epi_partial_bytes(const Geom &g, int Ci, int Co, int num_sms);
 cudaError_t launch_epilogue(const Launch &L, const Geom &g, int dtype, int mode,
                             const EpiArgs &a);
