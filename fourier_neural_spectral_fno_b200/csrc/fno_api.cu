@@ -945,10 +945,18 @@ int fno_backward_ready(const fno_net_desc *desc, const void *a, const fno_params
   float *partial = reinterpret_cast<float *>(wsb + w.partial);
   void *dv[2] = {wsb + w.act0, wsb + w.act1};
 
-  FNO_TRY(launch_proj_bwd(L, g, desc->dtype, width, hidden, outc, sv + sm.vlast(nl), du,
-                          params->Q1, params->q1, params->Q2, dv[nl & 1], partial),
-          "projection backward");
-  const int np = proj_bwd_grid(g, L.num_sms);
+  int np = proj_bwd_grid(g, L.num_sms);
+  if ((L.tc == 1 || L.tc == 3 || L.tc == 4) &&
+      proj_bwd_pipe_supported(g, desc->dtype, width, hidden, outc, sv + sm.vlast(nl), du,
+                              dv[nl & 1])) {
+    FNO_TRY(launch_proj_bwd_pipe(L, g, desc->dtype, width, hidden, outc, sv + sm.vlast(nl), du,
+                                 params->Q1, params->q1, params->Q2, dv[nl & 1], partial, &np),
+            "projection backward");
+  } else {
+    FNO_TRY(launch_proj_bwd(L, g, desc->dtype, width, hidden, outc, sv + sm.vlast(nl), du,
+                            params->Q1, params->q1, params->Q2, dv[nl & 1], partial),
+            "projection backward");
+  }
   const long long pstride = (long long)proj_bwd_partial_floats(width, hidden, outc);
   FNO_TRY(launch_reduce_rows(L, partial, np, pstride, 0, hidden, width, grads->Q1, grads->q1),
           "dQ1 reduction");

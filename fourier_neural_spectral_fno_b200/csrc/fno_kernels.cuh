@@ -223,6 +223,14 @@ cudaError_t launch_proj_pipe(const Launch &L, const Geom &g, int dtype, int widt
 cudaError_t launch_proj_fwd_tc(const Launch &L, const Geom &g, int dtype, int width, int hidden,
                                int out_ch, const void *v, const void *Q1, const void *q1,
                                const void *Q2, const void *q2, void *u);
+// tcgen05 projection backward, 16-bit storage, width % 16 == 0, hidden <= 128:
+// dv, and per-CTA partials in the layout of launch_proj_bwd (*nparts of them)
+bool proj_bwd_pipe_supported(const Geom &g, int dtype, int width, int hidden, int out_ch,
+                             const void *v, const void *du, const void *dv);
+cudaError_t launch_proj_bwd_pipe(const Launch &L, const Geom &g, int dtype, int width, int hidden,
+                                 int out_ch, const void *v, const void *du, const void *Q1,
+                                 const void *q1, const void *Q2, void *dv, float *partial,
+                                 int *nparts);
 int proj_bwd_grid(const Geom &g, int num_sms);
 size_t proj_bwd_partial_floats(int width, int hidden, int out_ch);
 size_t proj_bwd_smem_bytes(int width, int hidden, int out_ch);

@@ -445,6 +445,500 @@ cudaError_t launch_t(const Launch &L, const Geom &g, const ProjArgs &a, const vo
   return cudaGetLastError();
 }
 
+// ===========================================================================
+// Projection backward (16-bit storage, hidden <= 128) as a tcgen05 pipeline.
+// For a tile of 128 consecutive points p of one sample:
+//   z = v Q1^T + q1, g = GELU(z), dh = (du Q2) GELU'(z)
+//   dv = dh Q1;  dQ1 += dh^T v, dq1 += sum dh;  dQ2 += du^T g, dq2 += sum du
+// Four MMA chains: (1) Z = v Q1^T (A = v staged into TMEM, B = Q1 resident),
+// (2) [dQ1 | dq1] += dh^T [v; 1] (A = dh^T in shared memory, B = the v tile
+// straight from the ring stage: TMA boxes with 128-byte swizzle followed by
+// sixteen rows of ones), (3) dv = dh Q1 (A = dh in TMEM, B = Q1^T resident,
+// written over the tile's Z buffer), (4) dQ2^T += g^T du (A = g^T, B = du).
+// The epilogue warps evaluate GELU and GELU' between chain (1) and the rest.
+//
+//   warp 21      TMA: v (two swizzled 64-point boxes) and du of tile j
+//   warps 0-3    staging: v -> A_v (TMEM), from the swizzled boxes
+//   warp 20      MMA: chain (1) of tile j, then chains (3), (2), (4) of j - 1
+//   warps 4-19   epilogue (four per TMEM lane quarter, a quarter of the hidden
+//                units each): z -> dh, g -> A_dh, dh^T, g^T, du; then dv of
+//                the previous tile from TMEM to global; at the end the dQ1 /
+//                dQ2 accumulators -> per-CTA partials
+// ===========================================================================
+constexpr int PB_STAGES = 4;
+constexpr int PB_XBOX = 64;
+
+struct PbGeom {
+  int Cw, HP, NWq, NS;
+  int col_z, col_av, col_ah, col_q1, col_q2, used, cols;
+  uint32_t sbo_q1, sbo_q1t, sbo_t, bytes_tx;
+  size_t xbox, du_off, stage, bq1, bq1t, adht, agt, bdu, q1s, q2s, dq2, bar, tbase, total;
+};
+
+__host__ __device__ inline PbGeom pb_geom(int width, int out_ch) {
+  PbGeom e;
+  e.Cw = width;                   // multiple of 16
+  e.HP = ROWS;                    // hidden padded to 128 (the M of chains 2 and 4)
+  e.NWq = width + 16;             // N of chain (2): v rows, then ones
+  e.col_z = 0;                    // two Z / dv buffers
+  e.col_av = 2 * e.HP;
+  e.col_ah = e.col_av + width;    // two A_v buffers of width / 2 columns
+  e.col_q1 = e.col_ah + e.HP / 2;
+  e.col_q2 = e.col_q1 + rup(e.NWq, 16);
+  e.used = e.col_q2 + 16;
+  e.cols = 32;
+  while (e.cols < e.used && e.cols < 1024) e.cols *= 2;
+  e.sbo_q1 = (uint32_t)(width * 2 / 16) * 128u;     // B of (1): rows h, K = c
+  e.sbo_q1t = (uint32_t)(e.HP * 2 / 16) * 128u;     // B of (3): rows c, K = h
+  e.sbo_t = (uint32_t)(ROWS * 2 / 16) * 128u;       // K = 128 points
+  e.xbox = (size_t)e.NWq * 128;
+  e.du_off = 2 * e.xbox;
+  e.stage = alg(e.du_off + (size_t)kMaxOut * ROWS * 2, 1024);
+  e.bytes_tx = (uint32_t)(2 * (size_t)width * 128 + (size_t)out_ch * ROWS * 2);
+  size_t off = 0;
+  const size_t fixed = alg((size_t)e.HP * width * 2, 1024) + alg((size_t)width * e.HP * 2, 1024) +
+                       2 * (size_t)ROWS * ROWS * 2 + (size_t)16 * ROWS * 2 +
+                       sizeof(float) * (e.HP + kMaxOut * e.HP + 8) +
+                       sizeof(uint64_t) * (2 * PB_STAGES + 12) + 16 + 1024;
+  const size_t room = kSmemMax > fixed ? kSmemMax - fixed : 0;
+  const size_t ns = room / e.stage;
+  e.NS = (int)(ns < (size_t)PB_STAGES ? ns : (size_t)PB_STAGES);
+  off = (size_t)(e.NS > 0 ? e.NS : 0) * e.stage;
+  e.bq1 = off; off = alg(off + (size_t)e.HP * width * 2, 1024);
+  e.bq1t = off; off = alg(off + (size_t)width * e.HP * 2, 1024);
+  e.adht = off; off += (size_t)ROWS * ROWS * 2;
+  e.agt = off; off += (size_t)ROWS * ROWS * 2;
+  e.bdu = off; off += (size_t)16 * ROWS * 2;
+  e.q1s = off; off += sizeof(float) * e.HP;
+  e.q2s = off; off += sizeof(float) * kMaxOut * e.HP;
+  e.dq2 = off; off += sizeof(float) * 8;
+  off = alg(off, 8);
+  e.bar = off; off += sizeof(uint64_t) * (2 * PB_STAGES + 12);
+  e.tbase = off; off += 16;
+  e.total = off < 116 * 1024 ? 116 * 1024 : off;
+  return e;
+}
+
+__device__ __forceinline__ uint64_t pb_desc_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// byte offset of element (row c, point pp < 64) in a 128-byte-swizzled box
+__device__ __forceinline__ uint32_t sw128_off(int c, int pp) {
+  const int byte = pp * 2;
+  return (uint32_t)(c * 128 + ((((byte >> 4) ^ (c & 7)) & 7) << 4) + (byte & 15));
+}
+
+template <typename T, int CX>
+__global__ void __launch_bounds__(THREADS, 1)
+    k_proj_bwd_pipe(const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdu,
+                    ProjArgs a, const void *du_unused, void *dv_out, float *partial) {
+  using K = QKind<T>;
+  static_assert(!QKind<T>::tf32, "16-bit storage only");
+  (void)du_unused;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const int width = a.width, hidden = a.hidden, out_ch = a.out_ch;
+  const PbGeom e = pb_geom(width, out_ch);
+  unsigned char *bq1 = smem + e.bq1;
+  unsigned char *bq1t = smem + e.bq1t;
+  unsigned char *adht = smem + e.adht;
+  unsigned char *agt = smem + e.agt;
+  unsigned char *bdu = smem + e.bdu;
+  float *q1s = reinterpret_cast<float *>(smem + e.q1s);
+  float *q2s = reinterpret_cast<float *>(smem + e.q2s);
+  float *dq2s = reinterpret_cast<float *>(smem + e.dq2);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + e.bar);
+  uint64_t *empty = full + PB_STAGES;
+  uint64_t *aready = empty + PB_STAGES;   // [2]
+  uint64_t *zdone = aready + 2;           // [2]
+  uint64_t *zfree = zdone + 2;            // [2]
+  uint64_t *hready = zfree + 2;           // [1]
+  uint64_t *hdone = hready + 1;           // [1]
+  uint64_t *fin = hdone + 1;              // [1]
+  uint32_t *tbase_s = reinterpret_cast<uint32_t *>(smem + e.tbase);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long N = a.N;
+
+  if (warp == 0) {
+    tc::tmem_alloc(tbase_s, e.cols);
+    tc::tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int s = 0; s < PB_STAGES; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&aready[i], NCONV);
+      tc::mbar_init(&zdone[i], 1);
+      tc::mbar_init(&zfree[i], NEPI);
+    }
+    tc::mbar_init(hready, NEPI);
+    tc::mbar_init(hdone, 1);
+    tc::mbar_init(fin, 1);
+    tma::fence_barrier_init();
+  }
+  if (warp == WARP_TMA && lane == 0) {
+    tma::prefetch_map(&tmv);
+    tma::prefetch_map(&tmdu);
+  }
+  // zero the resident operands (padded rows stay zero), ones rows of the boxes
+  for (size_t i = (size_t)tid * 16; i < e.q1s - e.bq1; i += THREADS * 16)
+    *reinterpret_cast<uint4 *>(bq1 + i) = make_uint4(0, 0, 0, 0);
+  {
+    const uint32_t one2 = QKind<T>::fmt == tc::FMT_BF16 ? 0x3F803F80u : 0x3C003C00u;
+    const int per_box = 16 * 128 / 16;
+    for (int i = tid; i < e.NS * 2 * per_box; i += THREADS) {
+      const int sb = i / per_box, c = i - sb * per_box;
+      unsigned char *dst = smem + (size_t)(sb >> 1) * e.stage + (size_t)(sb & 1) * e.xbox +
+                           (size_t)width * 128 + (size_t)c * 16;
+      *reinterpret_cast<uint4 *>(dst) = make_uint4(one2, one2, one2, one2);
+    }
+  }
+  __syncthreads();
+  {  // Q1 [hidden][width] -> B of (1) (rows h, K = c) and B of (3) (rows c, K = h)
+    const T *Q1 = reinterpret_cast<const T *>(a.Q1);
+    for (int i = tid; i < hidden * width; i += THREADS) {
+      const int h = i / width, c = i - h * width;
+      *reinterpret_cast<T *>(bq1 + boff(h, c, 2, e.sbo_q1)) = Q1[i];
+      *reinterpret_cast<T *>(bq1t + boff(c, h, 2, e.sbo_q1t)) = Q1[i];
+    }
+    const T *q1 = reinterpret_cast<const T *>(a.q1);
+    const T *Q2 = reinterpret_cast<const T *>(a.Q2);
+    for (int h = tid; h < e.HP; h += THREADS) q1s[h] = h < hidden ? to_f<T>(q1[h]) : 0.f;
+    for (int i = tid; i < kMaxOut * e.HP; i += THREADS) {
+      const int o = i / e.HP, h = i - o * e.HP;
+      q2s[i] = (o < out_ch && h < hidden) ? to_f<T>(Q2[o * hidden + h]) : 0.f;
+    }
+    if (tid < 8) dq2s[tid] = 0.f;
+  }
+  tc::fence_proxy_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = *tbase_s;
+
+  const long long tpb = N / ROWS;
+  const long long ntiles = a.B * tpb;
+  const long long per_cta = (ntiles + gridDim.x - 1) / gridDim.x;
+  const long long t_begin = blockIdx.x * per_cta;
+  const long long t_end = t_begin + per_cta < ntiles ? t_begin + per_cta : ntiles;
+  const int ntl = t_begin < t_end ? (int)(t_end - t_begin) : 0;
+
+  if (warp == WARP_TMA) {
+    // ------------------------------------------------------------ TMA producer
+    int j = 0;
+    for (; j < ntl; ++j) {
+      const int s = j % e.NS;
+      const bool w = j < e.NS || tc::mbar_wait(&empty[s], ((j / e.NS) - 1) & 1, a.err);
+      if (!__all_sync(0xffffffffu, w)) break;
+      if (lane == 0) {
+        const long long tile = t_begin + j;
+        const long long b = tile / tpb;
+        const int n0 = (int)((tile - b * tpb) * ROWS);
+        unsigned char *st = smem + (size_t)s * e.stage;
+        tma::arrive_expect_tx(&full[s], e.bytes_tx);
+        tma::load_4d(st, &tmv, &full[s], n0, 0, 0, (int)b);
+        tma::load_4d(st + e.xbox, &tmv, &full[s], n0 + PB_XBOX, 0, 0, (int)b);
+        tma::load_4d(st + e.du_off, &tmdu, &full[s], n0, 0, 0, (int)b);
+      }
+      __syncwarp();
+    }
+    for (int jj = j - 1; jj >= 0 && jj >= j - e.NS; --jj)
+      tc::mbar_wait(&full[jj % e.NS], (jj / e.NS) & 1, nullptr);
+  } else if (warp < NCONV) {
+    // ------------------------------------------------------------ staging
+    const int t = tid;
+    const uint32_t arow = tbase + ((uint32_t)(warp * 32) << 16);
+    const int box = t / PB_XBOX, pp = t - box * PB_XBOX;
+    for (int j = 0; j < ntl; ++j) {
+      const int s = j % e.NS;
+      bool w = tc::mbar_wait(&full[s], (j / e.NS) & 1, a.err);
+      if (w && j >= 2) w = tc::mbar_wait(&zdone[j & 1], ((j - 2) >> 1) & 1, a.err);
+      if (!__all_sync(0xffffffffu, w)) break;
+      tc::fence_after_sync();
+      const unsigned char *xs = smem + (size_t)s * e.stage + (size_t)box * e.xbox;
+      const uint32_t ac = arow + e.col_av + (j & 1) * (width / 2);
+#pragma unroll
+      for (int c0 = 0; c0 < CX; c0 += 16) {
+        if (c0 < width) {
+          float vals[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            vals[i] = to_f<T>(*reinterpret_cast<const T *>(xs + sw128_off(c0 + i, pp)));
+          stage16<T>(ac + c0 / 2, 0u, vals);
+        }
+      }
+      tc::tmem_wait_st();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tma::arrive(&aready[j & 1]);
+    }
+  } else if (warp == WARP_MMA) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t id1 = tc::instr_desc(K::fmt, ROWS, e.HP);
+    const uint32_t id3 = tc::instr_desc(K::fmt, ROWS, width);
+    const uint32_t id2 = tc::instr_desc(K::fmt, ROWS, e.NWq);
+    const uint32_t id4 = tc::instr_desc(K::fmt, ROWS, 16);
+    const uint64_t b1 = tc::smem_desc_kmajor(tc::smem_u32(bq1), 128, e.sbo_q1);
+    const uint64_t b3 = tc::smem_desc_kmajor(tc::smem_u32(bq1t), 128, e.sbo_q1t);
+    const uint64_t a2 = tc::smem_desc_kmajor(tc::smem_u32(adht), 128, e.sbo_t);
+    const uint64_t a4 = tc::smem_desc_kmajor(tc::smem_u32(agt), 128, e.sbo_t);
+    const uint64_t b4 = tc::smem_desc_kmajor(tc::smem_u32(bdu), 128, e.sbo_t);
+    const int n1 = width / 16;
+    // chains (3), (2), (4) of local tile jj
+    auto second = [&](int jj) -> bool {
+      const bool w = tc::mbar_wait(hready, jj & 1, a.err);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      tc::fence_after_sync();
+      if (tc::elect_one()) {
+        const uint32_t dz = tbase + e.col_z + (jj & 1) * e.HP;
+#pragma unroll
+        for (int k = 0; k < ROWS / 16; ++k)   // dv = dh Q1 (K = 128 hidden)
+          tc::mma_f16_ts(dz, tbase + e.col_ah + 8 * k, b3 + (uint64_t)(16 * k), id3,
+                         k > 0 ? 1u : 0u);
+        const unsigned char *xs = smem + (size_t)(jj % e.NS) * e.stage;
+        const uint64_t x0 = pb_desc_sw128(tc::smem_u32(xs)), x1 = pb_desc_sw128(tc::smem_u32(xs + e.xbox));
+#pragma unroll
+        for (int k = 0; k < ROWS / 16; ++k)   // [dQ1 | dq1] += dh^T [v; 1]
+          tc::mma_f16_ss(tbase + e.col_q1, a2 + (uint64_t)(16 * k),
+                         (k < 4 ? x0 : x1) + (uint64_t)(2 * (k & 3)), id2,
+                         (jj > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < ROWS / 16; ++k)   // dQ2^T += g^T du
+          tc::mma_f16_ss(tbase + e.col_q2, a4 + (uint64_t)(16 * k), b4 + (uint64_t)(16 * k), id4,
+                         (jj > 0 || k > 0) ? 1u : 0u);
+        tc::mma_commit(&empty[jj % e.NS]);
+        tc::mma_commit(hdone);
+      }
+      __syncwarp();
+      return true;
+    };
+    int j = 0;
+    bool ok = true;
+    for (; j < ntl && ok; ++j) {
+      bool w = tc::mbar_wait(&aready[j & 1], (j >> 1) & 1, a.err);
+      if (w && j >= 2) w = tc::mbar_wait(&zfree[j & 1], ((j - 2) >> 1) & 1, a.err);
+      if (!__all_sync(0xffffffffu, w)) break;
+      tc::fence_after_sync();
+      if (tc::elect_one()) {
+        const uint32_t dz = tbase + e.col_z + (j & 1) * e.HP;
+        const uint32_t av = tbase + e.col_av + (j & 1) * (width / 2);
+        switch (n1) {   // Z = v Q1^T (K = width)
+          case 4:
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              tc::mma_f16_ts(dz, av + 8 * k, b1 + (uint64_t)(16 * k), id1, k > 0 ? 1u : 0u);
+            break;
+          default:
+            for (int k = 0; k < n1; ++k)
+              tc::mma_f16_ts(dz, av + 8 * k, b1 + (uint64_t)(16 * k), id1, k > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(&zdone[j & 1]);
+      }
+      __syncwarp();
+      if (j >= 1) ok = second(j - 1);
+    }
+    if (ok && j == ntl && ntl > 0) ok = second(ntl - 1);
+    if (tc::elect_one()) tc::mma_commit(fin);
+    __syncwarp();
+    tc::mbar_wait(fin, 0, nullptr);
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3, part = (warp - NCONV) >> 2;
+    const int t = q * 32 + lane;
+    const uint32_t arow = tbase + ((uint32_t)(q * 32) << 16);
+    const int h0 = part * (e.HP / 4);          // 32 hidden units of this warp
+    const int cw = width / 4;                  // dv columns of this warp (multiple of 4)
+    T *dv = reinterpret_cast<T *>(dv_out);
+    float dq2acc[kMaxOut];
+#pragma unroll
+    for (int o = 0; o < kMaxOut; ++o) dq2acc[o] = 0.f;
+    // dv of local tile jj from its Z buffer to global, then the buffer is free
+    auto store_dv = [&](int jj) {
+      const long long tile = t_begin + jj;
+      const long long b = tile / tpb;
+      const long long n = (tile - b * tpb) * ROWS + t;
+      const uint32_t dcol = arow + e.col_z + (jj & 1) * e.HP + part * cw;
+      for (int c0 = 0; c0 < cw; c0 += 4) {
+        uint32_t dd[4];
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(dd[0]), "=r"(dd[1]), "=r"(dd[2]), "=r"(dd[3])
+                     : "r"(dcol + c0)
+                     : "memory");
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          dv[(b * width + part * cw + c0 + i) * N + n] = from_f<T>(__uint_as_float(dd[i]));
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tma::arrive(&zfree[jj & 1]);
+    };
+    int j = 0;
+    for (; j < ntl; ++j) {
+      if (!epi_all(tc::mbar_wait(&zdone[j & 1], (j >> 1) & 1, a.err))) break;
+      tc::fence_after_sync();
+      const int s = j % e.NS;
+      const T *dus = reinterpret_cast<const T *>(smem + (size_t)s * e.stage + e.du_off);
+      float du_t[kMaxOut];
+#pragma unroll
+      for (int o = 0; o < kMaxOut; ++o) du_t[o] = o < out_ch ? to_f<T>(dus[o * ROWS + t]) : 0.f;
+      // z of this warp's 32 hidden units -> g, dh
+      float gv[32], dhv[32];
+      {
+        uint32_t z0[16], z1[16];
+        const uint32_t zc = arow + e.col_z + (j & 1) * e.HP + h0;
+        tc::tmem_ld16(zc, z0);
+        tc::tmem_ld16(zc + 16, z1);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int h = h0 + i;
+          const float z = __uint_as_float(i < 16 ? z0[i] : z1[i - 16]) + q1s[h];
+          float gz, gp;
+          gelu_and_grad_f(z, gz, gp);
+          float dg = 0.f;
+#pragma unroll
+          for (int o = 0; o < kMaxOut; ++o)
+            if (o < out_ch) dg = fmaf(q2s[o * e.HP + h], du_t[o], dg);
+          gv[i] = gz;
+          dhv[i] = dg * gp;
+        }
+      }
+      // the previous tile's chains (2)-(4) are done with A_dh, dh^T, g^T, du
+      if (j >= 1 && !epi_all(tc::mbar_wait(hdone, (j - 1) & 1, a.err))) break;
+      tc::fence_after_sync();
+      {
+        const uint32_t ah = arow + e.col_ah + h0 / 2;
+        float v16[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v16[i] = dhv[i];
+        stage16<T>(ah, 0u, v16);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v16[i] = dhv[16 + i];
+        stage16<T>(ah + 8, 0u, v16);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          *reinterpret_cast<T *>(adht + boff(h0 + i, t, 2, e.sbo_t)) = from_f<T>(dhv[i]);
+          *reinterpret_cast<T *>(agt + boff(h0 + i, t, 2, e.sbo_t)) = from_f<T>(gv[i]);
+        }
+        if (part == 0) {
+#pragma unroll
+          for (int o = 0; o < kMaxOut; ++o) {
+            if (o < out_ch) {
+              *reinterpret_cast<T *>(bdu + boff(o, t, 2, e.sbo_t)) = from_f<T>(du_t[o]);
+              dq2acc[o] += du_t[o];
+            }
+          }
+        }
+      }
+      tc::tmem_wait_st();
+      tc::fence_proxy_async_smem();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tma::arrive(hready);
+      if (j >= 1) store_dv(j - 1);
+    }
+    const bool done_all = epi_all(j == ntl);
+    if (done_all && ntl > 0) {
+      if (epi_all(tc::mbar_wait(hdone, (ntl - 1) & 1, a.err))) {
+        tc::fence_after_sync();
+        store_dv(ntl - 1);
+      }
+    }
+    // dq2: warp sums of the part-0 warps into shared memory
+    if (part == 0) {
+#pragma unroll
+      for (int o = 0; o < kMaxOut; ++o) {
+        float v = dq2acc[o];
+        for (int m = 16; m > 0; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+        if (lane == 0 && o < out_ch) atomicAdd(&dq2s[o], v);
+      }
+    }
+    epi_sync();
+    tc::fence_after_sync();
+    // accumulators -> partials: row h = lane t of the quarter
+    float *dst = partial + (long long)blockIdx.x * (hidden * (width + 1) + out_ch * (hidden + 1));
+    const bool row = t < hidden && done_all;
+    for (int c0 = part * 16; c0 < e.NWq; c0 += 64) {
+      uint32_t dd[16];
+      tc::tmem_ld16(arow + e.col_q1 + c0, dd);
+      tc::tmem_wait_ld();
+      if (row) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int col = c0 + i;
+          const float val = ntl > 0 ? __uint_as_float(dd[i]) : 0.f;
+          if (col < width) dst[t * (width + 1) + col] = val;
+          else if (col == width) dst[t * (width + 1) + width] = val;
+        }
+      }
+    }
+    if (part == 1) {
+      uint32_t dd[16];
+      tc::tmem_ld16(arow + e.col_q2, dd);
+      tc::tmem_wait_ld();
+      if (row) {
+        float *d2 = dst + hidden * (width + 1);
+#pragma unroll
+        for (int o = 0; o < kMaxOut; ++o)
+          if (o < out_ch) d2[o * (hidden + 1) + t] = ntl > 0 ? __uint_as_float(dd[o]) : 0.f;
+      }
+    }
+    if (part == 2 && q == 0 && lane < out_ch) {
+      float *d2 = dst + hidden * (width + 1);
+      d2[lane * (hidden + 1) + hidden] = dq2s[lane];
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tbase, e.cols);
+  }
+}
+
+template <typename T>
+cudaError_t launch_proj_bwd_t(const Launch &L, const Geom &g, const ProjArgs &a, const void *v,
+                              const void *du, void *dv, float *partial, int *nparts) {
+  using K = QKind<T>;
+  const PbGeom e = pb_geom(a.width, a.out_ch);
+  CUtensorMap tmv, tmdu;
+  memset(&tmv, 0, sizeof(tmv));
+  memset(&tmdu, 0, sizeof(tmdu));
+  const uint64_t rowb = (uint64_t)g.N * 2;
+  {
+    const uint64_t dims[4] = {(uint64_t)g.N, 1u, (uint64_t)a.width, (uint64_t)g.B};
+    const uint64_t str[3] = {rowb, rowb, rowb * (uint64_t)a.width};
+    const uint32_t box[4] = {(uint32_t)PB_XBOX, 1u, (uint32_t)a.width, 1u};
+    if (!encode_tmap_4d(&tmv, K::tmap, v, dims, str, box, true)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[4] = {(uint64_t)g.N, 1u, (uint64_t)a.out_ch, (uint64_t)g.B};
+    const uint64_t str[3] = {rowb, rowb, rowb * (uint64_t)a.out_ch};
+    const uint32_t box[4] = {(uint32_t)ROWS, 1u, (uint32_t)a.out_ch, 1u};
+    if (!encode_tmap_4d(&tmdu, K::tmap, du, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  const long long ntiles = g.B * (g.N / ROWS);
+  const int grid = (int)(ntiles < L.num_sms ? ntiles : L.num_sms);
+  *nparts = grid;
+  auto go = [&](auto kern) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)e.total);
+    kern<<<grid, THREADS, e.total, L.stream>>>(tmv, tmdu, a, du, dv, partial);
+  };
+  if (a.width <= 16) go(k_proj_bwd_pipe<T, 16>);
+  else if (a.width <= 32) go(k_proj_bwd_pipe<T, 32>);
+  else go(k_proj_bwd_pipe<T, 64>);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 bool proj_pipe_supported(const Geom &g, int dtype, int width, int hidden, int out_ch,
@@ -478,6 +972,42 @@ cudaError_t launch_proj_pipe(const Launch &L, const Geom &g, int dtype, int widt
                     : dtype == DT_F16 ? launch_t<__half>(L, g, a, v)
                                       : launch_t<__nv_bfloat16>(L, g, a, v);
   launch_end(L, "proj_fwd_pipe");
+  return err;
+}
+
+
+bool proj_bwd_pipe_supported(const Geom &g, int dtype, int width, int hidden, int out_ch,
+                             const void *v, const void *du, const void *dv) {
+  if (dtype == DT_F32) return false;
+  if (g.N % ROWS != 0 || g.N > (1LL << 30) || g.B > (1LL << 30)) return false;
+  if (width % 16 != 0 || width > 64 || hidden < 1 || hidden > ROWS) return false;
+  if (out_ch < 1 || out_ch > kMaxOut) return false;
+  if (((reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(du) |
+        reinterpret_cast<uintptr_t>(dv)) & 15) != 0)
+    return false;
+  const PbGeom e = pb_geom(width, out_ch);
+  return e.used <= 512 && e.NS >= 2 && e.total <= kSmemMax;
+}
+
+cudaError_t launch_proj_bwd_pipe(const Launch &L, const Geom &g, int dtype, int width, int hidden,
+                                 int out_ch, const void *v, const void *du, const void *Q1,
+                                 const void *q1, const void *Q2, void *dv, float *partial,
+                                 int *nparts) {
+  ProjArgs a{};
+  a.Q1 = Q1;
+  a.q1 = q1;
+  a.Q2 = Q2;
+  a.err = L.err;
+  a.B = g.B;
+  a.N = g.N;
+  a.width = width;
+  a.hidden = hidden;
+  a.out_ch = out_ch;
+  launch_begin(L);
+  cudaError_t err = dtype == DT_F16
+                        ? launch_proj_bwd_t<__half>(L, g, a, v, du, dv, partial, nparts)
+                        : launch_proj_bwd_t<__nv_bfloat16>(L, g, a, v, du, dv, partial, nparts);
+  launch_end(L, "proj_bwd_pipe");
   return err;
 }
 
