@@ -698,17 +698,18 @@ cudaError_t launch_pipe_img(const Launch &L, const Geom &g, const PipeArgs &a, c
 // accumulator that persists over all tiles of the CTA.  Sixteen rows of ones
 // after the x rows make the last sixteen accumulator columns db.
 //
-//   warp 17       TMA producer: x (two 64-point boxes, swizzled), dy, pre and
+//   warp 25       TMA producer: x (two 64-point boxes, swizzled), dy, pre and
 //                 the Udx rows of tile j into ring stage j % NS
-//   warps 0-7     staging: dz -> A (TMEM) and dz^T -> A_dW (shared memory);
-//                 Udx rows -> the spectral columns of the dx B operand
-//   warp 16       MMA issuer: both chains of tile j; one commit frees the ring
+//   warps 0-15    staging, four per TMEM lane quarter, one 16-channel group
+//                 each: dz -> A (TMEM) and dz^T -> A_dW (shared memory); Udx
+//                 rows -> the spectral columns of the dx B operand
+//   warp 24       MMA issuer: both chains of tile j; one commit frees the ring
 //                 stage, another signals D_dx full and the A/B buffers free
-//   warps 8-15    epilogue: D_dx -> dx; at the end, D_dW -> per-CTA partials
+//   warps 16-23   epilogue: D_dx -> dx; at the end, D_dW -> per-CTA partials
 // ===========================================================================
-constexpr int BW_NCONV = 8, BW_NEPI = 8;
-constexpr int BW_WARP_MMA = BW_NCONV + BW_NEPI;   // 16
-constexpr int BW_WARP_TMA = BW_WARP_MMA + 1;      // 17
+constexpr int BW_NCONV = 16, BW_NEPI = 8;
+constexpr int BW_WARP_MMA = BW_NCONV + BW_NEPI;   // 24
+constexpr int BW_WARP_TMA = BW_WARP_MMA + 1;      // 25
 constexpr int BW_THREADS = (BW_WARP_TMA + 1) * 32;
 constexpr int BW_MAX_STAGES = 4;
 constexpr int BW_XBOX = 64;                       // points per swizzled x box (128 bytes)
@@ -935,10 +936,10 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
   } else if (warp < BW_NCONV) {
     // ---------------------------------------------------------- staging
     const int t = tid & (ROWS - 1);
-    const int shalf = tid / ROWS;
+    const int part = tid / ROWS;               // 16-channel groups part, part + 4, ..
     const uint32_t arow = tbase + ((uint32_t)((warp & 3) * 32) << 16);
     // resident spectral A per variant, as in the forward (16-bit: two per column)
-    for (int v = 0; v < (shalf == 0 ? e.nvar : 0); ++v) {
+    for (int v = 0; v < (part == 0 ? e.nvar : 0); ++v) {
       const int n = e.Rt > 1 ? t % NL : v * ROWS + t;
       const int rl = e.Rt > 1 ? t / NL : 0;
       const uint32_t c0v = arow + e.col_spec + v * e.cs_cols;
@@ -1005,12 +1006,19 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         unsigned char *awb = awbase + aw * e.abuf;
 #pragma unroll
         for (int c0 = 0; c0 < CX; c0 += 16) {
-          if (c0 < Co && ((c0 >> 4) & 1) == shalf) {
+          if (c0 < Co && ((c0 >> 4) & 3) == part) {
             float vals[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float d = to_f<T>(dys[(c0 + i) * ROWS + t]);
-              vals[i] = act ? d * gelu_grad_f(to_f<T>(prs[(c0 + i) * ROWS + t])) : d;
+            for (int i = 0; i < 16; ++i) vals[i] = to_f<T>(dys[(c0 + i) * ROWS + t]);
+            if (act) {
+#pragma unroll
+              for (int i = 0; i < 16; i += 2) {
+                float g0 = to_f<T>(prs[(c0 + i) * ROWS + t]);
+                float g1 = to_f<T>(prs[(c0 + i + 1) * ROWS + t]);
+                gelu_grad2(g0, g1);
+                vals[i] *= g0;
+                vals[i + 1] *= g1;
+              }
             }
             stage16<T>(zc + c0 / 2, 0u, vals);
 #pragma unroll

@@ -206,6 +206,41 @@ __device__ __forceinline__ void gelu2(float &a, float &b) {
   b = b >= 0.0f ? b - wb : wb;
 }
 
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// GELU'(p) = Phi(p) + p phi(p) of two values at once (the backward's dz), on
+// packed pairs: Phi as erfc_pos (q - 1 carried through the squarings, 1 / sqrt 2
+// folded into the coefficients), phi(p) = exp(-p^2 / 2) / sqrt(2 pi) as
+// 2^(-p^2 log2(e) / 2).
+__device__ __forceinline__ void gelu_grad2(float &a, float &b) {
+  const f32x2 p = f2pack(a, b);
+  const f32x2 t = f2pack(fabsf(a), fabsf(b));
+  f32x2 u = f2fma(f2splat(5.38297490493278e-06f), t, f2splat(4.889063711743802e-05f));
+  u = f2fma(u, t, f2splat(3.8003574445610866e-05f));
+  u = f2fma(u, t, f2splat(0.0032776263542473316f));
+  u = f2fma(u, t, f2splat(0.02114100567996502f));
+  u = f2fma(u, t, f2splat(0.04986734688282013f));
+  u = f2mul(u, t);
+  u = f2mul(u, f2add(u, f2splat(2.0f)));
+  u = f2mul(u, f2add(u, f2splat(2.0f)));
+  u = f2mul(u, f2add(u, f2splat(2.0f)));
+  u = f2mul(u, f2add(u, f2splat(2.0f)));
+  float qa, qb;
+  f2unpack(f2add(u, f2splat(1.0f)), qa, qb);
+  float ha, hb;                                   // Phi(-|p|) = erfc(|p| / sqrt 2) / 2
+  f2unpack(f2mul(f2pack(rcp_approx(qa), rcp_approx(qb)), f2splat(0.5f)), ha, hb);
+  float ea, eb;                                   // -p^2 log2(e) / 2
+  f2unpack(f2mul(f2mul(p, p), f2splat(-0.72134752044448170368f)), ea, eb);
+  const f32x2 phi =
+      f2mul(f2pack(ex2_approx(ea), ex2_approx(eb)), f2splat(0.39894228040143267794f));
+  const f32x2 cdf = f2pack(a >= 0.0f ? 1.0f - ha : ha, b >= 0.0f ? 1.0f - hb : hb);
+  f2unpack(f2fma(p, phi, cdf), a, b);
+}
+
 // weight c_k / N of last-axis mode k_l (1 on DC and Nyquist, else 2)
 __device__ __forceinline__ float mode_weight(int k_l, int n_l, float inv_n) {
   bool edge = (k_l == 0) || ((n_l % 2 == 0) && (2 * k_l == n_l));

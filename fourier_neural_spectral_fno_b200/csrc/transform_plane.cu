@@ -244,8 +244,9 @@ __global__ void __launch_bounds__(PL_THREADS, 1) k_fwd_plane(PlaneArgs a) {
             const TS *src1 = reinterpret_cast<const TS *>(st + (size_t)(RB + rl) * RS) + 2 * jj;
 #pragma unroll
             for (int t = 0; t < 16; ++t) {
-              const float2 p = valid ? ld_pair(src1 + t * Q) : make_float2(0.f, 0.f);
-              z[t] = make_float2(z[t].x * gelu_grad_f(p.x), z[t].y * gelu_grad_f(p.y));
+              float2 p = valid ? ld_pair(src1 + t * Q) : make_float2(0.f, 0.f);
+              gelu_grad2(p.x, p.y);
+              z[t] = make_float2(z[t].x * p.x, z[t].y * p.y);
             }
           } else if (a.tanh_in) {
 #pragma unroll
