@@ -120,3 +120,30 @@ def test_paired_gelu_in_float32():
     assert np.all(z == 0.0)
     assert np.abs(g[pd < -9.0]).max() < 1e-15
     np.testing.assert_allclose(g[pd > 9.0], pd[pd > 9.0], rtol=1e-7, atol=0)
+
+
+def _grad_constants():
+    body = open(HDR).read().split("void gelu_grad2(float &a, float &b)")[1].split("u = f2mul(u, t)")[0]
+    return [float(v) for v in re.findall(r"f2splat\((-?\d+\.\d+(?:e-?\d+)?)f\)", body)]
+
+
+def test_paired_gelu_grad_constants_match_the_paired_gelu():
+    """gelu_grad2 folds 1 / sqrt 2 into the printed constants exactly as gelu2."""
+    np.testing.assert_array_equal(F(_grad_constants()), F(_paired_constants()[:6]))
+
+
+def test_paired_gelu_grad_in_float32():
+    """GELU'(p) = Phi(p) + p phi(p), step by step as gelu_grad2: Phi through the
+    q - 1 form (the reciprocal rounded once), phi through 2^(-p^2 log2(e) / 2)
+    (the power of two evaluated exactly, then rounded, as ex2.approx is within
+    2^-22 of it)."""
+    c = _grad_constants()[::-1]           # lowest order first
+    p = np.linspace(-12.0, 12.0, 2_400_001).astype(F)
+    h = (F(0.5) * _erfc_pos_f32(np.abs(p), c)).astype(F)
+    cdf = np.where(p >= 0, (F(1) - h).astype(F), h)
+    ex = ((p * p).astype(F) * F(-0.72134752044448170368)).astype(F)
+    phi = (np.exp2(ex.astype(np.float64)).astype(F) * F(0.39894228040143267794)).astype(F)
+    got = (p.astype(np.float64) * phi + cdf).astype(F).astype(np.float64)
+    pd = p.astype(np.float64)
+    exact = 0.5 * erfc(-pd / np.sqrt(2.0)) + pd * np.exp(-0.5 * pd * pd) / np.sqrt(2.0 * np.pi)
+    assert np.abs(got - exact).max() < 4.0e-7
