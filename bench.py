@@ -222,6 +222,10 @@ def algorithmic_bytes(tag: str, wl) -> float:
     table["proj_bwd"] = 2 * act + 2 * wl.batch * wl.out_ch * wl.points * s
     table["fwd_transform_pipe"] = table["fwd_transform"]
     table["proj_fwd_pipe"] = table["proj_fwd"]
+    # tensor-core backward: read dy, pre, x and the slab-inverted dxhat rows
+    # ([B][C][rows][m_L] complex), write dx
+    table["epi_block_bwd_pipe"] = 4 * act + rows * wl.width * wl.modes[-1] * 8
+    table["proj_bwd_pipe"] = table["proj_bwd"]
     return float(table.get(tag, 0.0))
 
 
@@ -236,7 +240,8 @@ def kernel_source_sha(tag: str) -> str:
              "fwd_transform_tc_dz": "transform_tc.cu", "fwd_transform_dz": "transform.cu",
              "fwd_fft": "transform_fft.cu", "fwd_fft_dz": "transform_fft.cu",
              "fwd_plane": "transform_plane.cu", "fwd_plane_dz": "transform_plane.cu",
-             "inv_slab_img": "spec_mid.cu", "inv_slab_fft": "spec_mid.cu"}
+             "inv_slab_img": "spec_mid.cu", "inv_slab_fft": "spec_mid.cu",
+             "epi_block_bwd_pipe": "epilogue_pipe.cu", "proj_bwd_pipe": "proj_pipe.cu"}
     path = os.path.join(ROOT, "fourier_neural_spectral_fno_b200", "csrc", files.get(tag, ""))
     if not os.path.isfile(path):
         return ""

@@ -1,7 +1,8 @@
 """Record per-launch DRAM traffic of the library's kernels from an ncu capture.
 
-Reads the CSV that ``ncu -i <report> --page raw --csv`` prints (a capture that
-collected ``dram__bytes_read.sum`` and ``dram__bytes_write.sum``), averages the
+Reads the CSV that ``ncu -i <report> --page raw --csv`` prints, or the long
+form that ``ncu --metrics ... --csv --log-file`` writes during a run (either
+with ``dram__bytes_read.sum`` and ``dram__bytes_write.sum``), averages the
 launches of each kernel, and stores them in ``profiles/traffic.json`` under the
 workload name, keyed by the kernel's timing tag together with the hash of the
 source file it was built from (bench.py ignores a record whose source changed).
@@ -39,6 +40,13 @@ KERNELS = {
     "k_lift": ("lift", "net.cu"),
     "k_proj_bwd": ("proj_bwd", "net.cu"),
     "k_lift_bwd": ("lift_bwd", "net.cu"),
+    "k_fwd_fft": ("fwd_fft", "transform_fft.cu"),
+    "k_inv_slab_img": ("inv_slab_img", "spec_mid.cu"),
+    "k_inv_slab_fft": ("inv_slab_fft", "spec_mid.cu"),
+    "k_epi_bwd_pipe": ("epi_block_bwd_pipe", "epilogue_pipe.cu"),
+    "k_proj_bwd_pipe": ("proj_bwd_pipe", "proj_pipe.cu"),
+    "k_mix_bwd_dx": ("mix_bwd_dx", "mix.cu"),
+    "k_mix_bwd_dr": ("mix_bwd_dr", "mix.cu"),
 }
 
 # k_epilogue<T, MODE, ...>: the timing tag follows the epilogue mode
@@ -63,6 +71,10 @@ def _kernel_key(name: str):
     if not m:
         return None
     base, targs = m.group(1), m.group(2)
+    if base == "k_fwd_plane":   # k_fwd_plane<TS, T, MP, DZ>: the dz form has its own tag
+        args = [t.strip() for t in (targs or "").split(",")]
+        dz = bool(args) and args[-1] in ("true", "1")
+        return ("fwd_plane_dz" if dz else "fwd_plane", "transform_plane.cu")
     if base == "k_epilogue":
         args = [t.strip() for t in (targs or "").split(",")]
         tag = EPILOGUE_TAGS.get(args[1]) if len(args) > 1 else None
@@ -70,9 +82,41 @@ def _kernel_key(name: str):
     return KERNELS.get(base)
 
 
+def _parse_long(rows):
+    """The long form (one row per launch and metric) that a live run with
+    ``--metrics ... --csv --log-file`` writes."""
+    col = {h: i for i, h in enumerate(rows[0])}
+    per_launch = defaultdict(dict)
+    names = {}
+    for r in rows[1:]:
+        if len(r) != len(rows[0]):
+            continue
+        m = r[col["Metric Name"]]
+        if m not in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            continue
+        try:
+            v = float(r[col["Metric Value"]].replace(",", ""))
+        except ValueError:
+            continue
+        per_launch[r[col["ID"]]][m] = v * UNIT_SCALE.get(r[col["Metric Unit"]], 1.0)
+        names[r[col["ID"]]] = r[col["Kernel Name"]]
+    acc = defaultdict(lambda: [0.0, 0.0, 0])
+    for i, mets in per_launch.items():
+        key = _kernel_key(names[i])
+        if key is None or len(mets) != 2:
+            continue
+        a = acc[key]
+        a[0] += mets["dram__bytes_read.sum"]
+        a[1] += mets["dram__bytes_write.sum"]
+        a[2] += 1
+    return acc
+
+
 def parse(csv_path: str):
-    rows = list(csv.reader(open(csv_path)))
+    rows = [r for r in csv.reader(open(csv_path)) if r and not r[0].startswith("==")]
     hdr = rows[0]
+    if "Metric Name" in hdr:
+        return _parse_long(rows)
     col = {h: i for i, h in enumerate(hdr)}
     acc = defaultdict(lambda: [0.0, 0.0, 0])
     for r in rows[2:]:                       # row 1 holds the units
