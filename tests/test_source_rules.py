@@ -43,4 +43,6 @@ def test_no_deliberate_traps():
     for name, text in _sources().items():
         assert "__trap" not in text, name
         assert not re.search(r'asm[^;]*"\s*trap', text), name
-        assert "assert(" not in text, name
+        # device asserts (a failing one traps the kernel); static_assert is a
+        # compile-time check and cannot reach the GPU
+        assert not re.search(r"(?<!static_)\bassert\(", text), name
