@@ -549,26 +549,30 @@ def run_fno(args, dist):
               "in_ev": torch.cuda.Event(), "done_ev": torch.cuda.Event(),
               "out_ev": torch.cuda.Event()}
         slots.append(sl)
-    copy_stream = torch.cuda.Stream(device=dev)
+    h2d_stream = torch.cuda.Stream(device=dev)
+    d2h_stream = torch.cuda.Stream(device=dev)
 
     def e2e_step(i):
+        # inputs in on one copy stream, results out on another, so that step
+        # i + 1's input copy never queues behind step i's result copy (which
+        # waits for step i's compute)
         sl = slots[i & 1]
-        with torch.cuda.stream(copy_stream):
+        with torch.cuda.stream(h2d_stream):
             if i >= 2:
-                copy_stream.wait_event(sl["out_ev"])    # slot free: step i-2 fully done
+                h2d_stream.wait_event(sl["out_ev"])     # slot free: step i-2 fully done
             for t, h in zip(sl["ins"], ins_host):
                 t.copy_(h, non_blocking=True)
-            sl["in_ev"].record(copy_stream)
+            sl["in_ev"].record(h2d_stream)
         stream.wait_event(sl["in_ev"])
         if train:
             step(sl["ins"][0], sl["ins"][1], None, sl["out"])
         else:
             step(sl["ins"][0], None, sl["out"], None)
         sl["done_ev"].record(stream)
-        with torch.cuda.stream(copy_stream):
-            copy_stream.wait_event(sl["done_ev"])
+        with torch.cuda.stream(d2h_stream):
+            d2h_stream.wait_event(sl["done_ev"])
             sl["host"].copy_(sl["out"], non_blocking=True)
-            sl["out_ev"].record(copy_stream)
+            sl["out_ev"].record(d2h_stream)
 
     def host_read(i):
         sl = slots[i & 1]
@@ -582,19 +586,19 @@ def run_fno(args, dist):
     torch.cuda.synchronize()
     dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(copy_stream)
+    e0.record(h2d_stream)
     for i in range(e_steps):
         e2e_step(i)
         if i >= 1:
             host_read(i - 1)
     host_read(e_steps - 1)
-    e1.record(copy_stream)
+    e1.record(d2h_stream)
     torch.cuda.synchronize()
     e_ms = dist.max(e0.elapsed_time(e1) / e_steps)
     e2e = {"value": dist.world * wl.batch / (e_ms / 1e3), "unit": "samples/s",
            "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in ins),
            "d2h_bytes_per_step": out.numel() * out.element_size(), "ms_per_step": e_ms,
-           "copies": "pinned host buffers; H2D and D2H on a copy stream overlapping the "
+           "copies": "pinned host buffers; H2D and D2H on two copy streams overlapping the "
                      "neighbouring steps' compute (two buffer slots)"}
 
     clocks = clk.summary()
