@@ -2,10 +2,11 @@
 // HBM-streaming form of the pruned radix-16 FFT of transform_fft.cu.
 //
 // One persistent CTA per SM walks the (sample, channel[, outer]) planes.  A
-// producer warp streams the plane's rows into a shared-memory ring with
-// untiled bulk async copies (one per row, into rows padded so that the
-// consumers' reads are free of bank conflicts), signalled through
-// mbarrier transaction counts; fifteen consumer warps turn each batch of rows
+// producer warp streams the plane's rows into a shared-memory ring with one
+// untiled bulk async copy per batch of rows (the batch is contiguous in the
+// plane; measured, a copy per row left the consumers waiting a third of the
+// time on the copy engine), signalled through mbarrier transaction counts;
+// fifteen consumer warps turn each batch of rows
 // into last-axis spectra (the pruned FFT of transform_fft.cu: one register
 // FFT16 of a packed pair of real subsequences per thread, the real-pair
 // combine, a shuffle reduce-scatter over the row's threads) and keep them in
@@ -55,10 +56,8 @@ __host__ __device__ inline PlaneGeom plane_geom(int S, int NL, int mL, int QS, i
   p.MP = pl_mp(mL, p.T);
   p.Qs = S / 16;
   p.nin = nin;
-  // a row's 2T threads read 2T consecutive 8-byte (4-byte) pairs; the pad
-  // shifts consecutive rows onto the next banks
-  const int pad = es == 4 ? 16 * (p.T % 8) : (p.T == 1 ? 16 : 8 * p.T);
-  p.RS = NL * es + pad;
+  // rows dense, so a batch of rows is one contiguous bulk copy (per input)
+  p.RS = NL * es;
   p.stage = pl_al((size_t)nin * p.RB * p.RS, 128);
   const size_t x1 = sizeof(float2) * (size_t)S * (p.MP + 1);
   const size_t twc = sizeof(float2) * 4 * (size_t)p.MP * p.T;
@@ -206,10 +205,10 @@ __global__ void __launch_bounds__(PL_THREADS, 1) k_fwd_plane(PlaneArgs a) {
         __syncwarp();
         unsigned char *st = smem + (size_t)s * G.stage;
         const long long row0 = plane * S + (long long)b * RB;
-        for (int i = lane; i < rows; i += 32) {
-          tma::load_bulk(st + (size_t)i * RS, in0 + (row0 + i) * NL, (uint32_t)row_bytes, &full[s]);
+        if (lane == 0) {   // the batch's rows are contiguous in the plane
+          tma::load_bulk(st, in0 + row0 * NL, (uint32_t)(rows * row_bytes), &full[s]);
           if (DZ)
-            tma::load_bulk(st + (size_t)(RB + i) * RS, in1 + (row0 + i) * NL, (uint32_t)row_bytes,
+            tma::load_bulk(st + (size_t)RB * RS, in1 + row0 * NL, (uint32_t)(rows * row_bytes),
                            &full[s]);
         }
         __syncwarp();
