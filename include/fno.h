@@ -43,7 +43,11 @@
  * `stream` (NULL = legacy default stream) with no host synchronisation.  The
  * workspace is scratch device memory of at least fno_*workspace_size() bytes;
  * its contents on entry do not matter.  Gradient outputs are overwritten, not
- * accumulated.  Device pointers must be 16-byte aligned.
+ * accumulated.  Device pointers must be 16-byte aligned.  Because nothing is
+ * allocated and nothing synchronises, a sequence of calls on a capturing stream
+ * records into a CUDA graph (stream capture, relaxed mode) whose replays give
+ * the same results as the calls; the graph holds the pointers, so the buffers
+ * must stay in place.
  *
  * Errors: every call returns FNO_OK (0) or a negative FNO_ERR_* code and
  * leaves a message for fno_last_error() (thread-local).  Invalid descriptors,

@@ -362,3 +362,40 @@ def test_factorised_weights_backward(grid, modes, rank, dtype, flags):
     assert_close(host(outs[5]), dw_ref, TOL[dtype], "dW (block)")
     assert_close(host(outs[6]), db_ref, TOL[dtype], "db (block)")
     del torch
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_forward_replays_as_cuda_graph(dtype):
+    """The network forward allocates nothing and never synchronises, so it can be
+    captured into a CUDA graph: every replay equals the eager call bit for bit,
+    including after the input is rewritten in place (the graph reads the buffers,
+    not copies of them), and the replay matches the oracle."""
+    import torch
+    grid, modes = (256, 256), (16, 16)
+    wl, inp = _tiny_network(grid, modes, dtype, batch=2, width=32, hidden=128, layers=4, in_ch=3)
+    d = capi.net_desc(wl.batch, grid, modes, wl.in_ch, wl.width, wl.hidden, 1, wl.n_layers, dtype)
+    pd = params_to_device(inp["params"], dtype)    # kept alive: cp holds raw pointers
+    cp = capi.make_params(pd)
+    ws = torch.empty(capi.fno_net_workspace_size(d, capi.FNO_OP_NET_FWD), dtype=torch.uint8,
+                     device="cuda")
+    a_d = dev(inp["a"], dtype)
+    u_eager = empty((wl.batch, 1) + grid, dtype)
+    u_graph = empty((wl.batch, 1) + grid, dtype)
+    capi.fno_forward(d, a_d, cp, u_eager, None, ws, torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="relaxed"):
+        capi.fno_forward(d, a_d, cp, u_graph, None, ws, torch.cuda.current_stream())
+    for _ in range(2):
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(u_graph, u_eager)
+    a2 = np.random.default_rng(7).standard_normal(inp["a"].shape)
+    a2 = synth.quantize(a2, dtype)
+    a_d.copy_(dev(a2, dtype))
+    g.replay()
+    capi.fno_forward(d, a_d, cp, u_eager, None, ws, torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    assert torch.equal(u_graph, u_eager)
+    assert_close(host(u_graph), O.forward(a2, inp["params"], modes), TOL[dtype], "u")
