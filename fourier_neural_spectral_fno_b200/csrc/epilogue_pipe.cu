@@ -78,7 +78,7 @@ __host__ __device__ inline size_t alg(size_t v, size_t a) { return (v + a - 1) /
 // Shared memory: NS ring stages (x tile, U rows), NA B buffers (hi rows then
 // lo rows), the last-axis twiddles, the bias, mbarriers.
 struct PipeGeom {
-  int Rt, nvar, KS, KSp, KXp, KA, NP, DC, cs_cols, ax_cols;
+  int Rt, nvar, KS, KSp, KXp, KA, NP, DC, DA, cs_cols, ax_cols;
   int NA, NS, NB;
   int col_spec, col_x, used_cols, cols;
   uint32_t sbo, sbo_s, x_bytes, u_bytes;
@@ -97,10 +97,11 @@ __host__ __device__ inline PipeGeom pipe_geom(const Geom &g, bool has_x, int Ci,
   e.KXp = has_x ? rup(Ci, 16) : 0;
   e.KA = e.KSp + e.KXp;
   e.NP = rup(Co, 16);
-  e.DC = tf32 ? 2 * e.NP : e.NP;
+  e.DC = tf32 ? 2 * e.NP : e.NP;           // rows of B (tf32: hi rows, then lo rows)
+  e.DA = e.NP;                             // accumulator columns
   e.cs_cols = tf32 ? 2 * e.KSp : e.KSp / 2;
   e.ax_cols = tf32 ? 2 * e.KXp : e.KXp / 2;
-  e.col_spec = 2 * e.DC;
+  e.col_spec = 2 * e.DA;
   e.col_x = e.col_spec + e.nvar * e.cs_cols;
   e.NA = e.col_x + 2 * e.ax_cols <= 512 ? 2 : 1;
   e.used_cols = e.col_x + e.NA * e.ax_cols;
@@ -237,13 +238,14 @@ __device__ __forceinline__ void cursor_next(Cursor &c, int Rt, const Geom &g) {
 // step).  acc_first: the first step accumulates onto D as well.
 template <typename K, int NSTEP>
 __device__ __forceinline__ void issue_exact(uint32_t d, uint32_t a, uint32_t lo, uint64_t b,
-                                            uint32_t idesc, bool acc_first) {
+                                            uint64_t blo, uint32_t idesc, bool acc_first) {
 #pragma unroll
   for (int s = 0; s < NSTEP; ++s) {
     const uint32_t acc = (acc_first || s > 0) ? 1u : 0u;
-    if (K::tf32) {
+    if (K::tf32) {   // A_hi B_hi + A_lo B_hi + A_hi B_lo
       tc::mma_tf32_ts(d, a + 8 * s, b + (uint64_t)(16 * s), idesc, acc);
       tc::mma_tf32_ts(d, a + lo + 8 * s, b + (uint64_t)(16 * s), idesc, 1u);
+      tc::mma_tf32_ts(d, a + 8 * s, b + blo + (uint64_t)(16 * s), idesc, 1u);
     } else {
       tc::mma_f16_ts(d, a + 8 * s, b + (uint64_t)(16 * s), idesc, acc);
     }
@@ -254,22 +256,23 @@ __device__ __forceinline__ void issue_exact(uint32_t d, uint32_t a, uint32_t lo,
 // loop (no branch inside either)
 template <typename K>
 __device__ __forceinline__ void issue_steps(uint32_t d, uint32_t a, uint32_t lo, uint64_t b,
-                                            uint32_t idesc, int n, bool acc_first) {
+                                            uint64_t blo, uint32_t idesc, int n, bool acc_first) {
   switch (n) {
-    case 1: issue_exact<K, 1>(d, a, lo, b, idesc, acc_first); return;
-    case 2: issue_exact<K, 2>(d, a, lo, b, idesc, acc_first); return;
-    case 3: issue_exact<K, 3>(d, a, lo, b, idesc, acc_first); return;
-    case 4: issue_exact<K, 4>(d, a, lo, b, idesc, acc_first); return;
-    case 6: issue_exact<K, 6>(d, a, lo, b, idesc, acc_first); return;
-    case 8: issue_exact<K, 8>(d, a, lo, b, idesc, acc_first); return;
+    case 1: issue_exact<K, 1>(d, a, lo, b, blo, idesc, acc_first); return;
+    case 2: issue_exact<K, 2>(d, a, lo, b, blo, idesc, acc_first); return;
+    case 3: issue_exact<K, 3>(d, a, lo, b, blo, idesc, acc_first); return;
+    case 4: issue_exact<K, 4>(d, a, lo, b, blo, idesc, acc_first); return;
+    case 6: issue_exact<K, 6>(d, a, lo, b, blo, idesc, acc_first); return;
+    case 8: issue_exact<K, 8>(d, a, lo, b, blo, idesc, acc_first); return;
     default: break;
   }
   if (n <= 0) return;
-  issue_exact<K, 1>(d, a, lo, b, idesc, acc_first);
+  issue_exact<K, 1>(d, a, lo, b, blo, idesc, acc_first);
   for (int s = 1; s < n; ++s) {
     if (K::tf32) {
       tc::mma_tf32_ts(d, a + 8 * s, b + (uint64_t)(16 * s), idesc, 1u);
       tc::mma_tf32_ts(d, a + lo + 8 * s, b + (uint64_t)(16 * s), idesc, 1u);
+      tc::mma_tf32_ts(d, a + 8 * s, b + blo + (uint64_t)(16 * s), idesc, 1u);
     } else {
       tc::mma_f16_ts(d, a + 8 * s, b + (uint64_t)(16 * s), idesc, 1u);
     }
@@ -383,7 +386,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     // (the whole warp walks the loop and waits; lane 0 issues)
     {
       Cursor c = cursor_at(t_begin, tps, g);
-      const uint32_t idesc = tc::instr_desc(K::fmt, ROWS, e.DC);
+      const uint32_t idesc = tc::instr_desc(K::fmt, ROWS, e.DA);
+      // descriptor offset (16-byte units) of the lo rows of B: after the NP hi rows
+      const uint64_t blo_img = K::tf32 ? (uint64_t)(e.NP / 8) * e.sbo_s / 16 : 0;
+      const uint64_t blo_buf = K::tf32 ? (uint64_t)(e.bhalf / 16) : 0;
       const uint32_t lo_spec = K::tf32 ? (uint32_t)e.KSp : 0u;
       const uint32_t lo_x = K::tf32 ? (uint32_t)e.KXp : 0u;
       const int ns = e.KSp / K::KSTEP, nx = e.KXp / K::KSTEP;
@@ -400,11 +406,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc::fence_after_sync();
         const int variant = e.Rt > 1 ? 0 : c.n0 / ROWS;
         const int ab = e.NA == 2 ? (j & 1) : 0;
-        const uint32_t d = tbase + (uint32_t)((j & 1) * e.DC);
-        // one elected thread issues the tile's K steps (tf32: the A_hi and A_lo
-        // products of each K step, both against [B_hi; B_lo]); one K step
-        // advances B by 256 bytes (16 in descriptor units, no carry out of the
-        // 14-bit field) and A by 8 TMEM columns
+        const uint32_t d = tbase + (uint32_t)((j & 1) * e.DA);
+        // one elected thread issues the tile's K steps (tf32: A_hi B_hi, A_lo B_hi
+        // and A_hi B_lo of each K step into one accumulator of NP columns, so the
+        // epilogue reads one column set); one K step advances B by 256 bytes (16
+        // in descriptor units, no carry out of the 14-bit field) and A by 8 TMEM
+        // columns
         if (tc::elect_one()) {
           // IMG: the spectral steps read this tile's ring stage, the x steps W;
           // else both read the staged B buffer, the x steps after the spectral
@@ -413,9 +420,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                         tc::smem_u32(smem + (size_t)(j % e.NS) * e.stage + e.uoff), 128, e.sbo_s)
                   : (ab ? bdesc1 : bdesc0);
           const uint64_t bx = IMG ? bdesc0 : bspec + (uint64_t)(16 * ns);
-          issue_steps<K>(d, tbase + e.col_spec + variant * e.cs_cols, lo_spec, bspec, idesc, ns,
-                         false);
-          issue_steps<K>(d, tbase + e.col_x + ab * e.ax_cols, lo_x, bx, idesc, nx, true);
+          issue_steps<K>(d, tbase + e.col_spec + variant * e.cs_cols, lo_spec, bspec,
+                         IMG ? blo_img : blo_buf, idesc, ns, false);
+          issue_steps<K>(d, tbase + e.col_x + ab * e.ax_cols, lo_x, bx, blo_buf, idesc, nx, true);
           tc::mma_commit(&mdone[j & 1]);
         }
         __syncwarp();
@@ -574,7 +581,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!__all_sync(0xffffffffu, tc::mbar_wait(&mdone[j & 1], (j >> 1) & 1, a.err))) break;
       tc::fence_after_sync();
       if (IMG && lane == 0) tma::arrive(&empty[j % e.NS]);   // tile j's MMAs are done with it
-      const uint32_t dcol = arow + (uint32_t)((j & 1) * e.DC);
+      const uint32_t dcol = arow + (uint32_t)((j & 1) * e.DA);
       float v[GPH][16];
 #pragma unroll
       for (int gi = 0; gi < GPH; ++gi) {
@@ -582,20 +589,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (c0 < Co) {
           uint32_t dv[16];
           tc::tmem_ld16(dcol + c0, dv);
-          if (K::tf32) {   // A [B_hi; B_lo]: add the two column halves
-            uint32_t dl[16];
-            tc::tmem_ld16(dcol + e.NP + c0, dl);
-            tc::tmem_wait_ld();
+          tc::tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; i += 2)
-              f2unpack(f2add(f2pack(__uint_as_float(dv[i]), __uint_as_float(dv[i + 1])),
-                             f2pack(__uint_as_float(dl[i]), __uint_as_float(dl[i + 1]))),
-                       v[gi][i], v[gi][i + 1]);
-          } else {
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) v[gi][i] = __uint_as_float(dv[i]);
-          }
+          for (int i = 0; i < 16; ++i) v[gi][i] = __uint_as_float(dv[i]);
         }
       }
       tc::fence_before_sync();
@@ -916,10 +912,10 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         const uint64_t bdesc =
             tc::smem_desc_kmajor(tc::smem_u32(bbase + (j & 1) * e.bbuf), 128, e.sbo);
         // dx: spectral steps (resident basis A, Udx columns of B), then dz steps
-        issue_steps<K>(d, tbase + e.col_spec + variant * e.cs_cols, 0u, bdesc, idx_desc, nss,
-                       false);
+        issue_steps<K>(d, tbase + e.col_spec + variant * e.cs_cols, 0u, bdesc, 0u, idx_desc,
+                       nss, false);
         issue_steps<K>(d, tbase + e.col_z + (j & 1) * (Co / 2), 0u,
-                       bdesc + (uint64_t)(16 * nss), idx_desc, nzs, true);
+                       bdesc + (uint64_t)(16 * nss), 0u, idx_desc, nzs, true);
         // dW, db: A = dz^T, B = the stage's x boxes and ones rows
         const unsigned char *xs = smem + (size_t)s * e.stage + e.x_off;
         issue_dw(tbase + e.col_dw,
