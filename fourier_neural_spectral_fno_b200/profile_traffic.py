@@ -47,6 +47,9 @@ KERNELS = {
     "k_proj_bwd_pipe": ("proj_bwd_pipe", "proj_pipe.cu"),
     "k_mix_bwd_dx": ("mix_bwd_dx", "mix.cu"),
     "k_mix_bwd_dr": ("mix_bwd_dr", "mix.cu"),
+    "k_mix_fwd_1": ("mix_fwd", "mix.cu"),          # the small-shape forms
+    "k_mix_bwd_dx_1": ("mix_bwd_dx", "mix.cu"),
+    "k_mix_bwd_dr_1": ("mix_bwd_dr", "mix.cu"),
 }
 
 # k_epilogue<T, MODE, ...>: the timing tag follows the epilogue mode
