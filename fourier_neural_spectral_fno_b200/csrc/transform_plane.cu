@@ -2,9 +2,9 @@
 // HBM-streaming form of the pruned radix-16 FFT of transform_fft.cu.
 //
 // One persistent CTA per SM walks the (sample, channel[, outer]) planes.  A
-// producer warp streams the plane's rows into a shared-memory ring with one
-// untiled bulk async copy per batch of rows (the batch is contiguous in the
-// plane; measured, a copy per row left the consumers waiting a third of the
+// producer warp streams the plane's rows into a shared-memory ring with a few
+// untiled bulk async copies per batch of rows (one per group of 15 consecutive
+// rows; measured, a copy per row left the consumers waiting a third of the
 // time on the copy engine), signalled through mbarrier transaction counts;
 // fifteen consumer warps turn each batch of rows
 // into last-axis spectra (the pruned FFT of transform_fft.cu: one register
@@ -36,9 +36,16 @@ constexpr int PL_THREADS = PL_CONSUMERS + 32;   // + the producer warp
 constexpr int PL_MAXSTAGES = 4;
 constexpr size_t PL_SMEM_MAX = 227 * 1024;
 
+// A batch of RB = 15 G rows (G = rows per consumer warp) sits in G groups of 15
+// consecutive rows, one bulk copy each; warp w takes the rows w, w + 15, ...,
+// one per group, and the groups are GS = 15 RS + PADG bytes apart, PADG being
+// the bytes a row's threads read at once, so a warp's rows lie on successive
+// banks and its loads take the minimal number of wavefronts.
+constexpr int PL_WARPS = PL_CONSUMERS / 32;   // rows per group
+
 struct PlaneGeom {
-  int T, RB, MP, Qs, NS, nin, RS;
-  size_t stage, x1, twc, tw2, bar, total;
+  int T, RB, G, MP, Qs, NS, nin, RS;
+  size_t GS, stage, x1, twc, tw2, bar, total;
 };
 
 // modes padded so that the 2T threads of a row split them evenly
@@ -53,12 +60,13 @@ __host__ __device__ inline PlaneGeom plane_geom(int S, int NL, int mL, int QS, i
   PlaneGeom p{};
   p.T = NL / 64;
   p.RB = PL_CONSUMERS / (2 * p.T);
+  p.G = 32 / (2 * p.T);
   p.MP = pl_mp(mL, p.T);
   p.Qs = S / 16;
   p.nin = nin;
-  // rows dense, so a batch of rows is one contiguous bulk copy (per input)
-  p.RS = NL * es;
-  p.stage = pl_al((size_t)nin * p.RB * p.RS, 128);
+  p.RS = NL * es;                                  // rows dense within a group
+  p.GS = pl_al((size_t)PL_WARPS * p.RS + (size_t)(2 * p.T) * 2 * es, 16);   // copy alignment
+  p.stage = pl_al((size_t)nin * p.G * p.GS, 128);
   const size_t x1 = sizeof(float2) * (size_t)S * (p.MP + 1);
   const size_t twc = sizeof(float2) * 4 * (size_t)p.MP * p.T;
   const size_t tw2 = sizeof(float2) * (size_t)QS * p.Qs;
@@ -205,11 +213,15 @@ __global__ void __launch_bounds__(PL_THREADS, 1) k_fwd_plane(PlaneArgs a) {
         __syncwarp();
         unsigned char *st = smem + (size_t)s * G.stage;
         const long long row0 = plane * S + (long long)b * RB;
-        if (lane == 0) {   // the batch's rows are contiguous in the plane
-          tma::load_bulk(st, in0 + row0 * NL, (uint32_t)(rows * row_bytes), &full[s]);
+        // one copy per group of 15 consecutive rows (lane g: group g)
+        const int gr = min(PL_WARPS, rows - PL_WARPS * lane);   // rows of group `lane`
+        if (lane < G.G && gr > 0) {
+          const long long r0 = row0 + (long long)PL_WARPS * lane;
+          tma::load_bulk(st + (size_t)lane * G.GS, in0 + r0 * NL, (uint32_t)(gr * row_bytes),
+                         &full[s]);
           if (DZ)
-            tma::load_bulk(st + (size_t)RB * RS, in1 + row0 * NL, (uint32_t)(rows * row_bytes),
-                           &full[s]);
+            tma::load_bulk(st + (size_t)(G.G + lane) * G.GS, in1 + r0 * NL,
+                           (uint32_t)(gr * row_bytes), &full[s]);
         }
         __syncwarp();
       }
@@ -221,7 +233,9 @@ __global__ void __launch_bounds__(PL_THREADS, 1) k_fwd_plane(PlaneArgs a) {
     // ------------------------------------------------------------ consumers
     // thread (rl, jj) of a batch owns the subsequences r_u = 4 (jj / 2) + 2 (jj % 2)
     // and r_v = r_u + 1 of row rl: one complex FFT16 of the pair u + i v
-    const int rl = tid / T2, jj = tid - rl * T2;
+    const int grp = (tid & 31) / T2, jj = (tid & 31) - grp * T2;
+    const int rl = PL_WARPS * grp + (tid >> 5);          // row of the batch
+    const size_t row_off = (size_t)grp * G.GS + (size_t)(tid >> 5) * RS;
     const int Q = NL / 16;
     const float2 *twj = twc + 2 * jj;
     long long it = 0;
@@ -236,11 +250,12 @@ __global__ void __launch_bounds__(PL_THREADS, 1) k_fwd_plane(PlaneArgs a) {
         const unsigned char *st = smem + (size_t)s * G.stage;
         float2 z[16];
         {
-          const TS *src = reinterpret_cast<const TS *>(st + (size_t)rl * RS) + 2 * jj;
+          const TS *src = reinterpret_cast<const TS *>(st + row_off) + 2 * jj;
 #pragma unroll
           for (int t = 0; t < 16; ++t) z[t] = valid ? ld_pair(src + t * Q) : make_float2(0.f, 0.f);
           if (DZ) {
-            const TS *src1 = reinterpret_cast<const TS *>(st + (size_t)(RB + rl) * RS) + 2 * jj;
+            const TS *src1 =
+                reinterpret_cast<const TS *>(st + (size_t)G.G * G.GS + row_off) + 2 * jj;
 #pragma unroll
             for (int t = 0; t < 16; ++t) {
               float2 p = valid ? ld_pair(src1 + t * Q) : make_float2(0.f, 0.f);
