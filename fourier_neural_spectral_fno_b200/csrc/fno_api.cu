@@ -686,7 +686,7 @@ int fno_block_fwd(const fno_block_desc *desc, const void *x, const void *R, cons
   return rc;
 }
 
-static int check_cp(const fno_block_desc *desc, const Geom &g, int rank, const void *lam,
+static int check_cp(const fno_block_desc *desc, int rank, const void *lam,
                     const void *A, const void *B, const void *C) {
   if (rank < 1) return fail(FNO_ERR_INVALID_ARG, "rank %d < 1", rank);
   if (rank > kMaxCpRank)
@@ -697,7 +697,6 @@ static int check_cp(const fno_block_desc *desc, const Geom &g, int rank, const v
   REQUIRE_PTR(C, "C");
   const size_t smem = sizeof(float2) * (size_t)(desc->cin + desc->cout) * kMaxCpRank;
   if (smem > kSmemLimit) return fail(FNO_ERR_UNSUPPORTED, "factor staging needs %zu B", smem);
-  (void)g;
   return FNO_OK;
 }
 
@@ -708,7 +707,7 @@ int fno_spectral_conv_fwd_cp(const fno_block_desc *desc, int rank, const void *x
   int rc = check_block(desc, &g);
   if (rc) return rc;
   if ((rc = check_smem(g, desc->cin, desc->cout, FNO_OP_SPECTRAL_FWD))) return rc;
-  if ((rc = check_cp(desc, g, rank, lam, A, B, C))) return rc;
+  if ((rc = check_cp(desc, rank, lam, A, B, C))) return rc;
   REQUIRE_PTR(x, "x");
   REQUIRE_PTR(y, "y");
   OPTIONAL_PTR(xhat_save, "xhat_save");
@@ -731,7 +730,7 @@ int fno_block_fwd_cp(const fno_block_desc *desc, int rank, const void *x, const 
   int rc = check_block(desc, &g);
   if (rc) return rc;
   if ((rc = check_smem(g, desc->cin, desc->cout, FNO_OP_BLOCK_FWD))) return rc;
-  if ((rc = check_cp(desc, g, rank, lam, A, B, C))) return rc;
+  if ((rc = check_cp(desc, rank, lam, A, B, C))) return rc;
   REQUIRE_PTR(x, "x");
   REQUIRE_PTR(W, "W");
   REQUIRE_PTR(b, "b");
@@ -760,7 +759,7 @@ static int bwd_cp(const fno_block_desc *desc, int rank, const void *x, const voi
   const int op = block ? FNO_OP_BLOCK_BWD_CP : FNO_OP_SPECTRAL_BWD_CP;
   if ((rc = check_smem(g, desc->cin, desc->cout, block ? FNO_OP_BLOCK_BWD : FNO_OP_SPECTRAL_BWD)))
     return rc;
-  if ((rc = check_cp(desc, g, rank, lam, A, B, C))) return rc;
+  if ((rc = check_cp(desc, rank, lam, A, B, C))) return rc;
   REQUIRE_PTR(x, "x");
   REQUIRE_PTR(dy, "dy");
   REQUIRE_PTR(dx, "dx");
@@ -884,11 +883,9 @@ int fno_forward(const fno_net_desc *desc, const void *a, const fno_params *param
                      EPI_BLOCK_FWD);
     if (rc) return rc;
   }
-  const int launches = g_launches;
   FNO_TRY(launch_proj_fwd(L, g, desc->dtype, desc->width, desc->hidden, desc->out_channels,
                           act_buf(nl), params->Q1, params->q1, params->Q2, params->q2, u),
           "projection");
-  (void)launches;
   g_err[0] = 0;
   return FNO_OK;
 }

@@ -186,7 +186,9 @@ __device__ __forceinline__ f32x2 f2splat(float c) { return f2pack(c, c); }
 // w = (p / 2) erfc(|p| / sqrt 2) and GELU(p) = p - w (p >= 0) or w (p < 0).
 // The error of q^16 near p = 0 is scaled by p here: |GELU error| <= 4e-7
 // max(1, |p|) in float32.
-__device__ __forceinline__ void gelu2(float &a, float &b) {
+// (1 + a_1 t + ... + a_6 t^6)^16 of two |p| at once, the coefficients holding
+// the 1 / sqrt 2 of erf(p / sqrt 2)
+__device__ __forceinline__ void erf_q16(float a, float b, float &qa, float &qb) {
   const f32x2 t = f2pack(fabsf(a), fabsf(b));
   f32x2 q = f2fma(f2splat(5.38297490493278e-06f), t, f2splat(4.889063711743802e-05f));
   q = f2fma(q, t, f2splat(3.8003574445610866e-05f));
@@ -198,12 +200,27 @@ __device__ __forceinline__ void gelu2(float &a, float &b) {
   q = f2mul(q, q);
   q = f2mul(q, q);
   q = f2mul(q, q);
-  float qa, qb, wa, wb;
   f2unpack(q, qa, qb);
+}
+
+__device__ __forceinline__ void gelu2(float &a, float &b) {
+  float qa, qb, wa, wb;
+  erf_q16(a, b, qa, qb);
   f2unpack(f2mul(f2pack(rcp_approx(qa), rcp_approx(qb)), f2mul(f2pack(a, b), f2splat(0.5f))), wa,
            wb);
   a = a >= 0.0f ? a - wa : wa;
   b = b >= 0.0f ? b - wb : wb;
+}
+
+// 2 GELU of two values at once, for a caller that folds the 1/2 into its next
+// multiply: w = p erfc(|p| / sqrt 2), 2 GELU(p) = 2 p - w (p >= 0) or w (p < 0);
+// one multiply fewer than gelu2.
+__device__ __forceinline__ void gelu2_dbl(float &a, float &b) {
+  float qa, qb, wa, wb;
+  erf_q16(a, b, qa, qb);
+  f2unpack(f2mul(f2pack(rcp_approx(qa), rcp_approx(qb)), f2pack(a, b)), wa, wb);
+  a = a >= 0.0f ? fmaf(2.0f, a, -wa) : wa;
+  b = b >= 0.0f ? fmaf(2.0f, b, -wb) : wb;
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -220,17 +220,25 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   {  // B = Q1 [hidden][width] (head rows block, remainder block), q1, Q2
     const T *Q1 = reinterpret_cast<const T *>(a.Q1);
-    for (int i = tid; i < hidden * width; i += THREADS) {
-      const int h = i / width, c = i - h * width;
-      const float v = to_f<T>(Q1[i]);
-      const uint32_t o = boff(h, c, K::EB, e.sbo);
-      if (K::tf32) {
-        uint32_t hi, lo;
-        tc::split_tf32(v, hi, lo);
-        *reinterpret_cast<uint32_t *>(bsm + o) = hi;
-        *reinterpret_cast<uint32_t *>(bsm + e.bhalf + o) = lo;
-      } else {
-        *reinterpret_cast<T *>(bsm + o) = from_f<T>(v);
+    const int nq = hidden * width;
+    for (int i0 = tid; i0 < nq; i0 += 8 * THREADS) {   // eight loads in flight
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = i0 + u * THREADS < nq ? to_f<T>(Q1[i0 + u * THREADS]) : 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * THREADS;
+        if (i >= nq) break;
+        const int h = i / width, c = i - h * width;
+        const uint32_t o = boff(h, c, K::EB, e.sbo);
+        if (K::tf32) {
+          uint32_t hi, lo;
+          tc::split_tf32(v[u], hi, lo);
+          *reinterpret_cast<uint32_t *>(bsm + o) = hi;
+          *reinterpret_cast<uint32_t *>(bsm + e.bhalf + o) = lo;
+        } else {
+          *reinterpret_cast<T *>(bsm + o) = from_f<T>(v[u]);
+        }
       }
     }
     const T *q1 = reinterpret_cast<const T *>(a.q1);
@@ -238,7 +246,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int h = tid; h < e.HP; h += THREADS) q1s[h] = h < hidden ? to_f<T>(q1[h]) : 0.f;
     for (int i = tid; i < kMaxOut * e.HP; i += THREADS) {
       const int o = i / e.HP, h = i - o * e.HP;
-      q2s[i] = (o < out_ch && h < hidden) ? to_f<T>(Q2[o * hidden + h]) : 0.f;
+      q2s[i] = (o < out_ch && h < hidden) ? 0.5f * to_f<T>(Q2[o * hidden + h]) : 0.f;
     }
   }
   tc::fence_proxy_async_smem();
@@ -356,8 +364,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         float z1 = __uint_as_float(dv[i + 1]) + qa.y;
         float z2 = __uint_as_float(dv[i + 2]) + qa.z;
         float z3 = __uint_as_float(dv[i + 3]) + qa.w;
-        gelu2(z0, z1);
-        gelu2(z2, z3);
+        gelu2_dbl(z0, z1);   // 2 GELU: q2s holds Q2 / 2
+        gelu2_dbl(z2, z3);
 #pragma unroll
         for (int o = 0; o < kMaxOut; ++o) {
           if (o < out_ch) {
@@ -538,10 +546,9 @@ __device__ __forceinline__ uint32_t sw128_off(int c, int pp) {
 template <typename T, int CX>
 __global__ void __launch_bounds__(THREADS, 1)
     k_proj_bwd_pipe(const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdu,
-                    ProjArgs a, const void *du_unused, void *dv_out, float *partial) {
+                    ProjArgs a, void *dv_out, float *partial) {
   using K = QKind<T>;
   static_assert(!QKind<T>::tf32, "16-bit storage only");
-  (void)du_unused;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int width = a.width, hidden = a.hidden, out_ch = a.out_ch;
   const PbGeom e = pb_geom(width, out_ch);
@@ -931,7 +938,7 @@ cudaError_t launch_proj_bwd_t(const Launch &L, const Geom &g, const ProjArgs &a,
   *nparts = grid;
   auto go = [&](auto kern) {
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)e.total);
-    kern<<<grid, THREADS, e.total, L.stream>>>(tmv, tmdu, a, du, dv, partial);
+    kern<<<grid, THREADS, e.total, L.stream>>>(tmv, tmdu, a, dv, partial);
   };
   if (a.width <= 16) go(k_proj_bwd_pipe<T, 16>);
   else if (a.width <= 32) go(k_proj_bwd_pipe<T, 32>);

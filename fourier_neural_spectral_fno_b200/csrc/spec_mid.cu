@@ -26,6 +26,7 @@ namespace {
 
 constexpr int IS_THREADS = 256;
 constexpr int SM_MAXQS = 64;
+constexpr int IS_FILL = 16;     // loads in flight per thread while filling shared memory
 
 // hi = x rounded to tf32 (nearest), lo = x - hi rounded to tf32: the
 // operand split of the float32 tensor-core path
@@ -60,7 +61,15 @@ __global__ void __launch_bounds__(IS_THREADS)
   const size_t slab = blockIdx.x;
   const int tid = threadIdx.x;
   const float2 *src = yhat + slab * QS * mL;
-  for (int e = tid; e < QS * mL; e += IS_THREADS) ys[e] = __ldg(src + e);
+  for (int e0 = tid; e0 < QS * mL; e0 += IS_FILL * IS_THREADS) {   // IS_FILL loads in flight
+    float2 v[IS_FILL];
+#pragma unroll
+    for (int u = 0; u < IS_FILL; ++u)
+      if (e0 + u * IS_THREADS < QS * mL) v[u] = __ldg(src + e0 + u * IS_THREADS);
+#pragma unroll
+    for (int u = 0; u < IS_FILL; ++u)
+      if (e0 + u * IS_THREADS < QS * mL) ys[e0 + u * IS_THREADS] = v[u];
+  }
   for (int e = tid; e < QS * Qp; e += IS_THREADS) {   // exp(+2 pi i kq(slot) r / S)
     const int slot = e / Qp, rr = e - slot * Qp;
     float sn, cs;
@@ -98,33 +107,50 @@ __global__ void __launch_bounds__(IS_THREADS)
 
 // The same inverse writing the epilogue's B images: a CTA owns eight
 // consecutive output channels (one 8-row group of the operand's core matrices)
-// and a quarter of the r's, and thread t takes channel t % 8 and mode
+// and a range of the r's, and thread t takes channel t % 8 and mode
 // (t / 8) % mL, so that the sixteen-byte rows of the core matrices of one grid
 // row leave a warp as one contiguous 256-byte store (the (re, im) pairs of two
-// modes of eight channels).  IMG 1: float32 images (tf32 high parts in rows
-// [0, Co), low parts in [Co, 2 Co)); 2 / 3: float16 / bfloat16 images; the
-// bias is folded into column 0.
-constexpr int IMG_RSPLIT = 4;
+// modes of eight channels); the grid's y dimension splits the r's.  IMG 1:
+// float32 images (tf32 high parts in rows [0, Co), low parts in [Co, 2 Co));
+// 2 / 3: float16 / bfloat16 images; the bias is folded into column 0.
+constexpr int IMG_RSPLIT = 4;   // r ranges per (sample, channel group)
 template <int NDM, bool FULL, int IMG, typename TB>
 __global__ void __launch_bounds__(IS_THREADS)
     k_inv_slab_img(const float2 *__restrict__ yhat, unsigned char *__restrict__ img, const TB *__restrict__ bias, int S, int mS,
                    int QS, int mL, int Co) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int Qp = S / 16;
-  float2 *ys = reinterpret_cast<float2 *>(smem);      // [slot][k][8 channels]
-  float2 *twr = ys + (size_t)QS * mL * 8;              // [slot][Qp]
+  const int nsk = QS * mL, ysl = nsk + 4;                // padded channel rows
+  float2 *ys = reinterpret_cast<float2 *>(smem);      // [8 channels][slot][k]
+  float2 *twr = ys + (size_t)8 * ysl;                  // [slot][Qp]
   const int groups = Co / 8;
   const int b = blockIdx.x / groups, o0 = (blockIdx.x - b * groups) * 8;
   const int tid = threadIdx.x;
-  for (int e = tid; e < 8 * QS * mL; e += IS_THREADS) {
-    const int oo = e / (QS * mL), sk = e - oo * (QS * mL);
-    ys[sk * 8 + oo] = __ldg(yhat + ((size_t)b * Co + o0 + oo) * QS * mL + sk);
+  // sixteen loads in flight per thread before their stores; consecutive
+  // threads take consecutive (slot, k), so the stores meet no bank conflict
+  const float2 *src = yhat + ((size_t)b * Co + o0) * nsk;
+  for (int s0 = tid; s0 < nsk; s0 += 2 * IS_THREADS) {
+    float2 v[2][8];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        if (s0 + h * IS_THREADS < nsk) v[h][c] = __ldg(src + (size_t)c * nsk + s0 + h * IS_THREADS);
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        if (s0 + h * IS_THREADS < nsk) ys[c * ysl + s0 + h * IS_THREADS] = v[h][c];
   }
-  for (int e = tid; e < QS * Qp; e += IS_THREADS) {
-    const int slot = e / Qp, rr = e - slot * Qp;
+  const int rchunk = (Qp + (int)gridDim.y - 1) / (int)gridDim.y;
+  const int r_lo = blockIdx.y * rchunk;
+  const int r_hi = min(Qp, r_lo + rchunk);
+  const int rn = r_hi - r_lo;
+  for (int e = tid; e < QS * rn; e += IS_THREADS) {   // this CTA's r only
+    const int slot = e / rn, rr = r_lo + (e - slot * rn);
     float sn, cs;
     sincospif(2.0f * (float)mulmod(kept_k(slot, mS, S), rr, S) / (float)S, &sn, &cs);
-    twr[e] = make_float2(cs, sn);
+    twr[slot * Qp + rr] = make_float2(cs, sn);
   }
   __syncthreads();
   constexpr int EB = IMG == 1 ? 4 : 2;
@@ -134,9 +160,7 @@ __global__ void __launch_bounds__(IS_THREADS)
   const int o = o0 + oo;
   const float bias_o = bias ? to_f<TB>(bias[o]) : 0.f;
   const int per_r = 8 * mL;
-  const int r_lo = blockIdx.y * ((Qp + IMG_RSPLIT - 1) / IMG_RSPLIT);
-  const int r_hi = min(Qp, r_lo + (Qp + IMG_RSPLIT - 1) / IMG_RSPLIT);
-  for (int task = tid; task < (r_hi - r_lo) * per_r; task += IS_THREADS) {
+  for (int task = tid; task < rn * per_r; task += IS_THREADS) {
     const int r = r_lo + task / per_r, k = (task / 8) % mL;
     float2 v[16];
 #pragma unroll
@@ -147,7 +171,7 @@ __global__ void __launch_bounds__(IS_THREADS)
         const int kq = p + 16 * d;
         if (FULL || (kq >= -mS && kq < mS)) {
           const int slot = kq >= 0 ? kq : kq + QS;
-          cfma(acc, ys[(slot * mL + k) * 8 + oo], twr[slot * Qp + r]);
+          cfma(acc, ys[oo * ysl + slot * mL + k], twr[slot * Qp + r]);
         }
       }
       v[p] = acc;
@@ -205,10 +229,15 @@ cudaError_t launch_inv_slab_fft(const Launch &L, const Geom &g, long long C, con
   return e;
 }
 
+// shared memory of k_inv_slab_img: eight padded channel rows of the slab
+// spectrum, then the twiddle table
+inline size_t img_smem(const Geom &g) {
+  return sizeof(float2) * ((size_t)8 * (g.QS * g.mL + 4) + (size_t)g.QS * (g.S / 16));
+}
+
 bool spec_mid_img_supported(const Geom &g, int Co) {
   if (Co % 8 != 0) return false;
-  const size_t smem = sizeof(float2) * ((size_t)8 * g.QS * g.mL + (size_t)g.QS * (g.S / 16));
-  return smem <= 200 * 1024;
+  return img_smem(g) <= 200 * 1024;
 }
 
 bool spec_mid_supported(const Geom &g, int Ci, int Co) {
@@ -242,9 +271,8 @@ cudaError_t launch_spec_mid(const Launch &L, const Geom &g, int dtype, int Ci, i
     else if (g.mS > 16) e = go2(k_inv_slab_fft<2, false>);
     else e = go2(k_inv_slab_fft<1, false>);
   } else {
-    const size_t smem3 =
-        sizeof(float2) * ((size_t)8 * g.QS * g.mL + (size_t)g.QS * (g.S / 16));
-    dim3 grid3((unsigned)(g.B * (Co / 8)), IMG_RSPLIT);
+    const size_t smem3 = img_smem(g);
+    dim3 grid3((unsigned)(g.B * (Co / 8)), (unsigned)(g.S / 16 < IMG_RSPLIT ? g.S / 16 : IMG_RSPLIT));
     auto go3 = [&](auto kern, const auto *bp) {
       cudaError_t e3 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             (int)smem3);

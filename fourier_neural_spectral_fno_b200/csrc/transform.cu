@@ -308,7 +308,6 @@ cudaError_t launch_fwd_slab(const Launch &L, const Geom &g, int dtype, int load_
   const size_t smem = fwd_slab_smem(g.S, g.NL, g.mL, g.QS);
   dim3 grid((unsigned)planes, (unsigned)nb);
   cudaError_t err;
-  (void)tiles;
   launch_begin(L);
   if (dtype == DT_F32)
     err = launch_fwd_slab_t<float>(L, load_mode, grid, smem, args);

@@ -27,7 +27,7 @@ def _compiled_constants():
 
 
 def _paired_constants():
-    body = open(HDR).read().split("void gelu2(float &a, float &b)")[1].split("f2unpack(q")[0]
+    body = open(HDR).read().split("void erf_q16(")[1].split("f2unpack(q")[0]
     return [float(v) for v in re.findall(r"f2splat\((-?\d+\.\d+(?:e-?\d+)?)f\)", body)]
 
 
@@ -120,6 +120,21 @@ def test_paired_gelu_in_float32():
     assert np.all(z == 0.0)
     assert np.abs(g[pd < -9.0]).max() < 1e-15
     np.testing.assert_allclose(g[pd > 9.0], pd[pd > 9.0], rtol=1e-7, atol=0)
+
+
+def test_doubled_paired_gelu_in_float32():
+    """gelu2_dbl (the projection's activation, whose caller halves Q2): 2 GELU as
+    2 p - p r or p r, step by step in float32."""
+    c = _paired_constants()[:6][::-1]
+    p = np.linspace(-12.0, 12.0, 2_400_001).astype(F)
+    r = _erfc_f32(np.abs(p), c)
+    w = (r * p).astype(F)
+    g2 = np.where(p >= 0, (F(2) * p - w).astype(F), w).astype(np.float64)
+    pd = p.astype(np.float64)
+    exact = pd * erfc(-pd / np.sqrt(2.0))
+    assert (np.abs(g2 - exact) / np.maximum(np.abs(pd), 1.0)).max() < 8.0e-7
+    body = open(HDR).read().split("void gelu2_dbl(float &a, float &b)")[1].split("}")[0]
+    assert "erf_q16(a, b, qa, qb)" in body and "fmaf(2.0f, a, -wa)" in body
 
 
 def _grad_constants():
