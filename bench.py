@@ -229,6 +229,8 @@ def algorithmic_bytes(tag: str, wl) -> float:
     # ([B][C][rows][m_L] complex), write dx
     table["epi_block_bwd_pipe"] = 4 * act + rows * wl.width * wl.modes[-1] * 8
     table["proj_bwd_pipe"] = table["proj_bwd"]
+    table["mix_fwd_tc"] = table["mix_fwd"]          # read spectrum and R, write spectrum
+    table["mix_bwd_dx"] = table["mix_bwd_dx_tc"] = table["mix_fwd"]
     return float(table.get(tag, 0.0))
 
 
@@ -244,7 +246,8 @@ def kernel_source_sha(tag: str) -> str:
              "fwd_fft": "transform_fft.cu", "fwd_fft_dz": "transform_fft.cu",
              "fwd_plane": "transform_plane.cu", "fwd_plane_dz": "transform_plane.cu",
              "inv_slab_img": "spec_mid.cu", "inv_slab_fft": "spec_mid.cu",
-             "epi_block_bwd_pipe": "epilogue_pipe.cu", "proj_bwd_pipe": "proj_pipe.cu"}
+             "epi_block_bwd_pipe": "epilogue_pipe.cu", "proj_bwd_pipe": "proj_pipe.cu",
+             "mix_fwd_tc": "mix_tc.cu", "mix_bwd_dx_tc": "mix_tc.cu"}
     path = os.path.join(ROOT, "fourier_neural_spectral_fno_b200", "csrc", files.get(tag, ""))
     if not os.path.isfile(path):
         return ""

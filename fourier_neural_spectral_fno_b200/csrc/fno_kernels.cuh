@@ -127,6 +127,12 @@ cudaError_t launch_cp_grads(const Launch &L, const Geom &g, int dtype, int Ci, i
 
 // ---- mixing (S3) -----------------------------------------------------------
 // yhat[b,o,k] = (c_k / N) sum_i xhat[b,i,k] R[i,o,k]
+// tcgen05 mixing (mix_tc.cu): bfloat16 weights, 64 output channels (Co for
+// the forward, Ci for the adjoint dxhat), batch <= 64, K a multiple of 4
+bool mix_tc_supported(const Geom &g, int dtype, bool adj, int Ci, int Co, const void *X,
+                      const void *R, const void *Y);
+cudaError_t launch_mix_tc(const Launch &L, const Geom &g, bool adj, int Ci, int Co,
+                          const float2 *X, const void *R, float2 *Y);
 cudaError_t launch_mix_fwd(const Launch &L, const Geom &g, int dtype, int Ci, int Co,
                            const float2 *xhat, const void *R, float2 *yhat);
 // dR[i,o,k] = sum_b conj(xhat[b,i,k]) (c_k/N) D[b,o,k]

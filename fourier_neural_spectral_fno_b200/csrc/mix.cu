@@ -1,4 +1,6 @@
-// Per-mode complex channel mixing (step S3) and its two adjoints.
+// Per-mode complex channel mixing (step S3) and its two adjoints on the CUDA
+// cores (the tensor-core form for bfloat16 weights at 64 channels is in
+// mix_tc.cu and is taken where it applies).
 //
 // For every kept mode k the block multiplies the batch of spectra
 // xhat[:, :, k] (B x Ci) by the mode's weight matrix R[:, :, k] (Ci x Co).
@@ -268,9 +270,12 @@ cudaError_t mix_dx_small(const Launch &L, const Geom &g, int Ci, int Co, const f
 cudaError_t launch_mix_fwd(const Launch &L, const Geom &g, int dtype, int Ci, int Co,
                            const float2 *xhat, const void *R, float2 *yhat) {
   const bool big = big_tiles(g.K, Co, g.B, L.num_sms);
+  const bool tc = L.tc != 0 && L.tc != 2 && mix_tc_supported(g, dtype, false, Ci, Co, xhat, R, yhat);
   launch_begin(L);
   cudaError_t e;
-  if (dtype == DT_F32)
+  if (tc)
+    e = launch_mix_tc(L, g, false, Ci, Co, xhat, R, yhat);
+  else if (dtype == DT_F32)
     e = big ? mix_fwd_t<float, 4, 8>(L, g, Ci, Co, xhat, R, yhat)
             : mix_fwd_small<float>(L, g, Ci, Co, xhat, R, yhat);
   else if (dtype == DT_F16)
@@ -279,7 +284,7 @@ cudaError_t launch_mix_fwd(const Launch &L, const Geom &g, int dtype, int Ci, in
   else
     e = big ? mix_fwd_t<__nv_bfloat16, 4, 8>(L, g, Ci, Co, xhat, R, yhat)
             : mix_fwd_small<__nv_bfloat16>(L, g, Ci, Co, xhat, R, yhat);
-  launch_end(L, "mix_fwd");
+  launch_end(L, tc ? "mix_fwd_tc" : "mix_fwd");
   return e;
 }
 
@@ -304,9 +309,12 @@ cudaError_t launch_mix_bwd_dr(const Launch &L, const Geom &g, int Ci, int Co, co
 cudaError_t launch_mix_bwd_dx(const Launch &L, const Geom &g, int dtype, int Ci, int Co,
                               const float2 *D, const void *R, float2 *dxhat) {
   const bool big = big_tiles(g.K, Ci, g.B, L.num_sms);
+  const bool tc = L.tc != 0 && L.tc != 2 && mix_tc_supported(g, dtype, true, Ci, Co, D, R, dxhat);
   launch_begin(L);
   cudaError_t e;
-  if (dtype == DT_F32)
+  if (tc)
+    e = launch_mix_tc(L, g, true, Ci, Co, D, R, dxhat);
+  else if (dtype == DT_F32)
     e = big ? mix_dx_t<float, 4, 8>(L, g, Ci, Co, D, R, dxhat)
             : mix_dx_small<float>(L, g, Ci, Co, D, R, dxhat);
   else if (dtype == DT_F16)
@@ -315,7 +323,7 @@ cudaError_t launch_mix_bwd_dx(const Launch &L, const Geom &g, int dtype, int Ci,
   else
     e = big ? mix_dx_t<__nv_bfloat16, 4, 8>(L, g, Ci, Co, D, R, dxhat)
             : mix_dx_small<__nv_bfloat16>(L, g, Ci, Co, D, R, dxhat);
-  launch_end(L, "mix_bwd_dx");
+  launch_end(L, tc ? "mix_bwd_dx_tc" : "mix_bwd_dx");
   return e;
 }
 

@@ -1,0 +1,309 @@
+// Per-mode complex channel mixing (step S3) on the tensor cores, for bfloat16
+// weights and 64 output channels: the forward yhat = w_k R^T xhat and the
+// input adjoint dxhat = w_k conj(R) D as one real GEMM per mode.
+//
+// For a mode k, write the complex reduction  Y[b, n] = sum_r X[b, r] A_k(n, r)
+// in real form: with K index 2 r + c' (c' = 0 real, 1 imaginary part of X)
+// and row index 2 n + c (c = 0 real, 1 imaginary part of Y),
+//     D[2n + c, b] = sum_{r, c'} Ablk[2n + c, 2r + c'] X[b, 2r + c']
+// where each 2 x 2 block of Ablk is the real matrix of multiplication by
+//     forward:  A(n, r) = R[r, n]         ( Rr  -Ri )   rows 2n, 2n + 1
+//                                        ( Ri   Rr )
+//     adjoint:  A(n, r) = conj R[n, r]    ( Rr   Ri )
+//                                        (-Ri   Rr )
+// M = 2 x 64 = 128 rows (TMEM lanes), N = the batch (padded to a multiple of
+// 16 with zero rows), K = 2 x (reduced channels).  The weights are bfloat16
+// and enter exactly; X (float32 spectra) enters as a bfloat16 pair hi + lo
+// (hi = X rounded, lo = X - hi rounded), two MMA chains into one fp32
+// accumulator, so the products keep about 16 mantissa bits of X.
+//
+// One CTA per MB (4 or 2) consecutive modes, K a multiple of 4: all threads
+// gather the modes' operands from global memory into shared memory in the
+// tcgen05 K-major core-matrix layout (R as one load of the MB modes' (re, im)
+// pairs per (i, o), X as 16-byte loads of the MB modes), one elected thread
+// issues the chains, every thread waits on
+// the commit (bounded), and the eight warps read the accumulators back: warp w
+// takes TMEM lane quarter w % 4 (32 rows = 16 output channels, real and
+// imaginary in neighbouring lanes) and half of the batch columns; each thread
+// writes, per batch entry, the MB modes of one output channel as 32 contiguous
+// bytes, scaled by the inverse transform's c_k / N.
+#include "fno_common.cuh"
+#include "fno_kernels.cuh"
+#include "tc_util.cuh"
+#include "tma_util.cuh"
+
+namespace fno {
+
+namespace {
+
+constexpr int MT_THREADS = 256;
+constexpr int MT_ROWS = 128;                 // 2 x 64 output channels
+constexpr size_t MT_SMEM_MAX = 227 * 1024;
+
+struct MtGeom {
+  int NB;            // batch padded to a multiple of 16 (the MMA's N)
+  uint32_t sbo;      // bytes between 8-row groups (K = 2 NR bf16 per row)
+  size_t a_bytes, b_bytes, a0, b0, bar, tslot, total;
+  uint32_t cols;     // TMEM columns allocated (power of two >= MB NB)
+};
+
+__host__ __device__ inline MtGeom mt_geom(long long B, int NR, int MB) {
+  MtGeom e;
+  e.NB = (int)((B + 15) / 16 * 16);
+  e.sbo = (uint32_t)(2 * NR * 2 / 16) * 128u;
+  e.a_bytes = (size_t)MT_ROWS * 2 * NR * 2;
+  e.b_bytes = (size_t)e.NB * 2 * NR * 2;
+  e.a0 = 0;
+  e.b0 = e.a0 + (size_t)MB * e.a_bytes;
+  e.bar = e.b0 + (size_t)MB * 2 * e.b_bytes;
+  e.tslot = e.bar + 8;
+  e.total = e.tslot + 8;
+  uint32_t c = 32;
+  while (c < (uint32_t)(MB * e.NB)) c *= 2;
+  e.cols = c;
+  return e;
+}
+
+// byte offset of element (row, kel) of a K-major no-swizzle bf16 operand
+__device__ __forceinline__ uint32_t mt_off(int row, int kel, uint32_t sbo) {
+  const int kb = kel * 2;
+  return (uint32_t)(row >> 3) * sbo + (uint32_t)(kb >> 4) * 128u + (uint32_t)(row & 7) * 16u +
+         (uint32_t)(kb & 15);
+}
+
+__device__ __forceinline__ uint32_t bf16_bits(float x) {
+  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+// X value -> (hi, lo) bfloat16 pairs packed as (re | im << 16)
+__device__ __forceinline__ void split_pair(float2 v, uint32_t &hi, uint32_t &lo) {
+  const __nv_bfloat16 hr = __float2bfloat16_rn(v.x), hi_ = __float2bfloat16_rn(v.y);
+  hi = (uint32_t)__bfloat16_as_ushort(hr) | ((uint32_t)__bfloat16_as_ushort(hi_) << 16);
+  lo = bf16_bits(v.x - __bfloat162float(hr)) | (bf16_bits(v.y - __bfloat162float(hi_)) << 16);
+}
+
+// X [B][NR][K] float2, R [Ci][Co][K] (re, im) bfloat16, Y [B][64][K] float2;
+// NR = Ci (forward) or Co (adjoint); the other channel count is 64.
+template <int MB, bool ADJ>
+__global__ void __launch_bounds__(MT_THREADS, 1)
+    k_mix_tc(const float2 *__restrict__ X, const __nv_bfloat16 *__restrict__ R,
+             float2 *__restrict__ Y, int B, int Ci, int Co, long long K, int mL, int NL,
+             float inv_n, int *err) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const int NR = ADJ ? Co : Ci;
+  const MtGeom e = mt_geom(B, NR, MB);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + e.bar);
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + e.tslot);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long k0 = (long long)blockIdx.x * MB;
+
+  if (warp == 0) {
+    tc::tmem_alloc(tslot, e.cols);
+    tc::tmem_relinquish();
+  }
+  if (tid == 0) {
+    tc::mbar_init(bar, 1);
+    tma::fence_barrier_init();
+  }
+
+  // ---- weights: pair p -> (n, r), the low bits on (n & 3, r & 3) so that a
+  // warp's four-byte stores fall in 16 banks of a core matrix row set
+  {
+    const int nq = 64 / 4;                       // n groups of four
+    const int npairs = 64 * NR;
+    for (int p0 = tid; p0 < npairs; p0 += 8 * MT_THREADS) {
+      uint4 rv[8];
+      int nn[8], rr[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int p = p0 + u * MT_THREADS;
+        const int q = p >> 4;
+        nn[u] = (q % nq) * 4 + (p & 3);
+        rr[u] = (q / nq) * 4 + ((p >> 2) & 3);
+        rv[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (p < npairs) {
+          const int i = ADJ ? nn[u] : rr[u], o = ADJ ? rr[u] : nn[u];
+          const __nv_bfloat16 *src = R + 2 * (((long long)i * Co + o) * K + k0);
+          if constexpr (MB == 4) {
+            rv[u] = __ldg(reinterpret_cast<const uint4 *>(src));
+          } else {
+            const uint2 t = __ldg(reinterpret_cast<const uint2 *>(src));
+            rv[u].x = t.x;
+            rv[u].y = t.y;
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (p0 + u * MT_THREADS >= npairs) break;
+        const uint32_t w4[4] = {rv[u].x, rv[u].y, rv[u].z, rv[u].w};   // (re | im << 16) per mode
+        const uint32_t o0 = mt_off(2 * nn[u], 2 * rr[u], e.sbo);
+        const uint32_t o1 = mt_off(2 * nn[u] + 1, 2 * rr[u], e.sbo);
+#pragma unroll
+        for (int m = 0; m < MB; ++m) {
+          const uint32_t re = w4[m] & 0xFFFFu, im = w4[m] >> 16;
+          const uint32_t nim = im ^ 0x8000u, nre = re;
+          // forward rows (Rr, -Ri) / (Ri, Rr); adjoint rows (Rr, Ri) / (-Ri, Rr)
+          const uint32_t row0 = ADJ ? (re | (im << 16)) : (re | (nim << 16));
+          const uint32_t row1 = ADJ ? (nim | (nre << 16)) : (im | (re << 16));
+          unsigned char *am = smem + e.a0 + (size_t)m * e.a_bytes;
+          *reinterpret_cast<uint32_t *>(am + o0) = row0;
+          *reinterpret_cast<uint32_t *>(am + o1) = row1;
+        }
+      }
+    }
+  }
+  // ---- spectra: pair p -> (b, r), the low bits on (b & 7, r & 3); rows
+  // b >= B are zero
+  {
+    const int nbq = e.NB / 8;
+    const int npairs = e.NB * NR;
+    for (int p0 = tid; p0 < npairs; p0 += 8 * MT_THREADS) {
+      float4 xv[8][2];
+      int bb[8], rr[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int p = p0 + u * MT_THREADS;
+        const int q = p >> 5;
+        bb[u] = (q % nbq) * 8 + (p & 7);
+        rr[u] = (q / nbq) * 4 + ((p >> 3) & 3);
+        xv[u][0] = xv[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (p < npairs && bb[u] < B) {
+          const float4 *src =
+              reinterpret_cast<const float4 *>(X + ((long long)bb[u] * NR + rr[u]) * K + k0);
+          xv[u][0] = __ldg(src);
+          if constexpr (MB == 4) xv[u][1] = __ldg(src + 1);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (p0 + u * MT_THREADS >= npairs) break;
+        const float2 v4[4] = {make_float2(xv[u][0].x, xv[u][0].y), make_float2(xv[u][0].z, xv[u][0].w),
+                              make_float2(xv[u][1].x, xv[u][1].y), make_float2(xv[u][1].z, xv[u][1].w)};
+        const uint32_t off = mt_off(bb[u], 2 * rr[u], e.sbo);
+#pragma unroll
+        for (int m = 0; m < MB; ++m) {
+          uint32_t hi, lo;
+          split_pair(v4[m], hi, lo);
+          unsigned char *bm = smem + e.b0 + (size_t)(2 * m) * e.b_bytes;
+          *reinterpret_cast<uint32_t *>(bm + off) = hi;
+          *reinterpret_cast<uint32_t *>(bm + e.b_bytes + off) = lo;
+        }
+      }
+    }
+  }
+  tc::fence_proxy_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = *tslot;
+
+  // ---- MMA: per mode, the hi chain then the lo chain into D_m
+  if (warp == 0) {
+    if (tc::elect_one()) {
+      const uint32_t idesc = tc::instr_desc(tc::FMT_BF16, MT_ROWS, e.NB);
+      const int nks = 2 * NR / 16;
+      for (int m = 0; m < MB; ++m) {
+        const uint32_t d = tbase + (uint32_t)(m * e.NB);
+        const uint64_t ad = tc::smem_desc_kmajor(tc::smem_u32(smem + e.a0 + (size_t)m * e.a_bytes),
+                                                 128, e.sbo);
+        const uint64_t bh = tc::smem_desc_kmajor(
+            tc::smem_u32(smem + e.b0 + (size_t)(2 * m) * e.b_bytes), 128, e.sbo);
+        const uint64_t bl = tc::smem_desc_kmajor(
+            tc::smem_u32(smem + e.b0 + (size_t)(2 * m + 1) * e.b_bytes), 128, e.sbo);
+        for (int ks = 0; ks < nks; ++ks)
+          tc::mma_f16_ss(d, ad + 16u * ks, bh + 16u * ks, idesc, ks > 0 ? 1u : 0u);
+        for (int ks = 0; ks < nks; ++ks) tc::mma_f16_ss(d, ad + 16u * ks, bl + 16u * ks, idesc, 1u);
+      }
+      tc::mma_commit(bar);
+    }
+    __syncwarp();
+  }
+  bool ok = tc::mbar_wait(bar, 0, err);
+  if (!ok) tc::mbar_wait(bar, 0, nullptr);   // drain before TMEM is released
+  tc::fence_after_sync();
+
+  // ---- epilogue: warp w reads lanes 32 (w % 4) .. and batch columns of half w / 4
+  if (ok) {
+    const int q = warp & 3, half = warp >> 2;
+    const int row = 32 * q + lane;               // 2 n + c
+    const int n = row >> 1, c = row & 1;
+    const uint32_t lane_base = tbase + ((uint32_t)(32 * q) << 16);
+    float wk[MB];
+#pragma unroll
+    for (int m = 0; m < MB; ++m) wk[m] = mode_weight((int)((k0 + m) % mL), NL, inv_n);
+    const int cols = e.NB / 2, cbeg = half * cols;
+    for (int c0 = cbeg; c0 < cbeg + cols; c0 += 8) {
+      uint32_t v[MB][8];
+#pragma unroll
+      for (int m = 0; m < MB; ++m) tc::tmem_ld8(lane_base + (uint32_t)(m * e.NB + c0), v[m]);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float own[MB], oth[MB];
+#pragma unroll
+        for (int m = 0; m < MB; ++m) {
+          own[m] = __uint_as_float(v[m][j]);
+          oth[m] = __shfl_xor_sync(0xffffffffu, own[m], 1);
+        }
+        const int b = c0 + j;
+        // the real-part lane stores even j, the imaginary-part lane odd j
+        if ((j & 1) == c && b < B) {
+          float2 y[MB];
+#pragma unroll
+          for (int m = 0; m < MB; ++m) {
+            const float re = c == 0 ? own[m] : oth[m], im = c == 0 ? oth[m] : own[m];
+            y[m] = make_float2(wk[m] * re, wk[m] * im);
+          }
+          float4 *dst = reinterpret_cast<float4 *>(Y + ((long long)b * 64 + n) * K + k0);
+          dst[0] = make_float4(y[0].x, y[0].y, y[1].x, y[1].y);
+          if constexpr (MB == 4) dst[1] = make_float4(y[2].x, y[2].y, y[3].x, y[3].y);
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tbase, e.cols);
+  }
+}
+
+inline int mt_modes(long long B, int NR) {
+  if (mt_geom(B, NR, 4).total <= MT_SMEM_MAX) return 4;
+  if (mt_geom(B, NR, 2).total <= MT_SMEM_MAX) return 2;
+  return 0;
+}
+
+}  // namespace
+
+bool mix_tc_supported(const Geom &g, int dtype, bool adj, int Ci, int Co, const void *X,
+                      const void *R, const void *Y) {
+  const int NR = adj ? Co : Ci, NOUT = adj ? Ci : Co;
+  if (dtype != DT_BF16 || NOUT != 64) return false;
+  if (NR % 8 != 0 || NR > 64 || g.B < 1 || g.B > 64) return false;
+  if (g.K % 4 != 0) return false;   // 16-byte loads of four modes from aligned rows
+  if (((uintptr_t)X | (uintptr_t)R | (uintptr_t)Y) & 31) return false;
+  return mt_modes(g.B, NR) > 0;
+}
+
+cudaError_t launch_mix_tc(const Launch &L, const Geom &g, bool adj, int Ci, int Co,
+                          const float2 *X, const void *R, float2 *Y) {
+  const int NR = adj ? Co : Ci;
+  const int mb = mt_modes(g.B, NR);
+  const MtGeom e = mt_geom(g.B, NR, mb);
+  const unsigned grid = (unsigned)((g.K + mb - 1) / mb);
+  auto go = [&](auto kern) {
+    cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)e.total);
+    if (r != cudaSuccess) return r;
+    kern<<<grid, MT_THREADS, e.total, L.stream>>>(X, (const __nv_bfloat16 *)R, Y, (int)g.B, Ci,
+                                                   Co, g.K, g.mL, g.NL, g.inv_n, L.err);
+    return cudaGetLastError();
+  };
+  if (adj) return mb == 4 ? go(k_mix_tc<4, true>) : go(k_mix_tc<2, true>);
+  return mb == 4 ? go(k_mix_tc<4, false>) : go(k_mix_tc<2, false>);
+}
+
+}  // namespace fno

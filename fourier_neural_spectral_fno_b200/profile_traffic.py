@@ -78,6 +78,10 @@ def _kernel_key(name: str):
         args = [t.strip() for t in (targs or "").split(",")]
         dz = bool(args) and args[-1] in ("true", "1")
         return ("fwd_plane_dz" if dz else "fwd_plane", "transform_plane.cu")
+    if base == "k_mix_tc":      # k_mix_tc<MB, ADJ>: the adjoint has its own tag
+        args = [t.strip() for t in (targs or "").split(",")]
+        adj = bool(args) and args[-1] in ("true", "1")
+        return ("mix_bwd_dx_tc" if adj else "mix_fwd_tc", "mix_tc.cu")
     if base == "k_epilogue":
         args = [t.strip() for t in (targs or "").split(",")]
         tag = EPILOGUE_TAGS.get(args[1]) if len(args) > 1 else None

@@ -158,6 +158,32 @@ def test_block_bwd(grid, modes, dtype, flags, give_xhat):
     assert_close(host(db), db_ref, tol, "db")
 
 
+@pytest.mark.parametrize("grid,modes,batch", [((32, 32), (8, 8), 3), ((64, 48), (10, 12), 33),
+                                              ((32, 32), (8, 8), 64), ((15, 9), (5, 5), 20)])
+@pytest.mark.parametrize("ci,co", [(64, 64), (16, 64), (64, 40)])
+def test_mixing_64_channels_bf16(grid, modes, batch, ci, co):
+    """The tensor-core mixing (bfloat16 weights, 64 output channels of the
+    forward or of the adjoint dxhat; batch padded to the MMA's N) against the
+    oracle, through the spectral forward and backward; the last shape (K not a
+    multiple of four) and the channel pairs without 64 outputs take the CUDA
+    cores."""
+    x, r, _, _, dy = _block_inputs(grid, modes, batch, ci, co, "bf16", seed=5)
+    d = capi.block_desc(batch, ci, co, grid, modes, "bf16")
+    k = capi.num_modes(grid, modes)
+    y = empty((batch, co) + grid, "bf16")
+    xh = empty((batch, ci, k, 2))
+    capi.fno_spectral_conv_fwd(d, dev(x, "bf16"), dev_complex(r, "bf16"), y, xh)
+    y_ref, xh_ref = O.spectral_conv_fwd(x, r, modes)
+    assert_close(host(y), y_ref, TOL["bf16"], "y")
+    dx = empty((batch, ci) + grid, "bf16")
+    dr = empty((ci, co, k, 2))
+    capi.fno_spectral_conv_bwd(d, dev(x, "bf16"), dev_complex(xh_ref), dev_complex(r, "bf16"),
+                               dev(dy, "bf16"), dx, dr)
+    dx_ref, dr_ref = O.spectral_conv_bwd(x, r, xh_ref, dy, modes)
+    assert_close(host(dx), dx_ref, TOL["bf16"], "dx")
+    assert_close(host_complex(dr), dr_ref, TOL["bf16"], "dR")
+
+
 def test_block_bwd_wide_channels_f32():
     grid, modes = (32, 40), (5, 7)
     x, r, w, b, dy = _block_inputs(grid, modes, 3, 64, 48, "f32", seed=4)
