@@ -21,12 +21,14 @@
 // gather the modes' operands from global memory into shared memory in the
 // tcgen05 K-major core-matrix layout (R as one load of the MB modes' (re, im)
 // pairs per (i, o), X as 16-byte loads of the MB modes), one elected thread
-// issues the chains, every thread waits on
-// the commit (bounded), and the eight warps read the accumulators back: warp w
-// takes TMEM lane quarter w % 4 (32 rows = 16 output channels, real and
-// imaginary in neighbouring lanes) and half of the batch columns; each thread
-// writes, per batch entry, the MB modes of one output channel as 32 contiguous
-// bytes, scaled by the inverse transform's c_k / N.
+// issues the chains, every thread waits on the commit (bounded), and the
+// sixteen warps read the accumulators back: warp w takes TMEM lane quarter
+// w % 4 (32 rows = 16 output channels, real and imaginary in neighbouring
+// lanes) and every fourth 8-column chunk of the batch; each thread writes, per
+// batch entry, the MB modes of one output channel as one contiguous run,
+// scaled by the inverse transform's c_k / N.  Sixteen warps and one pass of
+// loads per thread keep the gather's memory latency to about one round trip
+// (eight warps and three passes left the kernel waiting on loads).
 #include "fno_common.cuh"
 #include "fno_kernels.cuh"
 #include "tc_util.cuh"
@@ -36,7 +38,8 @@ namespace fno {
 
 namespace {
 
-constexpr int MT_THREADS = 256;
+constexpr int MT_THREADS = 512;
+constexpr int MT_RB = 8, MT_XB = 4;          // weight / spectrum loads per thread and pass
 constexpr int MT_ROWS = 128;                 // 2 x 64 output channels
 constexpr size_t MT_SMEM_MAX = 227 * 1024;
 
@@ -106,22 +109,28 @@ __global__ void __launch_bounds__(MT_THREADS, 1)
     tma::fence_barrier_init();
   }
 
-  // ---- weights: pair p -> (n, r), the low bits on (n & 3, r & 3) so that a
-  // warp's four-byte stores fall in 16 banks of a core matrix row set
+  // ---- operands.  Weights: pair p -> (n, r) with the low bits on (n & 3,
+  // r & 3), so that a warp's four-byte stores fall in 16 banks of a core-matrix
+  // row set.  Spectra: pair p -> (b, r) with the low bits on (b & 7, r & 3);
+  // rows b >= B are zero.  Each pass issues MT_RB weight loads and MT_XB
+  // spectrum loads per thread before any store, so one pass waits out one
+  // memory latency.
   {
     const int nq = 64 / 4;                       // n groups of four
-    const int npairs = 64 * NR;
-    for (int p0 = tid; p0 < npairs; p0 += 8 * MT_THREADS) {
-      uint4 rv[8];
-      int nn[8], rr[8];
+    const int nrp = 64 * NR;                     // weight pairs
+    const int nbq = e.NB / 8;
+    const int nxp = e.NB * NR;                   // spectrum pairs
+    for (int it = 0; it * MT_RB * MT_THREADS < nrp || it * MT_XB * MT_THREADS < nxp; ++it) {
+      uint4 rv[MT_RB];
+      int nn[MT_RB], rr[MT_RB];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int p = p0 + u * MT_THREADS;
+      for (int u = 0; u < MT_RB; ++u) {
+        const int p = (it * MT_RB + u) * MT_THREADS + tid;
         const int q = p >> 4;
         nn[u] = (q % nq) * 4 + (p & 3);
         rr[u] = (q / nq) * 4 + ((p >> 2) & 3);
         rv[u] = make_uint4(0u, 0u, 0u, 0u);
-        if (p < npairs) {
+        if (p < nrp) {
           const int i = ADJ ? nn[u] : rr[u], o = ADJ ? rr[u] : nn[u];
           const __nv_bfloat16 *src = R + 2 * (((long long)i * Co + o) * K + k0);
           if constexpr (MB == 4) {
@@ -133,54 +142,46 @@ __global__ void __launch_bounds__(MT_THREADS, 1)
           }
         }
       }
+      float4 xv[MT_XB][2];
+      int bb[MT_XB], xr[MT_XB];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (p0 + u * MT_THREADS >= npairs) break;
+      for (int u = 0; u < MT_XB; ++u) {
+        const int p = (it * MT_XB + u) * MT_THREADS + tid;
+        const int q = p >> 5;
+        bb[u] = (q % nbq) * 8 + (p & 7);
+        xr[u] = (q / nbq) * 4 + ((p >> 3) & 3);
+        xv[u][0] = xv[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (p < nxp && bb[u] < B) {
+          const float4 *src =
+              reinterpret_cast<const float4 *>(X + ((long long)bb[u] * NR + xr[u]) * K + k0);
+          xv[u][0] = __ldg(src);
+          if constexpr (MB == 4) xv[u][1] = __ldg(src + 1);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < MT_RB; ++u) {
+        if ((it * MT_RB + u) * MT_THREADS + tid >= nrp) break;
         const uint32_t w4[4] = {rv[u].x, rv[u].y, rv[u].z, rv[u].w};   // (re | im << 16) per mode
         const uint32_t o0 = mt_off(2 * nn[u], 2 * rr[u], e.sbo);
         const uint32_t o1 = mt_off(2 * nn[u] + 1, 2 * rr[u], e.sbo);
 #pragma unroll
         for (int m = 0; m < MB; ++m) {
           const uint32_t re = w4[m] & 0xFFFFu, im = w4[m] >> 16;
-          const uint32_t nim = im ^ 0x8000u, nre = re;
+          const uint32_t nim = im ^ 0x8000u;
           // forward rows (Rr, -Ri) / (Ri, Rr); adjoint rows (Rr, Ri) / (-Ri, Rr)
           const uint32_t row0 = ADJ ? (re | (im << 16)) : (re | (nim << 16));
-          const uint32_t row1 = ADJ ? (nim | (nre << 16)) : (im | (re << 16));
+          const uint32_t row1 = ADJ ? (nim | (re << 16)) : (im | (re << 16));
           unsigned char *am = smem + e.a0 + (size_t)m * e.a_bytes;
           *reinterpret_cast<uint32_t *>(am + o0) = row0;
           *reinterpret_cast<uint32_t *>(am + o1) = row1;
         }
       }
-    }
-  }
-  // ---- spectra: pair p -> (b, r), the low bits on (b & 7, r & 3); rows
-  // b >= B are zero
-  {
-    const int nbq = e.NB / 8;
-    const int npairs = e.NB * NR;
-    for (int p0 = tid; p0 < npairs; p0 += 8 * MT_THREADS) {
-      float4 xv[8][2];
-      int bb[8], rr[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int p = p0 + u * MT_THREADS;
-        const int q = p >> 5;
-        bb[u] = (q % nbq) * 8 + (p & 7);
-        rr[u] = (q / nbq) * 4 + ((p >> 3) & 3);
-        xv[u][0] = xv[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (p < npairs && bb[u] < B) {
-          const float4 *src =
-              reinterpret_cast<const float4 *>(X + ((long long)bb[u] * NR + rr[u]) * K + k0);
-          xv[u][0] = __ldg(src);
-          if constexpr (MB == 4) xv[u][1] = __ldg(src + 1);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (p0 + u * MT_THREADS >= npairs) break;
+      for (int u = 0; u < MT_XB; ++u) {
+        if ((it * MT_XB + u) * MT_THREADS + tid >= nxp) break;
         const float2 v4[4] = {make_float2(xv[u][0].x, xv[u][0].y), make_float2(xv[u][0].z, xv[u][0].w),
                               make_float2(xv[u][1].x, xv[u][1].y), make_float2(xv[u][1].z, xv[u][1].w)};
-        const uint32_t off = mt_off(bb[u], 2 * rr[u], e.sbo);
+        const uint32_t off = mt_off(bb[u], 2 * xr[u], e.sbo);
 #pragma unroll
         for (int m = 0; m < MB; ++m) {
           uint32_t hi, lo;
@@ -223,17 +224,18 @@ __global__ void __launch_bounds__(MT_THREADS, 1)
   if (!ok) tc::mbar_wait(bar, 0, nullptr);   // drain before TMEM is released
   tc::fence_after_sync();
 
-  // ---- epilogue: warp w reads lanes 32 (w % 4) .. and batch columns of half w / 4
+  // ---- epilogue: warp w reads TMEM lanes 32 (w % 4) .. (16 output channels,
+  // real and imaginary parts in neighbouring lanes) and the 8-column batch
+  // chunks w / 4, w / 4 + 4, ...
   if (ok) {
-    const int q = warp & 3, half = warp >> 2;
+    const int q = warp & 3;
     const int row = 32 * q + lane;               // 2 n + c
     const int n = row >> 1, c = row & 1;
     const uint32_t lane_base = tbase + ((uint32_t)(32 * q) << 16);
     float wk[MB];
 #pragma unroll
     for (int m = 0; m < MB; ++m) wk[m] = mode_weight((int)((k0 + m) % mL), NL, inv_n);
-    const int cols = e.NB / 2, cbeg = half * cols;
-    for (int c0 = cbeg; c0 < cbeg + cols; c0 += 8) {
+    for (int c0 = (warp >> 2) * 8; c0 < e.NB; c0 += (MT_THREADS / 128) * 8) {
       uint32_t v[MB][8];
 #pragma unroll
       for (int m = 0; m < MB; ++m) tc::tmem_ld8(lane_base + (uint32_t)(m * e.NB + c0), v[m]);
