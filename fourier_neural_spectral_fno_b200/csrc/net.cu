@@ -413,6 +413,102 @@ __global__ void __launch_bounds__(PB)
     partial[(long long)blockIdx.x * width * (in_ch + 1) + e] = acc[e];
 }
 
+// Lift adjoint, streaming form (the same per-CTA partials): warp w owns the
+// eight channels of group w % NCG and keeps their [8][IN + 1] sums in
+// registers; its lanes walk chunks of 16 bytes of consecutive points (8 for
+// 16-bit storage, 4 for float32) of one sample, all eight channel loads and the
+// IN input loads of a chunk in flight at once.  Lanes, then the warps of a
+// point group, meet once at the end (shuffles, then shared memory), in a fixed
+// order.  The tiled kernel above waited out one load per channel per tile.
+constexpr int LB_THREADS = 256, LB_CPW = 8;
+
+template <typename T> struct Pack16 {   // 16 bytes of storage elements
+  static constexpr int n = 16 / (int)sizeof(T);
+};
+template <typename T>
+__device__ __forceinline__ void unpack16(const uint4 &r, float (&v)[Pack16<T>::n]) {
+  if constexpr (sizeof(T) == 4) {
+    v[0] = __uint_as_float(r.x);
+    v[1] = __uint_as_float(r.y);
+    v[2] = __uint_as_float(r.z);
+    v[3] = __uint_as_float(r.w);
+  } else {
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const T lo = *reinterpret_cast<const T *>(reinterpret_cast<const unsigned short *>(&w[i]));
+      const T hi =
+          *reinterpret_cast<const T *>(reinterpret_cast<const unsigned short *>(&w[i]) + 1);
+      v[2 * i] = to_f<T>(lo);
+      v[2 * i + 1] = to_f<T>(hi);
+    }
+  }
+}
+
+template <typename T, int IN>
+__global__ void __launch_bounds__(LB_THREADS)
+    k_lift_bwd16(const T *__restrict__ a, const T *__restrict__ dv, float *__restrict__ partial,
+                 long long B, long long N, int width, int ncg) {
+  constexpr int PP = Pack16<T>::n;            // points per chunk
+  constexpr int NW = LB_THREADS / 32;
+  __shared__ float red[NW][LB_CPW * (IN + 1)];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int npg = NW / ncg, cg = warp % ncg, pg = warp / ncg;
+  const int c0 = cg * LB_CPW;
+  float acc[LB_CPW][IN + 1];
+#pragma unroll
+  for (int c = 0; c < LB_CPW; ++c)
+#pragma unroll
+    for (int j = 0; j <= IN; ++j) acc[c][j] = 0.f;
+  const long long nchunk = B * N / PP;
+  if (pg < npg) {
+    const long long step = (long long)gridDim.x * npg * 32;
+    for (long long q = ((long long)blockIdx.x * npg + pg) * 32 + lane; q < nchunk; q += step) {
+      const long long t = q * PP, b = t / N, n = t - b * N;
+      uint4 ar[IN], dr[LB_CPW];
+#pragma unroll
+      for (int j = 0; j < IN; ++j)
+        ar[j] = __ldg(reinterpret_cast<const uint4 *>(a + (b * IN + j) * N + n));
+#pragma unroll
+      for (int c = 0; c < LB_CPW; ++c)
+        dr[c] = c0 + c < width
+                    ? __ldg(reinterpret_cast<const uint4 *>(dv + (b * width + c0 + c) * N + n))
+                    : make_uint4(0u, 0u, 0u, 0u);
+      float av[IN][PP];
+#pragma unroll
+      for (int j = 0; j < IN; ++j) unpack16<T>(ar[j], av[j]);
+#pragma unroll
+      for (int c = 0; c < LB_CPW; ++c) {
+        float d[PP];
+        unpack16<T>(dr[c], d);
+#pragma unroll
+        for (int i = 0; i < PP; ++i) {
+#pragma unroll
+          for (int j = 0; j < IN; ++j) acc[c][j] = fmaf(d[i], av[j][i], acc[c][j]);
+          acc[c][IN] += d[i];
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < LB_CPW; ++c)
+#pragma unroll
+    for (int j = 0; j <= IN; ++j) {
+      float v = acc[c][j];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      if (lane == 0) red[warp][c * (IN + 1) + j] = v;
+    }
+  __syncthreads();
+  for (int e = threadIdx.x; e < width * (IN + 1); e += LB_THREADS) {
+    const int c = e / (IN + 1), j = e - c * (IN + 1);
+    const int g = c / LB_CPW, cc = c - g * LB_CPW;
+    float v = 0.f;
+    for (int p2 = 0; p2 < npg; ++p2) v += red[p2 * ncg + g][cc * (IN + 1) + j];
+    partial[(long long)blockIdx.x * width * (IN + 1) + e] = v;
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256)
     k_mse(const T *__restrict__ u, const T *__restrict__ tg, float *__restrict__ loss,
@@ -568,10 +664,31 @@ int lift_bwd_grid(const Geom &g, int num_sms) {
 cudaError_t launch_lift_bwd(const Launch &L, const Geom &g, int dtype, int in_ch, int width,
                             const void *a, const void *dv, float *partial) {
   const int grid = lift_bwd_grid(g, L.num_sms);
+  // the streaming form: 16-byte chunks of points that stay inside a sample,
+  // 16-byte aligned rows, at most 64 channels, 2 to 4 inputs
+  const int pp = dtype == DT_F32 ? 4 : 8;
+  const bool stream16 = g.N % pp == 0 && width <= 64 && in_ch >= 2 && in_ch <= 4 &&
+                        ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(dv)) & 15) == 0;
+  const int groups = (width + LB_CPW - 1) / LB_CPW;
+  const int ncg = groups <= 1 ? 1 : groups <= 2 ? 2 : groups <= 4 ? 4 : 8;
   launch_begin(L);
-  FNO_DISPATCH_T(dtype, k_lift_bwd<T><<<grid, PB, 0, L.stream>>>((const T *)a, (const T *)dv,
-                                                                 partial, g.B, g.N, in_ch,
-                                                                 width));
+  if (stream16) {
+    FNO_DISPATCH_T(dtype, {
+      if (in_ch == 2)
+        k_lift_bwd16<T, 2><<<grid, LB_THREADS, 0, L.stream>>>((const T *)a, (const T *)dv, partial,
+                                                              g.B, g.N, width, ncg);
+      else if (in_ch == 3)
+        k_lift_bwd16<T, 3><<<grid, LB_THREADS, 0, L.stream>>>((const T *)a, (const T *)dv, partial,
+                                                              g.B, g.N, width, ncg);
+      else
+        k_lift_bwd16<T, 4><<<grid, LB_THREADS, 0, L.stream>>>((const T *)a, (const T *)dv, partial,
+                                                              g.B, g.N, width, ncg);
+    });
+  } else {
+    FNO_DISPATCH_T(dtype, k_lift_bwd<T><<<grid, PB, 0, L.stream>>>((const T *)a, (const T *)dv,
+                                                                   partial, g.B, g.N, in_ch,
+                                                                   width));
+  }
   launch_end(L, "lift_bwd");
   return cudaGetLastError();
 }
