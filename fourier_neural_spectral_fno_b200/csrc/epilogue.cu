@@ -437,18 +437,35 @@ cudaError_t launch_epi_m(const Launch &L, const Geom &g, int mode, const EpiArgs
   }
 }
 
-__global__ void k_reduce_partials(const float *__restrict__ partial, int nparts, long long stride,
-                                  long long offset, int rows, int cols, float *__restrict__ out_main,
-                                  float *__restrict__ out_last) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= rows * (cols + 1)) return;
+// Sum of the per-CTA partial rows: a CTA takes 32 columns, its eight warps
+// the parts w, w + 8, ... of them (eight loads in flight per thread), and the
+// eight part sums meet in shared memory in a fixed order.
+constexpr int RP_COLS = 32, RP_SLICES = 8;
+__global__ void __launch_bounds__(RP_COLS * RP_SLICES)
+    k_reduce_partials(const float *__restrict__ partial, int nparts, long long stride,
+                      long long offset, int rows, int cols, float *__restrict__ out_main,
+                      float *__restrict__ out_last) {
+  __shared__ float part[RP_SLICES][RP_COLS];
+  const int lane = threadIdx.x & 31, sl = threadIdx.x >> 5;
+  const int e = blockIdx.x * RP_COLS + lane;
+  const bool in = e < rows * (cols + 1);
   float s = 0.f;
-  for (int p = 0; p < nparts; ++p) s += partial[p * stride + offset + e];
+  if (in) {
+    const float *src = partial + offset + e;
+#pragma unroll 8
+    for (int p = sl; p < nparts; p += RP_SLICES) s += src[p * stride];
+  }
+  part[sl][lane] = s;
+  __syncthreads();
+  if (sl != 0 || !in) return;
+  float t = part[0][lane];
+#pragma unroll
+  for (int i = 1; i < RP_SLICES; ++i) t += part[i][lane];
   const int r = e / (cols + 1), c = e - r * (cols + 1);
   if (c < cols) {
-    if (out_main) out_main[r * cols + c] = s;
+    if (out_main) out_main[r * cols + c] = t;
   } else if (out_last) {
-    out_last[r] = s;
+    out_last[r] = t;
   }
 }
 
@@ -483,8 +500,8 @@ cudaError_t launch_reduce_rows(const Launch &L, const float *partial, int nparts
                                float *out_main, float *out_last) {
   const int n = rows * (cols + 1);
   launch_begin(L);
-  k_reduce_partials<<<(n + 255) / 256, 256, 0, L.stream>>>(partial, nparts, stride, offset, rows,
-                                                           cols, out_main, out_last);
+  k_reduce_partials<<<(n + RP_COLS - 1) / RP_COLS, RP_COLS * RP_SLICES, 0, L.stream>>>(
+      partial, nparts, stride, offset, rows, cols, out_main, out_last);
   launch_end(L, "reduce_partials");
   return cudaGetLastError();
 }
