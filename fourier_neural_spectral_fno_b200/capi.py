@@ -396,9 +396,10 @@ def fno_profile_read(max_kernels: int = 64) -> Dict[str, Dict[str, float]]:
 
 def fno_set_tensor_cores(mode) -> int:
     """Kernel selection: 1 / True = the default kernels (per shape the faster
-    design as measured: the streaming pruned-FFT transform, mixing and pruned
-    slab-axis inverse on the CUDA cores, tcgen05 TMA pipelines for the epilogue
-    and projection), 4 = the default with the clustered FFT transform, 3 =
+    design as measured: the streaming pruned-FFT transform, mixing (tcgen05
+    for bfloat16 weights with 64 output channels) and pruned slab-axis inverse
+    on the CUDA cores, tcgen05 TMA pipelines for the epilogue and projection),
+    4 = the default with the clustered FFT transform, 3 =
     tcgen05 TMA pipelines throughout (dense DFT-matrix transform), 2 = tcgen05
     kernels without the pipelines, 0 / False = the CUDA-core kernels.  Returns
     the previous setting."""

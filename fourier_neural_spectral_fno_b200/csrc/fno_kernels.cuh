@@ -37,7 +37,8 @@ struct Launch {
   int num_sms;
   int tc;           // 1: default (pruned-FFT transform, mixing and pruned slab-axis
                     //    inverse on CUDA cores where each is measured faster, tcgen05
-                    //    TMA pipelines for the epilogue and projection);
+                    //    mixing for bf16 weights at 64 outputs, tcgen05 TMA pipelines
+                    //    for the epilogue and projection);
                     // 4: as 1 with the clustered FFT transform;
                     // 3: tcgen05 TMA pipelines throughout (dense DFT-matrix transform);
                     // 2: tcgen05 without the pipelines; 0: CUDA cores only

@@ -161,12 +161,14 @@ int fno_last_launch_count(void);
 /* Kernel selection.  1 (default): per shape the design measured faster: the
  * truncated transform as a streaming pruned radix-16 FFT on the CUDA cores
  * (2D grids) or a dense DFT-matrix contraction on the tensor cores (3D grids,
- * and shapes the streaming kernel does not take), the mixing and a pruned
- * slab-axis inverse on the CUDA cores, the warp-specialised tcgen05 TMA
- * pipelines for the epilogue and the projection; 4: as 1 with the transform
- * as a clustered pruned FFT; 3: the tcgen05 TMA pipelines throughout with the
- * dense DFT-matrix transform; 2: the tensor-core kernels without the TMA
- * pipelines; 0: the CUDA-core kernels everywhere.  All are complete
+ * and shapes the streaming kernel does not take), the mixing on the CUDA
+ * cores (on the tensor cores for bfloat16 weights with 64 output channels),
+ * a pruned slab-axis inverse on the CUDA cores, the warp-specialised tcgen05
+ * TMA pipelines for the epilogue and the projection; 4: as 1 with the
+ * transform as a clustered pruned FFT; 3: the tcgen05 TMA pipelines
+ * throughout with the dense DFT-matrix transform; 2: the tensor-core kernels
+ * without the TMA pipelines (mixing on the CUDA cores); 0: the CUDA-core
+ * kernels everywhere.  All are complete
  * implementations; the switch exists to compare them.  Process-wide; any
  * other nonzero value means 1; returns the previous setting. */
 int fno_set_tensor_cores(int enable);
