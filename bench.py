@@ -247,7 +247,9 @@ def kernel_source_sha(tag: str) -> str:
              "fwd_plane": "transform_plane.cu", "fwd_plane_dz": "transform_plane.cu",
              "inv_slab_img": "spec_mid.cu", "inv_slab_fft": "spec_mid.cu",
              "epi_block_bwd_pipe": "epilogue_pipe.cu", "proj_bwd_pipe": "proj_pipe.cu",
-             "mix_fwd_tc": "mix_tc.cu", "mix_bwd_dx_tc": "mix_tc.cu"}
+             "mix_fwd_tc": "mix_tc.cu", "mix_bwd_dx_tc": "mix_tc.cu", "lift_bwd": "net.cu",
+             "mix_bwd_dx": "mix.cu", "mix_bwd_dr": "mix.cu", "epi_spec": "epilogue.cu",
+             "epi_spec_bwd": "epilogue.cu"}
     path = os.path.join(ROOT, "fourier_neural_spectral_fno_b200", "csrc", files.get(tag, ""))
     if not os.path.isfile(path):
         return ""

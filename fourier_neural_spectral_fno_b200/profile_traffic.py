@@ -40,6 +40,7 @@ KERNELS = {
     "k_lift": ("lift", "net.cu"),
     "k_proj_bwd": ("proj_bwd", "net.cu"),
     "k_lift_bwd": ("lift_bwd", "net.cu"),
+    "k_lift_bwd16": ("lift_bwd", "net.cu"),        # the streaming form
     "k_fwd_fft": ("fwd_fft", "transform_fft.cu"),
     "k_inv_slab_img": ("inv_slab_img", "spec_mid.cu"),
     "k_inv_slab_fft": ("inv_slab_fft", "spec_mid.cu"),

@@ -98,3 +98,21 @@ def test_roofline_hbm_for_the_forward_pipeline():
     assert rec["algorithmic_bytes_per_launch"] == 2 * act + spec
     assert rec["achieved"] == pytest.approx((2 * act + spec) / 0.1e-3 / 1e9)
     assert rec["peak"] == pytest.approx(bench.hbm_peak()[0])   # measured copy peak, else fallback
+
+
+def test_traffic_records_and_bench_name_the_same_source():
+    """A traffic record is keyed by (timing tag, hash of the kernel's source file); bench.py
+    looks the hash up through its own tag -> file table, so the two tables must agree for
+    every kernel the recorder knows, or a fresh record would never be used."""
+    import importlib.util
+    from fourier_neural_spectral_fno_b200 import profile_traffic as pt
+    spec = importlib.util.spec_from_file_location("bench_mod", BENCH)
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    pairs = set(pt.KERNELS.values()) | {(t, "epilogue.cu") for t in pt.EPILOGUE_TAGS.values()}
+    pairs |= {("fwd_plane_dz", "transform_plane.cu"), ("mix_fwd_tc", "mix_tc.cu"),
+              ("mix_bwd_dx_tc", "mix_tc.cu")}
+    for tag, src in sorted(pairs):
+        path = os.path.join(ROOT, "fourier_neural_spectral_fno_b200", "csrc", src)
+        assert os.path.isfile(path), src
+        assert bench.kernel_source_sha(tag) == pt.source_sha(src), (tag, src)
