@@ -231,6 +231,7 @@ def algorithmic_bytes(tag: str, wl) -> float:
     table["proj_bwd_pipe"] = table["proj_bwd"]
     table["mix_fwd_tc"] = table["mix_fwd"]          # read spectrum and R, write spectrum
     table["mix_bwd_dx"] = table["mix_bwd_dx_tc"] = table["mix_fwd"]
+    table["mix_bwd_dr"] = table["mix_bwd_dr_tc"] = 2 * spec + 2 * wl.width * wl.width * k * 4
     return float(table.get(tag, 0.0))
 
 
@@ -248,7 +249,8 @@ def kernel_source_sha(tag: str) -> str:
              "inv_slab_img": "spec_mid.cu", "inv_slab_fft": "spec_mid.cu",
              "epi_block_bwd_pipe": "epilogue_pipe.cu", "proj_bwd_pipe": "proj_pipe.cu",
              "mix_fwd_tc": "mix_tc.cu", "mix_bwd_dx_tc": "mix_tc.cu", "lift_bwd": "net.cu",
-             "mix_bwd_dx": "mix.cu", "mix_bwd_dr": "mix.cu", "epi_spec": "epilogue.cu",
+             "mix_bwd_dx": "mix.cu", "mix_bwd_dr": "mix.cu", "mix_bwd_dr_tc": "mix_tc.cu",
+             "epi_spec": "epilogue.cu",
              "epi_spec_bwd": "epilogue.cu"}
     path = os.path.join(ROOT, "fourier_neural_spectral_fno_b200", "csrc", files.get(tag, ""))
     if not os.path.isfile(path):

@@ -356,7 +356,7 @@ int run_backward(const Launch &L, const Geom &g, int dtype, unsigned flags, int 
   const bool act = block && !(flags & FNO_NO_ACT);
   FNO_TRY(launch_fwd_transform(L, g, dtype, act ? LOAD_DZ : LOAD_PLAIN, Co, dy, pre, zpart, D),
           "transform of dz");
-  FNO_TRY(launch_mix_bwd_dr(L, g, Ci, Co, xhat, D, dR), "dR");
+  FNO_TRY(launch_mix_bwd_dr(L, g, dtype, Ci, Co, xhat, D, dR), "dR");
   float2 *dxhat = reinterpret_cast<float2 *>(ws + w.dxhat);
   FNO_TRY(launch_mix_bwd_dx(L, g, dtype, Ci, Co, D, R, dxhat), "dxhat");
   const float2 *Z = dxhat;

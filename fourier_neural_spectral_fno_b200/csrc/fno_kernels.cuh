@@ -137,8 +137,13 @@ cudaError_t launch_mix_tc(const Launch &L, const Geom &g, bool adj, int Ci, int 
 cudaError_t launch_mix_fwd(const Launch &L, const Geom &g, int dtype, int Ci, int Co,
                            const float2 *xhat, const void *R, float2 *yhat);
 // dR[i,o,k] = sum_b conj(xhat[b,i,k]) (c_k/N) D[b,o,k]
-cudaError_t launch_mix_bwd_dr(const Launch &L, const Geom &g, int Ci, int Co,
+cudaError_t launch_mix_bwd_dr(const Launch &L, const Geom &g, int dtype, int Ci, int Co,
                               const float2 *xhat, const float2 *D, float *dR);
+// tcgen05 dR (mix_tc.cu): 16-bit storage, 64 input channels, batch <= 64
+bool mix_tc_dr_supported(const Geom &g, int dtype, int Ci, int Co, const void *X, const void *D,
+                         const void *dR);
+cudaError_t launch_mix_tc_dr(const Launch &L, const Geom &g, int Co, const float2 *X,
+                             const float2 *D, float *dR);
 // dxhat[b,i,k] = sum_o (c_k/N) D[b,o,k] conj(R[i,o,k])
 cudaError_t launch_mix_bwd_dx(const Launch &L, const Geom &g, int dtype, int Ci, int Co,
                               const float2 *D, const void *R, float2 *dxhat);

@@ -288,10 +288,16 @@ cudaError_t launch_mix_fwd(const Launch &L, const Geom &g, int dtype, int Ci, in
   return e;
 }
 
-cudaError_t launch_mix_bwd_dr(const Launch &L, const Geom &g, int Ci, int Co, const float2 *xhat,
-                              const float2 *D, float *dR) {
+cudaError_t launch_mix_bwd_dr(const Launch &L, const Geom &g, int dtype, int Ci, int Co,
+                              const float2 *xhat, const float2 *D, float *dR) {
   const bool big = big_tiles(g.K, Ci, Co * 2, L.num_sms);
+  const bool tc = L.tc != 0 && L.tc != 2 && mix_tc_dr_supported(g, dtype, Ci, Co, xhat, D, dR);
   launch_begin(L);
+  if (tc) {
+    const cudaError_t e = launch_mix_tc_dr(L, g, Co, xhat, D, dR);
+    launch_end(L, "mix_bwd_dr_tc");
+    return e;
+  }
   if (big) {
     dim3 grid((unsigned)((g.K + MX_THREADS - 1) / MX_THREADS), (unsigned)((Co + 3) / 4),
               (unsigned)((Ci + 3) / 4));

@@ -272,6 +272,216 @@ __global__ void __launch_bounds__(MT_THREADS, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// dR[i, o, k] = w_k sum_b conj(xhat[b, i, k]) D[b, o, k] for 64 input channels:
+// per mode the real GEMM, rows 2 i + c (c = 0 real, 1 imaginary part of dR),
+// columns o, K index 2 b + c',
+//     D_acc[2i + c, o] = sum_{b, c'} Ablk[2i + c, 2b + c'] Dv[o, 2b + c']
+//     rows 2i: (Xr, Xi)    rows 2i + 1: (-Xi, Xr)    Dv[o, 2b..2b+1] = (Dr, Di)
+// M = 128, N = Co padded to 16, K = 2 x batch padded to 8.  Both operands are
+// float32 spectra and enter as bfloat16 pairs hi + lo, in three chains
+// (A_hi B_hi, A_hi B_lo, A_lo B_hi) into one fp32 accumulator: about 16
+// mantissa bits per product, for 16-bit storage.  The gather, issue, bounded
+// wait and read-back follow k_mix_tc; the read-back writes, per (i, o), the MB
+// modes of dR contiguously.
+struct DrGeom {
+  int KB, NP;        // batch padded to 8, output channels padded to 16
+  uint32_t sbo;
+  size_t a_bytes, b_bytes, a0, b0, bar, tslot, total;
+  uint32_t cols;
+};
+
+__host__ __device__ inline DrGeom dr_geom(long long B, int Co, int MB) {
+  DrGeom e;
+  e.KB = (int)((B + 7) / 8 * 8);
+  e.NP = (Co + 15) / 16 * 16;
+  const int kel = 2 * e.KB;
+  e.sbo = (uint32_t)(kel * 2 / 16) * 128u;
+  e.a_bytes = (size_t)MT_ROWS * kel * 2;     // one of A_hi, A_lo
+  e.b_bytes = (size_t)e.NP * kel * 2;        // one of B_hi, B_lo
+  e.a0 = 0;
+  e.b0 = (size_t)MB * 2 * e.a_bytes;
+  e.bar = e.b0 + (size_t)MB * 2 * e.b_bytes;
+  e.tslot = e.bar + 8;
+  e.total = e.tslot + 8;
+  uint32_t c = 32;
+  while (c < (uint32_t)(MB * e.NP)) c *= 2;
+  e.cols = c;
+  return e;
+}
+
+__device__ __forceinline__ uint32_t neg_bf16_lo(uint32_t w) { return w ^ 0x8000u; }
+
+template <int MB>
+__global__ void __launch_bounds__(MT_THREADS, 1)
+    k_mix_tc_dr(const float2 *__restrict__ X, const float2 *__restrict__ Dsp,
+                float *__restrict__ dR, int B, int Co, long long K, int mL, int NL, float inv_n,
+                int *err) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  constexpr int Ci = 64;
+  const DrGeom e = dr_geom(B, Co, MB);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + e.bar);
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + e.tslot);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long k0 = (long long)blockIdx.x * MB;
+
+  if (warp == 0) {
+    tc::tmem_alloc(tslot, e.cols);
+    tc::tmem_relinquish();
+  }
+  if (tid == 0) {
+    tc::mbar_init(bar, 1);
+    tma::fence_barrier_init();
+  }
+  // ---- operands, one pass of loads per thread before the stores.  A from
+  // xhat: pair p -> (i, b) with the low bits on (i & 3, b & 3); B from D: pair
+  // p -> (o, b) with the low bits on (o & 7, b & 3); padded rows are zero.
+  {
+    const int nxp = 64 * e.KB, nq8 = e.NP / 8, ndp = e.NP * e.KB;
+    for (int it = 0; it * MT_XB * MT_THREADS < nxp || it * MT_XB * MT_THREADS < ndp; ++it) {
+      float4 xv[MT_XB][2], dv[MT_XB][2];
+      int xi_[MT_XB], xb_[MT_XB], dor[MT_XB], db_[MT_XB];
+#pragma unroll
+      for (int u = 0; u < MT_XB; ++u) {
+        const int p = (it * MT_XB + u) * MT_THREADS + tid;
+        const int q = p >> 4;
+        xi_[u] = (q % 16) * 4 + (p & 3);
+        xb_[u] = (q / 16) * 4 + ((p >> 2) & 3);
+        xv[u][0] = xv[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (p < nxp && xb_[u] < B) {
+          const float4 *src =
+              reinterpret_cast<const float4 *>(X + ((long long)xb_[u] * Ci + xi_[u]) * K + k0);
+          xv[u][0] = __ldg(src);
+          if constexpr (MB == 4) xv[u][1] = __ldg(src + 1);
+        }
+        const int q2 = p >> 5;
+        dor[u] = (q2 % nq8) * 8 + (p & 7);
+        db_[u] = (q2 / nq8) * 4 + ((p >> 3) & 3);
+        dv[u][0] = dv[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (p < ndp && db_[u] < B && dor[u] < Co) {
+          const float4 *src =
+              reinterpret_cast<const float4 *>(Dsp + ((long long)db_[u] * Co + dor[u]) * K + k0);
+          dv[u][0] = __ldg(src);
+          if constexpr (MB == 4) dv[u][1] = __ldg(src + 1);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < MT_XB; ++u) {
+        if ((it * MT_XB + u) * MT_THREADS + tid < nxp) {
+          const float2 v4[4] = {make_float2(xv[u][0].x, xv[u][0].y), make_float2(xv[u][0].z, xv[u][0].w),
+                                make_float2(xv[u][1].x, xv[u][1].y), make_float2(xv[u][1].z, xv[u][1].w)};
+          const uint32_t o0 = mt_off(2 * xi_[u], 2 * xb_[u], e.sbo);
+          const uint32_t o1 = mt_off(2 * xi_[u] + 1, 2 * xb_[u], e.sbo);
+#pragma unroll
+          for (int m = 0; m < MB; ++m) {
+            uint32_t hi, lo;                       // (re | im << 16)
+            split_pair(v4[m], hi, lo);
+            unsigned char *ah = smem + e.a0 + (size_t)(2 * m) * e.a_bytes;
+            unsigned char *al = ah + e.a_bytes;
+            // row 2i: (Xr, Xi); row 2i + 1: (-Xi, Xr)
+            *reinterpret_cast<uint32_t *>(ah + o0) = hi;
+            *reinterpret_cast<uint32_t *>(al + o0) = lo;
+            *reinterpret_cast<uint32_t *>(ah + o1) = neg_bf16_lo(hi >> 16) | (hi << 16);
+            *reinterpret_cast<uint32_t *>(al + o1) = neg_bf16_lo(lo >> 16) | (lo << 16);
+          }
+        }
+        if ((it * MT_XB + u) * MT_THREADS + tid < ndp) {
+          const float2 v4[4] = {make_float2(dv[u][0].x, dv[u][0].y), make_float2(dv[u][0].z, dv[u][0].w),
+                                make_float2(dv[u][1].x, dv[u][1].y), make_float2(dv[u][1].z, dv[u][1].w)};
+          const uint32_t off = mt_off(dor[u], 2 * db_[u], e.sbo);
+#pragma unroll
+          for (int m = 0; m < MB; ++m) {
+            uint32_t hi, lo;
+            split_pair(v4[m], hi, lo);
+            unsigned char *bh = smem + e.b0 + (size_t)(2 * m) * e.b_bytes;
+            *reinterpret_cast<uint32_t *>(bh + off) = hi;
+            *reinterpret_cast<uint32_t *>(bh + e.b_bytes + off) = lo;
+          }
+        }
+      }
+    }
+  }
+  tc::fence_proxy_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = *tslot;
+
+  if (warp == 0) {
+    if (tc::elect_one()) {
+      const uint32_t idesc = tc::instr_desc(tc::FMT_BF16, MT_ROWS, e.NP);
+      const int nks = 2 * e.KB / 16;
+      for (int m = 0; m < MB; ++m) {
+        const uint32_t d = tbase + (uint32_t)(m * e.NP);
+        unsigned char *am = smem + e.a0 + (size_t)(2 * m) * e.a_bytes;
+        unsigned char *bm = smem + e.b0 + (size_t)(2 * m) * e.b_bytes;
+        const uint64_t ah = tc::smem_desc_kmajor(tc::smem_u32(am), 128, e.sbo);
+        const uint64_t al = tc::smem_desc_kmajor(tc::smem_u32(am + e.a_bytes), 128, e.sbo);
+        const uint64_t bh = tc::smem_desc_kmajor(tc::smem_u32(bm), 128, e.sbo);
+        const uint64_t bl = tc::smem_desc_kmajor(tc::smem_u32(bm + e.b_bytes), 128, e.sbo);
+        for (int ks = 0; ks < nks; ++ks)
+          tc::mma_f16_ss(d, ah + 16u * ks, bh + 16u * ks, idesc, ks > 0 ? 1u : 0u);
+        for (int ks = 0; ks < nks; ++ks) tc::mma_f16_ss(d, ah + 16u * ks, bl + 16u * ks, idesc, 1u);
+        for (int ks = 0; ks < nks; ++ks) tc::mma_f16_ss(d, al + 16u * ks, bh + 16u * ks, idesc, 1u);
+      }
+      tc::mma_commit(bar);
+    }
+    __syncwarp();
+  }
+  bool ok = tc::mbar_wait(bar, 0, err);
+  if (!ok) tc::mbar_wait(bar, 0, nullptr);   // drain before TMEM is released
+  tc::fence_after_sync();
+
+  if (ok) {
+    const int q = warp & 3;
+    const int row = 32 * q + lane;               // 2 i + c
+    const int i = row >> 1, c = row & 1;
+    const uint32_t lane_base = tbase + ((uint32_t)(32 * q) << 16);
+    float wk[MB];
+#pragma unroll
+    for (int m = 0; m < MB; ++m) wk[m] = mode_weight((int)((k0 + m) % mL), NL, inv_n);
+    for (int c0 = (warp >> 2) * 8; c0 < e.NP; c0 += (MT_THREADS / 128) * 8) {
+      uint32_t v[MB][8];
+#pragma unroll
+      for (int m = 0; m < MB; ++m) tc::tmem_ld8(lane_base + (uint32_t)(m * e.NP + c0), v[m]);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float own[MB], oth[MB];
+#pragma unroll
+        for (int m = 0; m < MB; ++m) {
+          own[m] = __uint_as_float(v[m][j]);
+          oth[m] = __shfl_xor_sync(0xffffffffu, own[m], 1);
+        }
+        const int o = c0 + j;
+        if ((j & 1) == c && o < Co) {
+          float2 y[MB];
+#pragma unroll
+          for (int m = 0; m < MB; ++m) {
+            const float re = c == 0 ? own[m] : oth[m], im = c == 0 ? oth[m] : own[m];
+            y[m] = make_float2(wk[m] * re, wk[m] * im);
+          }
+          float4 *dst = reinterpret_cast<float4 *>(dR + 2 * (((long long)i * Co + o) * K + k0));
+          dst[0] = make_float4(y[0].x, y[0].y, y[1].x, y[1].y);
+          if constexpr (MB == 4) dst[1] = make_float4(y[2].x, y[2].y, y[3].x, y[3].y);
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tbase, e.cols);
+  }
+}
+
+inline int dr_modes(long long B, int Co) {
+  if (dr_geom(B, Co, 4).total <= MT_SMEM_MAX) return 4;
+  if (dr_geom(B, Co, 2).total <= MT_SMEM_MAX) return 2;
+  return 0;
+}
+
 inline int mt_modes(long long B, int NR) {
   if (mt_geom(B, NR, 4).total <= MT_SMEM_MAX) return 4;
   if (mt_geom(B, NR, 2).total <= MT_SMEM_MAX) return 2;
@@ -306,6 +516,34 @@ cudaError_t launch_mix_tc(const Launch &L, const Geom &g, bool adj, int Ci, int 
   };
   if (adj) return mb == 4 ? go(k_mix_tc<4, true>) : go(k_mix_tc<2, true>);
   return mb == 4 ? go(k_mix_tc<4, false>) : go(k_mix_tc<2, false>);
+}
+
+}  // namespace fno
+
+namespace fno {
+
+bool mix_tc_dr_supported(const Geom &g, int dtype, int Ci, int Co, const void *X, const void *D,
+                         const void *dR) {
+  if (dtype == DT_F32 || Ci != 64 || Co < 1 || Co > 64) return false;
+  if (g.B < 1 || g.B > 64 || g.K % 4 != 0) return false;
+  if (((uintptr_t)X | (uintptr_t)D | (uintptr_t)dR) & 31) return false;
+  return dr_modes(g.B, Co) > 0;
+}
+
+cudaError_t launch_mix_tc_dr(const Launch &L, const Geom &g, int Co, const float2 *X,
+                             const float2 *D, float *dR) {
+  const int mb = dr_modes(g.B, Co);
+  const DrGeom e = dr_geom(g.B, Co, mb);
+  const unsigned grid = (unsigned)((g.K + mb - 1) / mb);
+  auto go = [&](auto kern) {
+    cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)e.total);
+    if (r != cudaSuccess) return r;
+    kern<<<grid, MT_THREADS, e.total, L.stream>>>(X, D, dR, (int)g.B, Co, g.K, g.mL, g.NL,
+                                                   g.inv_n, L.err);
+    return cudaGetLastError();
+  };
+  return mb == 4 ? go(k_mix_tc_dr<4>) : go(k_mix_tc_dr<2>);
 }
 
 }  // namespace fno

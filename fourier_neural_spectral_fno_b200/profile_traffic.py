@@ -79,6 +79,8 @@ def _kernel_key(name: str):
         args = [t.strip() for t in (targs or "").split(",")]
         dz = bool(args) and args[-1] in ("true", "1")
         return ("fwd_plane_dz" if dz else "fwd_plane", "transform_plane.cu")
+    if base == "k_mix_tc_dr":
+        return ("mix_bwd_dr_tc", "mix_tc.cu")
     if base == "k_mix_tc":      # k_mix_tc<MB, ADJ>: the adjoint has its own tag
         args = [t.strip() for t in (targs or "").split(",")]
         adj = bool(args) and args[-1] in ("true", "1")

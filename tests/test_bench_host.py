@@ -111,7 +111,7 @@ def test_traffic_records_and_bench_name_the_same_source():
     spec.loader.exec_module(bench)
     pairs = set(pt.KERNELS.values()) | {(t, "epilogue.cu") for t in pt.EPILOGUE_TAGS.values()}
     pairs |= {("fwd_plane_dz", "transform_plane.cu"), ("mix_fwd_tc", "mix_tc.cu"),
-              ("mix_bwd_dx_tc", "mix_tc.cu")}
+              ("mix_bwd_dx_tc", "mix_tc.cu"), ("mix_bwd_dr_tc", "mix_tc.cu")}
     for tag, src in sorted(pairs):
         path = os.path.join(ROOT, "fourier_neural_spectral_fno_b200", "csrc", src)
         assert os.path.isfile(path), src
