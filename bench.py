@@ -320,7 +320,7 @@ def roofline_record(dom: str, avg_ms: float, wl, n_sms: int) -> dict:
                 "hbm_view": {"achieved": gbs, "peak": hbm, "unit": "GB/s",
                              "frac": (gbs / hbm) if gbs else None}}
     return {"kernel": dom, "bound": "hbm", "achieved": gbs, "peak": hbm,
-            "peak_source": f"{hbm_src} (MEASURED_PEAKS.json hbm_gbs, copy)",
+            "peak_source": hbm_src,
             "unit": "GB/s", "frac": (gbs / hbm) if gbs else None,
             "traffic": measured_traffic(dom, wl), "avg_launch_ms": avg_ms,
             "algorithmic_bytes_per_launch": alg}
@@ -352,18 +352,20 @@ def block_roofline_record(stats: dict, steps: int, wl) -> dict:
             break
         traffic += per_launch * stats[t]["launches"] / steps / wl.n_layers
     return {"scope": "one spectral block (all its kernels)", "bound": "hbm", "achieved": gbs,
-            "peak": hbm, "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs, copy)",
+            "peak": hbm, "peak_source": src,
             "unit": "GB/s", "frac": gbs / hbm, "block_ms": ms,
             "algorithmic_bytes_per_block": float(alg), "traffic": traffic,
             "kernels": sorted(tags)}
 
 
 def hbm_peak():
+    """The copy bandwidth the HBM fractions divide by, and where it came from."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
-        return float(json.load(open(path))["hbm_gbs"]), "measured"
+        return (float(json.load(open(path))["hbm_gbs"]),
+                "measured (MEASURED_PEAKS.json hbm_gbs, a STREAM-style copy)")
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback"
+        return FALLBACK_HBM_GBS, "fallback (MEASURED_PEAKS.json absent; an earlier copy measurement)"
 
 
 def cpu_threads() -> int:
